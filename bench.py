@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Render + analytic score replay throughput on B200.
+
+One step = the whole path over one synthetic scene: preprocess (EWA projection, SH colour),
+tile binning + depth sort, front-to-back compositing, score replay + token finalisation, for all
+target views. Default workload: the DepthSplat-scale dense scene (5,898,240 Gaussians, SH degree
+3, 4 target views 512x960). Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank renders and scores its own replica of the
+workload (no data-path collective); value = all ranks' pixels / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "render+score-replay Mpix/s & Gaussian-pixel pairs/s; % of FP32/HBM roofline"
+WORKLOADS = {
+    1: "two_plane_occlusion_64x64_1v_256g",
+    2: "three_layer_occlusion_128x128_4v_4096g",
+    3: "resplat_pixel_aligned_256x448_8v_917504g_sh2",
+    4: "atsplat_anchor_512x960_4v_311296g_sh2",
+    5: "depthsplat_dense_512x960_4v_5898240g_sh3",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-tiles", type=int, default=0,
+                    help="tiles per sample for the CPU oracle (0 = size for ~10-20 s)")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------------------------
+# clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, p in zip(names, parts[3:7]):
+                if p.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_id_for(dev) -> str | None:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------------------------
+# roofline bookkeeping (algorithmic bytes / work per launch; see the design notes)
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
+    """Bytes each kernel group must move by its definition (unique inputs + outputs)."""
+    G, V, H, W, d = sc.G, sc.V, sc.H, sc.W, sc.d
+    px = V * H * W
+    TX, TY = (W + 15) // 16, (H + 15) // 16
+    return {
+        # read the parameters once, write per (v, g) record (64 B), rectangle (16 B), count (4 B)
+        "project": G * (4 * (3 + 3 + 4 + 1) + 12 * d) + V * G * (64 + 16 + 4),
+        "scan_counts": V * G * (4 + 8),
+        # read rectangle + depth, write (tile, depth, g) per instance
+        "emit": V * G * (16 + 4) + n_inst * 12,
+        "tile_hist": n_inst * 4,
+        "tile_scatter": n_inst * (4 + 8 + 8),
+        "tile_sort": n_inst * (8 + 4),
+        # gather 36 B per list entry staged, write C_hat, T, n, last
+        "render": n_inst * (4 + 36) + px * 24,
+        "replay": n_inst * (4 + 36) + px * (12 + 12 + 4) + V * G * 64,
+        "finalize": V * G * (64 + 64) + G * 4 * (9 + 3 * d),
+        "tiles": V * TX * TY,
+    }
+
+
+# instructions per traversed (pixel, entry) pair in the fp32 pipe, counted from the kernels'
+# arithmetic (see the design notes): alpha evaluation incl. exp, compositing or replay terms
+ALU_OPS_PER_PAIR = {"render": 40, "replay": 75}
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU oracle baseline: bounded sample, extrapolated to the metric's unit
+
+def cpu_oracle_sample(sc, obs_np, seconds_hint=15.0, tiles=0):
+    import numpy as np
+    from oracle import oracle as O
+    one = _one_view(sc)
+    t0 = time.perf_counter()
+    p = O.project(one, "f")
+    L = O.bin_lists(p, one.H, one.W)
+    t_pb = time.perf_counter() - t0
+    TX, TY = O.n_tiles(one.H, one.W)
+    nt = TX * TY
+    rng = np.random.default_rng(0)
+    n_s = tiles or max(8, min(nt, int(nt * 0.04)))
+    sel = np.stack([np.zeros(n_s, np.int32), rng.choice(nt, n_s, replace=False).astype(np.int32)], 1)
+    t1 = time.perf_counter()
+    r = O.render(p, L, one.H, one.W, one.bg, "f", sel=sel)
+    O.replay(p, L, r, obs_np[:1], one.sh_degree, one.H, one.W, "f", sel=sel)
+    t_rr = time.perf_counter() - t1
+    t2 = time.perf_counter()
+    acc = np.zeros((1, one.G, 8))
+    O.finalize(p, acc, one)
+    t_fin = time.perf_counter() - t2
+    t_view = t_pb + t_rr * nt / n_s + t_fin
+    return {"value": one.H * one.W / t_view / 1e6, "unit": "Mpix/s",
+            "cores": int(O.lib().orc_num_threads()), "kind": "oracle",
+            "sample": (f"1 of {sc.V} views: projection + binning of all {sc.G} Gaussians "
+                       f"({t_pb:.2f} s), render + replay of {n_s}/{nt} random tiles "
+                       f"({t_rr:.2f} s, scaled to the view), finalisation ({t_fin:.2f} s)"),
+            "seconds": t_pb + t_rr + t_fin}
+
+
+def _one_view(sc):
+    import dataclasses
+    return dataclasses.replace(sc, viewmats=sc.viewmats[:1], intrin=sc.intrin[:1])
+
+
+# ----------------------------------------------------------------------------------------------
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, as it stands, on bounded samples of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    from oracle import oracle as O
+    from synth import scenes
+    sc = scenes.make(args.config)
+    obs = scenes.smooth_observation(99, 1, sc.H, sc.W)
+    times, samples = [], []
+    for it in range(args.warmup + args.steps):
+        s = cpu_oracle_sample(sc, obs, tiles=args.cpu_tiles or 0)
+        if it >= args.warmup:
+            times.append(s["seconds"])
+            samples.append(s)
+    val = statistics.median([s["value"] for s in samples])
+    ms = 1e3 * sc.H * sc.W / (val * 1e6)
+    line = {"metric": METRIC, "value": val, "unit": "Mpix/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOADS[args.config], "views_per_step": 1,
+                       "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": val, "unit": "Mpix/s", "cores": samples[0]["cores"],
+                             "kind": "oracle", "sample": samples[0]["sample"]},
+            "e2e": {"value": val, "unit": "Mpix/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import numpy as np
+    import torch
+
+    import gaussian_splatting_raster_b200 as P
+    from gaussian_splatting_raster_b200 import runner
+    from synth import scenes
+
+    rank, world, local = dist_setup()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    P.load_library()  # built in-tree by __graft_entry__.build(); fails loudly when missing
+    sc = scenes.make(args.config)
+    ds = runner.to_device(sc)
+    ws = runner.workspace_for(ds)
+    out = runner.alloc_outputs(ds)
+
+    # observation: render of the perturbed scene (+ pixel noise), made by the same path, untimed
+    obs_scene = runner.to_device(sc.observed_scene())
+    obs_out = runner.alloc_outputs(obs_scene)
+    runner.render(ws, obs_scene, obs_out)
+    obs = obs_out.img.clone()
+    if sc.obs_noise_sigma > 0:
+        obs += torch.from_numpy(sc.pixel_noise()).to(dev)
+    del obs_scene, obs_out
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    l2_flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        return runner.render_and_score(ws, ds, obs, out)
+
+    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
+        n_inst = step()
+    if args.warmup <= 0:
+        n_inst = step()
+    torch.cuda.synchronize()
+    pairs = ws.pair_count()
+    n_total = int(sum(n_inst))
+
+    # ---- timed region: device time per step (CUDA events), L2 flushed between steps ----------
+    sampler = ClockSampler(gpu_id_for(dev)) if rank == 0 else None
+    ws.profile(True)
+    ws.profile_read(reset=True)
+    barrier(world)
+    if sampler:
+        sampler.start()
+    launches_before = ws.launch_count
+    step_ms = []
+    for _ in range(args.steps):
+        l2_flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    launches = ws.launch_count - launches_before
+    kern = ws.profile_read(reset=True)
+    ws.profile(False)
+
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    px_step = sc.V * sc.H * sc.W
+    value = px_step * args.steps * world / (total_ms * 1e-3) / 1e6
+    pairs_per_s = pairs * args.steps * world / (total_ms * 1e-3)
+
+    # ---- end to end through the public API with host buffers ----------------------------------
+    e2e = None
+    if not args.no_e2e:
+        host = {k: torch.from_numpy(np.ascontiguousarray(getattr(sc, k))).pin_memory()
+                for k in ("means", "log_scales", "quats", "opac", "sh", "viewmats", "intrin",
+                          "bg")}
+        host["obs"] = obs.cpu().pin_memory()
+        dev_in = {"means": ds.means, "log_scales": ds.log_scales, "quats": ds.quats,
+                  "opac": ds.opac, "sh": ds.sh, "viewmats": ds.viewmats, "intrin": ds.intrin,
+                  "bg": ds.bg, "obs": obs}
+        h_out = {"tokens": torch.empty(out.tokens.shape, dtype=torch.float32).pin_memory(),
+                 "img": torch.empty(out.img.shape, dtype=torch.float32).pin_memory(),
+                 "T": torch.empty(out.T.shape, dtype=torch.float32).pin_memory(),
+                 "n_contrib": torch.empty(out.n_contrib.shape, dtype=torch.int32).pin_memory()}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+        e2e_ms = []
+        barrier(world)
+        for _ in range(args.steps):
+            l2_flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for k, t in host.items():
+                dev_in[k].copy_(t, non_blocking=True)
+            step()
+            h_out["tokens"].copy_(out.tokens, non_blocking=True)
+            h_out["img"].copy_(out.img, non_blocking=True)
+            h_out["T"].copy_(out.T, non_blocking=True)
+            h_out["n_contrib"].copy_(out.n_contrib, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            e2e_ms.append(e0.elapsed_time(e1))
+        barrier(world)
+        e2e_total = max_over_ranks(sum(e2e_ms), world)
+        e2e = {"value": px_step * args.steps * world / (e2e_total * 1e-3) / 1e6,
+               "unit": "Mpix/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_total / args.steps}
+
+    # ---- roofline of the dominant kernel ------------------------------------------------------
+    peaks = load_peaks()
+    ab = algorithmic_bytes(sc, n_total, pairs)
+    per_kernel = {k: {"ms_per_step": v[0] / args.steps, "launches": v[1]}
+                  for k, v in kern.items() if v[1] > 0}
+    dom = max(per_kernel, key=lambda k: per_kernel[k]["ms_per_step"])
+    dom_ms = per_kernel[dom]["ms_per_step"]
+    lanes = torch.cuda.get_device_properties(dev).multi_processor_count * 128
+    if dom in ALU_OPS_PER_PAIR:
+        ops = ALU_OPS_PER_PAIR[dom] * pairs
+        achieved = ops / (dom_ms * 1e-3) / 1e12
+        peak = lanes * peaks["sm_max_mhz"] * 1e6 / 1e12
+        roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "Tops/s (fp32 pipe)", "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{lanes} fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz "
+                               f"({peaks['source']} max clock)"}
+    else:
+        achieved = ab.get(dom, 0) / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peaks['source']} copy bandwidth"}
+    for k, v in per_kernel.items():
+        if k in ab:
+            v["algorithmic_GBps"] = ab[k] / (v["ms_per_step"] * 1e-3) / 1e9
+    render_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in
+                    ("project", "scan_counts", "emit", "tile_hist", "hist_scan", "tile_scatter",
+                     "tile_ranges", "tile_sort", "render", "other"))
+    replay_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in ("replay", "finalize"))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(sc, obs.cpu().numpy(), tiles=args.cpu_tiles)
+        cpu.pop("seconds", None)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.config], "gaussians": sc.G, "views": sc.V,
+                       "height": sc.H, "width": sc.W, "sh_degree": sc.sh_degree,
+                       "instances_per_step": n_total, "pairs_per_step": pairs,
+                       "l2": "256 MiB buffer written between timed steps",
+                       "parallelism": f"replicas x{world}"},
+            "pairs_per_s": pairs_per_s,
+            "ms_view": ms_per_step / sc.V,
+            "render_ms_per_step": render_ms, "replay_ms_per_step": replay_ms,
+            "replay_over_render": replay_ms / render_ms if render_ms else None,
+            "gpu_launches": int(launches), "per_kernel": per_kernel,
+            "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    ws.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

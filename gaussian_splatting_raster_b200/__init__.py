@@ -1,0 +1,228 @@
+"""B200-native tile-based Gaussian-splatting render + analytic score replay.
+
+Thin ctypes binding of ``libsplat.so`` (C ABI in ``include/splat.h``). Every step of the path runs
+in the library's CUDA kernels; this module only checks tensor arguments and passes device pointers
+and the current CUDA stream. There is no CPU fallback: without the built library or a CUDA device
+the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB, build  # noqa: F401
+
+__all__ = ["Workspace", "SplatError", "load_library", "LIB", "build", "token_dim"]
+
+_ERRORS = {
+    -1: "INVALID_ARG", -2: "CAPACITY", -3: "STATE", -4: "CUDA", -5: "BOUNDS",
+    -6: "DEVICE_TIMEOUT", -7: "OOM",
+}
+
+# every symbol include/splat.h declares (checked against the header by the tests)
+EXPORTS = [
+    "splat_ws_create", "splat_ws_destroy", "splat_last_error", "splat_project",
+    "splat_bin_sort", "splat_render", "splat_score_replay", "splat_copy_projection",
+    "splat_copy_tile_lists", "splat_copy_last", "splat_copy_accumulators", "splat_pair_count",
+    "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
+]
+
+
+KERNEL_GROUPS = 12  # SPLAT_NUM_KERNELS
+
+
+class SplatError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"splat error {code} ({_ERRORS.get(code, '?')}): {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Load libsplat.so (raises OSError when it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB
+    if not os.path.exists(p):
+        raise OSError(f"libsplat.so not built at {p}; run gaussian_splatting_raster_b200.build()")
+    L = ctypes.CDLL(p)
+    V, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+    L.splat_ws_create.argtypes = [ctypes.POINTER(V), I, I, I, I, I]
+    L.splat_ws_create.restype = I
+    L.splat_ws_destroy.argtypes = [V]
+    L.splat_ws_destroy.restype = None
+    L.splat_last_error.argtypes = [V]
+    L.splat_last_error.restype = ctypes.c_char_p
+    L.splat_project.argtypes = [V, V, V, V, V, V, I, I, V, V, I, I, I, V]
+    L.splat_project.restype = I
+    L.splat_bin_sort.argtypes = [V, ctypes.POINTER(LL), V]
+    L.splat_bin_sort.restype = I
+    L.splat_render.argtypes = [V, V, V, V, V, V]
+    L.splat_render.restype = I
+    L.splat_score_replay.argtypes = [V, V, F, V, V]
+    L.splat_score_replay.restype = I
+    L.splat_copy_projection.argtypes = [V, V, V, V]
+    L.splat_copy_projection.restype = I
+    L.splat_copy_tile_lists.argtypes = [V, V, V, V]
+    L.splat_copy_tile_lists.restype = I
+    L.splat_copy_last.argtypes = [V, V, V]
+    L.splat_copy_last.restype = I
+    L.splat_copy_accumulators.argtypes = [V, V, V]
+    L.splat_copy_accumulators.restype = I
+    L.splat_pair_count.argtypes = [V, ctypes.POINTER(LL), V]
+    L.splat_pair_count.restype = I
+    L.splat_launch_count.argtypes = [V]
+    L.splat_launch_count.restype = LL
+    L.splat_profile_enable.argtypes = [V, I]
+    L.splat_profile_enable.restype = I
+    L.splat_profile_read.argtypes = [V, V, V, I]
+    L.splat_profile_read.restype = I
+    L.splat_kernel_name.argtypes = [I]
+    L.splat_kernel_name.restype = ctypes.c_char_p
+    if path is None:
+        _lib = L
+    return L
+
+
+def token_dim(sh_degree: int) -> int:
+    return 9 + 3 * (sh_degree + 1) ** 2
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t, name, dtype, shape=None):
+    import torch
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Workspace:
+    """Library-owned workspace (records, tile lists, accumulators) for problems up to the given
+    maxima. Calls enqueue on the current torch CUDA stream unless one is passed."""
+
+    def __init__(self, max_G: int, max_V: int, max_H: int, max_W: int, max_sh_degree: int = 3):
+        self._L = load_library()
+        h = ctypes.c_void_p()
+        rc = self._L.splat_ws_create(ctypes.byref(h), max_G, max_V, max_H, max_W, max_sh_degree)
+        if rc != 0:
+            raise SplatError(rc, "workspace creation failed")
+        self._h = h
+        self.G = self.V = self.H = self.W = self.deg = 0
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._L.splat_ws_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, rc):
+        if rc != 0:
+            raise SplatError(rc, self._L.splat_last_error(self._h).decode())
+
+    # -- the path -------------------------------------------------------------------------------
+    def project(self, means, log_scales, quats, opac_logits, sh, viewmats, intrin, H, W,
+                stream=None):
+        import torch
+        G = means.shape[0]
+        V = viewmats.shape[0]
+        d = sh.shape[1] if sh.dim() == 3 else 1
+        deg = {1: 0, 4: 1, 9: 2, 16: 3}.get(d)
+        if deg is None:
+            raise ValueError("sh must be [G, (deg+1)^2, 3] with deg <= 3")
+        f = torch.float32
+        args = [_ptr(means, "means", f, (G, 3)), _ptr(log_scales, "log_scales", f, (G, 3)),
+                _ptr(quats, "quats", f, (G, 4)), _ptr(opac_logits, "opac_logits", f, (G,)),
+                _ptr(sh, "sh", f, (G, d, 3))]
+        self._check(self._L.splat_project(
+            self._h, *args, G, deg, _ptr(viewmats, "viewmats", f, (V, 4, 4)),
+            _ptr(intrin, "intrin", f, (V, 4)), V, H, W, _stream(stream)))
+        self.G, self.V, self.H, self.W, self.deg = G, V, H, W, deg
+
+    def bin_sort(self, stream=None) -> list[int]:
+        out = (ctypes.c_longlong * max(self.V, 1))()
+        self._check(self._L.splat_bin_sort(self._h, out, _stream(stream)))
+        return [int(out[i]) for i in range(self.V)]
+
+    def render(self, bg, img, T_final, n_contrib, stream=None):
+        import torch
+        V, H, W = self.V, self.H, self.W
+        self._check(self._L.splat_render(
+            self._h, _ptr(bg, "bg", torch.float32, (3,)),
+            _ptr(img, "img", torch.float32, (V, H, W, 3)),
+            _ptr(T_final, "T_final", torch.float32, (V, H, W)),
+            _ptr(n_contrib, "n_contrib", torch.int32, (V, H, W)), _stream(stream)))
+
+    def score_replay(self, obs, tokens, lam: float = 1.0, stream=None):
+        import torch
+        V, H, W = self.V, self.H, self.W
+        self._check(self._L.splat_score_replay(
+            self._h, _ptr(obs, "obs", torch.float32, (V, H, W, 3)), ctypes.c_float(lam),
+            _ptr(tokens, "tokens", torch.float32, (self.G, token_dim(self.deg))),
+            _stream(stream)))
+
+    # -- inspection -----------------------------------------------------------------------------
+    def copy_projection(self, rec, rect, stream=None):
+        import torch
+        self._check(self._L.splat_copy_projection(
+            self._h, _ptr(rec, "rec", torch.float32, (self.V, self.G, 16)),
+            _ptr(rect, "rect", torch.int32, (self.V, self.G, 4)), _stream(stream)))
+
+    def copy_tile_lists(self, tile_offsets, ids, stream=None):
+        import torch
+        self._check(self._L.splat_copy_tile_lists(
+            self._h, _ptr(tile_offsets, "tile_offsets", torch.int64),
+            _ptr(ids, "ids", torch.int32), _stream(stream)))
+
+    def copy_last(self, last, stream=None):
+        import torch
+        self._check(self._L.splat_copy_last(
+            self._h, _ptr(last, "last", torch.int32, (self.V, self.H, self.W)), _stream(stream)))
+
+    def copy_accumulators(self, acc, stream=None):
+        import torch
+        self._check(self._L.splat_copy_accumulators(
+            self._h, _ptr(acc, "acc", torch.float64, (self.V, self.G, 8)), _stream(stream)))
+
+    def pair_count(self, stream=None) -> int:
+        out = ctypes.c_longlong()
+        self._check(self._L.splat_pair_count(self._h, ctypes.byref(out), _stream(stream)))
+        return int(out.value)
+
+    @property
+    def launch_count(self) -> int:
+        return int(self._L.splat_launch_count(self._h))
+
+    def profile(self, enable: bool = True):
+        """Bracket every kernel with CUDA events (per-kernel device time)."""
+        self._check(self._L.splat_profile_enable(self._h, 1 if enable else 0))
+
+    def profile_read(self, reset: bool = True) -> dict:
+        """{kernel group name: (milliseconds, timed launches)} since the last reset."""
+        n = KERNEL_GROUPS
+        ms = (ctypes.c_double * n)()
+        cnt = (ctypes.c_longlong * n)()
+        self._check(self._L.splat_profile_read(self._h, ms, cnt, 1 if reset else 0))
+        return {self._L.splat_kernel_name(i).decode(): (float(ms[i]), int(cnt[i]))
+                for i in range(n)}

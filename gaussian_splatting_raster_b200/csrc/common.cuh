@@ -1,0 +1,224 @@
+// Internal definitions shared by the libsplat CUDA translation units.
+//
+// Every file of the library is compiled with -fmad=false (no implicit multiply-add
+// contraction), IEEE division and square root, and denormals preserved. The preprocess, render
+// and replay decisions that turn floating point into integers (tile rectangle, depth order, the
+// 1/255 and 1e-4 thresholds, the 0.99 clamp) therefore depend only on the stated sequence of
+// correctly rounded fp32 operations; fused multiply-adds appear only where written as fmaf().
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "splat.h"
+
+namespace splat {
+
+constexpr int kTile = 16;        // 16x16 pixel tiles
+constexpr int kTilePix = 256;
+constexpr int kRecF4 = 4;        // float4 per (v, g) record
+constexpr int kAccN = 8;         // doubles per (v, g) accumulator
+constexpr int kFlagVisible = 256;
+
+// Record of one (view, Gaussian), 4 x float4 = 64 bytes, array-of-structures so that the
+// render's gather of one list entry touches two 32-byte sectors:
+//   r0 = (mx, my, conic a, conic b)        r1 = (conic c, opacity, colour r, colour g)
+//   r2 = (colour b, depth z, x_c, y_c)     r3 = (dir x, dir y, dir z, flags as int bits)
+// flags: bits 0..2 colour clamp inactive per channel (M_color), bit 8 visible.
+
+// ---------------------------------------------------------------------------------------------
+// exp for the decision path, written from Cody & Waite (1980), "Software Manual for the
+// Elementary Functions": x = k ln2 + r with k = rint(x log2 e), ln2 split into a 16-bit high
+// part (k * hi exact for |k| <= 128) and a low correction, e^r by its Taylor series to degree 7
+// (Horner, fused multiply-adds) on |r| <= ln2 / 2, scaled by 2^k through the exponent field.
+// Zero below -87, +inf above 88.
+// ---------------------------------------------------------------------------------------------
+namespace cw {
+constexpr double kLn2 = 0.693147180559945309417232121458;
+constexpr float kLog2e = (float)(1.0 / kLn2);
+constexpr float kLn2Hi = 45426.0f / 65536.0f;  // floor(ln2 * 2^16) / 2^16
+constexpr float kLn2Lo = (float)(kLn2 - 45426.0 / 65536.0);
+constexpr float kC2 = (float)(1.0 / 2.0);
+constexpr float kC3 = (float)(1.0 / 6.0);
+constexpr float kC4 = (float)(1.0 / 24.0);
+constexpr float kC5 = (float)(1.0 / 120.0);
+constexpr float kC6 = (float)(1.0 / 720.0);
+constexpr float kC7 = (float)(1.0 / 5040.0);
+}  // namespace cw
+
+__device__ __forceinline__ float exp_cw(float x) {
+  if (x != x) return x;
+  if (!(x > -87.0f)) return 0.0f;
+  if (x > 88.0f) return __int_as_float(0x7f800000);
+  const float k = rintf(x * cw::kLog2e);
+  const float r = (x - k * cw::kLn2Hi) - k * cw::kLn2Lo;
+  float p = cw::kC7;
+  p = fmaf(p, r, cw::kC6);
+  p = fmaf(p, r, cw::kC5);
+  p = fmaf(p, r, cw::kC4);
+  p = fmaf(p, r, cw::kC3);
+  p = fmaf(p, r, cw::kC2);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  return p * __int_as_float(((int)k + 127) << 23);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Real spherical harmonics up to degree 3 of a unit direction, Condon-Shortley phase (the 3DGS
+// colour model), as Cartesian polynomials. Normalisations: Y00 = 1/(2 sqrt(pi));
+// l=1: sqrt(3/(4 pi)); l=2: sqrt(15/pi)/2, sqrt(5/pi)/4, sqrt(15/pi)/4;
+// l=3: sqrt(35/(2 pi))/4, sqrt(105/pi)/2, sqrt(21/(2 pi))/4, sqrt(7/pi)/4, sqrt(105/pi)/4.
+// ---------------------------------------------------------------------------------------------
+template <int DEG>
+__device__ __forceinline__ void sh_poly(float x, float y, float z, float* B) {
+  B[0] = 0.28209479177387814f;
+  if (DEG >= 1) {
+    const float c1 = 0.48860251190291992f;
+    B[1] = -c1 * y;
+    B[2] = c1 * z;
+    B[3] = -c1 * x;
+  }
+  if (DEG >= 2) {
+    const float xx = x * x, yy = y * y, zz = z * z;
+    B[4] = 1.0925484305920792f * (x * y);
+    B[5] = -1.0925484305920792f * (y * z);
+    B[6] = 0.31539156525252005f * (2.0f * zz - xx - yy);
+    B[7] = -1.0925484305920792f * (x * z);
+    B[8] = 0.54627421529603959f * (xx - yy);
+    if (DEG >= 3) {
+      B[9] = -0.59004358992664352f * y * (3.0f * xx - yy);
+      B[10] = 2.8906114426405538f * (x * y) * z;
+      B[11] = -0.45704579946446572f * y * (4.0f * zz - xx - yy);
+      B[12] = 0.37317633259011540f * z * (2.0f * zz - 3.0f * xx - 3.0f * yy);
+      B[13] = -0.45704579946446572f * x * (4.0f * zz - xx - yy);
+      B[14] = 1.4453057213202769f * z * (xx - yy);
+      B[15] = -0.59004358992664352f * x * (xx - 3.0f * yy);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// workspace
+// ---------------------------------------------------------------------------------------------
+struct Workspace {
+  int device = 0;
+  int max_G = 0, max_V = 0, max_H = 0, max_W = 0, max_deg = 0, max_nt = 0;
+  // current problem
+  int G = 0, V = 0, H = 0, W = 0, deg = 0, TX = 0, TY = 0, nt = 0;
+  int stage = 0;  // 0 empty, 1 projected, 2 binned, 3 rendered, 4 replayed
+  long long launches = 0;
+
+  // per (v, g)
+  float4* rec = nullptr;     // [V*G*4]
+  int4* rect = nullptr;      // [V*G]
+  int* counts = nullptr;     // [V*G] tiles touched
+  long long* offs = nullptr; // [V*G + 1] exclusive scan of counts
+  double* acc = nullptr;     // [V*G*8]
+  float* views = nullptr;    // [V*20]: viewmat (16) + intrinsics (4)
+  int* last = nullptr;       // [V*H*W]
+  const float* img = nullptr;  // C_hat written by the last render (caller-owned)
+
+  // scan partials (int64)
+  long long* part = nullptr;
+  size_t part_cap = 0;
+
+  // instances
+  size_t inst_cap = 0;
+  uint32_t* inst_tile = nullptr;  // [N] tile id within its view
+  uint2* inst_kv = nullptr;       // [N] (depth bits, g)
+  uint32_t* skey = nullptr;       // [N] depth bits, tile-major
+  uint32_t* sval = nullptr;       // [N] g, tile-major; after the depth sort: the tile lists
+  uint32_t* skey2 = nullptr;      // [N] ping-pong for long tiles
+  uint32_t* sval2 = nullptr;
+
+  // tile histogram [sum_v nt * blocks_v] (int32, scanned in place)
+  size_t hist_cap = 0;
+  int* hist = nullptr;
+  long long* tile_off = nullptr;  // [V*(nt+1)]
+
+  // per-view tables
+  long long* d_vstart = nullptr;  // [V+1] first instance of each view
+  int* d_bstart = nullptr;        // [V+1] first binning block of each view
+  long long* h_vstart = nullptr;  // pinned
+  int* h_bstart = nullptr;        // pinned
+  long long n_total = 0;
+  int n_blocks = 0;
+
+  long long* d_scratch = nullptr;  // small device scratch (reductions)
+  long long* h_scratch = nullptr;  // pinned
+
+  // per-kernel timing (off by default)
+  bool prof = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<int> ev_open;  // (id, start event, end event) triples of recorded launches
+  int ev_used = 0;
+  double prof_ms[SPLAT_NUM_KERNELS] = {0};
+  long long prof_n[SPLAT_NUM_KERNELS] = {0};
+
+  std::string err;
+};
+
+}  // namespace splat
+
+struct splat_ws {
+  splat::Workspace w;
+};
+
+// launch helpers ------------------------------------------------------------------------------
+namespace splat {
+
+inline int set_err(Workspace& w, int code, const std::string& msg) {
+  w.err = msg;
+  return code;
+}
+
+// Bracket a kernel with timing events when profiling is on. Returns a token for prof_end.
+inline int prof_begin(Workspace& w, cudaStream_t st, int id) {
+  if (!w.prof) return -1;
+  while ((int)w.ev_pool.size() < w.ev_used + 2) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return -1;
+    w.ev_pool.push_back(e);
+  }
+  const int a = w.ev_used;
+  w.ev_used += 2;
+  cudaEventRecord(w.ev_pool[a], st);
+  w.ev_open.push_back(id);
+  w.ev_open.push_back(a);
+  return a;
+}
+inline void prof_end(Workspace& w, cudaStream_t st, int tok) {
+  if (tok < 0) return;
+  cudaEventRecord(w.ev_pool[tok + 1], st);
+}
+
+inline int check_launch(Workspace& w, const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return set_err(w, SPLAT_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  w.launches += 1;
+  return SPLAT_OK;
+}
+
+// host entry points implemented in the .cu files
+int launch_project(Workspace& w, const float* means, const float* lsc, const float* quats,
+                   const float* opac, const float* sh, cudaStream_t st);
+int launch_scan_counts(Workspace& w, cudaStream_t st);
+int launch_binning(Workspace& w, cudaStream_t st);
+int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int* n_contrib,
+                  cudaStream_t st);
+int launch_replay(Workspace& w, const float* obs, cudaStream_t st);
+int launch_finalize(Workspace& w, float lambda, float* tokens, cudaStream_t st);
+int launch_pair_count(Workspace& w, cudaStream_t st);
+int binning_configure(Workspace& w);
+
+// reduce-then-scan over n int32 values into int64 exclusive prefixes (out has n + 1 entries; the
+// last is the total). Uses w.part as scratch.
+int scan_i32_to_i64(Workspace& w, const int* in, long long* out, long long n, cudaStream_t st);
+// same, int32 in place (values and total < 2^31)
+int scan_i32_inplace(Workspace& w, int* data, long long n, cudaStream_t st);
+
+}  // namespace splat

@@ -1,0 +1,163 @@
+// Token finalisation: per Gaussian, over the views in which it is visible, the cross-view
+// weights, the 3-D covector pullback of the projected-centre score, the conditioning statistics
+// and the cross-view appearance scores.
+//
+// Source: "Research Proposal: Renderer Score Tokens for Recurrent Gaussian Splatting",
+// "Exact Score Operators" (q_gv = eps + sum_p w; opacity-logit score; SH score; projected-centre
+// score with grad G = G Sigma2D^-1 (p - mu2D); J_gv = d pi_v(mu_g) / d mu_g;
+// gamma_gv = q_gv / (eps + sum_v' q_gv'); b = sum_v gamma J^T s^mu2D; A = lambda I +
+// sum_v gamma J^T J; e~ = eig(A) / (tr A + eps); l = log(tr A + eps); s^alpha_g and s^SH_g as
+// gamma-weighted sums) and "Final Token and Updater" (z_g = [b(3), s^alpha, s^SH(3 d_SH),
+// log q_g, e~(3), l], 9 + 3 d_SH entries).
+//
+// Because gamma_gv / q_gv = 1 / q_g for every view, each block is a plain sum over views divided
+// once by q_g (the linear rewrite; no second pass over the views). Sums and the eigenvalues are
+// evaluated in double; the SH block's per-view products in fp32.
+#include "common.cuh"
+
+namespace splat {
+namespace {
+
+constexpr int kFinThreads = 128;
+
+// eigenvalues of a symmetric 3x3 matrix, descending, by the trigonometric solution of the
+// characteristic cubic (O. K. Smith, "Eigenvalues of a symmetric 3x3 matrix", CACM 4(4), 1961)
+__device__ void eig3_sym(double a00, double a01, double a02, double a11, double a12, double a22,
+                         double ev[3]) {
+  const double p1 = a01 * a01 + a02 * a02 + a12 * a12;
+  const double q = (a00 + a11 + a22) / 3.0;
+  const double d0 = a00 - q, d1 = a11 - q, d2 = a22 - q;
+  const double p2 = d0 * d0 + d1 * d1 + d2 * d2 + 2.0 * p1;
+  if (p2 <= 0.0) {
+    ev[0] = ev[1] = ev[2] = q;
+    return;
+  }
+  const double p = sqrt(p2 / 6.0);
+  const double ip = 1.0 / p;
+  const double b00 = d0 * ip, b11 = d1 * ip, b22 = d2 * ip;
+  const double b01 = a01 * ip, b02 = a02 * ip, b12 = a12 * ip;
+  const double detB = b00 * (b11 * b22 - b12 * b12) - b01 * (b01 * b22 - b12 * b02) +
+                      b02 * (b01 * b12 - b11 * b02);
+  double r = 0.5 * detB;
+  r = fmin(1.0, fmax(-1.0, r));
+  const double phi = acos(r) / 3.0;
+  const double e1 = q + 2.0 * p * cos(phi);
+  const double e3 = q + 2.0 * p * cos(phi + 2.0943951023931954923);  // + 2 pi / 3
+  const double e2 = 3.0 * q - e1 - e3;
+  ev[0] = e1;
+  ev[1] = e2;
+  ev[2] = e3;
+  // e1 >= e2 >= e3 holds analytically; enforce it against rounding
+  if (ev[1] > ev[0]) { const double tt = ev[0]; ev[0] = ev[1]; ev[1] = tt; }
+  if (ev[2] > ev[1]) { const double tt = ev[1]; ev[1] = ev[2]; ev[2] = tt; }
+  if (ev[1] > ev[0]) { const double tt = ev[0]; ev[0] = ev[1]; ev[1] = tt; }
+}
+
+template <int DEG>
+__global__ void __launch_bounds__(kFinThreads)
+k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
+           const float* __restrict__ views, int G, int V, double lambda,
+           float* __restrict__ tokens) {
+  constexpr int D = (DEG + 1) * (DEG + 1);
+  constexpr int DT = 9 + 3 * D;
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= G) return;
+  const double eps = 1e-6;
+  double qsum = 0.0, b0 = 0.0, b1 = 0.0, b2 = 0.0, sa = 0.0;
+  double A00 = 0.0, A01 = 0.0, A02 = 0.0, A11 = 0.0, A12 = 0.0, A22 = 0.0;
+  float ssh[3 * D];
+#pragma unroll
+  for (int k = 0; k < 3 * D; ++k) ssh[k] = 0.0f;
+  for (int v = 0; v < V; ++v) {
+    const size_t i = (size_t)v * G + g;
+    const float4 r3 = rec[i * kRecF4 + 3];
+    const int flags = __float_as_int(r3.w);
+    if (!(flags & kFlagVisible)) continue;
+    const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1], r2 = rec[i * kRecF4 + 2];
+    const double* a = acc + i * kAccN;
+    const double qgv = eps + a[0];
+    qsum += qgv;
+    sa += (1.0 - (double)r1.y) * a[4];
+    const double qa = r0.z, qb = r0.w, qc = r1.x;
+    const double sm0 = qa * a[5] + qb * a[6];
+    const double sm1 = qb * a[5] + qc * a[6];
+    // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
+    const float* vw = views + 20 * v;
+    const double fx = vw[16], fy = vw[17];
+    const double x = r2.z, y = r2.w, z = r2.y;
+    const double j00 = fx / z, j02 = -fx * x / (z * z);
+    const double j11 = fy / z, j12 = -fy * y / (z * z);
+    double J0[3], J1[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      J0[c] = j00 * (double)vw[c] + j02 * (double)vw[8 + c];
+      J1[c] = j11 * (double)vw[4 + c] + j12 * (double)vw[8 + c];
+    }
+    b0 += J0[0] * sm0 + J1[0] * sm1;
+    b1 += J0[1] * sm0 + J1[1] * sm1;
+    b2 += J0[2] * sm0 + J1[2] * sm1;
+    A00 += qgv * (J0[0] * J0[0] + J1[0] * J1[0]);
+    A01 += qgv * (J0[0] * J0[1] + J1[0] * J1[1]);
+    A02 += qgv * (J0[0] * J0[2] + J1[0] * J1[2]);
+    A11 += qgv * (J0[1] * J0[1] + J1[1] * J1[1]);
+    A12 += qgv * (J0[1] * J0[2] + J1[1] * J1[2]);
+    A22 += qgv * (J0[2] * J0[2] + J1[2] * J1[2]);
+    float B[16];
+    sh_poly<DEG>(r3.x, r3.y, r3.z, B);
+    const float w0 = (flags & 1) ? (float)a[1] : 0.0f;
+    const float w1 = (flags & 2) ? (float)a[2] : 0.0f;
+    const float w2 = (flags & 4) ? (float)a[3] : 0.0f;
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+      ssh[3 * k + 0] += B[k] * w0;
+      ssh[3 * k + 1] += B[k] * w1;
+      ssh[3 * k + 2] += B[k] * w2;
+    }
+  }
+  const double qg = eps + qsum;
+  const double inv = 1.0 / qg;
+  A00 = A00 * inv + lambda;
+  A11 = A11 * inv + lambda;
+  A22 = A22 * inv + lambda;
+  A01 *= inv;
+  A02 *= inv;
+  A12 *= inv;
+  double ev[3];
+  eig3_sym(A00, A01, A02, A11, A12, A22, ev);
+  const double tr = A00 + A11 + A22;
+  float* zt = tokens + (size_t)g * DT;
+  zt[0] = (float)(b0 * inv);
+  zt[1] = (float)(b1 * inv);
+  zt[2] = (float)(b2 * inv);
+  zt[3] = (float)(sa * inv);
+#pragma unroll
+  for (int k = 0; k < 3 * D; ++k) zt[4 + k] = (float)((double)ssh[k] * inv);
+  zt[4 + 3 * D] = (float)log(qg);
+  const double itr = 1.0 / (tr + eps);
+  zt[5 + 3 * D] = (float)(ev[0] * itr);
+  zt[6 + 3 * D] = (float)(ev[1] * itr);
+  zt[7 + 3 * D] = (float)(ev[2] * itr);
+  zt[8 + 3 * D] = (float)log(tr + eps);
+}
+
+}  // namespace
+
+int launch_finalize(Workspace& w, float lambda, float* tokens, cudaStream_t st) {
+  if (w.G == 0) return SPLAT_OK;
+  const int blocks = (w.G + kFinThreads - 1) / kFinThreads;
+  const int tok = prof_begin(w, st, SPLAT_K_FINALIZE);
+#define SPLAT_FIN(DEG)                                                                     \
+  k_finalize<DEG><<<blocks, kFinThreads, 0, st>>>(w.rec, w.acc, w.views, w.G, w.V,        \
+                                                  (double)lambda, tokens)
+  switch (w.deg) {
+    case 0: SPLAT_FIN(0); break;
+    case 1: SPLAT_FIN(1); break;
+    case 2: SPLAT_FIN(2); break;
+    default: SPLAT_FIN(3); break;
+  }
+#undef SPLAT_FIN
+  prof_end(w, st, tok);
+  return check_launch(w, "finalize kernel");
+}
+
+}  // namespace splat

@@ -1,0 +1,206 @@
+// Stage 1 preprocess: EWA projection of every Gaussian into every view, tile rectangle,
+// opacity and SH colour.
+//
+// Sources: "Research Proposal: Renderer Score Tokens for Recurrent Gaussian Splatting",
+// "Two-Stage Algorithm" Stage 1 (standard gsplat render) and "Projected-Center Mean Partial
+// Score" (G and Sigma2D); "ATSplat: Compact Feed-forward 3D Gaussian Splatting with Adaptive Token
+// Expansion", prerequisites (the 3DGS primitive). The EWA details follow the standard 3DGS tile
+// rasteriser: tangent clamp at 1.3x the half field of view inside the covariance Jacobian,
+// 0.3 px^2 dilation, 3-sigma square footprint, near plane z = 0.01.
+//
+// One thread per Gaussian reads its parameters once (SH included) and writes one record per view:
+// the SH coefficients, which dominate the input bytes at degree 3, are never re-read per view.
+#include "common.cuh"
+
+namespace splat {
+namespace {
+
+constexpr int kProjThreads = 256;
+
+__device__ __forceinline__ int clamp_tile(float val, int hi) {
+  if (!(val > 0.0f)) return 0;  // NaN -> 0
+  if (val > (float)hi) return hi;
+  return (int)val;
+}
+
+template <int DEG>
+__global__ void __launch_bounds__(kProjThreads)
+k_project(const float* __restrict__ means, const float* __restrict__ lsc,
+          const float* __restrict__ quats, const float* __restrict__ opac,
+          const float* __restrict__ sh, const float* __restrict__ views_in, int G, int V, int H,
+          int W, int TX, int TY, float4* __restrict__ rec, int4* __restrict__ rect,
+          int* __restrict__ counts) {
+  constexpr int D = (DEG + 1) * (DEG + 1);
+  extern __shared__ float s_views[];  // [V][20]
+  for (int i = threadIdx.x; i < V * 20; i += blockDim.x) s_views[i] = views_in[i];
+  __syncthreads();
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= G) return;
+
+  const float m0 = means[3 * g], m1 = means[3 * g + 1], m2 = means[3 * g + 2];
+  const float l0 = lsc[3 * g], l1 = lsc[3 * g + 1], l2 = lsc[3 * g + 2];
+  const float q0 = quats[4 * g], q1 = quats[4 * g + 1], q2 = quats[4 * g + 2],
+              q3 = quats[4 * g + 3];
+  const float a_logit = opac[g];
+  float shc[D * 3];
+#pragma unroll
+  for (int k = 0; k < D * 3; ++k) shc[k] = sh[(size_t)g * D * 3 + k];
+
+  bool ok = isfinite(m0) && isfinite(m1) && isfinite(m2) && isfinite(l0) && isfinite(l1) &&
+            isfinite(l2) && isfinite(q0) && isfinite(q1) && isfinite(q2) && isfinite(q3) &&
+            isfinite(a_logit);
+
+  // view-independent part: rotation, scales, Sigma3D, opacity
+  float Sw[3][3];
+  float o = 0.0f;
+  {
+    const float n2 = q0 * q0 + q1 * q1 + q2 * q2 + q3 * q3;
+    if (!(n2 > 0.0f)) ok = false;
+    const float inv = 1.0f / sqrtf(n2);
+    const float qw = q0 * inv, qx = q1 * inv, qy = q2 * inv, qz = q3 * inv;
+    float Rq[3][3];
+    Rq[0][0] = 1.0f - 2.0f * (qy * qy + qz * qz);
+    Rq[0][1] = 2.0f * (qx * qy - qw * qz);
+    Rq[0][2] = 2.0f * (qx * qz + qw * qy);
+    Rq[1][0] = 2.0f * (qx * qy + qw * qz);
+    Rq[1][1] = 1.0f - 2.0f * (qx * qx + qz * qz);
+    Rq[1][2] = 2.0f * (qy * qz - qw * qx);
+    Rq[2][0] = 2.0f * (qx * qz - qw * qy);
+    Rq[2][1] = 2.0f * (qy * qz + qw * qx);
+    Rq[2][2] = 1.0f - 2.0f * (qx * qx + qy * qy);
+    const float S[3] = {exp_cw(l0), exp_cw(l1), exp_cw(l2)};
+    float M[3][3];
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int j = 0; j < 3; ++j) M[i][j] = Rq[i][j] * S[j];
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int j = 0; j < 3; ++j) Sw[i][j] = M[i][0] * M[j][0] + M[i][1] * M[j][1] + M[i][2] * M[j][2];
+    o = 1.0f / (1.0f + exp_cw(-a_logit));
+  }
+
+  for (int v = 0; v < V; ++v) {
+    const size_t i = (size_t)v * G + g;
+    const float* vw = s_views + 20 * v;
+    float4 r0 = make_float4(0, 0, 0, 0), r1 = r0, r2 = r0, r3 = r0;
+    int4 rc = make_int4(0, 0, 0, 0);
+    int cnt = 0;
+    bool vis = ok;
+    float Rv[3][3], t[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+#pragma unroll
+      for (int b = 0; b < 3; ++b) Rv[a][b] = vw[4 * a + b];
+      t[a] = vw[4 * a + 3];
+    }
+    const float fx = vw[16], fy = vw[17], cx = vw[18], cy = vw[19];
+    const float x = Rv[0][0] * m0 + Rv[0][1] * m1 + Rv[0][2] * m2 + t[0];
+    const float y = Rv[1][0] * m0 + Rv[1][1] * m1 + Rv[1][2] * m2 + t[1];
+    const float z = Rv[2][0] * m0 + Rv[2][1] * m1 + Rv[2][2] * m2 + t[2];
+    if (!(z > 0.01f)) vis = false;
+    if (vis) {
+      float T1[3][3], Sc[3][3];
+#pragma unroll
+      for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) T1[a][b] = Rv[a][0] * Sw[0][b] + Rv[a][1] * Sw[1][b] + Rv[a][2] * Sw[2][b];
+#pragma unroll
+      for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) Sc[a][b] = T1[a][0] * Rv[b][0] + T1[a][1] * Rv[b][1] + T1[a][2] * Rv[b][2];
+      const float u = x / z, vv = y / z;
+      const float limx = 1.3f * ((0.5f * (float)W) / fx);
+      const float limy = 1.3f * ((0.5f * (float)H) / fy);
+      const float uc = fminf(limx, fmaxf(-limx, u));
+      const float vc = fminf(limy, fmaxf(-limy, vv));
+      const float J00 = fx / z, J02 = -(fx * uc) / z;
+      const float J11 = fy / z, J12 = -(fy * vc) / z;
+      float T0[3], Tr1[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        T0[k] = J00 * Sc[0][k] + J02 * Sc[2][k];
+        Tr1[k] = J11 * Sc[1][k] + J12 * Sc[2][k];
+      }
+      float ca = T0[0] * J00 + T0[2] * J02;
+      const float cb = T0[1] * J11 + T0[2] * J12;
+      float cc = Tr1[1] * J11 + Tr1[2] * J12;
+      ca = ca + 0.3f;
+      cc = cc + 0.3f;
+      const float det = ca * cc - cb * cb;
+      if (!(det > 0.0f)) vis = false;
+      const float qa = cc / det, qb = -cb / det, qc = ca / det;
+      const float mid = 0.5f * (ca + cc);
+      const float lam = mid + sqrtf(fmaxf(0.1f, mid * mid - det));
+      const float rr = ceilf(3.0f * sqrtf(lam));
+      if (!(rr > 0.0f)) vis = false;
+      const float mx = fx * u + cx, my = fy * vv + cy;
+      const int x0 = clamp_tile(floorf((mx - rr) / 16.0f), TX);
+      const int x1 = clamp_tile(floorf((mx + rr) / 16.0f) + 1.0f, TX);
+      const int y0 = clamp_tile(floorf((my - rr) / 16.0f), TY);
+      const int y1 = clamp_tile(floorf((my + rr) / 16.0f) + 1.0f, TY);
+      if (x1 <= x0 || y1 <= y0) vis = false;
+      if (vis) {
+        // view direction (world) from the camera centre -R^T t
+        const float cam0 = -(Rv[0][0] * t[0] + Rv[1][0] * t[1] + Rv[2][0] * t[2]);
+        const float cam1 = -(Rv[0][1] * t[0] + Rv[1][1] * t[1] + Rv[2][1] * t[2]);
+        const float cam2 = -(Rv[0][2] * t[0] + Rv[1][2] * t[1] + Rv[2][2] * t[2]);
+        const float d0 = m0 - cam0, d1 = m1 - cam1, d2 = m2 - cam2;
+        const float len = sqrtf(d0 * d0 + d1 * d1 + d2 * d2);
+        const float dx = d0 / len, dy = d1 / len, dz = d2 / len;
+        float B[16];
+        sh_poly<DEG>(dx, dy, dz, B);
+        float col[3];
+        int flags = kFlagVisible;
+#pragma unroll
+        for (int ch = 0; ch < 3; ++ch) {
+          float s = 0.0f;
+#pragma unroll
+          for (int k = 0; k < D; ++k) s = s + B[k] * shc[3 * k + ch];
+          s = s + 0.5f;
+          if (s > 0.0f) flags |= 1 << ch;
+          col[ch] = fmaxf(s, 0.0f);
+        }
+        r0 = make_float4(mx, my, qa, qb);
+        r1 = make_float4(qc, o, col[0], col[1]);
+        r2 = make_float4(col[2], z, x, y);
+        r3 = make_float4(dx, dy, dz, __int_as_float(flags));
+        rc = make_int4(x0, y0, x1, y1);
+        cnt = (x1 - x0) * (y1 - y0);
+      }
+    }
+    float4* rp = rec + i * kRecF4;
+    rp[0] = r0;
+    rp[1] = r1;
+    rp[2] = r2;
+    rp[3] = r3;
+    rect[i] = rc;
+    counts[i] = cnt;
+  }
+}
+
+}  // namespace
+
+int launch_project(Workspace& w, const float* means, const float* lsc, const float* quats,
+                   const float* opac, const float* sh, cudaStream_t st) {
+  if (w.G == 0) return SPLAT_OK;
+  const int blocks = (w.G + kProjThreads - 1) / kProjThreads;
+  const size_t smem = (size_t)w.V * 20 * sizeof(float);
+  const int tok = prof_begin(w, st, SPLAT_K_PROJECT);
+#define SPLAT_PROJ(DEG)                                                                          \
+  k_project<DEG><<<blocks, kProjThreads, smem, st>>>(means, lsc, quats, opac, sh, w.views, w.G,  \
+                                                     w.V, w.H, w.W, w.TX, w.TY, w.rec, w.rect,  \
+                                                     w.counts)
+  switch (w.deg) {
+    case 0: SPLAT_PROJ(0); break;
+    case 1: SPLAT_PROJ(1); break;
+    case 2: SPLAT_PROJ(2); break;
+    default: SPLAT_PROJ(3); break;
+  }
+#undef SPLAT_PROJ
+  prof_end(w, st, tok);
+  return check_launch(w, "project kernel");
+}
+
+}  // namespace splat

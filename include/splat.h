@@ -1,0 +1,180 @@
+/*
+ * splat.h -- C ABI of libsplat: tile-based 3D Gaussian Splatting render followed by the analytic
+ * score replay, for NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages, cited by title and section):
+ *   [P1] "Research Proposal: Renderer Score Tokens for Recurrent Gaussian Splatting"
+ *        - "Two-Stage Algorithm", Stage 1 (standard render: gsplat tile binning, contributor
+ *          sorting, front-to-back compositing, residual; tile bins and sorted contributor
+ *          indices stay in the renderer workspace) and Stage 2 (analytic score replay, suffix
+ *          composite equation, masked per-Gaussian accumulation);
+ *        - "Exact Score Operators" (o = sigmoid(a), alpha = o G, w = T alpha; rho and q; opacity
+ *          logit score; SH score; projected-centre mean score; projection Jacobian J; cross-view
+ *          weights gamma; covector pullback b; conditioning matrix A and its statistics);
+ *        - "Final Token and Updater" (token z_g of dimension 9 + 3 d_SH).
+ *   [P5] "ATSplat: Compact Feed-forward 3D Gaussian Splatting with Adaptive Token Expansion",
+ *        prerequisites section (the 3DGS primitive: centre, rotation, scale, opacity, SH).
+ *
+ * Conventions for every call:
+ *   - All array arguments are DEVICE pointers (cudaMalloc / torch CUDA tensors) on the device
+ *     that was current when the workspace was created, C-contiguous fp32/int32 as stated, 4-byte
+ *     aligned. The caller owns them; the library never frees or retains them past the call
+ *     except where a call says so.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every call
+ *     only enqueues work on that stream and returns; the exception is splat_bin_sort, which
+ *     waits for the per-view instance counts (one device-to-host read).
+ *   - Return value: SPLAT_OK (0) or a negative splat_status. No C++ exception crosses the ABI.
+ *     On error, splat_last_error(ws) returns a NUL-terminated message owned by the workspace,
+ *     valid until the next call on it. Argument errors are detected before any work is
+ *     enqueued. A workspace is not thread-safe: one host thread at a time.
+ *   - Call order per problem: splat_project -> splat_bin_sort -> splat_render ->
+ *     splat_score_replay. A call made out of order returns SPLAT_ERR_STATE.
+ */
+#ifndef SPLAT_H
+#define SPLAT_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct splat_ws splat_ws; /* opaque, library-owned workspace */
+
+typedef enum splat_status {
+  SPLAT_OK = 0,
+  SPLAT_ERR_INVALID_ARG = -1,    /* null/misaligned/host pointer, size out of range */
+  SPLAT_ERR_CAPACITY = -2,       /* sizes above the workspace maxima or 2^31 instances */
+  SPLAT_ERR_STATE = -3,          /* calls out of order */
+  SPLAT_ERR_CUDA = -4,           /* a CUDA runtime call or kernel launch failed */
+  SPLAT_ERR_BOUNDS = -5,         /* a device-side bounds check failed (reported, access skipped) */
+  SPLAT_ERR_DEVICE_TIMEOUT = -6, /* reserved: a bounded device-side wait ran out */
+  SPLAT_ERR_OOM = -7             /* device allocation failed */
+} splat_status;
+
+/*
+ * Create a workspace on the current device for problems with at most max_G Gaussians, max_V
+ * views of at most max_H x max_W pixels and SH degree <= max_sh_degree (0..3). Allocates the
+ * per-(Gaussian, view) records and accumulators up front; the instance (tile, Gaussian) lists
+ * grow on demand inside splat_bin_sort. *ws is set to NULL on failure.
+ */
+int splat_ws_create(splat_ws** ws, int max_G, int max_V, int max_H, int max_W,
+                    int max_sh_degree);
+
+/* Free all device and host memory of the workspace (synchronises its device). NULL is a no-op. */
+void splat_ws_destroy(splat_ws* ws);
+
+/* Message describing the last error on this workspace ("" when none). */
+const char* splat_last_error(const splat_ws* ws);
+
+/*
+ * Stage 1 preprocess ([P1] Stage 1 "original gsplat"; [P5] 3DGS primitive; [P1] "Projected-Center
+ * Mean Partial Score" for G and Sigma2D): for every Gaussian g and view v, the camera-space centre,
+ * the EWA 2-D covariance Sigma2D = J W Sigma3D W^T J^T + 0.3 I and its inverse (the conic), the
+ * 3-sigma footprint radius and its rectangle of 16x16 tiles, the opacity o = sigmoid(a), the view
+ * direction and the SH colour c = max(0, B(dir) . sh + 0.5). Culled when z <= 0.01, when an input
+ * is not finite, for a zero quaternion, det(Sigma2D) <= 0 or an empty tile rectangle.
+ *   means       [G,3]   world-space centres
+ *   log_scales  [G,3]   per-axis log standard deviations
+ *   quats       [G,4]   rotation quaternions (w, x, y, z), normalised here
+ *   opac_logits [G]     opacity logits a
+ *   sh          [G,d,3] SH coefficients, d = (sh_degree + 1)^2, channel-minor
+ *   viewmats    [V,4,4] world-to-camera, row-major; camera x right, y down, z forward
+ *   intrin      [V,4]   fx, fy, cx, cy in pixels; pixel (i, j) has centre (i + 0.5, j + 0.5)
+ * G >= 0 (G = 0 renders background only), 1 <= V, 1 <= H, W. The input arrays are read by this
+ * call only.
+ */
+int splat_project(splat_ws* ws, const float* means, const float* log_scales, const float* quats,
+                  const float* opac_logits, const float* sh, int G, int sh_degree,
+                  const float* viewmats, const float* intrin, int V, int H, int W, void* stream);
+
+/*
+ * Stage 1 tile binning and contributor sort ([P1] Stage 1 step 1): every visible (g, v) emits one
+ * instance per tile of its rectangle; each tile's list is ordered by (camera depth z, Gaussian
+ * index) -- a stable counting sort by tile followed by a per-tile radix sort of the fp32 depth
+ * bits. The lists stay in the workspace ([P1] Stage 1: not exposed as a per-pixel tensor).
+ * n_instances_out (HOST pointer, may be NULL) receives V counts. Synchronises with the stream
+ * once (the counts size the sort).
+ */
+int splat_bin_sort(splat_ws* ws, long long* n_instances_out, void* stream);
+
+/*
+ * Stage 1 front-to-back compositing ([P1] Stage 1 step 2): per pixel, over its tile's list,
+ * alpha = min(0.99, o G); entries with a positive exponent or alpha < 1/255 are skipped; the
+ * traversal stops before an entry that would take T below 1e-4. Writes
+ *   img       [V,H,W,3] C_hat = sum T alpha c + T_final bg
+ *   T_final   [V,H,W]   final transmittance
+ *   n_contrib [V,H,W]   number of composited Gaussians (int32)
+ * bg is a device pointer to 3 floats. The replay reads img back (it is C_hat), so img must stay
+ * unmodified until splat_score_replay has run.
+ */
+int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int* n_contrib,
+                 void* stream);
+
+/*
+ * Stage 2 analytic score replay and token finalisation ([P1] Stage 2, "Exact Score Operators",
+ * "Final Token and Updater"). Re-traverses every pixel's list in the same order and with the same
+ * decisions as splat_render, keeps prefix colour P and transmittance T, recovers
+ *   C+ = (C_hat - P - T alpha c) / (T (1 - alpha) + 1e-12),
+ * masks with M_alpha = (T (1 - alpha) >= 1e-4 and alpha < 0.99) and M_color (colour clamp
+ * inactive), forms r = C_hat - C_obs, rho = <r, c - C+>, w = T alpha and accumulates per (g, v)
+ *   q = sum w, sum w r, sum M_alpha w rho, sum M_alpha w rho (p - mu2D)
+ * (CTA-level reduction per tile, then fp64 atomics). Then, per Gaussian over the views where it
+ * is visible: q_gv = 1e-6 + q, q_g = 1e-6 + sum_v q_gv, gamma = q_gv / q_g, and
+ *   tokens[g] = [ b_mu (3) = sum_v gamma J^T Sigma2D^-1 Sd / q_gv,
+ *                 s_alpha (1) = sum_v gamma (1 - o) Sa / q_gv,
+ *                 s_SH (3d) = sum_v gamma M_color (B(dir) (x) Swr) / q_gv   (index k*3 + channel),
+ *                 log q_g (1),
+ *                 eig(A) descending / (tr A + 1e-6) (3),  log(tr A + 1e-6) (1) ],
+ *   A = lambda I + sum_v gamma J^T J,  J = d pi_v(mu) / d mu (unclamped pinhole Jacobian).
+ *   obs    [V,H,W,3] observed images C_obs
+ *   lambda conditioning regulariser (fixed after scene normalisation; 1.0 by default)
+ *   tokens [G, 9 + 3d] fp32 output
+ */
+int splat_score_replay(splat_ws* ws, const float* obs, float lambda, float* tokens,
+                       void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Inspection calls (tests and benchmarks; not part of the render/replay path). They copy
+ * workspace state into caller-owned DEVICE buffers on `stream`, or report host-side counters.
+ * ------------------------------------------------------------------------------------------- */
+
+/* Per (v, g) record, fp32 [V,G,16]: mx, my, conic a, b, c, opacity, colour r, g, b, depth z,
+ * x_c, y_c, dir x, y, z, flags (int bits: bit 0..2 colour-clamp-inactive per channel, bit 8
+ * visible). rect [V,G,4] int32 tile rectangle x0, y0, x1, y1 (zeros when culled). Needs
+ * splat_project. */
+int splat_copy_projection(splat_ws* ws, float* rec, int* rect, void* stream);
+
+/* Tile lists after splat_bin_sort: tile_offsets [V, n_t + 1] int64 (global positions, view-major,
+ * n_t = ceil(W/16) ceil(H/16), tiles row-major) and ids [sum of counts] int32 Gaussian indices. */
+int splat_copy_tile_lists(splat_ws* ws, long long* tile_offsets, int* ids, void* stream);
+
+/* Per-pixel list bound after splat_render: last [V,H,W] int32 = 1 + the list position of the last
+ * composited entry (0 when none), i.e. the number of entries both passes traverse. */
+int splat_copy_last(splat_ws* ws, int* last, void* stream);
+
+/* Per-(v, g) sums after splat_score_replay: acc [V,G,8] fp64 = q, Swr(3), Sa, Sd(2), 0. */
+int splat_copy_accumulators(splat_ws* ws, double* acc, void* stream);
+
+/* Gaussian-pixel pairs traversed by the last render (sum over pixels of `last`); synchronises. */
+int splat_pair_count(splat_ws* ws, long long* pairs, void* stream);
+
+/* Number of kernels this workspace has launched since creation (host counter). */
+long long splat_launch_count(const splat_ws* ws);
+
+/* Per-kernel device timing. When enabled, every kernel of the path is bracketed by a pair of
+ * CUDA events on the launch stream; splat_profile_read synchronises on them and adds, per kernel
+ * group id (0 .. SPLAT_NUM_KERNELS-1), the elapsed milliseconds and the number of timed launches
+ * since the last reset (reset != 0 clears after reading). Off by default. */
+enum {
+  SPLAT_K_PROJECT = 0, SPLAT_K_SCAN_COUNTS, SPLAT_K_EMIT, SPLAT_K_TILE_HIST, SPLAT_K_HIST_SCAN,
+  SPLAT_K_TILE_SCATTER, SPLAT_K_TILE_RANGES, SPLAT_K_TILE_SORT, SPLAT_K_RENDER, SPLAT_K_REPLAY,
+  SPLAT_K_FINALIZE, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
+};
+int splat_profile_enable(splat_ws* ws, int enable);
+int splat_profile_read(splat_ws* ws, double* ms, long long* launches, int reset);
+/* Static name of a kernel group id ("?" when out of range). */
+const char* splat_kernel_name(int id);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPLAT_H */

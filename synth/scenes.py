@@ -121,10 +121,10 @@ def _random_quats(rng, n: int) -> np.ndarray:
 def _sh_from_colour(rng, colour: np.ndarray, deg: int, hi_sigma: float) -> np.ndarray:
     n = colour.shape[0]
     d = (deg + 1) ** 2
-    sh = np.zeros((n, d, 3), np.float64)
+    sh = np.empty((n, d, 3), np.float32)
     sh[:, 0, :] = (colour - 0.5) / _Y00
     if d > 1:
-        sh[:, 1:, :] = rng.normal(0.0, hi_sigma, (n, d - 1, 3))
+        sh[:, 1:, :] = rng.standard_normal((n, d - 1, 3), dtype=np.float32) * np.float32(hi_sigma)
     return sh
 
 
@@ -149,7 +149,7 @@ def _finish(name, seed, means, log_scales, quats, opac, sh, deg, viewmats, intri
     G = means.shape[0]
     obs_means = means + rng.normal(0.0, mean_sigma, (G, 3))
     obs_sh = sh.copy()
-    obs_sh[:, 0, :] += rng.normal(0.0, colour_sigma, (G, 3)) / _Y00
+    obs_sh[:, 0, :] += (rng.normal(0.0, colour_sigma, (G, 3)) / _Y00).astype(np.float32)
     means, log_scales, quats, opac, sh, obs_means, obs_sh = _f32(
         means, log_scales, quats, opac, sh, obs_means, obs_sh)
     viewmats, intrin = _f32(viewmats, intrin)

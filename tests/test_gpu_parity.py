@@ -1,0 +1,159 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Bars: visibility, tile rectangles, tile offsets, per-tile order, final transmittance, contributor
+counts and list bounds bit-exact; projected means/conics/opacity/depth bitwise; colour within
+1e-5; tokens within 1e-4 relative L2 per Gaussian (floor 1e-3 x median norm).
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from synth import scenes
+from tests import parity_util as PU
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for the gpu tests")
+    from gaussian_splatting_raster_b200 import build, load_library
+    build()
+    load_library()
+
+
+def _full_check(sc, obs, lam=1.0):
+    g = PU.gpu_run(sc, obs, lam)
+    o = O.run(sc, obs, "f", lam=lam)
+    near = PU.compare_projection(sc, g, o["proj"]) if sc.G > 0 else np.zeros(0, bool)
+    PU.compare_lists(g, o["lists"])
+    PU.compare_render(g, o)
+    assert g["pairs"] == int(o["last"].sum())
+    if sc.G > 0:
+        PU.compare_tokens(g["tokens"], o["tokens"], exclude=near)
+    return g, o
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_small_configs_full_parity(cfg):
+    sc = scenes.make(cfg)
+    obs = O.observe(sc, "f")
+    g, o = _full_check(sc, obs)
+    assert g["n_contrib"].max() > 1
+
+
+def test_exact_depth_ties_keep_index_order():
+    sc = scenes.make(1)  # every Gaussian of a plane has the same camera depth
+    obs = O.observe(sc, "f")
+    g = PU.gpu_run(sc, obs)
+    o = O.run(sc, obs, "f")
+    PU.compare_lists(g, o["lists"])
+    # inside each tile, equal depths appear in increasing index
+    rec = o["proj"]["rec"][0]
+    off, ids = g["off"][0], g["ids"]
+    for t in range(off.shape[0] - 1):
+        seg = ids[off[t]:off[t + 1]]
+        d = rec[seg, 5]
+        key = np.lexsort((seg, d))
+        assert (key == np.arange(len(seg))).all()
+
+
+@pytest.mark.parametrize("deg", [0, 2, 3])
+def test_sh_degrees_and_ragged_image(deg):
+    sc = scenes.tiny_scene(40 + deg, 300, 37, 53, V=3, deg=deg, hi_sigma=0.2)
+    obs = np.random.default_rng(deg).uniform(0, 1, (sc.V, sc.H, sc.W, 3)).astype(np.float32)
+    _full_check(sc, obs, lam=0.5)
+
+
+def test_long_tile_list_uses_global_sort():
+    """One 16x16 tile with 12000 overlapping Gaussians: longer than the shared-memory sort."""
+    sc = scenes.tiny_scene(7, 12000, 16, 16, V=1, deg=1, depth_range=(1.0, 60.0),
+                           log_scale_mean=math.log(0.05))
+    obs = np.full((1, 16, 16, 3), 0.3, np.float32)
+    g, o = _full_check(sc, obs)
+    assert o["lists"]["n"] > 8192
+
+
+def test_empty_scene_and_all_culled():
+    sc = scenes.tiny_scene(3, 5, 20, 24, V=2)
+    sc.means[:, 2] = -1.0  # all behind the cameras
+    obs = np.zeros((2, 20, 24, 3), np.float32)
+    g, o = _full_check(sc, obs)
+    assert sum(g["n_per_view"]) == 0
+    assert (g["img"] == 0).all() and (g["T"] == 1).all()
+    # G = 0
+    sc0 = scenes.tiny_scene(3, 1, 20, 24, V=1)
+    for name in ("means", "log_scales", "quats", "opac", "sh"):
+        setattr(sc0, name, getattr(sc0, name)[:0])
+    sc0.bg = np.array([0.25, 0.5, 0.75], np.float32)
+    g0 = PU.gpu_run(sc0, np.zeros((1, 20, 24, 3), np.float32), with_acc=False)
+    assert (g0["img"] == sc0.bg).all() and g0["tokens"].shape == (0, 21)
+
+
+def test_nonzero_background_and_lambda():
+    sc = scenes.tiny_scene(9, 200, 48, 64, V=2, deg=1)
+    sc.bg = np.array([0.1, 0.6, 0.3], np.float32)
+    obs = np.random.default_rng(1).uniform(0, 1, (2, 48, 64, 3)).astype(np.float32)
+    _full_check(sc, obs, lam=2.5)
+
+
+def test_calls_out_of_order_and_bad_arguments():
+    import torch
+    from gaussian_splatting_raster_b200 import SplatError, Workspace
+    ws = Workspace(16, 1, 16, 16, 1)
+    with pytest.raises(SplatError) as e:
+        ws.bin_sort()
+    assert e.value.code == -3
+    z = torch.zeros((16, 3), device="cuda")
+    with pytest.raises(SplatError) as e:  # more Gaussians than the workspace holds
+        ws.project(torch.zeros((17, 3), device="cuda"), torch.zeros((17, 3), device="cuda"),
+                   torch.zeros((17, 4), device="cuda"), torch.zeros((17,), device="cuda"),
+                   torch.zeros((17, 4, 3), device="cuda"), torch.eye(4, device="cuda")[None],
+                   torch.ones((1, 4), device="cuda"), 16, 16)
+    assert e.value.code == -2
+    with pytest.raises(TypeError):  # host tensor
+        ws.project(z.cpu(), z, z, z[:, 0], torch.zeros((16, 4, 3), device="cuda"),
+                   torch.eye(4, device="cuda")[None], torch.ones((1, 4), device="cuda"), 16, 16)
+    ws.close()
+
+
+@pytest.mark.parametrize("cfg", [3, 4, 5])
+def test_full_size_sampled(cfg):
+    """Full-size workloads: projection and every tile list compared in full; render on sampled
+    tiles; tokens of sampled Gaussians (the oracle replays every tile those Gaussians touch)."""
+    sc = scenes.make(cfg)
+    obs = scenes.smooth_observation(77 + cfg, sc.V, sc.H, sc.W)
+    g = PU.gpu_run(sc, obs)
+    p = O.project(sc, "f")
+    near = PU.compare_projection(sc, g, p)
+    L = O.bin_lists(p, sc.H, sc.W)
+    PU.compare_lists(g, L)
+    rng = np.random.default_rng(cfg)
+    TX, TY = O.n_tiles(sc.H, sc.W)
+    # sampled Gaussians (visible somewhere, no colour near-tie) and the tiles they touch
+    cand = np.nonzero(p["valid"].any(0) & ~near)[0]
+    gs = rng.choice(cand, size=24, replace=False)
+    sel = set()
+    for v in range(sc.V):
+        for gg in gs:
+            if p["valid"][v, gg]:
+                x0, y0, x1, y1 = p["rect"][v, gg]
+                sel.update((v, ty * TX + tx) for ty in range(y0, y1) for tx in range(x0, x1))
+    # plus random tiles for the image checks
+    sel.update((int(rng.integers(sc.V)), int(rng.integers(TX * TY))) for _ in range(16))
+    sel = np.array(sorted(sel), np.int32)
+    r = O.render(p, L, sc.H, sc.W, sc.bg, "f", sel=sel)
+    mask = np.zeros((sc.V, sc.H, sc.W), bool)
+    for v, t in sel:
+        tx, ty = t % TX, t // TX
+        mask[v, ty * 16:(ty + 1) * 16, tx * 16:(tx + 1) * 16] = True
+    PU.compare_render(g, r, mask)
+    acc = O.replay(p, L, r, obs, sc.sh_degree, sc.H, sc.W, "f", sel=sel)["acc"]
+    z = O.finalize(p, acc, sc)
+    PU.compare_tokens(g["tokens"], z, which=gs)
+    # the accumulated supports of the sampled Gaussians agree too
+    np.testing.assert_allclose(g["acc"][:, gs, 0], acc[:, gs, 0], rtol=1e-5, atol=1e-6)
