@@ -15,7 +15,7 @@
 namespace splat {
 namespace {
 
-constexpr int kProjThreads = 256;
+constexpr int kProjThreads = 128;
 
 __device__ __forceinline__ int clamp_tile(float val, int hi) {
   if (!(val > 0.0f)) return 0;  // NaN -> 0
@@ -31,8 +31,27 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
           int W, int TX, int TY, float4* __restrict__ rec, int4* __restrict__ rect,
           int* __restrict__ counts) {
   constexpr int D = (DEG + 1) * (DEG + 1);
-  extern __shared__ float s_views[];  // [V][20]
+  constexpr int NSH = D * 3;
+  // shared memory: the block's SH coefficients [kProjThreads][NSH], then the views [V][20]
+  extern __shared__ float s_dyn[];
+  float* s_sh = s_dyn;
+  float* s_views = s_dyn + kProjThreads * NSH;
   for (int i = threadIdx.x; i < V * 20; i += blockDim.x) s_views[i] = views_in[i];
+  // coalesced staging of the block's contiguous SH rows (they dominate the input bytes)
+  {
+    const long long g0 = (long long)blockIdx.x * kProjThreads;
+    const int ng = (int)min((long long)kProjThreads, (long long)G - g0);
+    const int nf = ng * NSH;
+    const float* src = sh + g0 * NSH;
+    if ((((uintptr_t)src) & 15) == 0) {
+      const float4* s4 = reinterpret_cast<const float4*>(src);
+      for (int k = threadIdx.x; k < nf / 4; k += blockDim.x)
+        reinterpret_cast<float4*>(s_sh)[k] = s4[k];
+      for (int k = (nf / 4) * 4 + threadIdx.x; k < nf; k += blockDim.x) s_sh[k] = src[k];
+    } else {
+      for (int k = threadIdx.x; k < nf; k += blockDim.x) s_sh[k] = src[k];
+    }
+  }
   __syncthreads();
   const int g = blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= G) return;
@@ -42,9 +61,7 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
   const float q0 = quats[4 * g], q1 = quats[4 * g + 1], q2 = quats[4 * g + 2],
               q3 = quats[4 * g + 3];
   const float a_logit = opac[g];
-  float shc[D * 3];
-#pragma unroll
-  for (int k = 0; k < D * 3; ++k) shc[k] = sh[(size_t)g * D * 3 + k];
+  const float* shc = s_sh + threadIdx.x * NSH;
 
   bool ok = isfinite(m0) && isfinite(m1) && isfinite(m2) && isfinite(l0) && isfinite(l1) &&
             isfinite(l2) && isfinite(q0) && isfinite(q1) && isfinite(q2) && isfinite(q3) &&
@@ -186,12 +203,19 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
                    const float* opac, const float* sh, cudaStream_t st) {
   if (w.G == 0) return SPLAT_OK;
   const int blocks = (w.G + kProjThreads - 1) / kProjThreads;
-  const size_t smem = (size_t)w.V * 20 * sizeof(float);
   const int tok = prof_begin(w, st, SPLAT_K_PROJECT);
 #define SPLAT_PROJ(DEG)                                                                          \
-  k_project<DEG><<<blocks, kProjThreads, smem, st>>>(means, lsc, quats, opac, sh, w.views, w.G,  \
-                                                     w.V, w.H, w.W, w.TX, w.TY, w.rec, w.rect,  \
-                                                     w.counts)
+  {                                                                                              \
+    const size_t smem = ((size_t)kProjThreads * 3 * (DEG + 1) * (DEG + 1) + (size_t)w.V * 20) * \
+                        sizeof(float);                                                           \
+    if (smem > 48 * 1024 &&                                                                      \
+        cudaFuncSetAttribute(k_project<DEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
+                             (int)smem) != cudaSuccess)                                          \
+      return set_err(w, SPLAT_ERR_CAPACITY, "too many views for the projection kernel");        \
+    k_project<DEG><<<blocks, kProjThreads, smem, st>>>(means, lsc, quats, opac, sh, w.views,     \
+                                                       w.G, w.V, w.H, w.W, w.TX, w.TY, w.rec,    \
+                                                       w.rect, w.counts);                        \
+  }
   switch (w.deg) {
     case 0: SPLAT_PROJ(0); break;
     case 1: SPLAT_PROJ(1); break;

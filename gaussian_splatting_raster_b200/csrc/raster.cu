@@ -9,31 +9,46 @@
 // SH and projected-centre scores).
 //
 // One CTA per (tile, view), one thread per pixel of the 16x16 tile. The tile's list is walked in
-// batches of 256 entries whose records (mean, conic, opacity, colour: 36 bytes) are staged in
-// shared memory by one coalesced gather per batch. Both passes evaluate alpha through the same
-// device function, so the replay takes exactly the render's decisions.
+// batches of 256 entries whose records (mean, conic, opacity, colour) are staged in shared memory
+// by one gather per batch. Both passes evaluate alpha through the same device function, so the
+// replay takes exactly the render's decisions.
 //
-// Replay accumulation: per entry of a batch, each warp reduces its 32 pixels' seven
-// contributions (q, w r (3), w rho, w rho (p - mu2D) (2)) with shuffles and adds them to a
-// shared-memory slot of that entry; at the end of the batch one thread per entry adds the CTA's
-// sums to the (view, Gaussian) accumulator with fp64 atomics -- seven global atomics per
-// (Gaussian, tile) instead of per (Gaussian, pixel). The SH block never enters the pixel loop:
-// its per-pixel term M_color w (B (x) r) factors into M_color B (x) (sum w r), and the mean block
-// Sigma^-1 (sum w rho d) is formed once per (Gaussian, view) in finalisation.
+// Early skip. Most (pixel, entry) pairs of a tile lie far outside the Gaussian's footprint. For
+// every staged entry the loader computes cut = log((1/255) / o) - 1e-3; an exponent below cut
+// gives o exp(pw) < (1/255) exp(-1e-3), far below 1/255 even after the few-ulp errors of the
+// exp and of the product, so the entry is skipped without evaluating exp -- the same decision the
+// full evaluation takes, never a different one.
+//
+// Replay arithmetic. rho = <r, c - C+> is evaluated as
+//   rho = <r,c> - (<r,C_hat> - <r,P> - w <r,c>) / (T (1 - alpha) + eps),
+// algebraically the suffix composite of the recovery equation dotted with r, keeping <r, P> as a
+// running scalar instead of the prefix colour vector. Per entry and warp the seven per-pixel terms
+// (w, w r (3), w rho, w rho (p - mu2D) (2)) are summed by a transpose-reduction (each exchange
+// step halves the values a lane carries: 9 shuffles instead of 35), the eight lanes holding a
+// result add it into a shared-memory slot of the entry, and at the end of the batch one thread per
+// entry adds the CTA's sums to the (view, Gaussian) accumulator with fp64 atomics -- seven global
+// atomics per (Gaussian, tile). The SH block never enters the pixel loop: M_color w (B (x) r)
+// factors into M_color B (x) (sum w r); the mean block Sigma^-1 (sum w rho d) is formed once per
+// (Gaussian, view) in finalisation.
 #include "common.cuh"
 
 namespace splat {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr float kAlphaMin = 1.0f / 255.0f;
 
 struct Entry {
   bool use;
   float alpha, dx, dy;
 };
 
+// exponent cut below which alpha < 1/255 is certain (see the file comment)
+__device__ __forceinline__ float skip_cut(float o) { return logf(kAlphaMin / o) - 1e-3f; }
+
 // alpha of one list entry at pixel centre (px, py), with the rasteriser's skip rules
-__device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float px, float py) {
+__device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
+                                            float py) {
   Entry e;
   e.dx = px - A.x;
   e.dy = py - A.y;
@@ -43,9 +58,9 @@ __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, flo
   const float pw = -0.5f * (t1 + t2) - t3;
   e.use = false;
   e.alpha = 0.0f;
-  if (pw > 0.0f) return e;
+  if (pw > 0.0f || pw < cut) return e;
   const float al = fminf(0.99f, Bq.y * exp_cw(pw));
-  if (al < 1.0f / 255.0f) return e;
+  if (al < kAlphaMin) return e;
   e.alpha = al;
   e.use = true;
   return e;
@@ -63,7 +78,7 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const long long e = tile_off[(size_t)v * (nt + 1) + t + 1];
   __shared__ float4 s_a[kThreads], s_b[kThreads];
-  __shared__ float s_c[kThreads];
+  __shared__ float2 s_c[kThreads];  // (colour b, exponent cut)
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int n = 0, lst = 0;
@@ -74,16 +89,18 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     const long long k = base + threadIdx.x;
     if (k < e) {
       const float4* r = recv + (size_t)ids[k] * kRecF4;
+      const float4 b = r[1];
       s_a[threadIdx.x] = r[0];
-      s_b[threadIdx.x] = r[1];
-      s_c[threadIdx.x] = r[2].x;
+      s_b[threadIdx.x] = b;
+      s_c[threadIdx.x] = make_float2(r[2].x, skip_cut(b.y));
     }
     __syncthreads();
     const int cnt = (int)min((long long)kThreads, e - base);
     if (!done) {
       for (int q = 0; q < cnt; ++q) {
         const float4 A = s_a[q], Bq = s_b[q];
-        const Entry E = eval_entry(A, Bq, px, py);
+        const float2 Cq = s_c[q];
+        const Entry E = eval_entry(A, Bq, Cq.y, px, py);
         if (!E.use) continue;
         const float Tn = T * (1.0f - E.alpha);
         if (Tn < 1e-4f) {
@@ -91,9 +108,10 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
           break;
         }
         const float wgt = E.alpha * T;
-        C0 = C0 + wgt * Bq.z;
-        C1 = C1 + wgt * Bq.w;
-        C2 = C2 + wgt * s_c[q];
+        // colour sums are not decisions: fused multiply-adds (within rounding of the oracle)
+        C0 = fmaf(wgt, Bq.z, C0);
+        C1 = fmaf(wgt, Bq.w, C1);
+        C2 = fmaf(wgt, Cq.x, C2);
         T = Tn;
         ++n;
         lst = (int)(base - s) + q + 1;
@@ -111,10 +129,16 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   }
 }
 
-__device__ __forceinline__ float warp_sum(float x) {
+// one butterfly step of the transpose-reduction: lanes with `hi` keep the upper half of their
+// values and send the lower half, the others the reverse; the received half is added
+template <int HALF>
+__device__ __forceinline__ void tr_step(float* x, bool hi, int off) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
+  for (int k = 0; k < HALF; ++k) {
+    const float send = hi ? x[k] : x[k + HALF];
+    const float keep = hi ? x[k + HALF] : x[k];
+    x[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -128,21 +152,20 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   __shared__ float4 s_a[kThreads], s_b[kThreads];
-  __shared__ float s_c[kThreads];
+  __shared__ float2 s_c[kThreads];
   __shared__ uint32_t s_g[kThreads];
-  __shared__ float s_acc[7][kThreads];
+  __shared__ float s_acc[8][kThreads];
   __shared__ int s_max;
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
-  float Ch0 = 0.0f, Ch1 = 0.0f, Ch2 = 0.0f, r0 = 0.0f, r1 = 0.0f, r2 = 0.0f;
+  float r0 = 0.0f, r1 = 0.0f, r2 = 0.0f, rC = 0.0f;
   int lst = 0;
   if (inside) {
     const size_t p = ((size_t)v * H + j) * W + i;
-    Ch0 = img[3 * p];
-    Ch1 = img[3 * p + 1];
-    Ch2 = img[3 * p + 2];
+    const float Ch0 = img[3 * p], Ch1 = img[3 * p + 1], Ch2 = img[3 * p + 2];
     r0 = Ch0 - obs[3 * p];
     r1 = Ch1 - obs[3 * p + 1];
     r2 = Ch2 - obs[3 * p + 2];
+    rC = fmaf(r2, Ch2, fmaf(r1, Ch1, r0 * Ch0));  // <r, C_hat>
     lst = last[p];
   }
   if (threadIdx.x == 0) s_max = 0;
@@ -152,72 +175,61 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const int maxl = s_max;
   const float4* recv = rec + (size_t)v * G * kRecF4;
   double* accv = acc + (size_t)v * G * kAccN;
-  float T = 1.0f, P0 = 0.0f, P1 = 0.0f, P2 = 0.0f;
+  float T = 1.0f, rP = 0.0f;  // transmittance, <r, P>
   const int lane = threadIdx.x & 31;
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  const int slot = (lane >> 2) & 7;  // value index this lane holds after the reduction
   for (int base = 0; base < maxl; base += kThreads) {
     const int cnt = min(kThreads, maxl - base);
     if ((int)threadIdx.x < cnt) {
       const uint32_t g = ids[s + base + threadIdx.x];
       const float4* r = recv + (size_t)g * kRecF4;
+      const float4 b = r[1];
       s_a[threadIdx.x] = r[0];
-      s_b[threadIdx.x] = r[1];
-      s_c[threadIdx.x] = r[2].x;
+      s_b[threadIdx.x] = b;
+      s_c[threadIdx.x] = make_float2(r[2].x, skip_cut(b.y));
       s_g[threadIdx.x] = g;
     }
 #pragma unroll
-    for (int c = 0; c < 7; ++c) s_acc[c][threadIdx.x] = 0.0f;
+    for (int c = 0; c < 8; ++c) s_acc[c][threadIdx.x] = 0.0f;
     __syncthreads();
     for (int q = 0; q < cnt; ++q) {
-      float v0 = 0.0f, v1 = 0.0f, v2 = 0.0f, v3 = 0.0f, v4 = 0.0f, v5 = 0.0f, v6 = 0.0f;
+      float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
       bool used = false;
       if (base + q < lst) {
         const float4 A = s_a[q], Bq = s_b[q];
-        const Entry E = eval_entry(A, Bq, px, py);
+        const float2 Cq = s_c[q];
+        const Entry E = eval_entry(A, Bq, Cq.y, px, py);
         if (E.use) {
           used = true;
           const float al = E.alpha;
           const float den = T * (1.0f - al);
           const float w = al * T;
-          const float c0 = Bq.z, c1 = Bq.w, c2 = s_c[q];
-          const float dd = den + 1e-12f;
-          const float Cp0 = ((Ch0 - P0) - w * c0) / dd;
-          const float Cp1 = ((Ch1 - P1) - w * c1) / dd;
-          const float Cp2 = ((Ch2 - P2) - w * c2) / dd;
+          const float rc = fmaf(r2, Cq.x, fmaf(r1, Bq.w, r0 * Bq.z));  // <r, c>
+          const float num = fmaf(-w, rc, rC - rP);                      // <r, C_hat - P - w c>
+          const float rho = rc - __fdividef(num, den + 1e-12f);
           const bool Ma = (den >= 1e-4f) && (al < 0.99f);
-          const float rho = r0 * (c0 - Cp0) + r1 * (c1 - Cp1) + r2 * (c2 - Cp2);
-          v0 = w;
-          v1 = w * r0;
-          v2 = w * r1;
-          v3 = w * r2;
+          x[0] = w;
+          x[1] = w * r0;
+          x[2] = w * r1;
+          x[3] = w * r2;
           if (Ma) {
             const float wr = w * rho;
-            v4 = wr;
-            v5 = wr * E.dx;
-            v6 = wr * E.dy;
+            x[4] = wr;
+            x[5] = wr * E.dx;
+            x[6] = wr * E.dy;
           }
-          P0 = P0 + w * c0;
-          P1 = P1 + w * c1;
-          P2 = P2 + w * c2;
+          rP = fmaf(w, rc, rP);
           T = den;
         }
       }
       if (__any_sync(0xffffffffu, used)) {
-        v0 = warp_sum(v0);
-        v1 = warp_sum(v1);
-        v2 = warp_sum(v2);
-        v3 = warp_sum(v3);
-        v4 = warp_sum(v4);
-        v5 = warp_sum(v5);
-        v6 = warp_sum(v6);
-        if (lane == 0) {
-          atomicAdd(&s_acc[0][q], v0);
-          atomicAdd(&s_acc[1][q], v1);
-          atomicAdd(&s_acc[2][q], v2);
-          atomicAdd(&s_acc[3][q], v3);
-          atomicAdd(&s_acc[4][q], v4);
-          atomicAdd(&s_acc[5][q], v5);
-          atomicAdd(&s_acc[6][q], v6);
-        }
+        tr_step<4>(x, b4, 16);
+        tr_step<2>(x, b3, 8);
+        tr_step<1>(x, b2, 4);
+        x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
+        x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
+        if ((lane & 3) == 0 && slot < 7) atomicAdd(&s_acc[slot][q], x[0]);
       }
     }
     __syncthreads();
