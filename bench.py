@@ -151,9 +151,11 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
     }
 
 
-# instructions per traversed (pixel, entry) pair in the fp32 pipe, counted from the kernels'
-# arithmetic (see the design notes): alpha evaluation incl. exp, compositing or replay terms
-ALU_OPS_PER_PAIR = {"render": 40, "replay": 75}
+# algorithmic fp32 operations per traversed (pixel, list entry) pair, from the arithmetic the
+# method defines (the design notes count them): render = alpha (conic quadratic form, exp,
+# clamp/threshold tests) + transmittance + colour = 17 fp32 + 1 transcendental; replay = the same
+# alpha + suffix recovery (3 channels) + rho + masks + 7 weighted terms = 45 fp32 + 2 special
+ALU_OPS_PER_PAIR = {"render": 18, "replay": 47}
 
 
 # ----------------------------------------------------------------------------------------------

@@ -19,10 +19,11 @@
 // exp and of the product, so the entry is skipped without evaluating exp -- the same decision the
 // full evaluation takes, never a different one.
 //
-// Replay arithmetic. rho = <r, c - C+> is evaluated as
-//   rho = <r,c> - (<r,C_hat> - <r,P> - w <r,c>) / (T (1 - alpha) + eps),
-// algebraically the suffix composite of the recovery equation dotted with r, keeping <r, P> as a
-// running scalar instead of the prefix colour vector. Per entry and warp the seven per-pixel terms
+// Replay arithmetic. The suffix numerators C_hat - P - T alpha c are formed per channel exactly
+// as the recovery equation writes them (their cancellation dominates the fp32 error of C+), then
+// multiplied by one correctly rounded reciprocal of T (1 - alpha) + eps. (Rewriting rho through
+// running dot products <r, P> is algebraically the same but moves that cancellation and costs
+// ~4e-4 relative token error.) Per entry and warp the seven per-pixel terms
 // (w, w r (3), w rho, w rho (p - mu2D) (2)) are summed by a transpose-reduction (each exchange
 // step halves the values a lane carries: 9 shuffles instead of 35), the eight lanes holding a
 // result add it into a shared-memory slot of the entry, and at the end of the batch one thread per
@@ -108,10 +109,11 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
           break;
         }
         const float wgt = E.alpha * T;
-        // colour sums are not decisions: fused multiply-adds (within rounding of the oracle)
-        C0 = fmaf(wgt, Bq.z, C0);
-        C1 = fmaf(wgt, Bq.w, C1);
-        C2 = fmaf(wgt, Cq.x, C2);
+        // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is then
+        // exactly the background term, and the suffix recovery sees no rounding mismatch
+        C0 = C0 + wgt * Bq.z;
+        C1 = C1 + wgt * Bq.w;
+        C2 = C2 + wgt * Cq.x;
         T = Tn;
         ++n;
         lst = (int)(base - s) + q + 1;
@@ -157,15 +159,16 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   __shared__ float s_acc[8][kThreads];
   __shared__ int s_max;
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
-  float r0 = 0.0f, r1 = 0.0f, r2 = 0.0f, rC = 0.0f;
+  float Ch0 = 0.0f, Ch1 = 0.0f, Ch2 = 0.0f, r0 = 0.0f, r1 = 0.0f, r2 = 0.0f;
   int lst = 0;
   if (inside) {
     const size_t p = ((size_t)v * H + j) * W + i;
-    const float Ch0 = img[3 * p], Ch1 = img[3 * p + 1], Ch2 = img[3 * p + 2];
+    Ch0 = img[3 * p];
+    Ch1 = img[3 * p + 1];
+    Ch2 = img[3 * p + 2];
     r0 = Ch0 - obs[3 * p];
     r1 = Ch1 - obs[3 * p + 1];
     r2 = Ch2 - obs[3 * p + 2];
-    rC = fmaf(r2, Ch2, fmaf(r1, Ch1, r0 * Ch0));  // <r, C_hat>
     lst = last[p];
   }
   if (threadIdx.x == 0) s_max = 0;
@@ -175,7 +178,7 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const int maxl = s_max;
   const float4* recv = rec + (size_t)v * G * kRecF4;
   double* accv = acc + (size_t)v * G * kAccN;
-  float T = 1.0f, rP = 0.0f;  // transmittance, <r, P>
+  float T = 1.0f, P0 = 0.0f, P1 = 0.0f, P2 = 0.0f;  // transmittance, prefix colour
   const int lane = threadIdx.x & 31;
   const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
   const int slot = (lane >> 2) & 7;  // value index this lane holds after the reduction
@@ -205,9 +208,15 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
           const float al = E.alpha;
           const float den = T * (1.0f - al);
           const float w = al * T;
-          const float rc = fmaf(r2, Cq.x, fmaf(r1, Bq.w, r0 * Bq.z));  // <r, c>
-          const float num = fmaf(-w, rc, rC - rP);                      // <r, C_hat - P - w c>
-          const float rho = rc - __fdividef(num, den + 1e-12f);
+          const float c0 = Bq.z, c1 = Bq.w, c2 = Cq.x;
+          // suffix numerators C_hat - P - w c per channel, in the recovery equation's order
+          // (their cancellation dominates the fp32 error of C+, so they are formed exactly as
+          // written), then one correctly rounded reciprocal of the denominator
+          const float n0 = (Ch0 - P0) - w * c0;
+          const float n1 = (Ch1 - P1) - w * c1;
+          const float n2 = (Ch2 - P2) - w * c2;
+          const float inv = __frcp_rn(den + 1e-12f);
+          const float rho = r0 * (c0 - n0 * inv) + r1 * (c1 - n1 * inv) + r2 * (c2 - n2 * inv);
           const bool Ma = (den >= 1e-4f) && (al < 0.99f);
           x[0] = w;
           x[1] = w * r0;
@@ -219,7 +228,9 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
             x[5] = wr * E.dx;
             x[6] = wr * E.dy;
           }
-          rP = fmaf(w, rc, rP);
+          P0 = P0 + w * c0;
+          P1 = P1 + w * c1;
+          P2 = P2 + w * c2;
           T = den;
         }
       }
