@@ -25,6 +25,7 @@ EXPORTS = [
     "splat_bin_sort", "splat_render", "splat_score_replay", "splat_copy_projection",
     "splat_copy_tile_lists", "splat_copy_last", "splat_copy_accumulators", "splat_pair_count",
     "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
+    "splat_sort_depths_noalloc",
 ]
 
 
