@@ -138,11 +138,15 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
         # read the parameters once, write per (v, g) record (64 B), rectangle (16 B), count (4 B)
         "project": G * (4 * (3 + 3 + 4 + 1) + 12 * d) + V * G * (64 + 16 + 4),
         "scan_counts": V * G * (4 + 8),
-        # read rectangle + depth, write (tile, depth, g) per instance
-        "emit": V * G * (16 + 4) + n_inst * 12,
+        # one depth-digit pass per launch over every (v, g): histogram reads the keys, the
+        # scatter reads key + index and writes both
+        "depth_hist": V * G * 4,
+        "depth_scatter": V * G * 16,
+        # rectangles gathered into depth order (16 B in, 16 B + count out), the counts scanned
+        # (4 B in, 8 B out), instances (tile, g) emitted (rectangle, index, offset in; 8 B out)
+        "emit": V * G * (16 + 20 + 12 + 28) + n_inst * 8,
         "tile_hist": n_inst * 4,
-        "tile_scatter": n_inst * (4 + 8 + 8),
-        "tile_sort": n_inst * (8 + 4),
+        "tile_scatter": n_inst * (4 + 4 + 4),
         # gather 36 B per list entry staged, write C_hat, T, n, last
         "render": n_inst * (4 + 36) + px * 24,
         "replay": n_inst * (4 + 36) + px * (12 + 12 + 4) + V * G * 64,
@@ -400,8 +404,8 @@ def main():
         if k in ab:
             v["algorithmic_GBps"] = ab[k] / (v["ms_per_step"] * 1e-3) / 1e9
     render_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in
-                    ("project", "scan_counts", "emit", "tile_hist", "hist_scan", "tile_scatter",
-                     "tile_ranges", "tile_sort", "render", "other"))
+                    ("project", "scan_counts", "depth_hist", "depth_scatter", "emit", "tile_hist",
+                     "hist_scan", "tile_scatter", "tile_ranges", "render", "other"))
     replay_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in ("replay", "finalize"))
 
     cpu = None

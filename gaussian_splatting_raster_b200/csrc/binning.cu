@@ -5,16 +5,19 @@
 // sorted indices stay in the renderer workspace). The required order inside each tile is
 // (camera depth, Gaussian index).
 //
-// Design (differs from a single 64-bit (tile | depth) key radix sort):
-//   1. scan of the per-(v, g) tile counts -> instance offsets (reduce-then-scan, no waits);
-//   2. emit: each visible (v, g) writes its instances (tile id, depth bits, g) in index order;
-//   3. stable counting sort by tile: per-warp tile histograms per block of 16K instances, an
-//      exclusive scan of the (tile, block) counts, then a scatter that ranks equal tiles in
-//      instance order with warp match -- one pass over the instances instead of one per digit;
-//      the scanned histogram also yields every tile's [start, end) for free;
-//   4. per tile, a stable LSD radix sort of the fp32 depth bits (only the bits that vary inside
-//      the tile), in shared memory for lists of up to 8192 entries, in global memory above.
-// Stability of 3 and 4 gives the index tie-break.
+// Design (instead of one radix sort of 64-bit (tile | depth) keys over all instances):
+//   1. per view, a stable LSD radix sort of the (v, g) depth keys -- one key per Gaussian, not per
+//      instance -- over only the bits that vary among the view's visible keys (the projection
+//      records per-view ORs of the keys and of their complements), 8..11-bit digits;
+//   2. the tile rectangles gathered into that depth order, their tile counts scanned, and the
+//      instances (tile, g) emitted in depth order;
+//   3. one stable counting sort of the instances by tile. Stability of 1 (index order of equal
+//      depths) and 3 (depth order inside each tile) gives exactly (depth, index) per tile, and the
+//      scanned (tile, block) histogram yields every tile's [start, end).
+// Every pass -- each depth digit and the tile pass -- is the same stable counting sort: per block
+// of 16K items, per-warp shared-memory histograms (ranks of equal buckets inside a warp from
+// match.any), an int32 exclusive scan of the (bucket, block) counts, and a scatter that replays
+// the ranking. Uniform, bandwidth-shaped work; no decoupled look-back, so no device-side waits.
 #include "common.cuh"
 
 namespace splat {
@@ -124,36 +127,49 @@ int ensure_part(Workspace& w, long long nb) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// emit
-__global__ void k_emit(const float4* __restrict__ rec, const int4* __restrict__ rect,
-                       const long long* __restrict__ offs, long long VG, int G, int TX,
-                       uint32_t* __restrict__ inst_tile, uint2* __restrict__ inst_kv) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= VG) return;
-  const int4 rc = rect[i];
-  if (rc.z <= rc.x || rc.w <= rc.y) return;
-  const uint32_t g = (uint32_t)(i % G);
-  const uint32_t depth = __float_as_uint(rec[i * kRecF4 + 2].y);
-  long long pos = offs[i];
-  for (int ty = rc.y; ty < rc.w; ++ty)
-    for (int tx = rc.x; tx < rc.z; ++tx) {
-      inst_tile[pos] = (uint32_t)(ty * TX + tx);
-      inst_kv[pos] = make_uint2(depth, g);
-      ++pos;
-    }
-}
-
-// ---------------------------------------------------------------------------------------------
-// stable counting sort by tile
+// the stable counting-sort pass
 constexpr int kBinWarps = 8;
 constexpr int kBinThreads = kBinWarps * 32;
-constexpr int kBinChunk = 16384;                 // instances per block
+constexpr int kBinChunk = 16384;  // items per block
 constexpr int kBinPerWarp = kBinChunk / kBinWarps;
 
-__device__ __forceinline__ int find_view(const int* bstart, int V, int b) {
-  int v = 0;
-  while (v + 1 < V && bstart[v + 1] <= b) ++v;
-  return v;
+// Items of view v are [start(v), start(v + 1)); each view is cut into blocks of kBinChunk.
+// Uniform layout (every view holds `per_view` items, blocks_per_view blocks) or tables.
+struct Segs {
+  long long per_view;        // >= 0: uniform layout
+  int blocks_per_view;
+  const long long* vstart;   // tables (per_view < 0): [V + 1] item starts
+  const int* bstart;         // [V + 1] block starts
+  int V;
+};
+
+struct BlockRange {
+  int v, lb, nbv, b0;  // view, block within view, blocks of the view, first block of the view
+  long long beg, end, vbeg;
+};
+
+__device__ __forceinline__ BlockRange block_range(const Segs& sg, int b) {
+  BlockRange r;
+  if (sg.per_view >= 0) {
+    r.nbv = sg.blocks_per_view;
+    r.v = b / r.nbv;
+    r.lb = b - r.v * r.nbv;
+    r.b0 = r.v * r.nbv;
+    r.vbeg = (long long)r.v * sg.per_view;
+    r.beg = r.vbeg + (long long)r.lb * kBinChunk;
+    r.end = min(r.beg + (long long)kBinChunk, r.vbeg + sg.per_view);
+  } else {
+    int v = 0;
+    while (v + 1 < sg.V && sg.bstart[v + 1] <= b) ++v;
+    r.v = v;
+    r.b0 = sg.bstart[v];
+    r.lb = b - r.b0;
+    r.nbv = sg.bstart[v + 1] - r.b0;
+    r.vbeg = sg.vstart[v];
+    r.beg = r.vbeg + (long long)r.lb * kBinChunk;
+    r.end = min(r.beg + (long long)kBinChunk, sg.vstart[v + 1]);
+  }
+  return r;
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -162,95 +178,138 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-__global__ void __launch_bounds__(kBinThreads)
-k_tile_hist(const uint32_t* __restrict__ inst_tile, const long long* __restrict__ vstart,
-            const int* __restrict__ bstart, int V, int nt, int* __restrict__ hist) {
-  extern __shared__ uint32_t s_cnt[];  // [kBinWarps][nt]
-  const int b = blockIdx.x;
-  const int v = find_view(bstart, V, b);
-  const int lb = b - bstart[v];
-  const int nbv = bstart[v + 1] - bstart[v];
-  const long long beg = vstart[v] + (long long)lb * kBinChunk;
-  const long long end = min(beg + (long long)kBinChunk, vstart[v + 1]);
-  for (int t = threadIdx.x; t < kBinWarps * nt; t += blockDim.x) s_cnt[t] = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t* cnt = s_cnt + warp * nt;
-  const long long wb = beg + (long long)warp * kBinPerWarp;
-  const long long we = min(wb + (long long)kBinPerWarp, end);
-  for (long long base = wb; base < we; base += 32) {
-    const long long i = base + lane;
-    const bool ok = i < we;
-    const uint32_t t = ok ? inst_tile[i] : (0x80000000u | lane);
-    const uint32_t peers = __match_any_sync(0xffffffffu, t);
-    if (ok && lane == __ffs(peers) - 1) cnt[t] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  int* h = hist + (size_t)nt * bstart[v];
-  for (int t = threadIdx.x; t < nt; t += blockDim.x) {
-    uint32_t s = 0;
+constexpr int kUnroll = 4;  // 32-item batches whose loads are issued together
+
+// per-warp bucket counts of this block's items into cnt[nbk]; the loads of kUnroll batches are
+// issued before the first is ranked, so each warp keeps several requests in flight
+__device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, int shift,
+                                            uint32_t mask, long long wb, long long we,
+                                            uint32_t* cnt) {
+  const int lane = threadIdx.x & 31;
+  for (long long base = wb; base < we; base += 32 * kUnroll) {
+    uint32_t bk[kUnroll];
 #pragma unroll
-    for (int ww = 0; ww < kBinWarps; ++ww) s += s_cnt[ww * nt + t];
-    h[(size_t)t * nbv + lb] = (int)s;
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = base + 32 * u + lane;
+      bk[u] = i < we ? (keys[i] >> shift) & mask : (0x80000000u | lane);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const bool ok = base + 32 * u + lane < we;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bk[u]);
+      if (ok && lane == __ffs(peers) - 1) cnt[bk[u]] += __popc(peers);
+      __syncwarp();
+    }
   }
 }
 
+// histogram: hist[nbk * b0 + bucket * nbv + lb] = count of the block's items in the bucket
 __global__ void __launch_bounds__(kBinThreads)
-k_tile_scatter(const uint32_t* __restrict__ inst_tile, const uint2* __restrict__ inst_kv,
-               const long long* __restrict__ vstart, const int* __restrict__ bstart, int V,
-               int nt, const int* __restrict__ hist_scan, uint32_t* __restrict__ skey,
-               uint32_t* __restrict__ sval) {
-  extern __shared__ uint32_t s_cnt[];  // [kBinWarps][nt]
-  const int b = blockIdx.x;
-  const int v = find_view(bstart, V, b);
-  const int lb = b - bstart[v];
-  const int nbv = bstart[v + 1] - bstart[v];
-  const long long beg = vstart[v] + (long long)lb * kBinChunk;
-  const long long end = min(beg + (long long)kBinChunk, vstart[v + 1]);
-  for (int t = threadIdx.x; t < kBinWarps * nt; t += blockDim.x) s_cnt[t] = 0;
+k_count_hist(const uint32_t* __restrict__ keys, int shift, uint32_t mask, int nbk, Segs sg,
+             int* __restrict__ hist) {
+  extern __shared__ uint32_t s_cnt[];  // [kBinWarps][nbk]
+  const BlockRange r = block_range(sg, blockIdx.x);
+  for (int t = threadIdx.x; t < kBinWarps * nbk; t += blockDim.x) s_cnt[t] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  const long long wb = r.beg + (long long)warp * kBinPerWarp;
+  const long long we = min(wb + (long long)kBinPerWarp, r.end);
+  warp_counts(keys, shift, mask, wb, we, s_cnt + warp * nbk);
+  __syncthreads();
+  int* h = hist + (size_t)nbk * r.b0;
+  for (int t = threadIdx.x; t < nbk; t += blockDim.x) {
+    uint32_t s = 0;
+#pragma unroll
+    for (int ww = 0; ww < kBinWarps; ++ww) s += s_cnt[ww * nbk + t];
+    h[(size_t)t * r.nbv + r.lb] = (int)s;
+  }
+}
+
+// stable scatter of (key, value) by bucket; vals == nullptr means value = index within the view;
+// kout == nullptr drops the keys
+__global__ void __launch_bounds__(kBinThreads)
+k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ vals, int shift,
+                uint32_t mask, int nbk, Segs sg, const int* __restrict__ hist_scan,
+                uint32_t* __restrict__ kout, uint32_t* __restrict__ vout) {
+  extern __shared__ uint32_t s_cnt[];  // [kBinWarps][nbk]
+  const BlockRange r = block_range(sg, blockIdx.x);
+  for (int t = threadIdx.x; t < kBinWarps * nbk; t += blockDim.x) s_cnt[t] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t* cnt = s_cnt + warp * nt;
-  const long long wb = beg + (long long)warp * kBinPerWarp;
-  const long long we = min(wb + (long long)kBinPerWarp, end);
-  for (long long base = wb; base < we; base += 32) {
-    const long long i = base + lane;
-    const bool ok = i < we;
-    const uint32_t t = ok ? inst_tile[i] : (0x80000000u | lane);
-    const uint32_t peers = __match_any_sync(0xffffffffu, t);
-    if (ok && lane == __ffs(peers) - 1) cnt[t] += __popc(peers);
-    __syncwarp();
-  }
+  uint32_t* cnt = s_cnt + warp * nbk;
+  const long long wb = r.beg + (long long)warp * kBinPerWarp;
+  const long long we = min(wb + (long long)kBinPerWarp, r.end);
+  warp_counts(keys, shift, mask, wb, we, cnt);
   __syncthreads();
-  // per tile: global start of this block's run, then one sub-run per warp in warp order
-  const int* h = hist_scan + (size_t)nt * bstart[v];
-  for (int t = threadIdx.x; t < nt; t += blockDim.x) {
-    uint32_t run = (uint32_t)h[(size_t)t * nbv + lb];
+  // per bucket: global start of this block's run, then one sub-run per warp in warp order
+  const int* h = hist_scan + (size_t)nbk * r.b0;
+  for (int t = threadIdx.x; t < nbk; t += blockDim.x) {
+    uint32_t run = (uint32_t)h[(size_t)t * r.nbv + r.lb];
 #pragma unroll
     for (int ww = 0; ww < kBinWarps; ++ww) {
-      const uint32_t c = s_cnt[ww * nt + t];
-      s_cnt[ww * nt + t] = run;
+      const uint32_t c = s_cnt[ww * nbk + t];
+      s_cnt[ww * nbk + t] = run;
       run += c;
     }
   }
   __syncthreads();
   const uint32_t lt = lanemask_lt();
-  for (long long base = wb; base < we; base += 32) {
-    const long long i = base + lane;
-    const bool ok = i < we;
-    const uint32_t t = ok ? inst_tile[i] : (0x80000000u | lane);
-    const uint32_t peers = __match_any_sync(0xffffffffu, t);
-    if (ok) {
-      const uint2 kv = inst_kv[i];
-      const uint32_t pos = cnt[t] + __popc(peers & lt);
-      skey[pos] = kv.x;
-      sval[pos] = kv.y;
+  for (long long base = wb; base < we; base += 32 * kUnroll) {
+    uint32_t key[kUnroll], val[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = base + 32 * u + lane;
+      const bool ok = i < we;
+      key[u] = ok ? keys[i] : 0u;
+      val[u] = ok ? (vals ? vals[i] : (uint32_t)(i - r.vbeg)) : 0u;
     }
-    __syncwarp();
-    if (ok && lane == __ffs(peers) - 1) cnt[t] += __popc(peers);
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const bool ok = base + 32 * u + lane < we;
+      const uint32_t bk = ok ? (key[u] >> shift) & mask : (0x80000000u | lane);
+      const uint32_t peers = __match_any_sync(0xffffffffu, bk);
+      if (ok) {
+        const uint32_t pos = cnt[bk] + __popc(peers & lt);
+        if (kout) kout[pos] = key[u];
+        vout[pos] = val[u];
+      }
+      __syncwarp();
+      if (ok && lane == __ffs(peers) - 1) cnt[bk] += __popc(peers);
+      __syncwarp();
+    }
   }
+}
+
+// tile rectangles and counts in depth order (order == nullptr: index order)
+__global__ void k_gather_rects(const int4* __restrict__ rect, const uint32_t* __restrict__ order,
+                               long long VG, int G, int4* __restrict__ rect_s,
+                               int* __restrict__ cnt_s) {
+  const long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= VG) return;
+  const long long v = k / G;
+  const uint32_t g = order ? order[k] : (uint32_t)(k - v * G);
+  const int4 rc = rect[v * G + g];
+  rect_s[k] = rc;
+  cnt_s[k] = (rc.z - rc.x) * (rc.w - rc.y);
+}
+
+// instances (tile, g) in depth order
+__global__ void k_emit(const int4* __restrict__ rect_s, const uint32_t* __restrict__ order,
+                       const long long* __restrict__ offs, long long VG, int G, int TX,
+                       uint32_t* __restrict__ inst_tile, uint32_t* __restrict__ inst_g) {
+  const long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= VG) return;
+  const int4 rc = rect_s[k];
+  if (rc.z <= rc.x || rc.w <= rc.y) return;
+  const long long v = k / G;
+  const uint32_t g = order ? order[k] : (uint32_t)(k - v * G);
+  long long pos = offs[k];
+  for (int ty = rc.y; ty < rc.w; ++ty)
+    for (int tx = rc.x; tx < rc.z; ++tx) {
+      inst_tile[pos] = (uint32_t)(ty * TX + tx);
+      inst_g[pos] = g;
+      ++pos;
+    }
 }
 
 __global__ void k_tile_ranges(const int* __restrict__ hist_scan, const long long* __restrict__ vstart,
@@ -267,116 +326,6 @@ __global__ void k_tile_ranges(const int* __restrict__ hist_scan, const long long
   tile_off[idx] = o;
 }
 
-// ---------------------------------------------------------------------------------------------
-// per-tile stable LSD radix sort of the depth bits
-constexpr int kSortWarps = 16;
-constexpr int kSortThreads = kSortWarps * 32;
-constexpr int kSortCap = 8192;  // entries sorted in shared memory
-
-// one stable 8-bit digit pass over n entries; cnt is [kSortWarps][256] in shared memory
-__device__ void radix_pass(const uint32_t* kin, const uint32_t* vin, uint32_t* kout,
-                           uint32_t* vout, int n, int shift, uint32_t* cnt, uint32_t* s_warp) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = (((n + kSortWarps - 1) / kSortWarps) + 31) & ~31;
-  const int wb = warp * per;
-  const int we = min(n, wb + per);
-  for (int d = lane; d < 256; d += 32) cnt[warp * 256 + d] = 0;
-  __syncwarp();
-  for (int base = wb; base < we; base += 32) {
-    const int i = base + lane;
-    const bool ok = i < we;
-    const uint32_t dig = ok ? (kin[i] >> shift) & 255u : 256u + lane;
-    const uint32_t peers = __match_any_sync(0xffffffffu, dig);
-    if (ok && lane == __ffs(peers) - 1) cnt[warp * 256 + dig] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  // exclusive scan in (digit, warp) order: thread t owns digit t/2, warps (t&1)*8 .. +8
-  {
-    const int d = threadIdx.x >> 1, w0 = (threadIdx.x & 1) * 8;
-    uint32_t vals[8];
-    uint32_t s = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t c = cnt[(w0 + k) * 256 + d];
-      vals[k] = s;
-      s += c;
-    }
-    const uint32_t ex = block_exclusive_scan<uint32_t>(s, s_warp, nullptr);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) cnt[(w0 + k) * 256 + d] = ex + vals[k];
-  }
-  __syncthreads();
-  const uint32_t lt = lanemask_lt();
-  for (int base = wb; base < we; base += 32) {
-    const int i = base + lane;
-    const bool ok = i < we;
-    const uint32_t key = ok ? kin[i] : 0u;
-    const uint32_t dig = ok ? (key >> shift) & 255u : 256u + lane;
-    const uint32_t peers = __match_any_sync(0xffffffffu, dig);
-    if (ok) {
-      const uint32_t pos = cnt[warp * 256 + dig] + __popc(peers & lt);
-      kout[pos] = key;
-      vout[pos] = vin[i];
-    }
-    __syncwarp();
-    if (ok && lane == __ffs(peers) - 1) cnt[warp * 256 + dig] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-}
-
-__global__ void __launch_bounds__(kSortThreads)
-k_tile_sort(const long long* __restrict__ tile_off, int nt, uint32_t* skey, uint32_t* sval,
-            uint32_t* skey2, uint32_t* sval2) {
-  extern __shared__ uint32_t s_mem[];
-  uint32_t* cnt = s_mem;                     // [16][256]
-  uint32_t* kbuf = s_mem + kSortWarps * 256; // [2][cap]
-  uint32_t* vbuf = kbuf + 2 * kSortCap;      // [2][cap]
-  __shared__ uint32_t s_warp[32];
-  __shared__ uint32_t s_diff;
-  const int seg = blockIdx.x;
-  const int v = seg / nt, t = seg % nt;
-  const long long s = tile_off[(size_t)v * (nt + 1) + t];
-  const long long e = tile_off[(size_t)v * (nt + 1) + t + 1];
-  const int n = (int)(e - s);
-  if (n <= 1) return;
-  if (threadIdx.x == 0) s_diff = 0;
-  __syncthreads();
-  const uint32_t k0 = skey[s];
-  uint32_t dl = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) dl |= skey[s + i] ^ k0;
-  atomicOr(&s_diff, dl);
-  __syncthreads();
-  const uint32_t diff = s_diff;
-  const int nbits = diff ? 32 - __clz(diff) : 0;
-  const int passes = (nbits + 7) >> 3;
-  if (passes == 0) return;  // equal depths: index order already holds
-  if (n <= kSortCap) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      kbuf[i] = skey[s + i];
-      vbuf[i] = sval[s + i];
-    }
-    __syncthreads();
-    for (int p = 0; p < passes; ++p) {
-      const int a = p & 1, bsel = a ^ 1;
-      radix_pass(kbuf + a * kSortCap, vbuf + a * kSortCap, kbuf + bsel * kSortCap,
-                 vbuf + bsel * kSortCap, n, 8 * p, cnt, s_warp);
-    }
-    const uint32_t* vf = vbuf + (passes & 1) * kSortCap;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) sval[s + i] = vf[i];
-  } else {
-    uint32_t* K[2] = {skey + s, skey2 + s};
-    uint32_t* Vv[2] = {sval + s, sval2 + s};
-    for (int p = 0; p < passes; ++p) {
-      const int a = p & 1, bsel = a ^ 1;
-      radix_pass(K[a], Vv[a], K[bsel], Vv[bsel], n, 8 * p, cnt, s_warp);
-    }
-    if (passes & 1)
-      for (int i = threadIdx.x; i < n; i += blockDim.x) sval[s + i] = sval2[s + i];
-  }
-}
-
 template <typename T>
 int grow(Workspace& w, T** p, size_t n, const char* what) {
   if (*p) cudaFree(*p);
@@ -386,6 +335,14 @@ int grow(Workspace& w, T** p, size_t n, const char* what) {
     return set_err(w, SPLAT_ERR_OOM, std::string("allocation failed: ") + what);
   }
   return SPLAT_OK;
+}
+
+int ensure_hist(Workspace& w, size_t n) {
+  if (n + 1 <= w.hist_cap) return SPLAT_OK;
+  const size_t cap = n + n / 4 + 1024;
+  const int rc = grow(w, &w.hist, cap, "bucket histogram");
+  w.hist_cap = rc ? 0 : cap;
+  return rc;
 }
 
 }  // namespace
@@ -429,88 +386,123 @@ int launch_scan_counts(Workspace& w, cudaStream_t st) {
   return rc;
 }
 
-// after the host has read the per-view instance starts into w.h_vstart
+// one stable counting-sort pass (histogram, scan, scatter)
+static int count_pass(Workspace& w, cudaStream_t st, const uint32_t* keys, const uint32_t* vals,
+                      int shift, uint32_t mask, int nbk, const Segs& sg, int nblocks,
+                      uint32_t* kout, uint32_t* vout, int id_hist, int id_scatter) {
+  int rc;
+  const size_t hist_n = (size_t)nbk * nblocks;
+  if ((rc = ensure_hist(w, hist_n))) return rc;
+  const size_t smem = (size_t)kBinWarps * nbk * sizeof(uint32_t);
+  int tok = prof_begin(w, st, id_hist);
+  k_count_hist<<<nblocks, kBinThreads, smem, st>>>(keys, shift, mask, nbk, sg, w.hist);
+  prof_end(w, st, tok);
+  if ((rc = check_launch(w, "histogram kernel"))) return rc;
+  tok = prof_begin(w, st, SPLAT_K_HIST_SCAN);
+  rc = scan_i32_inplace(w, w.hist, (long long)hist_n, st);
+  prof_end(w, st, tok);
+  if (rc) return rc;
+  tok = prof_begin(w, st, id_scatter);
+  k_count_scatter<<<nblocks, kBinThreads, smem, st>>>(keys, vals, shift, mask, nbk, sg, w.hist,
+                                                       kout, vout);
+  prof_end(w, st, tok);
+  return check_launch(w, "scatter kernel");
+}
+
+// after the host has read the per-view instance starts (h_vstart) and key statistics (h_kbits)
 int launch_binning(Workspace& w, cudaStream_t st) {
   int rc;
   const long long N = w.n_total;
-  // block table: ceil(N_v / chunk) blocks per view
+  const long long VG = (long long)w.V * w.G;
+  if (N > (long long)w.inst_cap) {
+    const size_t cap = (size_t)(N + N / 4 + 1024);
+    if ((rc = grow(w, &w.inst_tile, cap, "instance tiles"))) return rc;
+    if ((rc = grow(w, &w.inst_g, cap, "instance indices"))) return rc;
+    if ((rc = grow(w, &w.sval, cap, "tile lists"))) return rc;
+    w.inst_cap = cap;
+  }
+  // ---- 1. depth order of every view's Gaussians --------------------------------------------
+  // highest bit that varies among any view's visible keys -> number of digit passes
+  int hb = -1;
+  for (int v = 0; v < w.V; ++v) {
+    uint32_t k1 = 0, k0 = 0;
+    for (int sidx = 0; sidx < kKeyStripes; ++sidx) {
+      k1 |= w.h_kbits[2 * (v * kKeyStripes + sidx)];
+      k0 |= w.h_kbits[2 * (v * kKeyStripes + sidx) + 1];
+    }
+    const uint32_t vary = k1 & k0;
+    if (vary) hb = max(hb, 31 - __builtin_clz(vary));
+  }
+  const int bits = hb + 1;
+  const int passes = bits == 0 ? 0 : (bits + 10) / 11;
+  const int dbits = passes ? (bits + passes - 1) / passes : 0;
+  const uint32_t* order = nullptr;  // sorted Gaussian indices per view (nullptr: index order)
+  if (passes > 0 && VG > 0) {
+    Segs sg{w.G, (int)((w.G + kBinChunk - 1) / kBinChunk), nullptr, nullptr, w.V};
+    const int nblocks = sg.blocks_per_view * w.V;
+    const uint32_t* kin = w.dkey;
+    const uint32_t* vin = nullptr;
+    uint32_t* kb[2] = {w.dk1, w.dk2};
+    uint32_t* vb[2] = {w.dv0, w.dv1};
+    for (int p = 0; p < passes; ++p) {
+      const int shift = p * dbits;
+      const int width = min(dbits, 32 - shift);
+      const uint32_t mask = (width >= 32) ? 0xffffffffu : ((1u << width) - 1u);
+      uint32_t* kout = (p + 1 < passes) ? kb[p & 1] : nullptr;
+      uint32_t* vout = vb[p & 1];
+      if ((rc = count_pass(w, st, kin, vin, shift, mask, (int)mask + 1, sg, nblocks, kout, vout,
+                           SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER)))
+        return rc;
+      kin = kout;
+      vin = vout;
+    }
+    order = vin;
+  }
+  // ---- 2. rectangles in depth order, their offsets, instance emission -------------------------
+  if (VG > 0) {
+    int tok = prof_begin(w, st, SPLAT_K_EMIT);
+    const unsigned grid = (unsigned)((VG + 255) / 256);
+    k_gather_rects<<<grid, 256, 0, st>>>(w.rect, order, VG, w.G, w.rect_s, w.counts);
+    if ((rc = check_launch(w, "rectangle gather kernel"))) return rc;
+    if ((rc = scan_i32_to_i64(w, w.counts, w.offs, VG, st))) return rc;
+    k_emit<<<grid, 256, 0, st>>>(w.rect_s, order, w.offs, VG, w.G, w.TX, w.inst_tile, w.inst_g);
+    prof_end(w, st, tok);
+    if ((rc = check_launch(w, "emit kernel"))) return rc;
+  }
+  // ---- 3. stable counting sort by tile --------------------------------------------------------
   w.h_bstart[0] = 0;
   for (int v = 0; v < w.V; ++v) {
     const long long nv = w.h_vstart[v + 1] - w.h_vstart[v];
     w.h_bstart[v + 1] = w.h_bstart[v] + (int)((nv + kBinChunk - 1) / kBinChunk);
   }
   w.n_blocks = w.h_bstart[w.V];
-  const size_t hist_n = (size_t)w.nt * (size_t)w.n_blocks;
-  if (N > w.inst_cap) {
-    const size_t cap = (size_t)(N + N / 4 + 1024);
-    if ((rc = grow(w, &w.inst_tile, cap, "instance tiles"))) return rc;
-    if ((rc = grow(w, &w.inst_kv, cap, "instance keys"))) return rc;
-    if ((rc = grow(w, &w.skey, cap, "sort keys"))) return rc;
-    if ((rc = grow(w, &w.sval, cap, "sort values"))) return rc;
-    if ((rc = grow(w, &w.skey2, cap, "sort keys 2"))) return rc;
-    if ((rc = grow(w, &w.sval2, cap, "sort values 2"))) return rc;
-    w.inst_cap = cap;
-  }
-  if (hist_n + 1 > w.hist_cap) {
-    const size_t cap = hist_n + hist_n / 4 + 1024;
-    if ((rc = grow(w, &w.hist, cap, "tile histogram"))) return rc;
-    w.hist_cap = cap;
-  }
   cudaMemcpyAsync(w.d_vstart, w.h_vstart, (w.V + 1) * sizeof(long long),
                   cudaMemcpyHostToDevice, st);
   cudaMemcpyAsync(w.d_bstart, w.h_bstart, (w.V + 1) * sizeof(int), cudaMemcpyHostToDevice, st);
-  const long long VG = (long long)w.V * w.G;
   if (N > 0) {
-    int tok = prof_begin(w, st, SPLAT_K_EMIT);
-    k_emit<<<(unsigned)((VG + 255) / 256), 256, 0, st>>>(w.rec, w.rect, w.offs, VG, w.G, w.TX,
-                                                          w.inst_tile, w.inst_kv);
-    prof_end(w, st, tok);
-    if ((rc = check_launch(w, "emit kernel"))) return rc;
-    const size_t smem = (size_t)kBinWarps * w.nt * sizeof(uint32_t);
-    tok = prof_begin(w, st, SPLAT_K_TILE_HIST);
-    k_tile_hist<<<w.n_blocks, kBinThreads, smem, st>>>(w.inst_tile, w.d_vstart, w.d_bstart, w.V,
-                                                       w.nt, w.hist);
-    prof_end(w, st, tok);
-    if ((rc = check_launch(w, "tile histogram kernel"))) return rc;
-    tok = prof_begin(w, st, SPLAT_K_HIST_SCAN);
-    rc = scan_i32_inplace(w, w.hist, (long long)hist_n, st);
-    prof_end(w, st, tok);
-    if (rc) return rc;
-    tok = prof_begin(w, st, SPLAT_K_TILE_SCATTER);
-    k_tile_scatter<<<w.n_blocks, kBinThreads, smem, st>>>(w.inst_tile, w.inst_kv, w.d_vstart,
-                                                          w.d_bstart, w.V, w.nt, w.hist, w.skey,
-                                                          w.sval);
-    prof_end(w, st, tok);
-    if ((rc = check_launch(w, "tile scatter kernel"))) return rc;
+    Segs sg{-1, 0, w.d_vstart, w.d_bstart, w.V};
+    if ((rc = count_pass(w, st, w.inst_tile, w.inst_g, 0, 0xffffffffu, w.nt, sg, w.n_blocks,
+                         nullptr, w.sval, SPLAT_K_TILE_HIST, SPLAT_K_TILE_SCATTER)))
+      return rc;
+  } else if ((rc = ensure_hist(w, 1))) {
+    return rc;
   }
   const int nr = w.V * (w.nt + 1);
-  int tok_r = prof_begin(w, st, SPLAT_K_TILE_RANGES);
+  const int tok_r = prof_begin(w, st, SPLAT_K_TILE_RANGES);
   k_tile_ranges<<<(nr + 255) / 256, 256, 0, st>>>(w.hist, w.d_vstart, w.d_bstart, w.V, w.nt,
                                                   w.tile_off);
   prof_end(w, st, tok_r);
-  if ((rc = check_launch(w, "tile ranges kernel"))) return rc;
-  if (N > 0) {
-    const size_t smem = (size_t)(kSortWarps * 256 + 4 * kSortCap) * sizeof(uint32_t);
-    const int tok_s = prof_begin(w, st, SPLAT_K_TILE_SORT);
-    k_tile_sort<<<w.V * w.nt, kSortThreads, smem, st>>>(w.tile_off, w.nt, w.skey, w.sval, w.skey2,
-                                                         w.sval2);
-    prof_end(w, st, tok_s);
-    if ((rc = check_launch(w, "tile depth sort kernel"))) return rc;
-  }
-  return SPLAT_OK;
+  return check_launch(w, "tile ranges kernel");
 }
 
-// shared-memory opt-in for the binning kernels (called once per workspace)
+// shared-memory opt-in for the counting-sort kernels (called once per workspace)
 int binning_configure(Workspace& w) {
-  const int sort_smem = (kSortWarps * 256 + 4 * kSortCap) * sizeof(uint32_t);
-  const int bin_smem = kBinWarps * w.max_nt * sizeof(uint32_t);
-  cudaError_t e1 = cudaFuncSetAttribute(k_tile_sort, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        sort_smem);
-  cudaError_t e2 = cudaFuncSetAttribute(k_tile_hist, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        bin_smem);
-  cudaError_t e3 = cudaFuncSetAttribute(k_tile_scatter,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, bin_smem);
-  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
+  const int need = kBinWarps * max(w.max_nt, 2048) * (int)sizeof(uint32_t);
+  cudaError_t e2 = cudaFuncSetAttribute(k_count_hist, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        need);
+  cudaError_t e3 = cudaFuncSetAttribute(k_count_scatter,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+  if (e2 != cudaSuccess || e3 != cudaSuccess) {
     cudaGetLastError();
     return set_err(w, SPLAT_ERR_CAPACITY,
                    "image has too many tiles for the binning kernels' shared memory");

@@ -65,20 +65,21 @@ int alloc(Workspace& w, T** p, size_t n, const char* what) {
 
 void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
-                 w.inst_tile, w.inst_kv, w.skey, w.sval, w.skey2, w.sval2, w.hist, w.tile_off,
-                 w.d_vstart, w.d_bstart, w.d_scratch};
+                 w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
+                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s};
   for (void* p : dev)
     if (p) cudaFree(p);
   if (w.h_vstart) cudaFreeHost(w.h_vstart);
   if (w.h_bstart) cudaFreeHost(w.h_bstart);
   if (w.h_scratch) cudaFreeHost(w.h_scratch);
+  if (w.h_kbits) cudaFreeHost(w.h_kbits);
   for (cudaEvent_t e : w.ev_pool) cudaEventDestroy(e);
   w.ev_pool.clear();
 }
 
 const char* const kKernelNames[SPLAT_NUM_KERNELS] = {
-    "project", "scan_counts", "emit", "tile_hist", "hist_scan", "tile_scatter", "tile_ranges",
-    "tile_sort", "render", "replay", "finalize", "other"};
+    "project", "scan_counts", "depth_hist", "depth_scatter", "emit", "tile_hist", "hist_scan",
+    "tile_scatter", "tile_ranges", "render", "replay", "finalize", "other"};
 
 // fold every recorded (start, end) pair into the per-kernel sums
 int fold_events(Workspace& w) {
@@ -135,6 +136,16 @@ int splat_ws_create(splat_ws** out, int max_G, int max_V, int max_H, int max_W,
   if (!rc) rc = alloc(w, &w.d_vstart, (size_t)max_V + 1, "view starts");
   if (!rc) rc = alloc(w, &w.d_bstart, (size_t)max_V + 1, "block starts");
   if (!rc) rc = alloc(w, &w.d_scratch, 8, "scratch");
+  if (!rc) rc = alloc(w, &w.dkey, VG, "depth keys");
+  if (!rc) rc = alloc(w, &w.kbits, (size_t)2 * splat::kKeyStripes * max_V, "key statistics");
+  if (!rc) rc = alloc(w, &w.dk1, VG, "depth keys 2");
+  if (!rc) rc = alloc(w, &w.dk2, VG, "depth keys 3");
+  if (!rc) rc = alloc(w, &w.dv0, VG, "depth order");
+  if (!rc) rc = alloc(w, &w.dv1, VG, "depth order 2");
+  if (!rc) rc = alloc(w, &w.rect_s, VG, "rectangles in depth order");
+  if (!rc && cudaMallocHost(&w.h_kbits, (size_t)2 * splat::kKeyStripes * max_V * sizeof(uint32_t)) !=
+                  cudaSuccess)
+    rc = SPLAT_ERR_OOM;
   if (!rc && cudaMallocHost(&w.h_vstart, (max_V + 1) * sizeof(long long)) != cudaSuccess)
     rc = SPLAT_ERR_OOM;
   if (!rc && cudaMallocHost(&w.h_bstart, (max_V + 1) * sizeof(int)) != cudaSuccess)
@@ -218,6 +229,9 @@ int splat_bin_sort(splat_ws* ws, long long* n_instances_out, void* stream) {
   if ((rc = splat::check_launch(w, "view start gather"))) return rc;
   cudaError_t e = cudaMemcpyAsync(w.h_vstart, w.d_vstart, (w.V + 1) * sizeof(long long),
                                   cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(w.h_kbits, w.kbits, (size_t)2 * splat::kKeyStripes * w.V * sizeof(uint32_t),
+                        cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(w, "reading the instance counts", e);
   w.n_total = w.h_vstart[w.V];

@@ -22,6 +22,7 @@ constexpr int kTilePix = 256;
 constexpr int kRecF4 = 4;        // float4 per (v, g) record
 constexpr int kAccN = 8;         // doubles per (v, g) accumulator
 constexpr int kFlagVisible = 256;
+constexpr int kKeyStripes = 64;  // striped copies of the per-view depth-key statistics
 
 // Record of one (view, Gaussian), 4 x float4 = 64 bytes, array-of-structures so that the
 // render's gather of one list entry touches two 32-byte sectors:
@@ -125,14 +126,20 @@ struct Workspace {
   long long* part = nullptr;
   size_t part_cap = 0;
 
+  // per-(v, g) depth order
+  uint32_t* dkey = nullptr;    // [V*G] depth sort keys (written by the projection)
+  uint32_t* kbits = nullptr;   // [V][kKeyStripes][2]: OR of visible keys, OR of complements
+  uint32_t* dk1 = nullptr;     // [V*G] radix ping-pong keys (dkey itself is never overwritten)
+  uint32_t* dk2 = nullptr;     // [V*G]
+  uint32_t* dv0 = nullptr;     // [V*G] radix values (Gaussian index), ping
+  uint32_t* dv1 = nullptr;     // [V*G] pong
+  int4* rect_s = nullptr;      // [V*G] tile rectangles in depth order
+
   // instances
   size_t inst_cap = 0;
-  uint32_t* inst_tile = nullptr;  // [N] tile id within its view
-  uint2* inst_kv = nullptr;       // [N] (depth bits, g)
-  uint32_t* skey = nullptr;       // [N] depth bits, tile-major
-  uint32_t* sval = nullptr;       // [N] g, tile-major; after the depth sort: the tile lists
-  uint32_t* skey2 = nullptr;      // [N] ping-pong for long tiles
-  uint32_t* sval2 = nullptr;
+  uint32_t* inst_tile = nullptr;  // [N] tile id within its view, emitted in depth order
+  uint32_t* inst_g = nullptr;     // [N] Gaussian index
+  uint32_t* sval = nullptr;       // [N] the tile lists: Gaussian indices, tile-major
 
   // tile histogram [sum_v nt * blocks_v] (int32, scanned in place)
   size_t hist_cap = 0;
@@ -144,6 +151,7 @@ struct Workspace {
   int* d_bstart = nullptr;        // [V+1] first binning block of each view
   long long* h_vstart = nullptr;  // pinned
   int* h_bstart = nullptr;        // pinned
+  uint32_t* h_kbits = nullptr;    // pinned [V][kKeyStripes][2]
   long long n_total = 0;
   int n_blocks = 0;
 

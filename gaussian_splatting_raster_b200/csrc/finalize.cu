@@ -12,7 +12,9 @@
 //
 // Because gamma_gv / q_gv = 1 / q_g for every view, each block is a plain sum over views divided
 // once by q_g (the linear rewrite; no second pass over the views). Sums and the eigenvalues are
-// evaluated in double; the SH block's per-view products in fp32.
+// evaluated in double; the SH block's per-view products in fp32, accumulated in a shared-memory
+// tile of the block's token rows (keeps registers, hence occupancy, low) that is then written out
+// with coalesced stores.
 #include "common.cuh"
 
 namespace splat {
@@ -54,90 +56,103 @@ __device__ void eig3_sym(double a00, double a01, double a02, double a11, double 
 }
 
 template <int DEG>
-__global__ void __launch_bounds__(kFinThreads)
+__global__ void __launch_bounds__(kFinThreads, 4)
 k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
            const float* __restrict__ views, int G, int V, double lambda,
            float* __restrict__ tokens) {
   constexpr int D = (DEG + 1) * (DEG + 1);
   constexpr int DT = 9 + 3 * D;
-  const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= G) return;
-  const double eps = 1e-6;
-  double qsum = 0.0, b0 = 0.0, b1 = 0.0, b2 = 0.0, sa = 0.0;
-  double A00 = 0.0, A01 = 0.0, A02 = 0.0, A11 = 0.0, A12 = 0.0, A22 = 0.0;
-  float ssh[3 * D];
+  constexpr int P = kFinThreads + 1;  // padded column stride: conflict-free row/column access
+  // the block's token rows, column-major; the SH block is accumulated here directly
+  __shared__ float s_tok[DT * P];
+  const int g0 = blockIdx.x * kFinThreads;
+  const int g = g0 + threadIdx.x;
+  float* col = s_tok + threadIdx.x;
 #pragma unroll
-  for (int k = 0; k < 3 * D; ++k) ssh[k] = 0.0f;
-  for (int v = 0; v < V; ++v) {
-    const size_t i = (size_t)v * G + g;
-    const float4 r3 = rec[i * kRecF4 + 3];
-    const int flags = __float_as_int(r3.w);
-    if (!(flags & kFlagVisible)) continue;
-    const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1], r2 = rec[i * kRecF4 + 2];
-    const double* a = acc + i * kAccN;
-    const double qgv = eps + a[0];
-    qsum += qgv;
-    sa += (1.0 - (double)r1.y) * a[4];
-    const double qa = r0.z, qb = r0.w, qc = r1.x;
-    const double sm0 = qa * a[5] + qb * a[6];
-    const double sm1 = qb * a[5] + qc * a[6];
-    // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
-    const float* vw = views + 20 * v;
-    const double fx = vw[16], fy = vw[17];
-    const double x = r2.z, y = r2.w, z = r2.y;
-    const double j00 = fx / z, j02 = -fx * x / (z * z);
-    const double j11 = fy / z, j12 = -fy * y / (z * z);
-    double J0[3], J1[3];
+  for (int k = 0; k < 3 * D; ++k) col[(4 + k) * P] = 0.0f;
+  if (g < G) {
+    const double eps = 1e-6;
+    double qsum = 0.0, b0 = 0.0, b1 = 0.0, b2 = 0.0, sa = 0.0;
+    double A00 = 0.0, A01 = 0.0, A02 = 0.0, A11 = 0.0, A12 = 0.0, A22 = 0.0;
+    for (int v = 0; v < V; ++v) {
+      const size_t i = (size_t)v * G + g;
+      const float4 r3 = rec[i * kRecF4 + 3];
+      const int flags = __float_as_int(r3.w);
+      if (!(flags & kFlagVisible)) continue;
+      const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1], r2 = rec[i * kRecF4 + 2];
+      const double2* a2 = reinterpret_cast<const double2*>(acc + i * kAccN);
+      const double2 a01 = a2[0], a23 = a2[1], a45 = a2[2], a67 = a2[3];
+      const double qgv = eps + a01.x;
+      qsum += qgv;
+      sa += (1.0 - (double)r1.y) * a45.x;
+      const double qa = r0.z, qb = r0.w, qc = r1.x;
+      const double sm0 = qa * a45.y + qb * a67.x;
+      const double sm1 = qb * a45.y + qc * a67.x;
+      // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
+      const float* vw = views + 20 * v;
+      const double fx = vw[16], fy = vw[17];
+      const double x = r2.z, y = r2.w, z = r2.y;
+      const double j00 = fx / z, j02 = -fx * x / (z * z);
+      const double j11 = fy / z, j12 = -fy * y / (z * z);
+      double J0[3], J1[3];
 #pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      J0[c] = j00 * (double)vw[c] + j02 * (double)vw[8 + c];
-      J1[c] = j11 * (double)vw[4 + c] + j12 * (double)vw[8 + c];
+      for (int c = 0; c < 3; ++c) {
+        J0[c] = j00 * (double)vw[c] + j02 * (double)vw[8 + c];
+        J1[c] = j11 * (double)vw[4 + c] + j12 * (double)vw[8 + c];
+      }
+      b0 += J0[0] * sm0 + J1[0] * sm1;
+      b1 += J0[1] * sm0 + J1[1] * sm1;
+      b2 += J0[2] * sm0 + J1[2] * sm1;
+      A00 += qgv * (J0[0] * J0[0] + J1[0] * J1[0]);
+      A01 += qgv * (J0[0] * J0[1] + J1[0] * J1[1]);
+      A02 += qgv * (J0[0] * J0[2] + J1[0] * J1[2]);
+      A11 += qgv * (J0[1] * J0[1] + J1[1] * J1[1]);
+      A12 += qgv * (J0[1] * J0[2] + J1[1] * J1[2]);
+      A22 += qgv * (J0[2] * J0[2] + J1[2] * J1[2]);
+      float B[16];
+      sh_poly<DEG>(r3.x, r3.y, r3.z, B);
+      const float w0 = (flags & 1) ? (float)a01.y : 0.0f;
+      const float w1 = (flags & 2) ? (float)a23.x : 0.0f;
+      const float w2 = (flags & 4) ? (float)a23.y : 0.0f;
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        col[(4 + 3 * k) * P] += B[k] * w0;
+        col[(5 + 3 * k) * P] += B[k] * w1;
+        col[(6 + 3 * k) * P] += B[k] * w2;
+      }
     }
-    b0 += J0[0] * sm0 + J1[0] * sm1;
-    b1 += J0[1] * sm0 + J1[1] * sm1;
-    b2 += J0[2] * sm0 + J1[2] * sm1;
-    A00 += qgv * (J0[0] * J0[0] + J1[0] * J1[0]);
-    A01 += qgv * (J0[0] * J0[1] + J1[0] * J1[1]);
-    A02 += qgv * (J0[0] * J0[2] + J1[0] * J1[2]);
-    A11 += qgv * (J0[1] * J0[1] + J1[1] * J1[1]);
-    A12 += qgv * (J0[1] * J0[2] + J1[1] * J1[2]);
-    A22 += qgv * (J0[2] * J0[2] + J1[2] * J1[2]);
-    float B[16];
-    sh_poly<DEG>(r3.x, r3.y, r3.z, B);
-    const float w0 = (flags & 1) ? (float)a[1] : 0.0f;
-    const float w1 = (flags & 2) ? (float)a[2] : 0.0f;
-    const float w2 = (flags & 4) ? (float)a[3] : 0.0f;
+    const double qg = eps + qsum;
+    const double inv = 1.0 / qg;
+    A00 = A00 * inv + lambda;
+    A11 = A11 * inv + lambda;
+    A22 = A22 * inv + lambda;
+    A01 *= inv;
+    A02 *= inv;
+    A12 *= inv;
+    double ev[3];
+    eig3_sym(A00, A01, A02, A11, A12, A22, ev);
+    const double tr = A00 + A11 + A22;
+    col[0 * P] = (float)(b0 * inv);
+    col[1 * P] = (float)(b1 * inv);
+    col[2 * P] = (float)(b2 * inv);
+    col[3 * P] = (float)(sa * inv);
 #pragma unroll
-    for (int k = 0; k < D; ++k) {
-      ssh[3 * k + 0] += B[k] * w0;
-      ssh[3 * k + 1] += B[k] * w1;
-      ssh[3 * k + 2] += B[k] * w2;
-    }
+    for (int k = 0; k < 3 * D; ++k) col[(4 + k) * P] = (float)((double)col[(4 + k) * P] * inv);
+    col[(4 + 3 * D) * P] = (float)log(qg);
+    const double itr = 1.0 / (tr + eps);
+    col[(5 + 3 * D) * P] = (float)(ev[0] * itr);
+    col[(6 + 3 * D) * P] = (float)(ev[1] * itr);
+    col[(7 + 3 * D) * P] = (float)(ev[2] * itr);
+    col[(8 + 3 * D) * P] = (float)log(tr + eps);
   }
-  const double qg = eps + qsum;
-  const double inv = 1.0 / qg;
-  A00 = A00 * inv + lambda;
-  A11 = A11 * inv + lambda;
-  A22 = A22 * inv + lambda;
-  A01 *= inv;
-  A02 *= inv;
-  A12 *= inv;
-  double ev[3];
-  eig3_sym(A00, A01, A02, A11, A12, A22, ev);
-  const double tr = A00 + A11 + A22;
-  float* zt = tokens + (size_t)g * DT;
-  zt[0] = (float)(b0 * inv);
-  zt[1] = (float)(b1 * inv);
-  zt[2] = (float)(b2 * inv);
-  zt[3] = (float)(sa * inv);
-#pragma unroll
-  for (int k = 0; k < 3 * D; ++k) zt[4 + k] = (float)((double)ssh[k] * inv);
-  zt[4 + 3 * D] = (float)log(qg);
-  const double itr = 1.0 / (tr + eps);
-  zt[5 + 3 * D] = (float)(ev[0] * itr);
-  zt[6 + 3 * D] = (float)(ev[1] * itr);
-  zt[7 + 3 * D] = (float)(ev[2] * itr);
-  zt[8 + 3 * D] = (float)log(tr + eps);
+  __syncthreads();
+  // the block's rows are contiguous in the output: coalesced stores
+  const int ng = min(kFinThreads, G - g0);
+  float* out = tokens + (size_t)g0 * DT;
+  for (int L = threadIdx.x; L < ng * DT; L += kFinThreads) {
+    const int row = L / DT, c = L - row * DT;
+    out[L] = s_tok[c * P + row];
+  }
 }
 
 }  // namespace

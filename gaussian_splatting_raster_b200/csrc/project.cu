@@ -29,7 +29,7 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
           const float* __restrict__ quats, const float* __restrict__ opac,
           const float* __restrict__ sh, const float* __restrict__ views_in, int G, int V, int H,
           int W, int TX, int TY, float4* __restrict__ rec, int4* __restrict__ rect,
-          int* __restrict__ counts) {
+          int* __restrict__ counts, uint32_t* __restrict__ dkey, uint32_t* __restrict__ kbits) {
   constexpr int D = (DEG + 1) * (DEG + 1);
   constexpr int NSH = D * 3;
   // shared memory: the block's SH coefficients [kProjThreads][NSH], then the views [V][20]
@@ -194,6 +194,21 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
     rp[3] = r3;
     rect[i] = rc;
     counts[i] = cnt;
+    // depth sort key (fp32 bits of z > 0 order like the values; culled entries sort last) and,
+    // per view, the OR of the visible keys and of their complements: a bit varies among the
+    // visible keys exactly where both ORs have it set
+    const uint32_t key = cnt > 0 ? __float_as_uint(z) : 0xffffffffu;
+    dkey[i] = key;
+    const unsigned lanes = __activemask();
+    const uint32_t k1 = __reduce_or_sync(lanes, cnt > 0 ? key : 0u);
+    const uint32_t k0 = __reduce_or_sync(lanes, cnt > 0 ? ~key : 0u);
+    if ((threadIdx.x & 31) == __ffs(lanes) - 1 && (k1 | k0)) {
+      // one of kKeyStripes copies per view, chosen by block, keeps same-address atomics rare;
+      // the host ORs the stripes together
+      uint32_t* kb = kbits + 2 * (v * kKeyStripes + (blockIdx.x & (kKeyStripes - 1)));
+      atomicOr(kb, k1);
+      atomicOr(kb + 1, k0);
+    }
   }
 }
 
@@ -201,6 +216,10 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
 
 int launch_project(Workspace& w, const float* means, const float* lsc, const float* quats,
                    const float* opac, const float* sh, cudaStream_t st) {
+  cudaError_t e =
+      cudaMemsetAsync(w.kbits, 0, (size_t)2 * kKeyStripes * w.V * sizeof(uint32_t), st);
+  if (e != cudaSuccess)
+    return set_err(w, SPLAT_ERR_CUDA, std::string("key statistics clear: ") + cudaGetErrorString(e));
   if (w.G == 0) return SPLAT_OK;
   const int blocks = (w.G + kProjThreads - 1) / kProjThreads;
   const int tok = prof_begin(w, st, SPLAT_K_PROJECT);
@@ -214,7 +233,7 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
       return set_err(w, SPLAT_ERR_CAPACITY, "too many views for the projection kernel");        \
     k_project<DEG><<<blocks, kProjThreads, smem, st>>>(means, lsc, quats, opac, sh, w.views,     \
                                                        w.G, w.V, w.H, w.W, w.TX, w.TY, w.rec,    \
-                                                       w.rect, w.counts);                        \
+                                                       w.rect, w.counts, w.dkey, w.kbits);       \
   }
   switch (w.deg) {
     case 0: SPLAT_PROJ(0); break;

@@ -17,7 +17,9 @@
 // every staged entry the loader computes cut = log((1/255) / o) - 1e-3; an exponent below cut
 // gives o exp(pw) < (1/255) exp(-1e-3), far below 1/255 even after the few-ulp errors of the
 // exp and of the product, so the entry is skipped without evaluating exp -- the same decision the
-// full evaluation takes, never a different one.
+// full evaluation takes, never a different one. The loader also computes, per entry, which of the
+// CTA's eight warps (two pixel rows each) the ellipse {exponent >= cut} can reach at all; the
+// other warps skip the entry with one warp-uniform test.
 //
 // Replay arithmetic. The suffix numerators C_hat - P - T alpha c are formed per channel exactly
 // as the recovery equation writes them (their cancellation dominates the fp32 error of C+), then
@@ -46,6 +48,31 @@ struct Entry {
 
 // exponent cut below which alpha < 1/255 is certain (see the file comment)
 __device__ __forceinline__ float skip_cut(float o) { return logf(kAlphaMin / o) - 1e-3f; }
+
+// Warps of the CTA (warp w holds pixel rows 2w, 2w + 1 of the tile) whose pixel centres can reach
+// the entry's exponent >= cut ellipse {d : d^T Q d <= -2 cut}. Its half-extents are
+// sqrt(-2 cut (Q^-1)_xx) and sqrt(-2 cut (Q^-1)_yy), widened by 1 % + 0.05 px: far more than the
+// fp32 evaluation of the exponent (or of det Q when det Q > 1e-4 qa qc) can move the boundary.
+// Nearly singular conics get every warp. Warps outside the box would only skip the entry, so
+// leaving them out changes no decision.
+__device__ __forceinline__ uint32_t strip_mask(float4 A, float qc, float cut, float x0f,
+                                               float y0f) {
+  if (!(cut < 0.0f)) return 0u;
+  const float det = A.z * qc - A.w * A.w;
+  if (!(det > 1e-4f * (A.z * qc))) return 0xffu;
+  const float r2 = -2.0f * cut;
+  const float ex = sqrtf(r2 * qc / det) * 1.01f + 0.05f;
+  const float ey = sqrtf(r2 * A.z / det) * 1.01f + 0.05f;
+  // pixel centres of the tile: x0f + 0.5 .. x0f + 15.5, rows y0f + 0.5 + r, r = 0 .. 15
+  if (A.x + ex < x0f + 0.5f || A.x - ex > x0f + 15.5f) return 0u;
+  const float lo = A.y - ey - (y0f + 0.5f), hi = A.y + ey - (y0f + 0.5f);
+  if (hi < 0.0f || lo > 15.0f) return 0u;
+  const int r0 = lo <= 0.0f ? 0 : (int)ceilf(lo);
+  const int r1 = hi >= 15.0f ? 15 : (int)floorf(hi);
+  if (r1 < r0) return 0u;
+  const int w0 = r0 >> 1, w1 = r1 >> 1;
+  return ((2u << w1) - 1u) & ~((1u << w0) - 1u);
+}
 
 // alpha of one list entry at pixel centre (px, py), with the rasteriser's skip rules
 __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
@@ -78,47 +105,60 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const long long e = tile_off[(size_t)v * (nt + 1) + t + 1];
+  // Each warp walks the whole list on its own (no CTA barriers): it stages 32 entries into its
+  // slice of shared memory, ballots which of them can reach its two pixel rows, evaluates only
+  // those, and leaves as soon as its 32 pixels are done.
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];  // (colour b, exponent cut)
+  float4* wa = s_a + warp * 32;
+  float4* wb = s_b + warp * 32;
+  float2* wc = s_c + warp * 32;
+  const float x0f = (float)(tx * kTile), y0f = (float)(ty * kTile);
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int n = 0, lst = 0;
   bool done = !inside;
   const float4* recv = rec + (size_t)v * G * kRecF4;
-  for (long long base = s; base < e; base += kThreads) {
-    if (__syncthreads_count(done) == kThreads) break;
-    const long long k = base + threadIdx.x;
+  for (long long base = s; base < e; base += 32) {
+    if (__all_sync(0xffffffffu, done)) break;
+    const long long k = base + lane;
+    bool hit = false;
     if (k < e) {
       const float4* r = recv + (size_t)ids[k] * kRecF4;
-      const float4 b = r[1];
-      s_a[threadIdx.x] = r[0];
-      s_b[threadIdx.x] = b;
-      s_c[threadIdx.x] = make_float2(r[2].x, skip_cut(b.y));
+      const float4 a = r[0], b = r[1];
+      const float cut = skip_cut(b.y);
+      wa[lane] = a;
+      wb[lane] = b;
+      wc[lane] = make_float2(r[2].x, cut);
+      hit = (strip_mask(a, b.x, cut, x0f, y0f) >> warp) & 1u;
     }
-    __syncthreads();
-    const int cnt = (int)min((long long)kThreads, e - base);
-    if (!done) {
-      for (int q = 0; q < cnt; ++q) {
-        const float4 A = s_a[q], Bq = s_b[q];
-        const float2 Cq = s_c[q];
-        const Entry E = eval_entry(A, Bq, Cq.y, px, py);
-        if (!E.use) continue;
-        const float Tn = T * (1.0f - E.alpha);
-        if (Tn < 1e-4f) {
-          done = true;
-          break;
-        }
-        const float wgt = E.alpha * T;
-        // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is then
-        // exactly the background term, and the suffix recovery sees no rounding mismatch
-        C0 = C0 + wgt * Bq.z;
-        C1 = C1 + wgt * Bq.w;
-        C2 = C2 + wgt * Cq.x;
-        T = Tn;
-        ++n;
-        lst = (int)(base - s) + q + 1;
+    uint32_t bits = __ballot_sync(0xffffffffu, hit);
+    __syncwarp();
+    while (bits) {  // warp-uniform: entries that can reach this warp's rows, in list order
+      const int q = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (done) continue;
+      const float4 A = wa[q], Bq = wb[q];
+      const float2 Cq = wc[q];
+      const Entry E = eval_entry(A, Bq, Cq.y, px, py);
+      if (!E.use) continue;
+      const float Tn = T * (1.0f - E.alpha);
+      if (Tn < 1e-4f) {
+        done = true;
+        continue;
       }
+      const float wgt = E.alpha * T;
+      // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is then
+      // exactly the background term, and the suffix recovery sees no rounding mismatch
+      C0 = C0 + wgt * Bq.z;
+      C1 = C1 + wgt * Bq.w;
+      C2 = C2 + wgt * Cq.x;
+      T = Tn;
+      ++n;
+      lst = (int)(base - s) + q + 1;
     }
+    __syncwarp();
   }
   if (inside) {
     const size_t p = ((size_t)v * H + j) * W + i;
@@ -155,7 +195,10 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];
+  __shared__ uint32_t s_m[kThreads];
   __shared__ uint32_t s_g[kThreads];
+  const int warp = threadIdx.x >> 5;
+  const float x0f = (float)(tx * kTile), y0f = (float)(ty * kTile);
   __shared__ float s_acc[8][kThreads];
   __shared__ int s_max;
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
@@ -187,16 +230,29 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     if ((int)threadIdx.x < cnt) {
       const uint32_t g = ids[s + base + threadIdx.x];
       const float4* r = recv + (size_t)g * kRecF4;
-      const float4 b = r[1];
-      s_a[threadIdx.x] = r[0];
+      const float4 a = r[0], b = r[1];
+      const float cut = skip_cut(b.y);
+      s_a[threadIdx.x] = a;
       s_b[threadIdx.x] = b;
-      s_c[threadIdx.x] = make_float2(r[2].x, skip_cut(b.y));
+      s_c[threadIdx.x] = make_float2(r[2].x, cut);
+      s_m[threadIdx.x] = strip_mask(a, b.x, cut, x0f, y0f);
       s_g[threadIdx.x] = g;
     }
 #pragma unroll
     for (int c = 0; c < 8; ++c) s_acc[c][threadIdx.x] = 0.0f;
     __syncthreads();
-    for (int q = 0; q < cnt; ++q) {
+    // this warp's entries of the batch: those whose ellipse can reach its two pixel rows
+    uint32_t sel[kThreads / 32];
+#pragma unroll
+    for (int c = 0; c < kThreads / 32; ++c) {
+      const int q = c * 32 + lane;
+      sel[c] = __ballot_sync(0xffffffffu, q < cnt && ((s_m[q] >> warp) & 1u));
+    }
+#pragma unroll
+    for (int c = 0; c < kThreads / 32; ++c)
+    while (sel[c]) {  // warp-uniform, in list order
+      const int q = c * 32 + __ffs(sel[c]) - 1;
+      sel[c] &= sel[c] - 1;
       float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
       bool used = false;
       if (base + q < lst) {

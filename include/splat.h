@@ -165,9 +165,9 @@ long long splat_launch_count(const splat_ws* ws);
  * group id (0 .. SPLAT_NUM_KERNELS-1), the elapsed milliseconds and the number of timed launches
  * since the last reset (reset != 0 clears after reading). Off by default. */
 enum {
-  SPLAT_K_PROJECT = 0, SPLAT_K_SCAN_COUNTS, SPLAT_K_EMIT, SPLAT_K_TILE_HIST, SPLAT_K_HIST_SCAN,
-  SPLAT_K_TILE_SCATTER, SPLAT_K_TILE_RANGES, SPLAT_K_TILE_SORT, SPLAT_K_RENDER, SPLAT_K_REPLAY,
-  SPLAT_K_FINALIZE, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
+  SPLAT_K_PROJECT = 0, SPLAT_K_SCAN_COUNTS, SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER,
+  SPLAT_K_EMIT, SPLAT_K_TILE_HIST, SPLAT_K_HIST_SCAN, SPLAT_K_TILE_SCATTER, SPLAT_K_TILE_RANGES,
+  SPLAT_K_RENDER, SPLAT_K_REPLAY, SPLAT_K_FINALIZE, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
 };
 int splat_profile_enable(splat_ws* ws, int enable);
 int splat_profile_read(splat_ws* ws, double* ms, long long* launches, int reset);
