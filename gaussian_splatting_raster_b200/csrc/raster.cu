@@ -193,14 +193,18 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
+  // Like the render, each warp walks the list on its own: 32-entry chunks staged into its slice
+  // of shared memory, a ballot of the entries that can reach its two pixel rows, no CTA barriers.
+  // Its per-entry sums go straight from the seven lanes holding them to the fp64 accumulators.
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];
-  __shared__ uint32_t s_m[kThreads];
   __shared__ uint32_t s_g[kThreads];
-  const int warp = threadIdx.x >> 5;
+  float4* wa = s_a + warp * 32;
+  float4* wb = s_b + warp * 32;
+  float2* wc = s_c + warp * 32;
+  uint32_t* wg = s_g + warp * 32;
   const float x0f = (float)(tx * kTile), y0f = (float)(ty * kTile);
-  __shared__ float s_acc[8][kThreads];
-  __shared__ int s_max;
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   float Ch0 = 0.0f, Ch1 = 0.0f, Ch2 = 0.0f, r0 = 0.0f, r1 = 0.0f, r2 = 0.0f;
   int lst = 0;
@@ -214,50 +218,36 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     r2 = Ch2 - obs[3 * p + 2];
     lst = last[p];
   }
-  if (threadIdx.x == 0) s_max = 0;
-  __syncthreads();
-  atomicMax(&s_max, lst);
-  __syncthreads();
-  const int maxl = s_max;
+  const int wmax = __reduce_max_sync(0xffffffffu, lst);  // entries this warp must traverse
   const float4* recv = rec + (size_t)v * G * kRecF4;
   double* accv = acc + (size_t)v * G * kAccN;
   float T = 1.0f, P0 = 0.0f, P1 = 0.0f, P2 = 0.0f;  // transmittance, prefix colour
-  const int lane = threadIdx.x & 31;
   const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
   const int slot = (lane >> 2) & 7;  // value index this lane holds after the reduction
-  for (int base = 0; base < maxl; base += kThreads) {
-    const int cnt = min(kThreads, maxl - base);
-    if ((int)threadIdx.x < cnt) {
-      const uint32_t g = ids[s + base + threadIdx.x];
+  for (int base = 0; base < wmax; base += 32) {
+    const int k = base + lane;
+    bool hit = false;
+    if (k < wmax) {
+      const uint32_t g = ids[s + k];
       const float4* r = recv + (size_t)g * kRecF4;
       const float4 a = r[0], b = r[1];
       const float cut = skip_cut(b.y);
-      s_a[threadIdx.x] = a;
-      s_b[threadIdx.x] = b;
-      s_c[threadIdx.x] = make_float2(r[2].x, cut);
-      s_m[threadIdx.x] = strip_mask(a, b.x, cut, x0f, y0f);
-      s_g[threadIdx.x] = g;
+      wa[lane] = a;
+      wb[lane] = b;
+      wc[lane] = make_float2(r[2].x, cut);
+      wg[lane] = g;
+      hit = (strip_mask(a, b.x, cut, x0f, y0f) >> warp) & 1u;
     }
-#pragma unroll
-    for (int c = 0; c < 8; ++c) s_acc[c][threadIdx.x] = 0.0f;
-    __syncthreads();
-    // this warp's entries of the batch: those whose ellipse can reach its two pixel rows
-    uint32_t sel[kThreads / 32];
-#pragma unroll
-    for (int c = 0; c < kThreads / 32; ++c) {
-      const int q = c * 32 + lane;
-      sel[c] = __ballot_sync(0xffffffffu, q < cnt && ((s_m[q] >> warp) & 1u));
-    }
-#pragma unroll
-    for (int c = 0; c < kThreads / 32; ++c)
-    while (sel[c]) {  // warp-uniform, in list order
-      const int q = c * 32 + __ffs(sel[c]) - 1;
-      sel[c] &= sel[c] - 1;
+    uint32_t bits = __ballot_sync(0xffffffffu, hit);
+    __syncwarp();
+    while (bits) {  // warp-uniform: entries that can reach this warp's rows, in list order
+      const int q = __ffs(bits) - 1;
+      bits &= bits - 1;
       float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
       bool used = false;
       if (base + q < lst) {
-        const float4 A = s_a[q], Bq = s_b[q];
-        const float2 Cq = s_c[q];
+        const float4 A = wa[q], Bq = wb[q];
+        const float2 Cq = wc[q];
         const Entry E = eval_entry(A, Bq, Cq.y, px, py);
         if (E.use) {
           used = true;
@@ -296,16 +286,11 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         tr_step<1>(x, b2, 4);
         x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
         x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
-        if ((lane & 3) == 0 && slot < 7) atomicAdd(&s_acc[slot][q], x[0]);
+        if ((lane & 3) == 0 && slot < 7 && x[0] != 0.0f)
+          atomicAdd(accv + (size_t)wg[q] * kAccN + slot, (double)x[0]);
       }
     }
-    __syncthreads();
-    if ((int)threadIdx.x < cnt && s_acc[0][threadIdx.x] != 0.0f) {
-      double* a = accv + (size_t)s_g[threadIdx.x] * kAccN;
-#pragma unroll
-      for (int c = 0; c < 7; ++c) atomicAdd(a + c, (double)s_acc[c][threadIdx.x]);
-    }
-    __syncthreads();
+    __syncwarp();
   }
 }
 
