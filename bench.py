@@ -137,7 +137,7 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
     return {
         # read the parameters once, write per (v, g) record (64 B), rectangle (16 B), count (4 B)
         "project": G * (4 * (3 + 3 + 4 + 1) + 12 * d) + V * G * (64 + 16 + 4),
-        "scan_counts": V * G * (4 + 8),
+
         # one depth-digit pass per launch over every (v, g): histogram reads the keys, the
         # scatter reads key + index and writes both
         "depth_hist": V * G * 4,
@@ -404,7 +404,7 @@ def main():
         if k in ab:
             v["algorithmic_GBps"] = ab[k] / (v["ms_per_step"] * 1e-3) / 1e9
     render_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in
-                    ("project", "scan_counts", "depth_hist", "depth_scatter", "emit", "tile_hist",
+                    ("project", "depth_hist", "depth_scatter", "emit", "tile_hist",
                      "hist_scan", "tile_scatter", "tile_ranges", "render", "other"))
     replay_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in ("replay", "finalize"))
 

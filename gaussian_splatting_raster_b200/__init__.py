@@ -29,7 +29,7 @@ EXPORTS = [
 ]
 
 
-KERNEL_GROUPS = 13  # SPLAT_NUM_KERNELS
+KERNEL_GROUPS = 12  # SPLAT_NUM_KERNELS
 
 
 class SplatError(RuntimeError):

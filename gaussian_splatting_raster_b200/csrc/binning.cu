@@ -379,12 +379,6 @@ int scan_i32_inplace(Workspace& w, int* data, long long n, cudaStream_t st) {
   return check_launch(w, "hist scan downsweep");
 }
 
-int launch_scan_counts(Workspace& w, cudaStream_t st) {
-  const int tok = prof_begin(w, st, SPLAT_K_SCAN_COUNTS);
-  const int rc = scan_i32_to_i64(w, w.counts, w.offs, (long long)w.V * w.G, st);
-  prof_end(w, st, tok);
-  return rc;
-}
 
 // one stable counting-sort pass (histogram, scan, scatter)
 static int count_pass(Workspace& w, cudaStream_t st, const uint32_t* keys, const uint32_t* vals,
@@ -420,6 +414,14 @@ int launch_binning(Workspace& w, cudaStream_t st) {
     if ((rc = grow(w, &w.inst_g, cap, "instance indices"))) return rc;
     if ((rc = grow(w, &w.sval, cap, "tile lists"))) return rc;
     w.inst_cap = cap;
+  }
+  {
+    const size_t need = ((size_t)N / 32 + (size_t)w.V * w.nt + 2) * 8;
+    if (need > w.umask_cap) {
+      const size_t cap = need + need / 4;
+      if ((rc = grow(w, &w.umask, cap, "composited-entry masks"))) return rc;
+      w.umask_cap = cap;
+    }
   }
   // ---- 1. depth order of every view's Gaussians --------------------------------------------
   // highest bit that varies among any view's visible keys -> number of digit passes

@@ -66,19 +66,20 @@ int alloc(Workspace& w, T** p, size_t n, const char* what) {
 void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
-                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s};
+                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask};
   for (void* p : dev)
     if (p) cudaFree(p);
   if (w.h_vstart) cudaFreeHost(w.h_vstart);
   if (w.h_bstart) cudaFreeHost(w.h_bstart);
   if (w.h_scratch) cudaFreeHost(w.h_scratch);
   if (w.h_kbits) cudaFreeHost(w.h_kbits);
+  if (w.h_ntot) cudaFreeHost(w.h_ntot);
   for (cudaEvent_t e : w.ev_pool) cudaEventDestroy(e);
   w.ev_pool.clear();
 }
 
 const char* const kKernelNames[SPLAT_NUM_KERNELS] = {
-    "project", "scan_counts", "depth_hist", "depth_scatter", "emit", "tile_hist", "hist_scan",
+    "project", "depth_hist", "depth_scatter", "emit", "tile_hist", "hist_scan",
     "tile_scatter", "tile_ranges", "render", "replay", "finalize", "other"};
 
 // fold every recorded (start, end) pair into the per-kernel sums
@@ -97,10 +98,6 @@ int fold_events(Workspace& w) {
   return SPLAT_OK;
 }
 
-__global__ void k_gather_vstart(const long long* offs, int G, int V, long long* out) {
-  const int v = blockIdx.x * blockDim.x + threadIdx.x;
-  if (v <= V) out[v] = offs[(size_t)v * G];
-}
 
 }  // namespace
 
@@ -138,6 +135,10 @@ int splat_ws_create(splat_ws** out, int max_G, int max_V, int max_H, int max_W,
   if (!rc) rc = alloc(w, &w.d_scratch, 8, "scratch");
   if (!rc) rc = alloc(w, &w.dkey, VG, "depth keys");
   if (!rc) rc = alloc(w, &w.kbits, (size_t)2 * splat::kKeyStripes * max_V, "key statistics");
+  if (!rc) rc = alloc(w, &w.ntot, (size_t)splat::kKeyStripes * max_V, "instance counts");
+  if (!rc && cudaMallocHost(&w.h_ntot, (size_t)splat::kKeyStripes * max_V *
+                                           sizeof(unsigned long long)) != cudaSuccess)
+    rc = SPLAT_ERR_OOM;
   if (!rc) rc = alloc(w, &w.dk1, VG, "depth keys 2");
   if (!rc) rc = alloc(w, &w.dk2, VG, "depth keys 3");
   if (!rc) rc = alloc(w, &w.dv0, VG, "depth order");
@@ -211,7 +212,6 @@ int splat_project(splat_ws* ws, const float* means, const float* log_scales, con
                           4 * sizeof(float), V, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_fail(w, "copying the cameras", e);
   if ((rc = splat::launch_project(w, means, log_scales, quats, opac_logits, sh, st))) return rc;
-  if ((rc = splat::launch_scan_counts(w, st))) return rc;
   w.stage = 1;
   return SPLAT_OK;
 }
@@ -222,18 +222,23 @@ int splat_bin_sort(splat_ws* ws, long long* n_instances_out, void* stream) {
   w.err.clear();
   if (w.stage < 1) return fail(w, SPLAT_ERR_STATE, "splat_bin_sort before splat_project");
   cudaStream_t st = (cudaStream_t)stream;
-  const int tok = splat::prof_begin(w, st, SPLAT_K_OTHER);
-  k_gather_vstart<<<(w.V + 1 + 127) / 128, 128, 0, st>>>(w.offs, w.G, w.V, w.d_vstart);
-  splat::prof_end(w, st, tok);
   int rc;
-  if ((rc = splat::check_launch(w, "view start gather"))) return rc;
-  cudaError_t e = cudaMemcpyAsync(w.h_vstart, w.d_vstart, (w.V + 1) * sizeof(long long),
+  // the one synchronisation of the path: per-view instance counts and depth-key statistics,
+  // accumulated in striped copies by the projection, folded here
+  const int ns = splat::kKeyStripes;
+  cudaError_t e = cudaMemcpyAsync(w.h_ntot, w.ntot, (size_t)ns * w.V * sizeof(unsigned long long),
                                   cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess)
-    e = cudaMemcpyAsync(w.h_kbits, w.kbits, (size_t)2 * splat::kKeyStripes * w.V * sizeof(uint32_t),
+    e = cudaMemcpyAsync(w.h_kbits, w.kbits, (size_t)2 * ns * w.V * sizeof(uint32_t),
                         cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(w, "reading the instance counts", e);
+  w.h_vstart[0] = 0;
+  for (int v = 0; v < w.V; ++v) {
+    unsigned long long nv = 0;
+    for (int k = 0; k < ns; ++k) nv += w.h_ntot[v * ns + k];
+    w.h_vstart[v + 1] = w.h_vstart[v] + (long long)nv;
+  }
   w.n_total = w.h_vstart[w.V];
   if (w.n_total >= (1LL << 31) - 1)
     return fail(w, SPLAT_ERR_CAPACITY, "%lld instances exceed the 2^31 limit", w.n_total);

@@ -24,10 +24,13 @@ constexpr int kAccN = 8;         // doubles per (v, g) accumulator
 constexpr int kFlagVisible = 256;
 constexpr int kKeyStripes = 64;  // striped copies of the per-view depth-key statistics
 
-// Record of one (view, Gaussian), 4 x float4 = 64 bytes, array-of-structures so that the
-// render's gather of one list entry touches two 32-byte sectors:
+// Record of one (view, Gaussian), 4 x float4 = 64 bytes, array-of-structures: the render and the
+// replay gather r0..r2 (48 bytes), the finaliser r0, r1, r3.
 //   r0 = (mx, my, conic a, conic b)        r1 = (conic c, opacity, colour r, colour g)
-//   r2 = (colour b, depth z, x_c, y_c)     r3 = (dir x, dir y, dir z, flags as int bits)
+//   r2 = (colour b, cut, ex, ey)           r3 = (depth z, x_c, y_c, flags as int bits)
+// cut = log((1/255) / o) - 1e-3: an exponent below it gives alpha < 1/255 for certain;
+// (ex, ey) = half-extents of the ellipse {exponent >= cut} widened by 1 % + 0.05 px (+inf for a
+// nearly singular conic, -1 when no pixel can pass).
 // flags: bits 0..2 colour clamp inactive per channel (M_color), bit 8 visible.
 
 // ---------------------------------------------------------------------------------------------
@@ -129,6 +132,8 @@ struct Workspace {
   // per-(v, g) depth order
   uint32_t* dkey = nullptr;    // [V*G] depth sort keys (written by the projection)
   uint32_t* kbits = nullptr;   // [V][kKeyStripes][2]: OR of visible keys, OR of complements
+  unsigned long long* ntot = nullptr;  // [V][kKeyStripes] instance counts (striped)
+  unsigned long long* h_ntot = nullptr;  // pinned copy
   uint32_t* dk1 = nullptr;     // [V*G] radix ping-pong keys (dkey itself is never overwritten)
   uint32_t* dk2 = nullptr;     // [V*G]
   uint32_t* dv0 = nullptr;     // [V*G] radix values (Gaussian index), ping
@@ -140,6 +145,9 @@ struct Workspace {
   uint32_t* inst_tile = nullptr;  // [N] tile id within its view, emitted in depth order
   uint32_t* inst_g = nullptr;     // [N] Gaussian index
   uint32_t* sval = nullptr;       // [N] the tile lists: Gaussian indices, tile-major
+  // per (tile, 32-entry chunk, warp): entries some pixel of the warp composited (render -> replay)
+  uint32_t* umask = nullptr;
+  size_t umask_cap = 0;
 
   // tile histogram [sum_v nt * blocks_v] (int32, scanned in place)
   size_t hist_cap = 0;
@@ -214,7 +222,6 @@ inline int check_launch(Workspace& w, const char* what) {
 // host entry points implemented in the .cu files
 int launch_project(Workspace& w, const float* means, const float* lsc, const float* quats,
                    const float* opac, const float* sh, cudaStream_t st);
-int launch_scan_counts(Workspace& w, cudaStream_t st);
 int launch_binning(Workspace& w, cudaStream_t st);
 int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int* n_contrib,
                   cudaStream_t st);

@@ -76,10 +76,10 @@ k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
     double A00 = 0.0, A01 = 0.0, A02 = 0.0, A11 = 0.0, A12 = 0.0, A22 = 0.0;
     for (int v = 0; v < V; ++v) {
       const size_t i = (size_t)v * G + g;
-      const float4 r3 = rec[i * kRecF4 + 3];
+      const float4 r3 = rec[i * kRecF4 + 3];  // (z, x_c, y_c, flags)
       const int flags = __float_as_int(r3.w);
       if (!(flags & kFlagVisible)) continue;
-      const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1], r2 = rec[i * kRecF4 + 2];
+      const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1];
       const double2* a2 = reinterpret_cast<const double2*>(acc + i * kAccN);
       const double2 a01 = a2[0], a23 = a2[1], a45 = a2[2], a67 = a2[3];
       const double qgv = eps + a01.x;
@@ -91,7 +91,7 @@ k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
       // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
       const float* vw = views + 20 * v;
       const double fx = vw[16], fy = vw[17];
-      const double x = r2.z, y = r2.w, z = r2.y;
+      const double x = r3.y, y = r3.z, z = r3.x;
       const double j00 = fx / z, j02 = -fx * x / (z * z);
       const double j11 = fy / z, j12 = -fy * y / (z * z);
       double J0[3], J1[3];
@@ -109,8 +109,15 @@ k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
       A11 += qgv * (J0[1] * J0[1] + J1[1] * J1[1]);
       A12 += qgv * (J0[1] * J0[2] + J1[1] * J1[2]);
       A22 += qgv * (J0[2] * J0[2] + J1[2] * J1[2]);
+      // view direction (mu - camera centre) / |.| = R_v^T x_c / |x_c|
       float B[16];
-      sh_poly<DEG>(r3.x, r3.y, r3.z, B);
+      {
+        const float dw0 = vw[0] * r3.y + vw[4] * r3.z + vw[8] * r3.x;
+        const float dw1 = vw[1] * r3.y + vw[5] * r3.z + vw[9] * r3.x;
+        const float dw2 = vw[2] * r3.y + vw[6] * r3.z + vw[10] * r3.x;
+        const float il = rsqrtf(dw0 * dw0 + dw1 * dw1 + dw2 * dw2);
+        sh_poly<DEG>(dw0 * il, dw1 * il, dw2 * il, B);
+      }
       const float w0 = (flags & 1) ? (float)a01.y : 0.0f;
       const float w1 = (flags & 2) ? (float)a23.x : 0.0f;
       const float w2 = (flags & 4) ? (float)a23.y : 0.0f;

@@ -29,7 +29,8 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
           const float* __restrict__ quats, const float* __restrict__ opac,
           const float* __restrict__ sh, const float* __restrict__ views_in, int G, int V, int H,
           int W, int TX, int TY, float4* __restrict__ rec, int4* __restrict__ rect,
-          int* __restrict__ counts, uint32_t* __restrict__ dkey, uint32_t* __restrict__ kbits) {
+          int* __restrict__ counts, uint32_t* __restrict__ dkey, uint32_t* __restrict__ kbits,
+          unsigned long long* __restrict__ ntot) {
   constexpr int D = (DEG + 1) * (DEG + 1);
   constexpr int NSH = D * 3;
   // shared memory: the block's SH coefficients [kProjThreads][NSH], then the views [V][20]
@@ -179,10 +180,26 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
           if (s > 0.0f) flags |= 1 << ch;
           col[ch] = fmaxf(s, 0.0f);
         }
+        // the render's early-skip bound and the half-extents of the ellipse {exponent >= cut}
+        // (bounding box of every pixel centre that can reach alpha >= 1/255), widened by
+        // 1 % + 0.05 px -- far more than fp32 rounding of the exponent (or of det Q when
+        // det Q > 1e-4 qa qc) can move its boundary; nearly singular conics get an unbounded box
+        const float cut = logf((1.0f / 255.0f) / o) - 1e-3f;
+        float ex = -1.0f, ey = -1.0f;
+        if (cut < 0.0f) {
+          const float dq = qa * qc - qb * qb;
+          if (dq > 1e-4f * (qa * qc)) {
+            const float r2c = -2.0f * cut;
+            ex = sqrtf(r2c * qc / dq) * 1.01f + 0.05f;
+            ey = sqrtf(r2c * qa / dq) * 1.01f + 0.05f;
+          } else {
+            ex = ey = __int_as_float(0x7f800000);
+          }
+        }
         r0 = make_float4(mx, my, qa, qb);
         r1 = make_float4(qc, o, col[0], col[1]);
-        r2 = make_float4(col[2], z, x, y);
-        r3 = make_float4(dx, dy, dz, __int_as_float(flags));
+        r2 = make_float4(col[2], cut, ex, ey);
+        r3 = make_float4(z, x, y, __int_as_float(flags));
         rc = make_int4(x0, y0, x1, y1);
         cnt = (x1 - x0) * (y1 - y0);
       }
@@ -202,12 +219,15 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
     const unsigned lanes = __activemask();
     const uint32_t k1 = __reduce_or_sync(lanes, cnt > 0 ? key : 0u);
     const uint32_t k0 = __reduce_or_sync(lanes, cnt > 0 ? ~key : 0u);
+    const unsigned int ntile = __reduce_add_sync(lanes, (unsigned int)cnt);
     if ((threadIdx.x & 31) == __ffs(lanes) - 1 && (k1 | k0)) {
       // one of kKeyStripes copies per view, chosen by block, keeps same-address atomics rare;
-      // the host ORs the stripes together
-      uint32_t* kb = kbits + 2 * (v * kKeyStripes + (blockIdx.x & (kKeyStripes - 1)));
+      // the host folds the stripes (OR of the key statistics, sum of the instance counts)
+      const int stripe = v * kKeyStripes + (blockIdx.x & (kKeyStripes - 1));
+      uint32_t* kb = kbits + 2 * stripe;
       atomicOr(kb, k1);
       atomicOr(kb + 1, k0);
+      atomicAdd(ntot + stripe, (unsigned long long)ntile);
     }
   }
 }
@@ -218,6 +238,8 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
                    const float* opac, const float* sh, cudaStream_t st) {
   cudaError_t e =
       cudaMemsetAsync(w.kbits, 0, (size_t)2 * kKeyStripes * w.V * sizeof(uint32_t), st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(w.ntot, 0, (size_t)kKeyStripes * w.V * sizeof(unsigned long long), st);
   if (e != cudaSuccess)
     return set_err(w, SPLAT_ERR_CUDA, std::string("key statistics clear: ") + cudaGetErrorString(e));
   if (w.G == 0) return SPLAT_OK;
@@ -233,7 +255,8 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
       return set_err(w, SPLAT_ERR_CAPACITY, "too many views for the projection kernel");        \
     k_project<DEG><<<blocks, kProjThreads, smem, st>>>(means, lsc, quats, opac, sh, w.views,     \
                                                        w.G, w.V, w.H, w.W, w.TX, w.TY, w.rec,    \
-                                                       w.rect, w.counts, w.dkey, w.kbits);       \
+                                                       w.rect, w.counts, w.dkey, w.kbits,        \
+                                                       w.ntot);                                  \
   }
   switch (w.deg) {
     case 0: SPLAT_PROJ(0); break;

@@ -17,9 +17,9 @@
 // every staged entry the loader computes cut = log((1/255) / o) - 1e-3; an exponent below cut
 // gives o exp(pw) < (1/255) exp(-1e-3), far below 1/255 even after the few-ulp errors of the
 // exp and of the product, so the entry is skipped without evaluating exp -- the same decision the
-// full evaluation takes, never a different one. The loader also computes, per entry, which of the
-// CTA's eight warps (two pixel rows each) the ellipse {exponent >= cut} can reach at all; the
-// other warps skip the entry with one warp-uniform test.
+// full evaluation takes, never a different one. The projection stores cut and the half-extents of
+// the ellipse {exponent >= cut} with every record; a warp (two pixel rows) only evaluates the
+// entries whose box reaches its rows.
 //
 // Replay arithmetic. The suffix numerators C_hat - P - T alpha c are formed per channel exactly
 // as the recovery equation writes them (their cancellation dominates the fp32 error of C+), then
@@ -46,33 +46,18 @@ struct Entry {
   float alpha, dx, dy;
 };
 
-// exponent cut below which alpha < 1/255 is certain (see the file comment)
-__device__ __forceinline__ float skip_cut(float o) { return logf(kAlphaMin / o) - 1e-3f; }
-
-// Warps of the CTA (warp w holds pixel rows 2w, 2w + 1 of the tile) whose pixel centres can reach
-// the entry's exponent >= cut ellipse {d : d^T Q d <= -2 cut}. Its half-extents are
-// sqrt(-2 cut (Q^-1)_xx) and sqrt(-2 cut (Q^-1)_yy), widened by 1 % + 0.05 px: far more than the
-// fp32 evaluation of the exponent (or of det Q when det Q > 1e-4 qa qc) can move the boundary.
-// Nearly singular conics get every warp. Warps outside the box would only skip the entry, so
+// Can the entry's ellipse {exponent >= cut} (centre A.xy, half-extents ex, ey precomputed by the
+// projection, conservatively widened) reach a pixel centre of the warp's strip: columns
+// x0 + 0.5 .. x0 + 15.5, rows y0 + 0.5 .. y0 + 1.5? Entries outside would only be skipped, so
 // leaving them out changes no decision.
-__device__ __forceinline__ uint32_t strip_mask(float4 A, float qc, float cut, float x0f,
-                                               float y0f) {
-  if (!(cut < 0.0f)) return 0u;
-  const float det = A.z * qc - A.w * A.w;
-  if (!(det > 1e-4f * (A.z * qc))) return 0xffu;
-  const float r2 = -2.0f * cut;
-  const float ex = sqrtf(r2 * qc / det) * 1.01f + 0.05f;
-  const float ey = sqrtf(r2 * A.z / det) * 1.01f + 0.05f;
-  // pixel centres of the tile: x0f + 0.5 .. x0f + 15.5, rows y0f + 0.5 + r, r = 0 .. 15
-  if (A.x + ex < x0f + 0.5f || A.x - ex > x0f + 15.5f) return 0u;
-  const float lo = A.y - ey - (y0f + 0.5f), hi = A.y + ey - (y0f + 0.5f);
-  if (hi < 0.0f || lo > 15.0f) return 0u;
-  const int r0 = lo <= 0.0f ? 0 : (int)ceilf(lo);
-  const int r1 = hi >= 15.0f ? 15 : (int)floorf(hi);
-  if (r1 < r0) return 0u;
-  const int w0 = r0 >> 1, w1 = r1 >> 1;
-  return ((2u << w1) - 1u) & ~((1u << w0) - 1u);
+__device__ __forceinline__ bool reaches_strip(float4 A, float ex, float ey, float x0, float y0) {
+  return A.x + ex >= x0 + 0.5f && A.x - ex <= x0 + 15.5f && A.y + ey >= y0 + 0.5f &&
+         A.y - ey <= y0 + 1.5f;
 }
+
+// position of the composited-entry mask of (global tile gt, chunk starting at list position p):
+// distinct for every chunk of every tile, at most N / 32 + V * nt
+__device__ __forceinline__ long long chunk_index(long long p, int gt) { return (p >> 5) + gt; }
 
 // alpha of one list entry at pixel centre (px, py), with the rasteriser's skip rules
 __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
@@ -98,23 +83,25 @@ __global__ void __launch_bounds__(kThreads)
 k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
          const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
          const float* __restrict__ bgp, float* __restrict__ img, float* __restrict__ Tout,
-         int* __restrict__ ncout, int* __restrict__ last) {
+         int* __restrict__ ncout, int* __restrict__ last, uint32_t* __restrict__ umask) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
   const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const long long e = tile_off[(size_t)v * (nt + 1) + t + 1];
+  const int gt = v * nt + t;
   // Each warp walks the whole list on its own (no CTA barriers): it stages 32 entries into its
   // slice of shared memory, ballots which of them can reach its two pixel rows, evaluates only
-  // those, and leaves as soon as its 32 pixels are done.
+  // those, and leaves as soon as its 32 pixels are done. Per 32-entry chunk it records which
+  // entries some pixel of the warp composited: the replay visits exactly those.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];  // (colour b, exponent cut)
   float4* wa = s_a + warp * 32;
   float4* wb = s_b + warp * 32;
   float2* wc = s_c + warp * 32;
-  const float x0f = (float)(tx * kTile), y0f = (float)(ty * kTile);
+  const float x0f = (float)(tx * kTile), y0f = (float)(ty * kTile + 2 * warp);
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int n = 0, lst = 0;
@@ -126,38 +113,44 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     bool hit = false;
     if (k < e) {
       const float4* r = recv + (size_t)ids[k] * kRecF4;
-      const float4 a = r[0], b = r[1];
-      const float cut = skip_cut(b.y);
+      const float4 a = r[0], b = r[1], c = r[2];  // c = (colour b, cut, ex, ey)
       wa[lane] = a;
       wb[lane] = b;
-      wc[lane] = make_float2(r[2].x, cut);
-      hit = (strip_mask(a, b.x, cut, x0f, y0f) >> warp) & 1u;
+      wc[lane] = make_float2(c.x, c.y);
+      hit = reaches_strip(a, c.z, c.w, x0f, y0f);
     }
     uint32_t bits = __ballot_sync(0xffffffffu, hit);
+    uint32_t ubits = 0u;
     __syncwarp();
     while (bits) {  // warp-uniform: entries that can reach this warp's rows, in list order
       const int q = __ffs(bits) - 1;
       bits &= bits - 1;
-      if (done) continue;
-      const float4 A = wa[q], Bq = wb[q];
-      const float2 Cq = wc[q];
-      const Entry E = eval_entry(A, Bq, Cq.y, px, py);
-      if (!E.use) continue;
-      const float Tn = T * (1.0f - E.alpha);
-      if (Tn < 1e-4f) {
-        done = true;
-        continue;
+      bool comp = false;
+      if (!done) {
+        const float4 A = wa[q], Bq = wb[q];
+        const float2 Cq = wc[q];
+        const Entry E = eval_entry(A, Bq, Cq.y, px, py);
+        if (E.use) {
+          const float Tn = T * (1.0f - E.alpha);
+          if (Tn < 1e-4f) {
+            done = true;
+          } else {
+            const float wgt = E.alpha * T;
+            // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is
+            // then exactly the background term, and the suffix recovery sees no rounding mismatch
+            C0 = C0 + wgt * Bq.z;
+            C1 = C1 + wgt * Bq.w;
+            C2 = C2 + wgt * Cq.x;
+            T = Tn;
+            ++n;
+            lst = (int)(base - s) + q + 1;
+            comp = true;
+          }
+        }
       }
-      const float wgt = E.alpha * T;
-      // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is then
-      // exactly the background term, and the suffix recovery sees no rounding mismatch
-      C0 = C0 + wgt * Bq.z;
-      C1 = C1 + wgt * Bq.w;
-      C2 = C2 + wgt * Cq.x;
-      T = Tn;
-      ++n;
-      lst = (int)(base - s) + q + 1;
+      if (__any_sync(0xffffffffu, comp)) ubits |= 1u << q;
     }
+    if (lane == 0) umask[chunk_index(base, gt) * 8 + warp] = ubits;
     __syncwarp();
   }
   if (inside) {
@@ -187,15 +180,18 @@ __global__ void __launch_bounds__(kThreads)
 k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
          const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
          const float* __restrict__ img, const float* __restrict__ obs,
-         const int* __restrict__ last, double* __restrict__ acc) {
+         const int* __restrict__ last, const uint32_t* __restrict__ umask,
+         double* __restrict__ acc) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
   const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
-  // Like the render, each warp walks the list on its own: 32-entry chunks staged into its slice
-  // of shared memory, a ballot of the entries that can reach its two pixel rows, no CTA barriers.
-  // Its per-entry sums go straight from the seven lanes holding them to the fp64 accumulators.
+  const int gt = v * nt + t;
+  // Like the render, each warp walks the list on its own (no CTA barriers), in 32-entry chunks;
+  // per chunk it stages and evaluates only the entries the render recorded as composited by some
+  // pixel of the warp -- every other entry contributes nothing to any of its pixels. Its
+  // per-entry sums go straight from the seven lanes holding them to the fp64 accumulators.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];
@@ -204,7 +200,6 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   float4* wb = s_b + warp * 32;
   float2* wc = s_c + warp * 32;
   uint32_t* wg = s_g + warp * 32;
-  const float x0f = (float)(tx * kTile), y0f = (float)(ty * kTile);
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   float Ch0 = 0.0f, Ch1 = 0.0f, Ch2 = 0.0f, r0 = 0.0f, r1 = 0.0f, r2 = 0.0f;
   int lst = 0;
@@ -225,22 +220,19 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
   const int slot = (lane >> 2) & 7;  // value index this lane holds after the reduction
   for (int base = 0; base < wmax; base += 32) {
-    const int k = base + lane;
-    bool hit = false;
-    if (k < wmax) {
-      const uint32_t g = ids[s + k];
+    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
+    if (!bits) continue;  // warp-uniform
+    if ((bits >> lane) & 1u) {
+      const uint32_t g = ids[s + base + lane];
       const float4* r = recv + (size_t)g * kRecF4;
-      const float4 a = r[0], b = r[1];
-      const float cut = skip_cut(b.y);
-      wa[lane] = a;
-      wb[lane] = b;
-      wc[lane] = make_float2(r[2].x, cut);
+      const float4 c = r[2];
+      wa[lane] = r[0];
+      wb[lane] = r[1];
+      wc[lane] = make_float2(c.x, c.y);
       wg[lane] = g;
-      hit = (strip_mask(a, b.x, cut, x0f, y0f) >> warp) & 1u;
     }
-    uint32_t bits = __ballot_sync(0xffffffffu, hit);
     __syncwarp();
-    while (bits) {  // warp-uniform: entries that can reach this warp's rows, in list order
+    while (bits) {  // warp-uniform: entries some pixel of this warp composited, in list order
       const int q = __ffs(bits) - 1;
       bits &= bits - 1;
       float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
@@ -310,7 +302,7 @@ int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int
   dim3 grid(w.nt, w.V);
   const int tok = prof_begin(w, st, SPLAT_K_RENDER);
   k_render<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX, w.nt, bg,
-                                      img, T_final, n_contrib, w.last);
+                                      img, T_final, n_contrib, w.last, w.umask);
   prof_end(w, st, tok);
   return check_launch(w, "render kernel");
 }
@@ -324,7 +316,7 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
   }
   dim3 grid(w.nt, w.V);
   k_replay<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX, w.nt,
-                                      w.img, obs, w.last, w.acc);
+                                      w.img, obs, w.last, w.umask, w.acc);
   prof_end(w, st, tok);
   return check_launch(w, "replay kernel");
 }

@@ -137,10 +137,11 @@ int splat_score_replay(splat_ws* ws, const float* obs, float lambda, float* toke
  * workspace state into caller-owned DEVICE buffers on `stream`, or report host-side counters.
  * ------------------------------------------------------------------------------------------- */
 
-/* Per (v, g) record, fp32 [V,G,16]: mx, my, conic a, b, c, opacity, colour r, g, b, depth z,
- * x_c, y_c, dir x, y, z, flags (int bits: bit 0..2 colour-clamp-inactive per channel, bit 8
- * visible). rect [V,G,4] int32 tile rectangle x0, y0, x1, y1 (zeros when culled). Needs
- * splat_project. */
+/* Per (v, g) record, fp32 [V,G,16]: mx, my, conic a, b, c, opacity, colour r, g, b, cut,
+ * ex, ey, depth z, x_c, y_c, flags (int bits: bit 0..2 colour-clamp-inactive per channel, bit 8
+ * visible). cut = log((1/255)/opacity) - 1e-3 bounds the exponent below which alpha < 1/255;
+ * (ex, ey) are the conservatively widened half-extents of the ellipse where it is not.
+ * rect [V,G,4] int32 tile rectangle x0, y0, x1, y1 (zeros when culled). Needs splat_project. */
 int splat_copy_projection(splat_ws* ws, float* rec, int* rect, void* stream);
 
 /* Tile lists after splat_bin_sort: tile_offsets [V, n_t + 1] int64 (global positions, view-major,
@@ -165,7 +166,7 @@ long long splat_launch_count(const splat_ws* ws);
  * group id (0 .. SPLAT_NUM_KERNELS-1), the elapsed milliseconds and the number of timed launches
  * since the last reset (reset != 0 clears after reading). Off by default. */
 enum {
-  SPLAT_K_PROJECT = 0, SPLAT_K_SCAN_COUNTS, SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER,
+  SPLAT_K_PROJECT = 0, SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER,
   SPLAT_K_EMIT, SPLAT_K_TILE_HIST, SPLAT_K_HIST_SCAN, SPLAT_K_TILE_SCATTER, SPLAT_K_TILE_RANGES,
   SPLAT_K_RENDER, SPLAT_K_REPLAY, SPLAT_K_FINALIZE, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
 };

@@ -57,7 +57,8 @@ def compare_projection(scene, g, p):
     assert (valid_g == (p["valid"] == 1)).all(), "visibility differs"
     v = valid_g
     gr, orr = g["rec"][v].astype(np.float64), p["rec"][v]
-    pairs = [(0, 0), (1, 1), (2, 2), (3, 3), (4, 4), (5, 6), (9, 5), (10, 10), (11, 11)]
+    # GPU record: mx my a b c o cr cg cb cut ex ey z xc yc flags
+    pairs = [(0, 0), (1, 1), (2, 2), (3, 3), (4, 4), (5, 6), (12, 5), (13, 10), (14, 11)]
     for gi, oi in pairs:
         bad = gr[:, gi] != orr[:, oi]
         assert not bad.any(), f"record field {gi} differs in {bad.sum()} places"

@@ -48,7 +48,7 @@ def _one_tile_lists(seed, G):
     ws.copy_tile_lists(off, ids)
     torch.cuda.synchronize()
     ws.close()
-    return rec[0, :, 9].clone(), ids[:n].clone()  # camera depth z per Gaussian, the tile list
+    return rec[0, :, 12].clone(), ids[:n].clone()  # camera depth z per Gaussian, the tile list
 
 
 @pytest.mark.parametrize("G", [3000, 20000])
