@@ -129,6 +129,27 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture (profiles/dram_traffic.json), only
+    when the kernel's sources still hash to what was captured and the workload matches."""
+    import hashlib
+    try:
+        d = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))["kernels"][kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if d.get("workload") != workload:
+        return None
+    m = hashlib.sha256()
+    for f in d["sources"]:
+        try:
+            m.update(open(os.path.join(ROOT, f), "rb").read())
+        except OSError:
+            return None
+    if m.hexdigest() != d["sha256"]:
+        return None
+    return int(d["dram_read_bytes"]) + int(d["dram_write_bytes"])
+
+
 def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
     """Bytes each kernel group must move by its definition (unique inputs + outputs)."""
     G, V, H, W, d = sc.G, sc.V, sc.H, sc.W, sc.d
@@ -341,43 +362,72 @@ def main():
     pairs_per_s = pairs * args.steps * world / (total_ms * 1e-3)
 
     # ---- end to end through the public API with host buffers ----------------------------------
+    # Every step copies its inputs from pinned host memory and its outputs (tokens, image, final
+    # transmittance, contributor counts) back, all inside the timed region. The steps are
+    # pipelined with double-buffered device inputs/outputs: step k+1's host->device copy and step
+    # k-1's device->host copy run on two copy streams while step k computes.
     e2e = None
     if not args.no_e2e:
+        names = ("means", "log_scales", "quats", "opac", "sh", "viewmats", "intrin", "bg")
         host = {k: torch.from_numpy(np.ascontiguousarray(getattr(sc, k))).pin_memory()
-                for k in ("means", "log_scales", "quats", "opac", "sh", "viewmats", "intrin",
-                          "bg")}
+                for k in names}
         host["obs"] = obs.cpu().pin_memory()
-        dev_in = {"means": ds.means, "log_scales": ds.log_scales, "quats": ds.quats,
-                  "opac": ds.opac, "sh": ds.sh, "viewmats": ds.viewmats, "intrin": ds.intrin,
-                  "bg": ds.bg, "obs": obs}
-        h_out = {"tokens": torch.empty(out.tokens.shape, dtype=torch.float32).pin_memory(),
-                 "img": torch.empty(out.img.shape, dtype=torch.float32).pin_memory(),
-                 "T": torch.empty(out.T.shape, dtype=torch.float32).pin_memory(),
-                 "n_contrib": torch.empty(out.n_contrib.shape, dtype=torch.int32).pin_memory()}
+        dsets = [ds, runner.DeviceScene(*[getattr(ds, k).clone() for k in names], ds.H, ds.W)]
+        dobs = [obs, obs.clone()]
+        outs = [out, runner.alloc_outputs(ds)]
+
+        def h_outputs():
+            return {"tokens": torch.empty(out.tokens.shape, dtype=torch.float32).pin_memory(),
+                    "img": torch.empty(out.img.shape, dtype=torch.float32).pin_memory(),
+                    "T": torch.empty(out.T.shape, dtype=torch.float32).pin_memory(),
+                    "n_contrib": torch.empty(out.n_contrib.shape, dtype=torch.int32).pin_memory()}
+        h_out = [h_outputs(), h_outputs()]
         h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
-        e2e_ms = []
+        d2h = sum(t.numel() * t.element_size() for t in h_out[0].values())
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
+        in_ready, comp_done, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+        def enqueue_h2d(b):
+            with torch.cuda.stream(s_in):
+                for k in names:
+                    getattr(dsets[b], k).copy_(host[k], non_blocking=True)
+                dobs[b].copy_(host["obs"], non_blocking=True)
+                in_ready[b].record(s_in)
+
         barrier(world)
-        for _ in range(args.steps):
-            l2_flush.zero_()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for k, t in host.items():
-                dev_in[k].copy_(t, non_blocking=True)
-            step()
-            h_out["tokens"].copy_(out.tokens, non_blocking=True)
-            h_out["img"].copy_(out.img, non_blocking=True)
-            h_out["T"].copy_(out.T, non_blocking=True)
-            h_out["n_contrib"].copy_(out.n_contrib, non_blocking=True)
-            e1.record(stream)
-            e1.synchronize()
-            e2e_ms.append(e0.elapsed_time(e1))
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        s_in.wait_event(t0)
+        s_out.wait_event(t0)
+        enqueue_h2d(0)
+        for k in range(args.steps):
+            b = k & 1
+            if k + 1 < args.steps:
+                if k >= 1:
+                    s_in.wait_event(comp_done[1 - b])  # step k-1 has read that input set
+                enqueue_h2d(1 - b)
+            stream.wait_event(in_ready[b])
+            if k >= 2:
+                stream.wait_event(out_free[b])  # step k-2's outputs have been copied out
+            runner.render_and_score(ws, dsets[b], dobs[b], outs[b])
+            comp_done[b].record(stream)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                h_out[b]["tokens"].copy_(outs[b].tokens, non_blocking=True)
+                h_out[b]["img"].copy_(outs[b].img, non_blocking=True)
+                h_out[b]["T"].copy_(outs[b].T, non_blocking=True)
+                h_out[b]["n_contrib"].copy_(outs[b].n_contrib, non_blocking=True)
+                out_free[b].record(s_out)
+        t1.record(s_out)
+        t1.synchronize()
         barrier(world)
-        e2e_total = max_over_ranks(sum(e2e_ms), world)
+        e2e_total = max_over_ranks(t0.elapsed_time(t1), world)
         e2e = {"value": px_step * args.steps * world / (e2e_total * 1e-3) / 1e6,
                "unit": "Mpix/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e2e_total / args.steps}
+               "ms_per_step": e2e_total / args.steps, "pipelined": True}
+        del dsets, dobs, outs, h_out
 
     # ---- roofline of the dominant kernel ------------------------------------------------------
     peaks = load_peaks()
@@ -392,13 +442,15 @@ def main():
         achieved = ops / (dom_ms * 1e-3) / 1e12
         peak = lanes * peaks["sm_max_mhz"] * 1e6 / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
-                "unit": "Tops/s (fp32 pipe)", "frac": achieved / peak, "traffic": None,
+                "unit": "Tops/s (fp32 pipe)", "frac": achieved / peak,
+                "traffic": recorded_traffic(dom, WORKLOADS[args.config]),
                 "peak_source": f"{lanes} fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz "
                                f"({peaks['source']} max clock)"}
     else:
         achieved = ab.get(dom, 0) / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": recorded_traffic(dom, WORKLOADS[args.config]),
                 "peak_source": f"{peaks['source']} copy bandwidth"}
     for k, v in per_kernel.items():
         if k in ab:
