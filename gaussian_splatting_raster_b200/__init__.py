@@ -12,7 +12,8 @@ import os
 
 from .build import LIB, build  # noqa: F401
 
-__all__ = ["Workspace", "SplatError", "load_library", "LIB", "build", "token_dim"]
+__all__ = ["Workspace", "SplatError", "load_library", "LIB", "build", "token_dim",
+           "partials_dim", "finalize_partials"]
 
 _ERRORS = {
     -1: "INVALID_ARG", -2: "CAPACITY", -3: "STATE", -4: "CUDA", -5: "BOUNDS",
@@ -25,7 +26,7 @@ EXPORTS = [
     "splat_bin_sort", "splat_render", "splat_score_replay", "splat_copy_projection",
     "splat_copy_tile_lists", "splat_copy_last", "splat_copy_accumulators", "splat_pair_count",
     "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
-    "splat_sort_depths_noalloc",
+    "splat_sort_depths_noalloc", "splat_score_partials", "splat_finalize_partials",
 ]
 
 
@@ -83,6 +84,10 @@ def load_library(path: str | None = None):
     L.splat_profile_read.restype = I
     L.splat_kernel_name.argtypes = [I]
     L.splat_kernel_name.restype = ctypes.c_char_p
+    L.splat_score_partials.argtypes = [V, V, V, V]
+    L.splat_score_partials.restype = I
+    L.splat_finalize_partials.argtypes = [V, I, I, F, V, V]
+    L.splat_finalize_partials.restype = I
     if path is None:
         _lib = L
     return L
@@ -90,6 +95,22 @@ def load_library(path: str | None = None):
 
 def token_dim(sh_degree: int) -> int:
     return 9 + 3 * (sh_degree + 1) ** 2
+
+
+def partials_dim(sh_degree: int) -> int:
+    return 11 + 3 * (sh_degree + 1) ** 2
+
+
+def finalize_partials(partials, sh_degree: int, tokens, lam: float = 1.0, stream=None):
+    """Tokens [n, 9 + 3d] from summed per-Gaussian partials [n, 11 + 3d] (any slice of rows)."""
+    import torch
+    n = partials.shape[0]
+    rc = load_library().splat_finalize_partials(
+        _ptr(partials, "partials", torch.float32, (n, partials_dim(sh_degree))), n, sh_degree,
+        ctypes.c_float(lam), _ptr(tokens, "tokens", torch.float32, (n, token_dim(sh_degree))),
+        _stream(stream))
+    if rc != 0:
+        raise SplatError(rc, "finalize from partials failed")
 
 
 def _stream(stream):
@@ -181,6 +202,15 @@ class Workspace:
         self._check(self._L.splat_score_replay(
             self._h, _ptr(obs, "obs", torch.float32, (V, H, W, 3)), ctypes.c_float(lam),
             _ptr(tokens, "tokens", torch.float32, (self.G, token_dim(self.deg))),
+            _stream(stream)))
+
+    def score_partials(self, obs, partials, stream=None):
+        """Replay of this workspace's views; per-Gaussian sums [G, 11 + 3d] instead of tokens."""
+        import torch
+        V, H, W = self.V, self.H, self.W
+        self._check(self._L.splat_score_partials(
+            self._h, _ptr(obs, "obs", torch.float32, (V, H, W, 3)),
+            _ptr(partials, "partials", torch.float32, (self.G, partials_dim(self.deg))),
             _stream(stream)))
 
     # -- inspection -----------------------------------------------------------------------------

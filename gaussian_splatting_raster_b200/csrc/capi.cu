@@ -284,6 +284,33 @@ int splat_score_replay(splat_ws* ws, const float* obs, float lambda, float* toke
   return SPLAT_OK;
 }
 
+int splat_score_partials(splat_ws* ws, const float* obs, float* partials, void* stream) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  Workspace& w = ws->w;
+  w.err.clear();
+  if (w.stage < 3) return fail(w, SPLAT_ERR_STATE, "splat_score_partials before splat_render");
+  int rc;
+  if ((rc = check_dev_ptr(w, obs, "obs"))) return rc;
+  if ((rc = check_dev_ptr(w, partials, "partials", w.G == 0))) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((rc = splat::launch_replay(w, obs, st))) return rc;
+  if ((rc = splat::launch_partials(w, partials, st))) return rc;
+  w.stage = 4;
+  return SPLAT_OK;
+}
+
+int splat_finalize_partials(const float* partials, int G, int sh_degree, float lambda,
+                            float* tokens, void* stream) {
+  if (G < 0 || sh_degree < 0 || sh_degree > 3 || !(lambda >= 0.0f) || !std::isfinite(lambda))
+    return SPLAT_ERR_INVALID_ARG;
+  if (G == 0) return SPLAT_OK;
+  if (!partials || !tokens || (((uintptr_t)partials | (uintptr_t)tokens) & 3u))
+    return SPLAT_ERR_INVALID_ARG;
+  cudaError_t e = splat::launch_finalize_partials(partials, G, sh_degree, (double)lambda, tokens,
+                                                  (cudaStream_t)stream);
+  return e == cudaSuccess ? SPLAT_OK : SPLAT_ERR_CUDA;
+}
+
 // ----------------------------------------------------------------------------------------------
 int splat_copy_projection(splat_ws* ws, float* rec, int* rect, void* stream) {
   if (!ws) return SPLAT_ERR_INVALID_ARG;

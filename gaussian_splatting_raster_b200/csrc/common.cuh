@@ -227,6 +227,9 @@ int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int
                   cudaStream_t st);
 int launch_replay(Workspace& w, const float* obs, cudaStream_t st);
 int launch_finalize(Workspace& w, float lambda, float* tokens, cudaStream_t st);
+int launch_partials(Workspace& w, float* partials, cudaStream_t st);
+cudaError_t launch_finalize_partials(const float* partials, int G, int deg, double lambda,
+                                     float* tokens, cudaStream_t st);
 int launch_pair_count(Workspace& w, cudaStream_t st);
 int binning_configure(Workspace& w);
 

@@ -55,6 +55,116 @@ __device__ void eig3_sym(double a00, double a01, double a02, double a11, double 
   if (ev[1] > ev[0]) { const double tt = ev[0]; ev[0] = ev[1]; ev[1] = tt; }
 }
 
+// Per-Gaussian sums over the views where g is visible, all linear in the per-view terms (so the
+// sums of disjoint view sets add): qsum = sum_v q_gv, b = sum_v J^T Sigma^-1 Sd,
+// sa = sum_v (1 - o) Sa, A = sum_v q_gv J^T J (6 entries) in registers (double); the SH block
+// sum_v M_color (Swr (x) B) is added into the shared-memory column `col` (stride P) at 4 + k.
+template <int DEG, int P>
+__device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
+                                          const double* __restrict__ acc,
+                                          const float* __restrict__ views, int G, int V, int g,
+                                          double& qsum, double b[3], double& sa, double A[6],
+                                          float* col) {
+  constexpr int D = (DEG + 1) * (DEG + 1);
+  const double eps = 1e-6;
+  for (int v = 0; v < V; ++v) {
+    const size_t i = (size_t)v * G + g;
+    const float4 r3 = rec[i * kRecF4 + 3];  // (z, x_c, y_c, flags)
+    const int flags = __float_as_int(r3.w);
+    if (!(flags & kFlagVisible)) continue;
+    const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1];
+    const double2* a2 = reinterpret_cast<const double2*>(acc + i * kAccN);
+    const double2 a01 = a2[0], a23 = a2[1], a45 = a2[2], a67 = a2[3];
+    const double qgv = eps + a01.x;
+    qsum += qgv;
+    sa += (1.0 - (double)r1.y) * a45.x;
+    const double qa = r0.z, qb = r0.w, qc = r1.x;
+    const double sm0 = qa * a45.y + qb * a67.x;
+    const double sm1 = qb * a45.y + qc * a67.x;
+    // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
+    const float* vw = views + 20 * v;
+    const double fx = vw[16], fy = vw[17];
+    const double x = r3.y, y = r3.z, z = r3.x;
+    const double j00 = fx / z, j02 = -fx * x / (z * z);
+    const double j11 = fy / z, j12 = -fy * y / (z * z);
+    double J0[3], J1[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      J0[c] = j00 * (double)vw[c] + j02 * (double)vw[8 + c];
+      J1[c] = j11 * (double)vw[4 + c] + j12 * (double)vw[8 + c];
+    }
+    b[0] += J0[0] * sm0 + J1[0] * sm1;
+    b[1] += J0[1] * sm0 + J1[1] * sm1;
+    b[2] += J0[2] * sm0 + J1[2] * sm1;
+    A[0] += qgv * (J0[0] * J0[0] + J1[0] * J1[0]);
+    A[1] += qgv * (J0[0] * J0[1] + J1[0] * J1[1]);
+    A[2] += qgv * (J0[0] * J0[2] + J1[0] * J1[2]);
+    A[3] += qgv * (J0[1] * J0[1] + J1[1] * J1[1]);
+    A[4] += qgv * (J0[1] * J0[2] + J1[1] * J1[2]);
+    A[5] += qgv * (J0[2] * J0[2] + J1[2] * J1[2]);
+    // view direction (mu - camera centre) / |.| = R_v^T x_c / |x_c|
+    float B[16];
+    {
+      const float dw0 = vw[0] * r3.y + vw[4] * r3.z + vw[8] * r3.x;
+      const float dw1 = vw[1] * r3.y + vw[5] * r3.z + vw[9] * r3.x;
+      const float dw2 = vw[2] * r3.y + vw[6] * r3.z + vw[10] * r3.x;
+      const float il = rsqrtf(dw0 * dw0 + dw1 * dw1 + dw2 * dw2);
+      sh_poly<DEG>(dw0 * il, dw1 * il, dw2 * il, B);
+    }
+    const float w0 = (flags & 1) ? (float)a01.y : 0.0f;
+    const float w1 = (flags & 2) ? (float)a23.x : 0.0f;
+    const float w2 = (flags & 4) ? (float)a23.y : 0.0f;
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+      col[(4 + 3 * k) * P] += B[k] * w0;
+      col[(5 + 3 * k) * P] += B[k] * w1;
+      col[(6 + 3 * k) * P] += B[k] * w2;
+    }
+  }
+}
+
+// token from the sums: q_g = eps + qsum, everything divided once by q_g (gamma_gv / q_gv = 1/q_g),
+// A = lambda I + (sum q_gv J^T J) / q_g, conditioning statistics of A. Writes columns 0..DT-1 of
+// `col`; the SH block must already sit in columns 4 .. 4 + 3d - 1 (it is scaled in place).
+template <int DEG, int P>
+__device__ __forceinline__ void finish_token(double qsum, const double b[3], double sa,
+                                             const double An[6], double lambda, float* col) {
+  constexpr int D = (DEG + 1) * (DEG + 1);
+  const double eps = 1e-6;
+  const double qg = eps + qsum;
+  const double inv = 1.0 / qg;
+  const double A00 = An[0] * inv + lambda, A11 = An[3] * inv + lambda, A22 = An[5] * inv + lambda;
+  const double A01 = An[1] * inv, A02 = An[2] * inv, A12 = An[4] * inv;
+  double ev[3];
+  eig3_sym(A00, A01, A02, A11, A12, A22, ev);
+  const double tr = A00 + A11 + A22;
+  col[0 * P] = (float)(b[0] * inv);
+  col[1 * P] = (float)(b[1] * inv);
+  col[2 * P] = (float)(b[2] * inv);
+  col[3 * P] = (float)(sa * inv);
+#pragma unroll
+  for (int k = 0; k < 3 * D; ++k) col[(4 + k) * P] = (float)((double)col[(4 + k) * P] * inv);
+  col[(4 + 3 * D) * P] = (float)log(qg);
+  const double itr = 1.0 / (tr + eps);
+  col[(5 + 3 * D) * P] = (float)(ev[0] * itr);
+  col[(6 + 3 * D) * P] = (float)(ev[1] * itr);
+  col[(7 + 3 * D) * P] = (float)(ev[2] * itr);
+  col[(8 + 3 * D) * P] = (float)log(tr + eps);
+}
+
+// the block's rows (ncols each) are contiguous in the output: coalesced stores from the tile
+template <int P>
+__device__ __forceinline__ void store_rows(const float* s_tile, int ncols, int g0, int G,
+                                           float* out_rows) {
+  const int ng = min(kFinThreads, G - g0);
+  float* out = out_rows + (size_t)g0 * ncols;
+  for (int L = threadIdx.x; L < ng * ncols; L += kFinThreads) {
+    const int row = L / ncols, c = L - row * ncols;
+    out[L] = s_tile[c * P + row];
+  }
+}
+
+// fused single-device path: sums over all views, then the token
 template <int DEG>
 __global__ void __launch_bounds__(kFinThreads, 4)
 k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
@@ -71,95 +181,85 @@ k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
 #pragma unroll
   for (int k = 0; k < 3 * D; ++k) col[(4 + k) * P] = 0.0f;
   if (g < G) {
-    const double eps = 1e-6;
-    double qsum = 0.0, b0 = 0.0, b1 = 0.0, b2 = 0.0, sa = 0.0;
-    double A00 = 0.0, A01 = 0.0, A02 = 0.0, A11 = 0.0, A12 = 0.0, A22 = 0.0;
-    for (int v = 0; v < V; ++v) {
-      const size_t i = (size_t)v * G + g;
-      const float4 r3 = rec[i * kRecF4 + 3];  // (z, x_c, y_c, flags)
-      const int flags = __float_as_int(r3.w);
-      if (!(flags & kFlagVisible)) continue;
-      const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1];
-      const double2* a2 = reinterpret_cast<const double2*>(acc + i * kAccN);
-      const double2 a01 = a2[0], a23 = a2[1], a45 = a2[2], a67 = a2[3];
-      const double qgv = eps + a01.x;
-      qsum += qgv;
-      sa += (1.0 - (double)r1.y) * a45.x;
-      const double qa = r0.z, qb = r0.w, qc = r1.x;
-      const double sm0 = qa * a45.y + qb * a67.x;
-      const double sm1 = qb * a45.y + qc * a67.x;
-      // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
-      const float* vw = views + 20 * v;
-      const double fx = vw[16], fy = vw[17];
-      const double x = r3.y, y = r3.z, z = r3.x;
-      const double j00 = fx / z, j02 = -fx * x / (z * z);
-      const double j11 = fy / z, j12 = -fy * y / (z * z);
-      double J0[3], J1[3];
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        J0[c] = j00 * (double)vw[c] + j02 * (double)vw[8 + c];
-        J1[c] = j11 * (double)vw[4 + c] + j12 * (double)vw[8 + c];
-      }
-      b0 += J0[0] * sm0 + J1[0] * sm1;
-      b1 += J0[1] * sm0 + J1[1] * sm1;
-      b2 += J0[2] * sm0 + J1[2] * sm1;
-      A00 += qgv * (J0[0] * J0[0] + J1[0] * J1[0]);
-      A01 += qgv * (J0[0] * J0[1] + J1[0] * J1[1]);
-      A02 += qgv * (J0[0] * J0[2] + J1[0] * J1[2]);
-      A11 += qgv * (J0[1] * J0[1] + J1[1] * J1[1]);
-      A12 += qgv * (J0[1] * J0[2] + J1[1] * J1[2]);
-      A22 += qgv * (J0[2] * J0[2] + J1[2] * J1[2]);
-      // view direction (mu - camera centre) / |.| = R_v^T x_c / |x_c|
-      float B[16];
-      {
-        const float dw0 = vw[0] * r3.y + vw[4] * r3.z + vw[8] * r3.x;
-        const float dw1 = vw[1] * r3.y + vw[5] * r3.z + vw[9] * r3.x;
-        const float dw2 = vw[2] * r3.y + vw[6] * r3.z + vw[10] * r3.x;
-        const float il = rsqrtf(dw0 * dw0 + dw1 * dw1 + dw2 * dw2);
-        sh_poly<DEG>(dw0 * il, dw1 * il, dw2 * il, B);
-      }
-      const float w0 = (flags & 1) ? (float)a01.y : 0.0f;
-      const float w1 = (flags & 2) ? (float)a23.x : 0.0f;
-      const float w2 = (flags & 4) ? (float)a23.y : 0.0f;
-#pragma unroll
-      for (int k = 0; k < D; ++k) {
-        col[(4 + 3 * k) * P] += B[k] * w0;
-        col[(5 + 3 * k) * P] += B[k] * w1;
-        col[(6 + 3 * k) * P] += B[k] * w2;
-      }
-    }
-    const double qg = eps + qsum;
-    const double inv = 1.0 / qg;
-    A00 = A00 * inv + lambda;
-    A11 = A11 * inv + lambda;
-    A22 = A22 * inv + lambda;
-    A01 *= inv;
-    A02 *= inv;
-    A12 *= inv;
-    double ev[3];
-    eig3_sym(A00, A01, A02, A11, A12, A22, ev);
-    const double tr = A00 + A11 + A22;
-    col[0 * P] = (float)(b0 * inv);
-    col[1 * P] = (float)(b1 * inv);
-    col[2 * P] = (float)(b2 * inv);
-    col[3 * P] = (float)(sa * inv);
-#pragma unroll
-    for (int k = 0; k < 3 * D; ++k) col[(4 + k) * P] = (float)((double)col[(4 + k) * P] * inv);
-    col[(4 + 3 * D) * P] = (float)log(qg);
-    const double itr = 1.0 / (tr + eps);
-    col[(5 + 3 * D) * P] = (float)(ev[0] * itr);
-    col[(6 + 3 * D) * P] = (float)(ev[1] * itr);
-    col[(7 + 3 * D) * P] = (float)(ev[2] * itr);
-    col[(8 + 3 * D) * P] = (float)log(tr + eps);
+    double qsum = 0.0, sa = 0.0, b[3] = {0.0, 0.0, 0.0}, A[6] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    view_sums<DEG, P>(rec, acc, views, G, V, g, qsum, b, sa, A, col);
+    finish_token<DEG, P>(qsum, b, sa, A, lambda, col);
   }
   __syncthreads();
-  // the block's rows are contiguous in the output: coalesced stores
-  const int ng = min(kFinThreads, G - g0);
-  float* out = tokens + (size_t)g0 * DT;
-  for (int L = threadIdx.x; L < ng * DT; L += kFinThreads) {
-    const int row = L / DT, c = L - row * DT;
-    out[L] = s_tok[c * P + row];
+  store_rows<P>(s_tok, DT, g0, G, tokens);
+}
+
+// sharded path, part 1: this device's per-Gaussian partial sums over its views,
+// [qsum, b(3), sa, A(6: 00 01 02 11 12 22), SH block (3d)] = 11 + 3d floats per Gaussian
+template <int DEG>
+__global__ void __launch_bounds__(kFinThreads, 4)
+k_partials(const float4* __restrict__ rec, const double* __restrict__ acc,
+           const float* __restrict__ views, int G, int V, float* __restrict__ partials) {
+  constexpr int D = (DEG + 1) * (DEG + 1);
+  constexpr int K = 11 + 3 * D;
+  constexpr int P = kFinThreads + 1;
+  __shared__ float s_tile[K * P];
+  const int g0 = blockIdx.x * kFinThreads;
+  const int g = g0 + threadIdx.x;
+  float* col = s_tile + threadIdx.x;
+  // the SH sums are accumulated at columns 4.. (the layout view_sums writes), then moved behind
+  // the eleven scalar sums
+#pragma unroll
+  for (int k = 0; k < 3 * D; ++k) col[(4 + k) * P] = 0.0f;
+  if (g < G) {
+    double qsum = 0.0, sa = 0.0, b[3] = {0.0, 0.0, 0.0}, A[6] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    view_sums<DEG, P>(rec, acc, views, G, V, g, qsum, b, sa, A, col);
+#pragma unroll
+    for (int k = 3 * D - 1; k >= 0; --k) col[(11 + k) * P] = col[(4 + k) * P];
+    col[0] = (float)qsum;
+    col[1 * P] = (float)b[0];
+    col[2 * P] = (float)b[1];
+    col[3 * P] = (float)b[2];
+    col[4 * P] = (float)sa;
+#pragma unroll
+    for (int k = 0; k < 6; ++k) col[(5 + k) * P] = (float)A[k];
   }
+  __syncthreads();
+  store_rows<P>(s_tile, K, g0, G, partials);
+}
+
+// sharded path, part 2: tokens from (summed) partials; needs no workspace
+template <int DEG>
+__global__ void __launch_bounds__(kFinThreads, 4)
+k_finalize_partials(const float* __restrict__ partials, int G, double lambda,
+                    float* __restrict__ tokens) {
+  constexpr int D = (DEG + 1) * (DEG + 1);
+  constexpr int K = 11 + 3 * D;
+  constexpr int DT = 9 + 3 * D;
+  constexpr int P = kFinThreads + 1;
+  __shared__ float s_tile[K * P];
+  const int g0 = blockIdx.x * kFinThreads;
+  const int ng = min(kFinThreads, G - g0);
+  const float* in = partials + (size_t)g0 * K;
+  for (int L = threadIdx.x; L < ng * K; L += kFinThreads) {
+    const int row = L / K, c = L - row * K;
+    s_tile[c * P + row] = in[L];
+  }
+  __syncthreads();
+  float* col = s_tile + threadIdx.x;
+  double qsum = 0.0, sa = 0.0, b[3], A[6];
+  if (threadIdx.x < ng) {
+    qsum = col[0];
+    b[0] = col[1 * P];
+    b[1] = col[2 * P];
+    b[2] = col[3 * P];
+    sa = col[4 * P];
+#pragma unroll
+    for (int k = 0; k < 6; ++k) A[k] = col[(5 + k) * P];
+  }
+  __syncthreads();  // the token overwrites the tile's columns in place
+  if (threadIdx.x < ng) {
+#pragma unroll
+    for (int k = 0; k < 3 * D; ++k) col[(4 + k) * P] = col[(11 + k) * P];
+    finish_token<DEG, P>(qsum, b, sa, A, lambda, col);
+  }
+  __syncthreads();
+  store_rows<P>(s_tile, DT, g0, G, tokens);
 }
 
 }  // namespace
@@ -180,6 +280,36 @@ int launch_finalize(Workspace& w, float lambda, float* tokens, cudaStream_t st) 
 #undef SPLAT_FIN
   prof_end(w, st, tok);
   return check_launch(w, "finalize kernel");
+}
+
+int launch_partials(Workspace& w, float* partials, cudaStream_t st) {
+  if (w.G == 0) return SPLAT_OK;
+  const int blocks = (w.G + kFinThreads - 1) / kFinThreads;
+  const int tok = prof_begin(w, st, SPLAT_K_FINALIZE);
+#define SPLAT_PART(DEG) \
+  k_partials<DEG><<<blocks, kFinThreads, 0, st>>>(w.rec, w.acc, w.views, w.G, w.V, partials)
+  switch (w.deg) {
+    case 0: SPLAT_PART(0); break;
+    case 1: SPLAT_PART(1); break;
+    case 2: SPLAT_PART(2); break;
+    default: SPLAT_PART(3); break;
+  }
+#undef SPLAT_PART
+  prof_end(w, st, tok);
+  return check_launch(w, "partial sums kernel");
+}
+
+cudaError_t launch_finalize_partials(const float* partials, int G, int deg, double lambda,
+                                     float* tokens, cudaStream_t st) {
+  if (G == 0) return cudaSuccess;
+  const int blocks = (G + kFinThreads - 1) / kFinThreads;
+  switch (deg) {
+    case 0: k_finalize_partials<0><<<blocks, kFinThreads, 0, st>>>(partials, G, lambda, tokens); break;
+    case 1: k_finalize_partials<1><<<blocks, kFinThreads, 0, st>>>(partials, G, lambda, tokens); break;
+    case 2: k_finalize_partials<2><<<blocks, kFinThreads, 0, st>>>(partials, G, lambda, tokens); break;
+    default: k_finalize_partials<3><<<blocks, kFinThreads, 0, st>>>(partials, G, lambda, tokens); break;
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace splat

@@ -8,18 +8,21 @@
 // (o = sigmoid(a), alpha = o G, w = T alpha, rho = <r, c - C+>, q = sum w; the opacity-logit,
 // SH and projected-centre scores).
 //
-// One CTA per (tile, view), one thread per pixel of the 16x16 tile. The tile's list is walked in
-// batches of 256 entries whose records (mean, conic, opacity, colour) are staged in shared memory
-// by one gather per batch. Both passes evaluate alpha through the same device function, so the
-// replay takes exactly the render's decisions.
+// One CTA per (tile, view), one thread per pixel of the 16x16 tile; the eight warps (two pixel
+// rows each) walk the tile's list independently, with no CTA barrier: each warp stages 32-entry
+// chunks of records in its own shared-memory slice, keeps by ballot the entries whose precomputed
+// box reaches its rows, and stops when all its pixels are saturated. Both passes evaluate alpha
+// through the same device function, so the replay takes exactly the render's decisions; the
+// render also leaves, per (tile, warp, chunk), the mask of entries that composited some pixel of
+// the warp, and the replay visits only those.
 //
-// Early skip. Most (pixel, entry) pairs of a tile lie far outside the Gaussian's footprint. For
-// every staged entry the loader computes cut = log((1/255) / o) - 1e-3; an exponent below cut
+// Early skip. Most (pixel, entry) pairs of a tile lie far outside the Gaussian's footprint. The
+// projection stores with every record cut = log((1/255) / o) - 1e-3; an exponent below cut
 // gives o exp(pw) < (1/255) exp(-1e-3), far below 1/255 even after the few-ulp errors of the
 // exp and of the product, so the entry is skipped without evaluating exp -- the same decision the
-// full evaluation takes, never a different one. The projection stores cut and the half-extents of
-// the ellipse {exponent >= cut} with every record; a warp (two pixel rows) only evaluates the
-// entries whose box reaches its rows.
+// full evaluation takes, never a different one. The record also holds the half-extents of the
+// ellipse {exponent >= cut}; a warp (two pixel rows) only evaluates the entries whose box reaches
+// its rows.
 //
 // Replay arithmetic. The suffix numerators C_hat - P - T alpha c are formed per channel exactly
 // as the recovery equation writes them (their cancellation dominates the fp32 error of C+), then
@@ -27,10 +30,9 @@
 // running dot products <r, P> is algebraically the same but moves that cancellation and costs
 // ~4e-4 relative token error.) Per entry and warp the seven per-pixel terms
 // (w, w r (3), w rho, w rho (p - mu2D) (2)) are summed by a transpose-reduction (each exchange
-// step halves the values a lane carries: 9 shuffles instead of 35), the eight lanes holding a
-// result add it into a shared-memory slot of the entry, and at the end of the batch one thread per
-// entry adds the CTA's sums to the (view, Gaussian) accumulator with fp64 atomics -- seven global
-// atomics per (Gaussian, tile). The SH block never enters the pixel loop: M_color w (B (x) r)
+// step halves the values a lane carries: 9 shuffles instead of 35), and the seven lanes holding a
+// result add it to the (view, Gaussian) accumulator with one fp64 atomic each -- seven global
+// atomics per (Gaussian, warp-strip). The SH block never enters the pixel loop: M_color w (B (x) r)
 // factors into M_color B (x) (sum w r); the mean block Sigma^-1 (sum w rho d) is formed once per
 // (Gaussian, view) in finalisation.
 #include "common.cuh"

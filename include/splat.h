@@ -132,6 +132,24 @@ int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int*
 int splat_score_replay(splat_ws* ws, const float* obs, float lambda, float* tokens,
                        void* stream);
 
+/*
+ * View-sharded replay ([P1] "Exact Score Operators": every cross-view quantity of the token --
+ * q_g, the covector pullback, s^alpha, s^SH and A -- is a per-Gaussian sum over views, so the sums
+ * of disjoint view sets add). splat_score_partials runs the replay of splat_score_replay for this
+ * workspace's views and writes, instead of tokens, the per-Gaussian sums over those views:
+ *   partials [G, 11 + 3d] fp32 = [sum_v (1e-6 + q_gv), sum_v J^T Sigma2D^-1 Sd (3),
+ *                                 sum_v (1 - o) Sa, sum_v q_gv J^T J (00 01 02 11 12 22),
+ *                                 sum_v M_color (B (x) Swr) (3d, index k*3 + channel)].
+ * Devices that replay disjoint view sets of one scene add their partials (e.g. an NCCL
+ * reduce-scatter over the Gaussian axis) and call splat_finalize_partials on any slice of rows:
+ * it turns summed partials [n, 11 + 3d] into tokens [n, 9 + 3d] exactly as splat_score_replay
+ * would. splat_finalize_partials needs no workspace and allocates nothing; both are asynchronous
+ * on `stream`. On one device, partials of all views give the tokens of splat_score_replay.
+ */
+int splat_score_partials(splat_ws* ws, const float* obs, float* partials, void* stream);
+int splat_finalize_partials(const float* partials, int G, int sh_degree, float lambda,
+                            float* tokens, void* stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Inspection calls (tests and benchmarks; not part of the render/replay path). They copy
  * workspace state into caller-owned DEVICE buffers on `stream`, or report host-side counters.

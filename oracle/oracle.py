@@ -68,6 +68,8 @@ def lib():
         L.orc_bin.argtypes = [P, P, P, i32, i32, i32, i32, P, P]
         L.orc_bin.restype = i64
         L.orc_finalize.argtypes = [P, P, P, P, P, P, i32, i32, i32, f64, P]
+        L.orc_partials.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, P]
+        L.orc_finalize_partials.argtypes = [P, i32, i32, f64, P]
         _lib = L
     return _lib
 
@@ -184,6 +186,30 @@ def finalize(proj, acc, scene, lam: float = 1.0) -> np.ndarray:
     lib().orc_finalize(_p(proj["valid"]), _p(proj["rec"]), _p(proj["B"]), _p(_c(acc, np.float64)),
                        _p(_c(scene.viewmats, np.float32)), _p(_c(scene.intrin, np.float32)),
                        G, V, scene.sh_degree, float(lam), _p(tokens))
+    return tokens
+
+
+def partials(proj, acc, scene, views=None) -> np.ndarray:
+    """Per-Gaussian sums [G, 11 + 3d] over the views in `views` (all when None)."""
+    V, G = proj["valid"].shape
+    d = (scene.sh_degree + 1) ** 2
+    out = np.zeros((G, 11 + 3 * d))
+    use = None
+    if views is not None:
+        use = np.zeros(V, np.int32)
+        use[list(views)] = 1
+    lib().orc_partials(_p(proj["valid"]), _p(proj["rec"]), _p(proj["B"]), _p(_c(acc, np.float64)),
+                       _p(_c(scene.viewmats, np.float32)), _p(_c(scene.intrin, np.float32)),
+                       _p(use) if use is not None else None, G, V, scene.sh_degree, _p(out))
+    return out
+
+
+def finalize_partials(P, sh_degree: int, lam: float = 1.0) -> np.ndarray:
+    """Tokens from summed partials."""
+    P = _c(P, np.float64)
+    G = P.shape[0]
+    tokens = np.zeros((G, 9 + 3 * (sh_degree + 1) ** 2))
+    lib().orc_finalize_partials(_p(P), G, sh_degree, float(lam), _p(tokens))
     return tokens
 
 

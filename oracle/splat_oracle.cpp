@@ -756,4 +756,83 @@ int orc_finalize(const int* valid, const double* rec, const double* B, const dou
   return 0;
 }
 
+
+// Per-Gaussian sums over the views in `use_view` (null = all) for view-sharded finalisation
+// ([P1] "Exact Score Operators": gamma_gv / q_gv = 1 / q_g makes every block a sum over views
+// divided once by q_g). out [G, 11 + 3d] = [sum (eps + q_gv), sum J^T Sigma^-1 Sd (3),
+// sum (1 - o) Sa, sum q_gv J^T J (00 01 02 11 12 22), sum M_color Swr (x) B (3d)].
+int orc_partials(const int* valid, const double* rec, const double* B, const double* acc,
+                 const float* viewmats, const float* intrin, const int* use_view, int G, int V,
+                 int deg, double* out) {
+  const int d = (deg + 1) * (deg + 1);
+  const int K = 11 + 3 * d;
+  const double eps = 1e-6;
+#pragma omp parallel for schedule(static)
+  for (int g = 0; g < G; ++g) {
+    double* o = out + (long long)g * K;
+    for (int k = 0; k < K; ++k) o[k] = 0.0;
+    for (int v = 0; v < V; ++v) {
+      const long long i = (long long)v * G + g;
+      if (!valid[i] || (use_view && !use_view[v])) continue;
+      const double* a = acc + i * ACC_N;
+      const double* rc = rec + i * F_NFIELDS;
+      const double qgv = eps + a[0];
+      o[0] += qgv;
+      const double smu[2] = {rc[F_QA] * a[5] + rc[F_QB] * a[6], rc[F_QB] * a[5] + rc[F_QC] * a[6]};
+      const float* vm = viewmats + 16 * v;
+      const double fx = intrin[4 * v], fy = intrin[4 * v + 1];
+      const double x = rc[F_XC], y = rc[F_YC], z = rc[F_ZC];
+      const double Jc[2][3] = {{fx / z, 0.0, -fx * x / (z * z)}, {0.0, fy / z, -fy * y / (z * z)}};
+      double J[2][3];
+      for (int r = 0; r < 2; ++r)
+        for (int c = 0; c < 3; ++c)
+          J[r][c] = Jc[r][0] * vm[0 * 4 + c] + Jc[r][1] * vm[1 * 4 + c] + Jc[r][2] * vm[2 * 4 + c];
+      for (int c = 0; c < 3; ++c) o[1 + c] += J[0][c] * smu[0] + J[1][c] * smu[1];
+      o[4] += (1.0 - rc[F_OPAC]) * a[4];
+      const int pr[6][2] = {{0, 0}, {0, 1}, {0, 2}, {1, 1}, {1, 2}, {2, 2}};
+      for (int e = 0; e < 6; ++e) {
+        const int r = pr[e][0], c = pr[e][1];
+        o[5 + e] += qgv * (J[0][r] * J[0][c] + J[1][r] * J[1][c]);
+      }
+      const int cm = (int)rc[F_CMASK];
+      const double* Bg = B + i * NB;
+      for (int k = 0; k < d; ++k)
+        for (int ch = 0; ch < 3; ++ch)
+          if ((cm >> ch) & 1) o[11 + 3 * k + ch] += a[1 + ch] * Bg[k];
+    }
+  }
+  return 0;
+}
+
+// Tokens from summed partials: q_g = eps + sum (eps + q_gv); every block divided by q_g;
+// A = lambda I + (sum q_gv J^T J) / q_g; eigenvalues descending; same layout as orc_finalize.
+int orc_finalize_partials(const double* P, int G, int deg, double lambda, double* tokens) {
+  const int d = (deg + 1) * (deg + 1);
+  const int K = 11 + 3 * d, D = 9 + 3 * d;
+  const double eps = 1e-6;
+#pragma omp parallel for schedule(static)
+  for (int g = 0; g < G; ++g) {
+    const double* p = P + (long long)g * K;
+    double* z = tokens + (long long)g * D;
+    const double qg = eps + p[0];
+    for (int c = 0; c < 3; ++c) z[c] = p[1 + c] / qg;
+    z[3] = p[4] / qg;
+    for (int k = 0; k < 3 * d; ++k) z[4 + k] = p[11 + k] / qg;
+    double A[9];
+    const int pr[6][2] = {{0, 0}, {0, 1}, {0, 2}, {1, 1}, {1, 2}, {2, 2}};
+    for (int e = 0; e < 6; ++e) {
+      const int r = pr[e][0], c = pr[e][1];
+      A[3 * r + c] = A[3 * c + r] = p[5 + e] / qg;
+    }
+    for (int r = 0; r < 3; ++r) A[4 * r] += lambda;
+    double ev[3];
+    eig3_jacobi(A, ev);
+    const double tr = A[0] + A[4] + A[8];
+    z[4 + 3 * d] = std::log(qg);
+    for (int r = 0; r < 3; ++r) z[5 + 3 * d + r] = ev[r] / (tr + eps);
+    z[8 + 3 * d] = std::log(tr + eps);
+  }
+  return 0;
+}
+
 }  // extern "C"
