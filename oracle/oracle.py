@@ -22,6 +22,8 @@ TILE = 16
 NF = 16        # fields per (view, Gaussian) record
 NB = 16        # SH basis slots
 ACC_N = 8      # q, Swr[3], Sa, Sd[2], composited pixel count
+ACCB_N = 10    # backward sums: q, Swr[3], H, Hd[2], Hdd[3]
+GRAD_BLOCKS = dict(mean=(0, 3), log_scale=(3, 6), quat=(6, 10), opacity=(10, 11))
 F = dict(mx=0, my=1, qa=2, qb=3, qc=4, depth=5, opac=6, c0=7, c1=8, c2=9, xc=10, yc=11, zc=12,
          cmask=13, tiles=14)
 
@@ -69,6 +71,12 @@ def lib():
         L.orc_bin.restype = i64
         L.orc_finalize.argtypes = [P, P, P, P, P, P, i32, i32, i32, f64, P]
         L.orc_partials.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, P]
+        for m in "fd":
+            getattr(L, f"orc_backward_{m}").argtypes = [P, P, P, i32, i32, i32, i32, P, P, P, P,
+                                                        P, i32, P]
+        L.orc_grad_finalize.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                        P, P, P, P]
+        L.orc_sh_poly_grad.argtypes = [i32, P, i64, P, P]
         L.orc_finalize_partials.argtypes = [P, i32, i32, f64, P]
         _lib = L
     return _lib
@@ -211,6 +219,58 @@ def finalize_partials(P, sh_degree: int, lam: float = 1.0) -> np.ndarray:
     tokens = np.zeros((G, 9 + 3 * (sh_degree + 1) ** 2))
     lib().orc_finalize_partials(_p(P), G, sh_degree, float(lam), _p(tokens))
     return tokens
+
+
+def sh_poly_grad(deg: int, dirs: np.ndarray):
+    """SH basis [n, d] and its gradient [n, d, 3] by the polynomial form of the basis."""
+    dirs = _c(dirs, np.float64).reshape(-1, 3)
+    n = dirs.shape[0]
+    B, dB = np.zeros((n, NB)), np.zeros((n, NB, 3))
+    lib().orc_sh_poly_grad(deg, _p(dirs), n, _p(B), _p(dB))
+    d = (deg + 1) ** 2
+    return B[:, :d], dB[:, :d]
+
+
+def backward(proj, lists, rend, obs, bg, H, W, mode="f", sel=None) -> np.ndarray:
+    """Per-(view, Gaussian) sums of the renderer backward [V, G, 10]."""
+    V, G = proj["valid"].shape
+    TX, TY = n_tiles(H, W)
+    s, ns = _sel(sel, V, TX * TY)
+    accb = np.zeros((V, G, ACCB_N))
+    ids = lists["ids"] if lists["n"] > 0 else np.zeros(1, np.int32)
+    getattr(lib(), f"orc_backward_{mode}")(
+        _p(proj["rec"]), _p(lists["off"]), _p(ids), G, V, H, W,
+        _p(_c(rend["img"], np.float64)), _p(_c(obs, np.float32)), _p(_c(bg, np.float32)),
+        _p(_c(rend["last"], np.int32)), _p(s) if s is not None else None, ns, _p(accb))
+    return accb
+
+
+def grad_dim(sh_degree: int) -> int:
+    return 11 + 3 * (sh_degree + 1) ** 2
+
+
+def gradients(proj, accb, scene, mode="f") -> dict:
+    """raw / detached / support / pscale gradients [G, 11 + 3d] from the backward sums."""
+    V, G = proj["valid"].shape
+    K = grad_dim(scene.sh_degree)
+    out = {k: np.zeros((G, K)) for k in ("raw", "detached", "support", "pscale")}
+    lib().orc_grad_finalize(
+        _p(proj["valid"]), _p(proj["rec"]), _p(_c(accb, np.float64)),
+        _p(_c(scene.means, np.float32)), _p(_c(scene.log_scales, np.float32)),
+        _p(_c(scene.quats, np.float32)), _p(_c(scene.sh, np.float32)),
+        _p(_c(scene.viewmats, np.float32)), _p(_c(scene.intrin, np.float32)), G, V, scene.H,
+        scene.W, scene.sh_degree, 1 if mode == "f" else 0, _p(out["raw"]), _p(out["detached"]),
+        _p(out["support"]), _p(out["pscale"]))
+    return out
+
+
+def run_backward(scene, obs, mode: str = "f") -> dict:
+    """Projection, binning, render and the renderer backward with its four gradient variants."""
+    p = project(scene, mode)
+    L = bin_lists(p, scene.H, scene.W)
+    r = render(p, L, scene.H, scene.W, scene.bg, mode)
+    accb = backward(p, L, r, obs, scene.bg, scene.H, scene.W, mode)
+    return dict(proj=p, lists=L, **r, accb=accb, **gradients(p, accb, scene, mode))
 
 
 def trace(proj, lists, H, W, bg, v, i, j, mode="d", cap=4096) -> np.ndarray:

@@ -489,6 +489,129 @@ void replay_pixel(const double* rec_v, const double* B_v, int d, const Lists& L,
   }
 }
 
+
+// ------------------------------------------------------------------------------------------
+// Gradient of the SH basis with respect to the view direction, for the renderer backward.
+// On the unit sphere each real SH function is a polynomial in (x, y, z):
+//   B_lm = N_lm (-1)^m [d^|m| P_l / dz^|m|](z) A_m(x, y),
+//   A_m = Re (x + i y)^m (m > 0), Im (x + i y)^|m| (m < 0), 1 (m = 0),
+// since (1 - z^2)^{m/2} e^{i m phi} = (x + i y)^m there (the associated Legendre function with
+// the Condon-Shortley phase is (-1)^m (1 - z^2)^{m/2} d^m P_l / dz^m). N_lm is the normalisation
+// of sh_basis_def (times sqrt 2 for m != 0). The Legendre polynomial coefficients come from
+// Bonnet's recurrence (n + 1) P_{n+1} = (2n + 1) z P_n - n P_{n-1}. This extension off the sphere
+// is differentiated by hand (product rule); the caller projects the gradient onto the tangent
+// plane, which removes any dependence on how the basis is extended off the sphere.
+// ------------------------------------------------------------------------------------------
+void sh_poly_grad_def(int deg, const double dir[3], double* B, double (*dB)[3]) {
+  const double x = dir[0], y = dir[1], z = dir[2];
+  double Pc[5][5] = {{0}};  // Pc[l][k]: coefficient of z^k in P_l
+  Pc[0][0] = 1.0;
+  Pc[1][1] = 1.0;
+  for (int n = 1; n + 1 <= 4; ++n)
+    for (int k = 0; k <= n + 1; ++k)
+      Pc[n + 1][k] = ((2.0 * n + 1.0) * (k > 0 ? Pc[n][k - 1] : 0.0) - n * Pc[n - 1][k]) / (n + 1.0);
+  // D^m P_l evaluated at z, for m = 0..l+1
+  auto dpoly = [&](int l, int m) {
+    double v = 0.0;
+    for (int k = m; k <= l; ++k) {
+      double c = Pc[l][k];
+      for (int t = 0; t < m; ++t) c *= (double)(k - t);
+      v += c * std::pow(z, k - m);
+    }
+    return v;
+  };
+  auto fact = [](int n) { double f = 1; for (int i = 2; i <= n; ++i) f *= i; return f; };
+  // (x + i y)^m and its x-derivative m (x + i y)^{m-1} (the y-derivative is i times that)
+  double re[5], im[5];
+  re[0] = 1.0; im[0] = 0.0;
+  for (int m = 1; m <= 4; ++m) {
+    re[m] = re[m - 1] * x - im[m - 1] * y;
+    im[m] = re[m - 1] * y + im[m - 1] * x;
+  }
+  for (int l = 0; l <= deg; ++l) {
+    for (int m = -l; m <= l; ++m) {
+      const int am = m < 0 ? -m : m;
+      double N = std::sqrt((2.0 * l + 1.0) / (4.0 * M_PI) * fact(l - am) / fact(l + am));
+      if (am) N *= std::sqrt(2.0);
+      if (am & 1) N = -N;
+      double A, Ax, Ay;
+      if (m == 0) { A = 1.0; Ax = 0.0; Ay = 0.0; }
+      else if (m > 0) { A = re[am]; Ax = am * re[am - 1]; Ay = -am * im[am - 1]; }
+      else { A = im[am]; Ax = am * im[am - 1]; Ay = am * re[am - 1]; }
+      const double Dm = dpoly(l, am), Dm1 = dpoly(l, am + 1);
+      const int k = l * l + l + m;
+      B[k] = N * Dm * A;
+      dB[k][0] = N * Dm * Ax;
+      dB[k][1] = N * Dm * Ay;
+      dB[k][2] = N * Dm1 * A;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Renderer backward of one pixel: derivatives of L = 1/2 sum_p |C_hat_p - C_obs_p|^2 ("Relation
+// to Gradient": the raw gradient the score tokens are compared with; RGB squared loss as in
+// "Exact Score Operators"), with the contributor order, the skip decisions, the early stop and
+// the clamp decisions held fixed. With the composited entries i = 1..n,
+//   C_hat = sum_i T_i alpha_i c_i + T_{n+1} bg,   T_{i+1} = T_i (1 - alpha_i),
+//   d C_hat / d c_i = T_i alpha_i,
+//   d C_hat / d alpha_i = T_i c_i - S_i / (1 - alpha_i),  S_i = sum_{j>i} T_j alpha_j c_j + T_{n+1} bg,
+// the suffix S_i being summed back to front (its definition; no recovery equation). With
+// ga_i = <r, d C_hat / d alpha_i> and, where alpha = o G is not clamped, d alpha = alpha d(pw) +
+// G d o with pw = -1/2 d^T Q d, d = p - mu2D, Q the conic, the pixel adds to its (Gaussian, view)
+//   q += w, Swr += w r (w = T alpha), and with h = ga alpha:  H += h, Hd += h d (2),
+//   Hdd += h (dx^2, dx dy, dy^2),
+// from which the per-Gaussian chain forms every parameter's derivative. T_i are products of
+// (1 - alpha) in double.
+// ------------------------------------------------------------------------------------------
+constexpr int ACCB_N = 10;  // q, Swr(3), H, Hdx, Hdy, Hdxdx, Hdxdy, Hdydy
+
+template <typename R>
+void backward_pixel(const double* rec_v, const Lists& L, long long ofs_base, int tile, int i,
+                    int j, const double* chat, const float* obs, const float* bg, int lst,
+                    double* accb_v) {
+  const long long s = L.off[ofs_base + tile];
+  const R px = (R)i + (R)0.5, py = (R)j + (R)0.5;
+  double r[3];
+  for (int ch = 0; ch < 3; ++ch) r[ch] = chat[ch] - (double)obs[ch];
+  struct Hit { int g; double al, dx, dy; };
+  std::vector<Hit> hits;
+  for (long long k = s; k < s + lst; ++k) {
+    const int g = L.ids[k];
+    EntryEval<R> E = eval_entry<R>(rec_v + (long long)g * F_NFIELDS, px, py);
+    if (E.use) hits.push_back({g, (double)E.alpha, (double)E.dx, (double)E.dy});
+  }
+  const int n = (int)hits.size();
+  std::vector<double> T(n + 1);
+  T[0] = 1.0;
+  for (int k = 0; k < n; ++k) T[k + 1] = T[k] * (1.0 - hits[k].al);
+  double S[3];
+  for (int ch = 0; ch < 3; ++ch) S[ch] = T[n] * (double)bg[ch];
+  for (int k = n - 1; k >= 0; --k) {
+    const Hit& e = hits[k];
+    const double* rec = rec_v + (long long)e.g * F_NFIELDS;
+    const double w = T[k] * e.al;
+    double ga = 0.0;
+    for (int ch = 0; ch < 3; ++ch) ga += r[ch] * (T[k] * rec[F_C0 + ch] - S[ch] / (1.0 - e.al));
+    double* a = accb_v + (long long)e.g * ACCB_N;
+    double add[ACCB_N] = {w, w * r[0], w * r[1], w * r[2], 0, 0, 0, 0, 0, 0};
+    if (e.al < 0.99) {
+      const double h = ga * e.al;
+      add[4] = h;
+      add[5] = h * e.dx;
+      add[6] = h * e.dy;
+      add[7] = h * e.dx * e.dx;
+      add[8] = h * e.dx * e.dy;
+      add[9] = h * e.dy * e.dy;
+    }
+    for (int q = 0; q < ACCB_N; ++q) {
+#pragma omp atomic
+      a[q] += add[q];
+    }
+    for (int ch = 0; ch < 3; ++ch) S[ch] += w * rec[F_C0 + ch];
+  }
+}
+
 }  // namespace
 
 // ==========================================================================================
@@ -833,6 +956,275 @@ int orc_finalize_partials(const double* P, int G, int deg, double lambda, double
     z[8 + 3 * d] = std::log(tr + eps);
   }
   return 0;
+}
+
+
+// Renderer backward over the listed (view, tile) pairs (all when n_sel < 0), adding into
+// accb [V, G, 10] (q, Swr[3], H, Hd[2], Hdd[3]; see backward_pixel). `img` is the render's
+// C_hat [V, H, W, 3], `last` its list bounds.
+#define ORC_BACKWARD(SUF, R)                                                                    \
+  void orc_backward_##SUF(const double* rec, const long long* off, const int* ids, int G,      \
+                          int V, int H, int W, const double* img, const float* obs,            \
+                          const float* bg, const int* last, const int* sel, int n_sel,         \
+                          double* accb) {                                                       \
+    const int TX = (W + TILE - 1) / TILE, TY = (H + TILE - 1) / TILE, nt = TX * TY;            \
+    const long long npairs = n_sel < 0 ? (long long)V * nt : n_sel;                             \
+    Lists L{off, ids};                                                                          \
+    _Pragma("omp parallel for schedule(dynamic, 4)")                                           \
+    for (long long q = 0; q < npairs; ++q) {                                                    \
+      const int v = n_sel < 0 ? (int)(q / nt) : sel[2 * q];                                     \
+      const int t = n_sel < 0 ? (int)(q % nt) : sel[2 * q + 1];                                 \
+      const int tx = t % TX, ty = t / TX;                                                       \
+      for (int j = ty * TILE; j < std::min(H, (ty + 1) * TILE); ++j)                            \
+        for (int i = tx * TILE; i < std::min(W, (tx + 1) * TILE); ++i) {                        \
+          const long long p = ((long long)v * H + j) * W + i;                                   \
+          backward_pixel<R>(rec + (long long)v * G * F_NFIELDS, L, (long long)v * (nt + 1), t, \
+                            i, j, img + 3 * p, obs + 3 * p, bg, last[p],                        \
+                            accb + (long long)v * G * ACCB_N);                                  \
+        }                                                                                       \
+    }                                                                                           \
+  }
+ORC_BACKWARD(f, float)
+ORC_BACKWARD(d, double)
+
+// Per-Gaussian chain of the renderer backward ("Relation to Gradient": raw, detached,
+// support-normalised and parameter-scale-normalised gradients). Rows [G, 11 + 3d]:
+//   [dL/dmu (3), dL/dlog_scale (3), dL/dquat (w, x, y, z), dL/dopacity_logit, dL/dsh (k-major)].
+// Per visible view, from the sums of backward_pixel (Q = stored conic, o = opacity):
+//   dL/da += (1 - o) H;  dL/dc_ch = Swr_ch where the colour clamp is inactive, else 0;
+//   dL/dsh_k += B_k dL/dc;  dL/dB_k = <dL/dc, sh_k>;  dL/d mu2D = Q Hd;
+//   dL/d(qa, qb, qc) = (-Hdxdx / 2, -Hdxdy, -Hdydy / 2);
+// then through the conic (qa, qb, qc) = (c, -b, a) / (a c - b^2) of Sigma2D = [[a, b], [b, c]]
+// (entry-wise partials), Sigma2D = J Sc J^T + 0.3 I (J the EWA Jacobian with the tangent clamped
+// at 1.3x the half field of view, Sc = R_v Sigma3D R_v^T), J and mu2D as functions of the camera
+// point x_c = R_v mu + t_v, the view direction dir = (mu - cam) / |mu - cam| of the SH colour,
+// and after the view loop Sigma3D = (Rq S)(Rq S)^T, S = diag(exp(log_scale)), Rq from q / |q|.
+// Variants ("Relation to Gradient" lists them; the readings are the plainest ones):
+//   detached: the same derivative with the paths the score operators stop -- Sigma2D, the view
+//     direction -- cut; it keeps the opacity-logit and SH blocks and the mean through mu2D only
+//     (sum_v J_gv^T Q Hd with J_gv = d pi_v / d mu), and is zero for scale and rotation;
+//   support: raw / q_g with q_g = eps + sum_v (eps + q_gv), the tokens' support normaliser;
+//   pscale: raw with the mean block times exp(mean of the three log-scales), the derivative with
+//     respect to the mean measured in units of the Gaussian's own size.
+// `fp32_decisions`: take the tangent-clamp decision in fp32 exactly as the fp32 projection does.
+// Any output pointer may be null.
+int orc_grad_finalize(const int* valid, const double* rec, const double* accb,
+                      const float* means, const float* lsc, const float* quats, const float* sh,
+                      const float* viewmats, const float* intrin, int G, int V, int H, int W,
+                      int deg, int fp32_decisions, double* raw, double* det, double* sup,
+                      double* psc) {
+  const int d = (deg + 1) * (deg + 1);
+  const int K = 11 + 3 * d;
+  const double eps = 1e-6;
+#pragma omp parallel for schedule(static)
+  for (int g = 0; g < G; ++g) {
+    std::vector<double> gr(K, 0.0), gd(K, 0.0);
+    double dSig[3][3] = {{0}};  // dL / dSigma3D (entry-wise)
+    double qg = eps;
+    const double mu[3] = {means[3 * g], means[3 * g + 1], means[3 * g + 2]};
+    // Gaussian frame (double, from the fp32 parameters)
+    double qv[4] = {quats[4 * g], quats[4 * g + 1], quats[4 * g + 2], quats[4 * g + 3]};
+    const double qn = std::sqrt(qv[0] * qv[0] + qv[1] * qv[1] + qv[2] * qv[2] + qv[3] * qv[3]);
+    const double w_ = qv[0] / qn, x_ = qv[1] / qn, y_ = qv[2] / qn, z_ = qv[3] / qn;
+    const double Rq[3][3] = {
+        {1 - 2 * (y_ * y_ + z_ * z_), 2 * (x_ * y_ - w_ * z_), 2 * (x_ * z_ + w_ * y_)},
+        {2 * (x_ * y_ + w_ * z_), 1 - 2 * (x_ * x_ + z_ * z_), 2 * (y_ * z_ - w_ * x_)},
+        {2 * (x_ * z_ - w_ * y_), 2 * (y_ * z_ + w_ * x_), 1 - 2 * (x_ * x_ + y_ * y_)}};
+    double Sd[3], Mm[3][3], Sig[3][3];
+    for (int k = 0; k < 3; ++k) Sd[k] = std::exp((double)lsc[3 * g + k]);
+    for (int i = 0; i < 3; ++i)
+      for (int k = 0; k < 3; ++k) Mm[i][k] = Rq[i][k] * Sd[k];
+    for (int i = 0; i < 3; ++i)
+      for (int j = 0; j < 3; ++j) {
+        Sig[i][j] = 0;
+        for (int k = 0; k < 3; ++k) Sig[i][j] += Mm[i][k] * Mm[j][k];
+      }
+    const float* shg = sh + (long long)g * d * 3;
+    for (int v = 0; v < V; ++v) {
+      const long long iv = (long long)v * G + g;
+      if (!valid[iv]) continue;
+      const double* rc = rec + iv * F_NFIELDS;
+      const double* a = accb + iv * ACCB_N;
+      qg += eps + a[0];
+      const float* vm = viewmats + 16 * v;
+      double Rv[3][3], tv[3];
+      for (int i = 0; i < 3; ++i) {
+        for (int j = 0; j < 3; ++j) Rv[i][j] = vm[4 * i + j];
+        tv[i] = vm[4 * i + 3];
+      }
+      const double fx = intrin[4 * v], fy = intrin[4 * v + 1];
+      const double o = rc[F_OPAC];
+      const double qa = rc[F_QA], qb = rc[F_QB], qc = rc[F_QC];
+      // opacity logit
+      gr[10] += (1.0 - o) * a[4];
+      // colour -> SH coefficients and view direction
+      const int cm = (int)rc[F_CMASK];
+      double gc[3];
+      for (int ch = 0; ch < 3; ++ch) gc[ch] = ((cm >> ch) & 1) ? a[1 + ch] : 0.0;
+      double cam[3], dv[3];
+      for (int i = 0; i < 3; ++i) cam[i] = -(Rv[0][i] * tv[0] + Rv[1][i] * tv[1] + Rv[2][i] * tv[2]);
+      for (int i = 0; i < 3; ++i) dv[i] = mu[i] - cam[i];
+      const double len = std::sqrt(dv[0] * dv[0] + dv[1] * dv[1] + dv[2] * dv[2]);
+      const double dir[3] = {dv[0] / len, dv[1] / len, dv[2] / len};
+      double Bv[16], dB[16][3];
+      sh_poly_grad_def(deg, dir, Bv, dB);
+      double gdir[3] = {0, 0, 0};
+      for (int k = 0; k < d; ++k) {
+        double gB = 0.0;
+        for (int ch = 0; ch < 3; ++ch) {
+          gr[11 + 3 * k + ch] += Bv[k] * gc[ch];
+          gB += gc[ch] * (double)shg[3 * k + ch];
+        }
+        for (int i = 0; i < 3; ++i) gdir[i] += gB * dB[k][i];
+      }
+      const double dg = dir[0] * gdir[0] + dir[1] * gdir[1] + dir[2] * gdir[2];
+      for (int i = 0; i < 3; ++i) gr[i] += (gdir[i] - dir[i] * dg) / len;
+      // projected centre and conic
+      const double gmx = qa * a[5] + qb * a[6], gmy = qb * a[5] + qc * a[6];
+      const double gqa = -0.5 * a[7], gqb = -a[8], gqc = -0.5 * a[9];
+      // camera point (double) and the EWA Jacobian with its clamp decision
+      double xc[3];
+      for (int i = 0; i < 3; ++i)
+        xc[i] = Rv[i][0] * mu[0] + Rv[i][1] * mu[1] + Rv[i][2] * mu[2] + tv[i];
+      const double x = xc[0], y = xc[1], z = xc[2];
+      bool in_u, in_v;
+      if (fp32_decisions) {
+        const float uf = (float)rc[F_XC] / (float)rc[F_ZC], vf = (float)rc[F_YC] / (float)rc[F_ZC];
+        const float lxf = 1.3f * ((0.5f * (float)W) / (float)fx);
+        const float lyf = 1.3f * ((0.5f * (float)H) / (float)fy);
+        in_u = uf >= -lxf && uf <= lxf;
+        in_v = vf >= -lyf && vf <= lyf;
+      } else {
+        const double ud = rc[F_XC] / rc[F_ZC], vd = rc[F_YC] / rc[F_ZC];
+        const double lxd = 1.3 * ((0.5 * W) / fx), lyd = 1.3 * ((0.5 * H) / fy);
+        in_u = ud >= -lxd && ud <= lxd;
+        in_v = vd >= -lyd && vd <= lyd;
+      }
+      const double lx = 1.3 * ((0.5 * W) / fx), ly = 1.3 * ((0.5 * H) / fy);
+      const double uc = in_u ? x / z : (x / z > 0 ? lx : -lx);
+      const double vc = in_v ? y / z : (y / z > 0 ? ly : -ly);
+      const double J[2][3] = {{fx / z, 0.0, -fx * uc / z}, {0.0, fy / z, -fy * vc / z}};
+      double Sc[3][3];
+      for (int i = 0; i < 3; ++i)
+        for (int j = 0; j < 3; ++j) {
+          double acc2 = 0.0;
+          for (int k = 0; k < 3; ++k)
+            for (int l = 0; l < 3; ++l) acc2 += Rv[i][k] * Sig[k][l] * Rv[j][l];
+          Sc[i][j] = acc2;
+        }
+      double s2a = 0.3, s2b = 0.0, s2c = 0.3;
+      for (int k = 0; k < 3; ++k)
+        for (int l = 0; l < 3; ++l) {
+          s2a += J[0][k] * Sc[k][l] * J[0][l];
+          s2b += J[0][k] * Sc[k][l] * J[1][l];
+          s2c += J[1][k] * Sc[k][l] * J[1][l];
+        }
+      const double D = s2a * s2c - s2b * s2b, D2 = D * D;
+      // d(qa, qb, qc) / d(a, b, c) entry by entry
+      const double ga_ = gqa * (-s2c * s2c / D2) + gqb * (s2b * s2c / D2) + gqc * (-s2b * s2b / D2);
+      const double gb_ = gqa * (2 * s2b * s2c / D2) + gqb * (-1.0 / D - 2 * s2b * s2b / D2) +
+                         gqc * (2 * s2a * s2b / D2);
+      const double gc_ = gqa * (-s2b * s2b / D2) + gqb * (s2a * s2b / D2) + gqc * (-s2a * s2a / D2);
+      // Sigma2D entries: a = J0 Sc J0^T, b = J0 Sc J1^T, c = J1 Sc J1^T
+      double dSc[3][3], dJ[2][3];
+      for (int k = 0; k < 3; ++k)
+        for (int l = 0; l < 3; ++l)
+          dSc[k][l] = ga_ * J[0][k] * J[0][l] + gb_ * J[0][k] * J[1][l] + gc_ * J[1][k] * J[1][l];
+      for (int k = 0; k < 3; ++k) {
+        double s00 = 0, s01 = 0, s11 = 0, s10 = 0;
+        for (int l = 0; l < 3; ++l) {
+          s00 += (Sc[k][l] + Sc[l][k]) * J[0][l];
+          s01 += Sc[k][l] * J[1][l];
+          s10 += J[0][l] * Sc[l][k];
+          s11 += (Sc[k][l] + Sc[l][k]) * J[1][l];
+        }
+        dJ[0][k] = ga_ * s00 + gb_ * s01;
+        dJ[1][k] = gb_ * s10 + gc_ * s11;
+      }
+      // camera-point gradient: mu2D = (fx x / z + cx, fy y / z + cy), and J(x, y, z)
+      double gx = gmx * fx / z, gy = gmy * fy / z;
+      double gz = -gmx * fx * x / (z * z) - gmy * fy * y / (z * z);
+      gz += dJ[0][0] * (-fx / (z * z)) + dJ[1][1] * (-fy / (z * z));
+      if (in_u) { gx += dJ[0][2] * (-fx / (z * z)); gz += dJ[0][2] * (2 * fx * x / (z * z * z)); }
+      else gz += dJ[0][2] * (fx * uc / (z * z));
+      if (in_v) { gy += dJ[1][2] * (-fy / (z * z)); gz += dJ[1][2] * (2 * fy * y / (z * z * z)); }
+      else gz += dJ[1][2] * (fy * vc / (z * z));
+      const double gxc[3] = {gx, gy, gz};
+      for (int i = 0; i < 3; ++i)
+        gr[i] += Rv[0][i] * gxc[0] + Rv[1][i] * gxc[1] + Rv[2][i] * gxc[2];
+      // detached mean: through mu2D only
+      const double gxd[3] = {gmx * fx / z, gmy * fy / z,
+                             -gmx * fx * x / (z * z) - gmy * fy * y / (z * z)};
+      for (int i = 0; i < 3; ++i)
+        gd[i] += Rv[0][i] * gxd[0] + Rv[1][i] * gxd[1] + Rv[2][i] * gxd[2];
+      // Sc = R_v Sigma3D R_v^T
+      for (int p2 = 0; p2 < 3; ++p2)
+        for (int q2 = 0; q2 < 3; ++q2) {
+          double acc2 = 0.0;
+          for (int i = 0; i < 3; ++i)
+            for (int j = 0; j < 3; ++j) acc2 += dSc[i][j] * Rv[i][p2] * Rv[j][q2];
+          dSig[p2][q2] += acc2;
+        }
+    }
+    // Sigma3D = M M^T, M = Rq diag(S)
+    double dM[3][3];
+    for (int i = 0; i < 3; ++i)
+      for (int k = 0; k < 3; ++k) {
+        dM[i][k] = 0.0;
+        for (int j = 0; j < 3; ++j) dM[i][k] += (dSig[i][j] + dSig[j][i]) * Mm[j][k];
+      }
+    double dR[3][3];
+    for (int k = 0; k < 3; ++k) {
+      double gS = 0.0;
+      for (int i = 0; i < 3; ++i) {
+        gS += dM[i][k] * Rq[i][k];
+        dR[i][k] = dM[i][k] * Sd[k];
+      }
+      gr[3 + k] = gS * Sd[k];
+    }
+    // rotation entries as functions of the unit quaternion (w, x, y, z)
+    const double gw = dR[0][1] * (-2 * z_) + dR[0][2] * (2 * y_) + dR[1][0] * (2 * z_) +
+                      dR[1][2] * (-2 * x_) + dR[2][0] * (-2 * y_) + dR[2][1] * (2 * x_);
+    const double gx_ = dR[0][1] * (2 * y_) + dR[0][2] * (2 * z_) + dR[1][0] * (2 * y_) +
+                       dR[1][1] * (-4 * x_) + dR[1][2] * (-2 * w_) + dR[2][0] * (2 * z_) +
+                       dR[2][1] * (2 * w_) + dR[2][2] * (-4 * x_);
+    const double gy_ = dR[0][0] * (-4 * y_) + dR[0][1] * (2 * x_) + dR[0][2] * (2 * w_) +
+                       dR[1][0] * (2 * x_) + dR[1][2] * (2 * z_) + dR[2][0] * (-2 * w_) +
+                       dR[2][1] * (2 * z_) + dR[2][2] * (-4 * y_);
+    const double gz_ = dR[0][0] * (-4 * z_) + dR[0][1] * (-2 * w_) + dR[0][2] * (2 * x_) +
+                       dR[1][0] * (2 * w_) + dR[1][1] * (-4 * z_) + dR[1][2] * (2 * y_) +
+                       dR[2][0] * (2 * x_) + dR[2][1] * (2 * y_);
+    // q_hat = q / |q|
+    const double qh[4] = {w_, x_, y_, z_}, gqh[4] = {gw, gx_, gy_, gz_};
+    const double dotq = qh[0] * gqh[0] + qh[1] * gqh[1] + qh[2] * gqh[2] + qh[3] * gqh[3];
+    for (int k = 0; k < 4; ++k) gr[6 + k] = (gqh[k] - qh[k] * dotq) / qn;
+    // detached keeps opacity and SH as they are
+    gd[10] = gr[10];
+    for (int k = 11; k < K; ++k) gd[k] = gr[k];
+    const double sig = std::exp(((double)lsc[3 * g] + (double)lsc[3 * g + 1] +
+                                 (double)lsc[3 * g + 2]) / 3.0);
+    for (int k = 0; k < K; ++k) {
+      const long long o = (long long)g * K + k;
+      if (raw) raw[o] = gr[k];
+      if (det) det[o] = gd[k];
+      if (sup) sup[o] = gr[k] / qg;
+      if (psc) psc[o] = k < 3 ? gr[k] * sig : gr[k];
+    }
+  }
+  return 0;
+}
+
+// SH basis and its gradient by the polynomial form (for the oracle's own checks):
+// dirs [n, 3] unit vectors -> B [n, 16], dB [n, 16, 3].
+void orc_sh_poly_grad(int deg, const double* dirs, long long n, double* B, double* dB) {
+  for (long long i = 0; i < n; ++i) {
+    double b[16] = {0}, db[16][3] = {{0}};
+    sh_poly_grad_def(deg, dirs + 3 * i, b, db);
+    for (int k = 0; k < 16; ++k) {
+      B[16 * i + k] = b[k];
+      for (int c = 0; c < 3; ++c) dB[48 * i + 3 * k + c] = db[k][c];
+    }
+  }
 }
 
 }  // extern "C"
