@@ -7,6 +7,10 @@ target views. Default workload: the DepthSplat-scale dense scene (5,898,240 Gaus
 3, 4 target views 512x960). Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
+                  [--path score|backward]
+
+--path backward times the renderer backward instead of the score replay (the gradient comparators:
+raw, detached, support- and parameter-scale-normalised gradients, all four per step).
 
 Multi-GPU: one process per GPU (torchrun); every rank renders and scores its own replica of the
 workload (no data-path collective); value = all ranks' pixels / the slowest rank's time.
@@ -26,6 +30,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "render+score-replay Mpix/s & Gaussian-pixel pairs/s; % of FP32/HBM roofline"
+METRICS = {"score": METRIC,
+           "backward": "render+backward Mpix/s & Gaussian-pixel pairs/s; % of FP32/HBM roofline"}
+PATHS = {"score": "render+score_replay+tokens",
+         "backward": "render+backward+gradients(raw,detached,support,pscale)"}
 WORKLOADS = {
     1: "two_plane_occlusion_64x64_1v_256g",
     2: "three_layer_occlusion_128x128_4v_4096g",
@@ -42,6 +50,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--path", choices=["score", "backward"], default="score")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=0,
@@ -172,6 +181,11 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
         "render": n_inst * (4 + 36) + px * 24,
         "replay": n_inst * (4 + 36) + px * (12 + 12 + 4) + V * G * 64,
         "finalize": V * G * (64 + 64) + G * 4 * (9 + 3 * d),
+        # backward: list entries as the replay, per pixel C_hat, C_obs, T_final, last; ten fp64
+        # sums per (v, g); the chain reads records (48 B) and sums (80 B) per (v, g), the
+        # parameters, and writes four gradient rows
+        "backward": n_inst * (4 + 36) + px * (12 + 12 + 4 + 4) + V * G * 80,
+        "grad": V * G * (48 + 80) + G * (12 + 16 + 12 * d) + 4 * G * 4 * (11 + 3 * d),
         "tiles": V * TX * TY,
     }
 
@@ -179,14 +193,16 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
 # algorithmic fp32 operations per traversed (pixel, list entry) pair, from the arithmetic the
 # method defines (the design notes count them): render = alpha (conic quadratic form, exp,
 # clamp/threshold tests) + transmittance + colour = 17 fp32 + 1 transcendental; replay = the same
-# alpha + suffix recovery (3 channels) + rho + masks + 7 weighted terms = 45 fp32 + 2 special
-ALU_OPS_PER_PAIR = {"render": 18, "replay": 47}
+# alpha + suffix recovery (3 channels) + rho + masks + 7 weighted terms = 45 fp32 + 2 special;
+# backward = the same alpha + transmittance recovery + d C_hat / d alpha (two 3-channel dot
+# products) + 10 weighted terms + suffix update = 49 fp32 + 2 special
+ALU_OPS_PER_PAIR = {"render": 18, "replay": 47, "backward": 51}
 
 
 # ----------------------------------------------------------------------------------------------
 # CPU oracle baseline: bounded sample, extrapolated to the metric's unit
 
-def cpu_oracle_sample(sc, obs_np, seconds_hint=15.0, tiles=0):
+def cpu_oracle_sample(sc, obs_np, seconds_hint=15.0, tiles=0, path="score"):
     import numpy as np
     from oracle import oracle as O
     one = _one_view(sc)
@@ -201,18 +217,25 @@ def cpu_oracle_sample(sc, obs_np, seconds_hint=15.0, tiles=0):
     sel = np.stack([np.zeros(n_s, np.int32), rng.choice(nt, n_s, replace=False).astype(np.int32)], 1)
     t1 = time.perf_counter()
     r = O.render(p, L, one.H, one.W, one.bg, "f", sel=sel)
-    O.replay(p, L, r, obs_np[:1], one.sh_degree, one.H, one.W, "f", sel=sel)
+    if path == "backward":
+        accb = O.backward(p, L, r, obs_np[:1], one.bg, one.H, one.W, "f", sel=sel)
+    else:
+        O.replay(p, L, r, obs_np[:1], one.sh_degree, one.H, one.W, "f", sel=sel)
     t_rr = time.perf_counter() - t1
     t2 = time.perf_counter()
-    acc = np.zeros((1, one.G, 8))
-    O.finalize(p, acc, one)
+    if path == "backward":
+        O.gradients(p, accb, one, "f")
+    else:
+        O.finalize(p, np.zeros((1, one.G, 8)), one)
     t_fin = time.perf_counter() - t2
+    second = "backward" if path == "backward" else "replay"
+    last = "gradient chain" if path == "backward" else "finalisation"
     t_view = t_pb + t_rr * nt / n_s + t_fin
     return {"value": one.H * one.W / t_view / 1e6, "unit": "Mpix/s",
             "cores": int(O.lib().orc_num_threads()), "kind": "oracle",
             "sample": (f"1 of {sc.V} views: projection + binning of all {sc.G} Gaussians "
-                       f"({t_pb:.2f} s), render + replay of {n_s}/{nt} random tiles "
-                       f"({t_rr:.2f} s, scaled to the view), finalisation ({t_fin:.2f} s)"),
+                       f"({t_pb:.2f} s), render + {second} of {n_s}/{nt} random tiles "
+                       f"({t_rr:.2f} s, scaled to the view), {last} ({t_fin:.2f} s)"),
             "seconds": t_pb + t_rr + t_fin}
 
 
@@ -269,18 +292,18 @@ def run_reference(args):
     obs = scenes.smooth_observation(99, 1, sc.H, sc.W)
     times, samples = [], []
     for it in range(args.warmup + args.steps):
-        s = cpu_oracle_sample(sc, obs, tiles=args.cpu_tiles or 0)
+        s = cpu_oracle_sample(sc, obs, tiles=args.cpu_tiles or 0, path=args.path)
         if it >= args.warmup:
             times.append(s["seconds"])
             samples.append(s)
     val = statistics.median([s["value"] for s in samples])
     ms = 1e3 * sc.H * sc.W / (val * 1e6)
-    line = {"metric": METRIC, "value": val, "unit": "Mpix/s", "n_gpus": args.gpus,
+    line = {"metric": METRICS[args.path], "value": val, "unit": "Mpix/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOADS[args.config], "views_per_step": 1,
-                       "l2": "n/a (CPU)"},
+                       "path": PATHS[args.path], "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": val, "unit": "Mpix/s", "cores": samples[0]["cores"],
                              "kind": "oracle", "sample": samples[0]["sample"]},
             "e2e": {"value": val, "unit": "Mpix/s", "h2d_bytes_per_step": 0,
@@ -320,8 +343,21 @@ def main():
     stream = torch.cuda.current_stream()
     l2_flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
+    K = P.grad_dim(ds.deg)
+
+    def alloc_grads():
+        return {k: torch.empty((ds.G, K), dtype=torch.float32, device=dev)
+                for k in ("raw", "detached", "support", "pscale")}
+
+    grads = alloc_grads() if args.path == "backward" else None
+
+    def run(ds_, obs_, out_, grads_):
+        if args.path == "backward":
+            return runner.render_and_backward(ws, ds_, obs_, out_, grads_)
+        return runner.render_and_score(ws, ds_, obs_, out_)
+
     def step():
-        return runner.render_and_score(ws, ds, obs, out)
+        return run(ds, obs, out, grads)
 
     for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
         n_inst = step()
@@ -375,12 +411,19 @@ def main():
         dsets = [ds, runner.DeviceScene(*[getattr(ds, k).clone() for k in names], ds.H, ds.W)]
         dobs = [obs, obs.clone()]
         outs = [out, runner.alloc_outputs(ds)]
+        dgrads = [grads, alloc_grads()] if args.path == "backward" else [None, None]
+
+        def d_outputs(b):
+            o = {"img": outs[b].img, "T": outs[b].T, "n_contrib": outs[b].n_contrib}
+            if args.path == "backward":
+                o.update(dgrads[b])
+            else:
+                o["tokens"] = outs[b].tokens
+            return o
 
         def h_outputs():
-            return {"tokens": torch.empty(out.tokens.shape, dtype=torch.float32).pin_memory(),
-                    "img": torch.empty(out.img.shape, dtype=torch.float32).pin_memory(),
-                    "T": torch.empty(out.T.shape, dtype=torch.float32).pin_memory(),
-                    "n_contrib": torch.empty(out.n_contrib.shape, dtype=torch.int32).pin_memory()}
+            return {k: torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                    for k, t in d_outputs(0).items()}
         h_out = [h_outputs(), h_outputs()]
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = sum(t.numel() * t.element_size() for t in h_out[0].values())
@@ -411,14 +454,12 @@ def main():
             stream.wait_event(in_ready[b])
             if k >= 2:
                 stream.wait_event(out_free[b])  # step k-2's outputs have been copied out
-            runner.render_and_score(ws, dsets[b], dobs[b], outs[b])
+            run(dsets[b], dobs[b], outs[b], dgrads[b])
             comp_done[b].record(stream)
             s_out.wait_event(comp_done[b])
             with torch.cuda.stream(s_out):
-                h_out[b]["tokens"].copy_(outs[b].tokens, non_blocking=True)
-                h_out[b]["img"].copy_(outs[b].img, non_blocking=True)
-                h_out[b]["T"].copy_(outs[b].T, non_blocking=True)
-                h_out[b]["n_contrib"].copy_(outs[b].n_contrib, non_blocking=True)
+                for k, t in d_outputs(b).items():
+                    h_out[b][k].copy_(t, non_blocking=True)
                 out_free[b].record(s_out)
         t1.record(s_out)
         t1.synchronize()
@@ -427,7 +468,7 @@ def main():
         e2e = {"value": px_step * args.steps * world / (e2e_total * 1e-3) / 1e6,
                "unit": "Mpix/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_total / args.steps, "pipelined": True}
-        del dsets, dobs, outs, h_out
+        del dsets, dobs, outs, h_out, dgrads
 
     # ---- roofline of the dominant kernel ------------------------------------------------------
     peaks = load_peaks()
@@ -458,28 +499,30 @@ def main():
     render_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in
                     ("project", "depth_hist", "depth_scatter", "emit", "tile_hist",
                      "hist_scan", "tile_scatter", "tile_ranges", "render", "other"))
-    replay_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in ("replay", "finalize"))
+    second = ("backward", "grad") if args.path == "backward" else ("replay", "finalize")
+    replay_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in second)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_sample(sc, obs.cpu().numpy(), tiles=args.cpu_tiles)
+        cpu = cpu_oracle_sample(sc, obs.cpu().numpy(), tiles=args.cpu_tiles, path=args.path)
         cpu.pop("seconds", None)
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world,
+            "metric": METRICS[args.path], "value": value, "unit": "Mpix/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": WORKLOADS[args.config], "gaussians": sc.G, "views": sc.V,
                        "height": sc.H, "width": sc.W, "sh_degree": sc.sh_degree,
+                       "path": PATHS[args.path],
                        "instances_per_step": n_total, "pairs_per_step": pairs,
                        "l2": "256 MiB buffer written between timed steps",
                        "parallelism": f"replicas x{world}"},
             "pairs_per_s": pairs_per_s,
             "ms_view": ms_per_step / sc.V,
-            "render_ms_per_step": render_ms, "replay_ms_per_step": replay_ms,
-            "replay_over_render": replay_ms / render_ms if render_ms else None,
+            "render_ms_per_step": render_ms, f"{second[0]}_ms_per_step": replay_ms,
+            f"{second[0]}_over_render": replay_ms / render_ms if render_ms else None,
             "gpu_launches": int(launches), "per_kernel": per_kernel,
             "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
         }

@@ -13,7 +13,7 @@ import os
 from .build import LIB, build  # noqa: F401
 
 __all__ = ["Workspace", "SplatError", "load_library", "LIB", "build", "token_dim",
-           "partials_dim", "finalize_partials"]
+           "partials_dim", "grad_dim", "finalize_partials"]
 
 _ERRORS = {
     -1: "INVALID_ARG", -2: "CAPACITY", -3: "STATE", -4: "CUDA", -5: "BOUNDS",
@@ -27,10 +27,11 @@ EXPORTS = [
     "splat_copy_tile_lists", "splat_copy_last", "splat_copy_accumulators", "splat_pair_count",
     "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
     "splat_sort_depths_noalloc", "splat_score_partials", "splat_finalize_partials",
+    "splat_backward",
 ]
 
 
-KERNEL_GROUPS = 12  # SPLAT_NUM_KERNELS
+KERNEL_GROUPS = 14  # SPLAT_NUM_KERNELS
 
 
 class SplatError(RuntimeError):
@@ -88,6 +89,8 @@ def load_library(path: str | None = None):
     L.splat_score_partials.restype = I
     L.splat_finalize_partials.argtypes = [V, I, I, F, V, V]
     L.splat_finalize_partials.restype = I
+    L.splat_backward.argtypes = [V, V, V, V, V, V, V, V, V, V]
+    L.splat_backward.restype = I
     if path is None:
         _lib = L
     return L
@@ -98,6 +101,11 @@ def token_dim(sh_degree: int) -> int:
 
 
 def partials_dim(sh_degree: int) -> int:
+    return 11 + 3 * (sh_degree + 1) ** 2
+
+
+def grad_dim(sh_degree: int) -> int:
+    """Row width of the gradients: mean (3), log-scale (3), quaternion (4), opacity logit, SH."""
     return 11 + 3 * (sh_degree + 1) ** 2
 
 
@@ -212,6 +220,21 @@ class Workspace:
             self._h, _ptr(obs, "obs", torch.float32, (V, H, W, 3)),
             _ptr(partials, "partials", torch.float32, (self.G, partials_dim(self.deg))),
             _stream(stream)))
+
+    def backward(self, obs, log_scales, quats, sh, raw=None, detached=None, support=None,
+                 pscale=None, stream=None):
+        """Renderer backward of 1/2 sum |C_hat - C_obs|^2 after render: the requested gradient
+        variants, each [G, 11 + 3d] fp32 (None skips a variant). log_scales, quats, sh are the
+        arrays given to project."""
+        import torch
+        G, d, f = self.G, (self.deg + 1) ** 2, torch.float32
+        K = grad_dim(self.deg)
+        outs = [_ptr(t, n, f, (G, K)) for t, n in ((raw, "raw"), (detached, "detached"),
+                                                    (support, "support"), (pscale, "pscale"))]
+        self._check(self._L.splat_backward(
+            self._h, _ptr(obs, "obs", f, (self.V, self.H, self.W, 3)),
+            _ptr(log_scales, "log_scales", f, (G, 3)), _ptr(quats, "quats", f, (G, 4)),
+            _ptr(sh, "sh", f, (G, d, 3)), *outs, _stream(stream)))
 
     # -- inspection -----------------------------------------------------------------------------
     def copy_projection(self, rec, rect, stream=None):

@@ -8,7 +8,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsplat.so")
-SOURCES = ["capi.cu", "project.cu", "binning.cu", "raster.cu", "finalize.cu", "noalloc.cu"]
+SOURCES = ["capi.cu", "project.cu", "binning.cu", "raster.cu", "finalize.cu", "backward.cu",
+           "noalloc.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -66,7 +66,7 @@ int alloc(Workspace& w, T** p, size_t n, const char* what) {
 void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
-                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask};
+                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.accb};
   for (void* p : dev)
     if (p) cudaFree(p);
   if (w.h_vstart) cudaFreeHost(w.h_vstart);
@@ -80,7 +80,7 @@ void free_all(Workspace& w) {
 
 const char* const kKernelNames[SPLAT_NUM_KERNELS] = {
     "project", "depth_hist", "depth_scatter", "emit", "tile_hist", "hist_scan",
-    "tile_scatter", "tile_ranges", "render", "replay", "finalize", "other"};
+    "tile_scatter", "tile_ranges", "render", "replay", "finalize", "backward", "grad", "other"};
 
 // fold every recorded (start, end) pair into the per-kernel sums
 int fold_events(Workspace& w) {
@@ -188,7 +188,6 @@ int splat_project(splat_ws* ws, const float* means, const float* log_scales, con
     return fail(w, SPLAT_ERR_CAPACITY, "sizes exceed the workspace maxima");
   int rc;
   const bool none = G == 0;
-  if ((rc = check_dev_ptr(w, means, "means", none))) return rc;
   if ((rc = check_dev_ptr(w, log_scales, "log_scales", none))) return rc;
   if ((rc = check_dev_ptr(w, quats, "quats", none))) return rc;
   if ((rc = check_dev_ptr(w, opac_logits, "opac_logits", none))) return rc;
@@ -262,6 +261,8 @@ int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int*
   if ((rc = check_dev_ptr(w, n_contrib, "n_contrib"))) return rc;
   if ((rc = splat::launch_render(w, bg, img, T_final, n_contrib, (cudaStream_t)stream))) return rc;
   w.img = img;
+  w.Tfin = T_final;
+  w.bg = bg;
   w.stage = 3;
   return SPLAT_OK;
 }
@@ -282,6 +283,34 @@ int splat_score_replay(splat_ws* ws, const float* obs, float lambda, float* toke
   if ((rc = splat::launch_finalize(w, lambda, tokens, st))) return rc;
   w.stage = 4;
   return SPLAT_OK;
+}
+
+int splat_backward(splat_ws* ws, const float* obs, const float* log_scales, const float* quats,
+                   const float* sh, float* grad_raw, float* grad_detached, float* grad_support,
+                   float* grad_pscale, void* stream) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  Workspace& w = ws->w;
+  w.err.clear();
+  if (w.stage < 3) return fail(w, SPLAT_ERR_STATE, "splat_backward before splat_render");
+  if (!grad_raw && !grad_detached && !grad_support && !grad_pscale)
+    return fail(w, SPLAT_ERR_INVALID_ARG, "splat_backward: no output requested");
+  int rc;
+  const bool none = w.G == 0;
+  if ((rc = check_dev_ptr(w, obs, "obs"))) return rc;
+  if ((rc = check_dev_ptr(w, log_scales, "log_scales", none))) return rc;
+  if ((rc = check_dev_ptr(w, quats, "quats", none))) return rc;
+  if ((rc = check_dev_ptr(w, sh, "sh", none))) return rc;
+  float* outs[4] = {grad_raw, grad_detached, grad_support, grad_pscale};
+  const char* names[4] = {"grad_raw", "grad_detached", "grad_support", "grad_pscale"};
+  for (int k = 0; k < 4; ++k)
+    if (outs[k] && (rc = check_dev_ptr(w, outs[k], names[k], none))) return rc;
+  if (!w.accb && (rc = alloc(w, &w.accb, (size_t)w.max_V * w.max_G * splat::kAccBN,
+                             "backward sums")))
+    return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((rc = splat::launch_backward(w, obs, st))) return rc;
+  return splat::launch_grad(w, log_scales, quats, sh, grad_raw, grad_detached, grad_support,
+                            grad_pscale, st);
 }
 
 int splat_score_partials(splat_ws* ws, const float* obs, float* partials, void* stream) {

@@ -21,6 +21,7 @@ constexpr int kTile = 16;        // 16x16 pixel tiles
 constexpr int kTilePix = 256;
 constexpr int kRecF4 = 4;        // float4 per (v, g) record
 constexpr int kAccN = 8;         // doubles per (v, g) accumulator
+constexpr int kAccBN = 10;       // doubles per (v, g) renderer-backward sums
 constexpr int kFlagVisible = 256;
 constexpr int kKeyStripes = 64;  // striped copies of the per-view depth-key statistics
 
@@ -121,9 +122,12 @@ struct Workspace {
   int* counts = nullptr;     // [V*G] tiles touched
   long long* offs = nullptr; // [V*G + 1] exclusive scan of counts
   double* acc = nullptr;     // [V*G*8]
+  double* accb = nullptr;    // [max_V*max_G*10] renderer-backward sums, allocated on first use
   float* views = nullptr;    // [V*20]: viewmat (16) + intrinsics (4)
   int* last = nullptr;       // [V*H*W]
-  const float* img = nullptr;  // C_hat written by the last render (caller-owned)
+  const float* img = nullptr;   // C_hat written by the last render (caller-owned)
+  const float* Tfin = nullptr;  // final transmittance written by the last render (caller-owned)
+  const float* bg = nullptr;    // background colour of the last render (caller-owned)
 
   // scan partials (int64)
   long long* part = nullptr;
@@ -230,6 +234,9 @@ int launch_finalize(Workspace& w, float lambda, float* tokens, cudaStream_t st);
 int launch_partials(Workspace& w, float* partials, cudaStream_t st);
 cudaError_t launch_finalize_partials(const float* partials, int G, int deg, double lambda,
                                      float* tokens, cudaStream_t st);
+int launch_backward(Workspace& w, const float* obs, cudaStream_t st);
+int launch_grad(Workspace& w, const float* lsc, const float* quats, const float* sh, float* raw,
+                float* det, float* sup, float* psc, cudaStream_t st);
 int launch_pair_count(Workspace& w, cudaStream_t st);
 int binning_configure(Workspace& w);
 

@@ -288,6 +288,120 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   }
 }
 
+// Renderer backward of L = 1/2 sum |C_hat - C_obs|^2 with the render's decisions held fixed.
+// Each warp walks its composited entries BACK TO FRONT (chunks from the last one down, entries in
+// a chunk from the highest position down), starting from the final transmittance and the
+// background term: per entry T_i = T_{i+1} / (1 - alpha_i), and the composite behind the entry,
+// S = sum_{j>i} T_j alpha_j c_j + T_final bg, is summed as it goes (no cancellation, unlike the
+// front-to-back recovery C_hat - P - T alpha c). With
+//   d C_hat / d alpha = T c - S / (1 - alpha),  ga = <r, d C_hat / d alpha>,
+// and, where alpha = o G is not clamped, h = ga alpha, the pixel adds to its (view, Gaussian)
+//   q += w, w r (3), h, h (dx, dy), h (dx^2, dx dy, dy^2)     (w = T alpha)
+// by a 16-slot transpose-reduction per entry and fp64 atomics from the ten lanes holding sums.
+__global__ void __launch_bounds__(kThreads)
+k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
+           const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
+           const float* __restrict__ img, const float* __restrict__ Tfin,
+           const float* __restrict__ bgp, const float* __restrict__ obs,
+           const int* __restrict__ last, const uint32_t* __restrict__ umask,
+           double* __restrict__ accb) {
+  const int t = blockIdx.x, v = blockIdx.y;
+  const int tx = t % TX, ty = t / TX;
+  const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
+  const bool inside = i < W && j < H;
+  const long long s = tile_off[(size_t)v * (nt + 1) + t];
+  const int gt = v * nt + t;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float4 s_a[kThreads], s_b[kThreads];
+  __shared__ float2 s_c[kThreads];
+  __shared__ uint32_t s_g[kThreads];
+  float4* wa = s_a + warp * 32;
+  float4* wb = s_b + warp * 32;
+  float2* wc = s_c + warp * 32;
+  uint32_t* wg = s_g + warp * 32;
+  const float px = (float)i + 0.5f, py = (float)j + 0.5f;
+  float r0 = 0.0f, r1 = 0.0f, r2 = 0.0f, T = 1.0f, S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
+  int lst = 0;
+  if (inside) {
+    const size_t p = ((size_t)v * H + j) * W + i;
+    r0 = img[3 * p] - obs[3 * p];
+    r1 = img[3 * p + 1] - obs[3 * p + 1];
+    r2 = img[3 * p + 2] - obs[3 * p + 2];
+    T = Tfin[p];
+    S0 = T * bgp[0];
+    S1 = T * bgp[1];
+    S2 = T * bgp[2];
+    lst = last[p];
+  }
+  const int wmax = __reduce_max_sync(0xffffffffu, lst);
+  const float4* recv = rec + (size_t)v * G * kRecF4;
+  double* accv = accb + (size_t)v * G * kAccBN;
+  const int slot = (lane >> 1) & 15;  // value index this lane holds after the reduction
+  for (int base = (wmax - 1) & ~31; base >= 0; base -= 32) {
+    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
+    if (!bits) continue;  // warp-uniform
+    if ((bits >> lane) & 1u) {
+      const uint32_t g = ids[s + base + lane];
+      const float4* r = recv + (size_t)g * kRecF4;
+      const float4 c = r[2];
+      wa[lane] = r[0];
+      wb[lane] = r[1];
+      wc[lane] = make_float2(c.x, c.y);
+      wg[lane] = g;
+    }
+    __syncwarp();
+    while (bits) {  // warp-uniform, from the highest list position down
+      const int q = 31 - __clz(bits);
+      bits &= ~(1u << q);
+      float x[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) x[k] = 0.0f;
+      bool used = false;
+      if (base + q < lst) {
+        const float4 A = wa[q], Bq = wb[q];
+        const float2 Cq = wc[q];
+        const Entry E = eval_entry(A, Bq, Cq.y, px, py);
+        if (E.use) {
+          used = true;
+          const float al = E.alpha;
+          const float i1m = __frcp_rn(1.0f - al);
+          T = T * i1m;  // transmittance in front of the entry
+          const float w = al * T;
+          const float c0 = Bq.z, c1 = Bq.w, c2 = Cq.x;
+          x[0] = w;
+          x[1] = w * r0;
+          x[2] = w * r1;
+          x[3] = w * r2;
+          if (al < 0.99f) {
+            const float ga = T * (r0 * c0 + r1 * c1 + r2 * c2) - (r0 * S0 + r1 * S1 + r2 * S2) * i1m;
+            const float h = ga * al;
+            const float hx = h * E.dx, hy = h * E.dy;
+            x[4] = h;
+            x[5] = hx;
+            x[6] = hy;
+            x[7] = hx * E.dx;
+            x[8] = hx * E.dy;
+            x[9] = hy * E.dy;
+          }
+          S0 = S0 + w * c0;
+          S1 = S1 + w * c1;
+          S2 = S2 + w * c2;
+        }
+      }
+      if (__any_sync(0xffffffffu, used)) {
+        tr_step<8>(x, lane & 16, 16);
+        tr_step<4>(x, lane & 8, 8);
+        tr_step<2>(x, lane & 4, 4);
+        tr_step<1>(x, lane & 2, 2);
+        x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
+        if ((lane & 1) == 0 && slot < kAccBN && x[0] != 0.0f)
+          atomicAdd(accv + (size_t)wg[q] * kAccBN + slot, (double)x[0]);
+      }
+    }
+    __syncwarp();
+  }
+}
+
 __global__ void k_pair_sum(const int* __restrict__ last, long long n, long long* out) {
   long long sacc = 0;
   for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
@@ -321,6 +435,20 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
                                       w.img, obs, w.last, w.umask, w.acc);
   prof_end(w, st, tok);
   return check_launch(w, "replay kernel");
+}
+
+int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {
+  const int tok = prof_begin(w, st, SPLAT_K_BACKWARD);
+  if (w.G > 0) {
+    cudaError_t e = cudaMemsetAsync(w.accb, 0, (size_t)w.V * w.G * kAccBN * sizeof(double), st);
+    if (e != cudaSuccess)
+      return set_err(w, SPLAT_ERR_CUDA, std::string("backward sums clear: ") + cudaGetErrorString(e));
+  }
+  dim3 grid(w.nt, w.V);
+  k_backward<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX, w.nt,
+                                        w.img, w.Tfin, w.bg, obs, w.last, w.umask, w.accb);
+  prof_end(w, st, tok);
+  return check_launch(w, "backward kernel");
 }
 
 int launch_pair_count(Workspace& w, cudaStream_t st) {

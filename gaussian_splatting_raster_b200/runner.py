@@ -75,5 +75,14 @@ def render_and_score(ws: Workspace, ds: DeviceScene, obs, out: Outputs, lam: flo
     return n
 
 
+def render_and_backward(ws: Workspace, ds: DeviceScene, obs, out: Outputs, grads: dict,
+                        stream=None) -> list[int]:
+    """Render, then the renderer backward into the variants named in `grads` (raw, detached,
+    support, pscale -> [G, 11 + 3d] fp32 tensors)."""
+    n = render(ws, ds, out, stream)
+    ws.backward(obs, ds.log_scales, ds.quats, ds.sh, stream=stream, **grads)
+    return n
+
+
 def workspace_for(ds: DeviceScene) -> Workspace:
     return Workspace(max(ds.G, 1), ds.V, ds.H, ds.W, ds.deg)

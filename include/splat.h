@@ -103,8 +103,9 @@ int splat_bin_sort(splat_ws* ws, long long* n_instances_out, void* stream);
  *   img       [V,H,W,3] C_hat = sum T alpha c + T_final bg
  *   T_final   [V,H,W]   final transmittance
  *   n_contrib [V,H,W]   number of composited Gaussians (int32)
- * bg is a device pointer to 3 floats. The replay reads img back (it is C_hat), so img must stay
- * unmodified until splat_score_replay has run.
+ * bg is a device pointer to 3 floats. The replay reads img back (it is C_hat), and the backward
+ * img, T_final and bg, so these must stay unmodified until splat_score_replay / splat_backward
+ * have run.
  */
 int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int* n_contrib,
                  void* stream);
@@ -150,6 +151,41 @@ int splat_score_partials(splat_ws* ws, const float* obs, float* partials, void* 
 int splat_finalize_partials(const float* partials, int G, int sh_degree, float lambda,
                             float* tokens, void* stream);
 
+/*
+ * Renderer backward: the gradient comparators of [P1] "Relation to Gradient" (raw, detached,
+ * support-normalised and parameter-scale-normalised gradients; the pages' "kill test" baseline).
+ * Derivatives of L = 1/2 sum over views and pixels of |C_hat - C_obs|^2 (RGB squared loss,
+ * [P1] "Exact Score Operators") with the contributor order, the skip and early-stop decisions and
+ * the clamp decisions of splat_render held fixed. One back-to-front traversal of the entries
+ * splat_render composited (same decisions), from T_final and the background term, forms per
+ * entry d C_hat / d alpha = T c - S / (1 - alpha), S the composite behind it (summed as the
+ * traversal goes), and per (Gaussian, view) the sums
+ *   q = sum w, sum w r, and where alpha = o G < 0.99 with h = <r, d C_hat / d alpha> alpha:
+ *   sum h, sum h (p - mu2D), sum h (dx^2, dx dy, dy^2);
+ * then one pass per Gaussian chains them through the conic, the EWA covariance
+ * Sigma2D = J R_v Sigma3D R_v^T J^T + 0.3 I (tangent clamp at 1.3x the half field of view
+ * included), the projected centre, the SH view direction, Sigma3D = R S S^T R^T with
+ * S = diag(exp(log_scale)) and R from the normalised quaternion. Output rows, fp32 [G, 11 + 3d]:
+ *   [dL/dmean (3), dL/dlog_scale (3), dL/dquat (w, x, y, z), dL/dopacity_logit,
+ *    dL/dsh (3d, index k*3 + channel)]
+ * for the variants (each pointer may be NULL; at least one must be given):
+ *   grad_raw      the derivative itself;
+ *   grad_detached the derivative with the paths the score operators stop cut (Sigma2D and the
+ *                 view direction): mean through the projected centre only, zero scale and
+ *                 rotation blocks, opacity and SH blocks as in grad_raw;
+ *   grad_support  grad_raw / q_g, q_g = 1e-6 + sum_v (1e-6 + q_gv), the tokens' normaliser;
+ *   grad_pscale   grad_raw with the mean block multiplied by exp(mean of the three log-scales)
+ *                 (the derivative per unit of the Gaussian's own size).
+ * log_scales, quats, sh must be the arrays given to the last splat_project, unchanged (the
+ * means enter through the camera points the projection recorded).
+ * Needs splat_render; obs [V,H,W,3]. Leaves the workspace stage as it was (the score replay may
+ * still follow). The first call allocates the backward sums, 80 bytes per (view, Gaussian) of the
+ * workspace maxima (SPLAT_ERR_OOM when that fails).
+ */
+int splat_backward(splat_ws* ws, const float* obs, const float* log_scales, const float* quats,
+                   const float* sh, float* grad_raw, float* grad_detached, float* grad_support,
+                   float* grad_pscale, void* stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Inspection calls (tests and benchmarks; not part of the render/replay path). They copy
  * workspace state into caller-owned DEVICE buffers on `stream`, or report host-side counters.
@@ -186,7 +222,8 @@ long long splat_launch_count(const splat_ws* ws);
 enum {
   SPLAT_K_PROJECT = 0, SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER,
   SPLAT_K_EMIT, SPLAT_K_TILE_HIST, SPLAT_K_HIST_SCAN, SPLAT_K_TILE_SCATTER, SPLAT_K_TILE_RANGES,
-  SPLAT_K_RENDER, SPLAT_K_REPLAY, SPLAT_K_FINALIZE, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
+  SPLAT_K_RENDER, SPLAT_K_REPLAY, SPLAT_K_FINALIZE, SPLAT_K_BACKWARD, SPLAT_K_GRAD,
+  SPLAT_K_OTHER, SPLAT_NUM_KERNELS
 };
 int splat_profile_enable(splat_ws* ws, int enable);
 int splat_profile_read(splat_ws* ws, double* ms, long long* launches, int reset);

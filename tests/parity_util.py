@@ -106,3 +106,78 @@ def compare_tokens(zg, zo, exclude=None, which=None):
     err = token_errors(zg[idx].astype(np.float64), zo[idx])
     assert err.max(initial=0) <= TOKEN_RTOL, f"token error {err.max()} at {idx[err.argmax()]}"
     return err
+
+
+# renderer backward -------------------------------------------------------------------------------
+GRAD_RTOL = 1e-4
+GRAD_BLOCK_RTOL = 1e-3
+GRAD_VARIANTS = ("raw", "detached", "support", "pscale")
+
+
+def grad_blocks(K):
+    return {"mean": (0, 3), "log_scale": (3, 6), "quat": (6, 10), "opacity": (10, 11),
+            "sh": (11, K)}
+
+
+def gpu_backward(scene, obs, variants=GRAD_VARIANTS):
+    import torch
+    from gaussian_splatting_raster_b200 import grad_dim, runner
+
+    ds = runner.to_device(scene)
+    ws = runner.workspace_for(ds)
+    out = runner.alloc_outputs(ds)
+    obs_t = torch.as_tensor(np.ascontiguousarray(obs, np.float32)).cuda()
+    K = grad_dim(ds.deg)
+    grads = {k: torch.full((ds.G, K), float("nan"), dtype=torch.float32, device="cuda")
+             for k in variants}
+    runner.render_and_backward(ws, ds, obs_t, out, grads)
+    res = {k: v for k, v in grads.items()}
+    res.update(img=out.img, T=out.T, n_contrib=out.n_contrib)
+    if ds.G > 0:
+        rec = torch.empty((ds.V, ds.G, 16), dtype=torch.float32, device="cuda")
+        rect = torch.empty((ds.V, ds.G, 4), dtype=torch.int32, device="cuda")
+        ws.copy_projection(rec, rect)
+        res["rec"], res["rect"] = rec, rect
+    torch.cuda.synchronize()
+    res = {k: v.cpu().numpy() for k, v in res.items()}
+    res["launches"] = ws.launch_count
+    ws.close()
+    return res
+
+
+def compare_grads(gg, go, which=None, exclude=None, rtol=GRAD_RTOL, block_rtol=GRAD_BLOCK_RTOL):
+    """Two bars. (1) Per Gaussian, the whole row with every block scaled by that block's median
+    norm over the Gaussians: relative L2 <= rtol (floor 1e-3), the bar the tokens meet. (2) Per
+    Gaussian and block: relative L2 <= block_rtol (floor 1e-3 x the block's median norm); looser,
+    because a block that is a sum of terms of both signs (the opacity logit's above all) can be
+    far smaller than its terms, and its fp32 rounding is relative to the terms. Returns the worst
+    block errors."""
+    K = go.shape[1]
+    idx = np.arange(go.shape[0]) if which is None else np.asarray(which)
+    if exclude is not None:
+        idx = idx[~exclude[idx]]
+    worst = {}
+    gs, os_ = [], []
+    for name, (lo, hi) in grad_blocks(K).items():
+        o = go[idx, lo:hi]
+        g = gg[idx, lo:hi].astype(np.float64)
+        assert np.isfinite(g).all(), f"{name}: non-finite gradient"
+        norms = np.linalg.norm(o, axis=1)
+        nz = norms[norms > 0]
+        if nz.size == 0:
+            assert (g == 0).all(), f"{name}: expected zeros"
+            worst[name] = 0.0
+            continue
+        med = np.median(nz)
+        err = np.linalg.norm(g - o, axis=1) / np.maximum(norms, TOKEN_FLOOR * med)
+        worst[name] = float(err.max())
+        assert err.max() <= block_rtol, f"{name}: error {err.max()} at Gaussian {idx[err.argmax()]}"
+        gs.append(g / med)
+        os_.append(o / med)
+    if gs:
+        g, o = np.concatenate(gs, 1), np.concatenate(os_, 1)
+        n = np.linalg.norm(o, axis=1)
+        err = np.linalg.norm(g - o, axis=1) / np.maximum(n, TOKEN_FLOOR)
+        worst["row"] = float(err.max())
+        assert err.max() <= rtol, f"row error {err.max()} at Gaussian {idx[err.argmax()]}"
+    return worst
