@@ -64,7 +64,7 @@ __device__ __forceinline__ void sh_dB(int k, double x, double y, double z, doubl
 }
 
 template <int DEG>
-__global__ void __launch_bounds__(kGradThreads, 2)
+__global__ void __launch_bounds__(kGradThreads, 3)
 k_grad(const float4* __restrict__ rec, const double* __restrict__ accb,
        const float* __restrict__ views, const float* __restrict__ lsc,
        const float* __restrict__ quats, const float* __restrict__ sh, int G, int V, int H, int W,
@@ -119,12 +119,14 @@ k_grad(const float4* __restrict__ rec, const double* __restrict__ accb,
     }
     for (int v = 0; v < V; ++v) {
       const size_t iv = (size_t)v * G + g;
+      // all loads of the view issued together (one memory round trip per view); the record and
+      // sums of a view where g is culled are read but not used
       const float4 r3 = rec[iv * kRecF4 + 3];  // (z, x_c, y_c, flags)
-      const int flags = __float_as_int(r3.w);
-      if (!(flags & kFlagVisible)) continue;
       const float4 r0 = rec[iv * kRecF4], r1 = rec[iv * kRecF4 + 1];
       const double2* a2 = reinterpret_cast<const double2*>(accb + iv * kAccBN);
       const double2 aq = a2[0], ar = a2[1], ah = a2[2], ad = a2[3], ae = a2[4];
+      const int flags = __float_as_int(r3.w);
+      if (!(flags & kFlagVisible)) continue;
       // aq = (q, w r0), ar = (w r1, w r2), ah = (h, h dx), ad = (h dy, h dx dx), ae = (h dx dy, h dy dy)
       qg += eps + aq.x;
       const double o = r1.y;
