@@ -77,6 +77,11 @@ def lib():
         L.orc_grad_finalize.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
                                         P, P, P, P]
         L.orc_sh_poly_grad.argtypes = [i32, P, i64, P, P]
+        for m in "fd":
+            getattr(L, f"orc_render_features_{m}").argtypes = [P, P, P, i32, i32, i32, i32, P, P,
+                                                               i32, P, i32, P]
+            getattr(L, f"orc_scatter_{m}").argtypes = [P, P, P, i32, i32, i32, i32, P, P, i32, P,
+                                                       i32, P]
         L.orc_finalize_partials.argtypes = [P, i32, i32, f64, P]
         _lib = L
     return _lib
@@ -271,6 +276,46 @@ def run_backward(scene, obs, mode: str = "f") -> dict:
     r = render(p, L, scene.H, scene.W, scene.bg, mode)
     accb = backward(p, L, r, obs, scene.bg, scene.H, scene.W, mode)
     return dict(proj=p, lists=L, **r, accb=accb, **gradients(p, accb, scene, mode))
+
+
+def render_features(proj, lists, rend, feats, H, W, mode="f", sel=None) -> np.ndarray:
+    """Per-Gaussian attributes [G, C] composited with the render's weights -> [V, H, W, C]."""
+    V, G = proj["valid"].shape
+    TX, TY = n_tiles(H, W)
+    s, ns = _sel(sel, V, TX * TY)
+    feats = _c(feats, np.float32).reshape(G, -1)
+    C = feats.shape[1]
+    out = np.zeros((V, H, W, C))
+    ids = lists["ids"] if lists["n"] > 0 else np.zeros(1, np.int32)
+    getattr(lib(), f"orc_render_features_{mode}")(
+        _p(proj["rec"]), _p(lists["off"]), _p(ids), G, V, H, W, _p(_c(rend["last"], np.int32)),
+        _p(feats) if G > 0 else None, C, _p(s) if s is not None else None, ns, _p(out))
+    return out
+
+
+def scatter(proj, lists, rend, pixel_map, H, W, mode="f", sel=None) -> np.ndarray:
+    """Per-pixel map [V, H, W, C] scattered to the Gaussians with the render's weights -> [G, C]."""
+    V, G = proj["valid"].shape
+    TX, TY = n_tiles(H, W)
+    s, ns = _sel(sel, V, TX * TY)
+    m = _c(pixel_map, np.float32).reshape(V, H, W, -1)
+    C = m.shape[3]
+    out = np.zeros((G, C))
+    ids = lists["ids"] if lists["n"] > 0 else np.zeros(1, np.int32)
+    getattr(lib(), f"orc_scatter_{mode}")(
+        _p(proj["rec"]), _p(lists["off"]), _p(ids), G, V, H, W, _p(_c(rend["last"], np.int32)),
+        _p(m), C, _p(s) if s is not None else None, ns, _p(out))
+    return out
+
+
+def attribution(proj, lists, rend, obs, H, W, mode="f", sel=None) -> np.ndarray:
+    """Scalar attribution per Gaussian [G, 3]: alphaT coverage sum w, PRIMU-style error
+    sum w |r| (r = C_hat - C_obs), and the error per coverage sum w |r| / (sum w + 1e-6)."""
+    r = np.asarray(rend["img"], np.float64) - np.asarray(obs, np.float64)
+    rn = np.sqrt((r * r).sum(-1)).astype(np.float32)
+    m = np.stack([np.ones_like(rn), rn], -1)
+    s = scatter(proj, lists, rend, m, H, W, mode, sel)
+    return np.concatenate([s, (s[:, 1] / (s[:, 0] + 1e-6))[:, None]], 1)
 
 
 def trace(proj, lists, H, W, bg, v, i, j, mode="d", cap=4096) -> np.ndarray:

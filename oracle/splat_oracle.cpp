@@ -612,6 +612,34 @@ void backward_pixel(const double* rec_v, const Lists& L, long long ofs_base, int
   }
 }
 
+
+// ------------------------------------------------------------------------------------------
+// Per-Gaussian attributes composited with the render's weights -- the multi-channel /
+// scalar-attribute render (learned feature channels rendered beside RGB, as in "ReCoSplat"
+// section 2.1; a per-Gaussian uncertainty score rendered by alpha compositing into a map, as in
+// "ATSplat", core method) -- and its transpose, the scatter of a per-pixel map back to the
+// Gaussians with the same weights (the mask-channel back-projection of a 2D gain, "L2D2-GS"
+// method; with a map of ones the alphaT coverage, with the residual norm the PRIMU-style error of
+// "Relation to Gradient" / "Novelty Boundary"):
+//   F_p = sum_i w_i f_{g_i},      s_g = sum_p sum_{i: g_i = g} w_i m_p,      w = T alpha,
+// over the entries render_pixel composited (same decisions; no background term for attributes).
+// ------------------------------------------------------------------------------------------
+template <typename R>
+void pixel_weights(const double* rec_v, const Lists& L, long long ofs_base, int tile, int i,
+                   int j, int lst, std::vector<std::pair<int, R>>& out) {
+  out.clear();
+  const long long s = L.off[ofs_base + tile];
+  const R px = (R)i + (R)0.5, py = (R)j + (R)0.5;
+  R T = (R)1;
+  for (long long k = s; k < s + lst; ++k) {
+    const int g = L.ids[k];
+    EntryEval<R> E = eval_entry<R>(rec_v + (long long)g * F_NFIELDS, px, py);
+    if (!E.use) continue;
+    out.push_back({g, E.alpha * T});
+    T = T * ((R)1 - E.alpha);
+  }
+}
+
 }  // namespace
 
 // ==========================================================================================
@@ -1226,5 +1254,66 @@ void orc_sh_poly_grad(int deg, const double* dirs, long long n, double* B, doubl
     }
   }
 }
+
+
+// Attribute render [V, H, W, C] (fp accumulation in the working precision, like the colour) and
+// map scatter [G, C] (double) over the listed (view, tile) pairs (all when n_sel < 0); `last` is
+// the render's list bound per pixel.
+#define ORC_FEATURES(SUF, R)                                                                    \
+  void orc_render_features_##SUF(const double* rec, const long long* off, const int* ids,      \
+                                 int G, int V, int H, int W, const int* last,                  \
+                                 const float* feats, int C, const int* sel, int n_sel,         \
+                                 double* out) {                                                 \
+    const int TX = (W + TILE - 1) / TILE, TY = (H + TILE - 1) / TILE, nt = TX * TY;            \
+    const long long nsel = n_sel < 0 ? (long long)V * nt : n_sel;                               \
+    Lists L{off, ids};                                                                          \
+    _Pragma("omp parallel for schedule(dynamic, 1)")                                           \
+    for (long long q = 0; q < nsel; ++q) {                                                      \
+      const int v = n_sel < 0 ? (int)(q / nt) : sel[2 * q];                                     \
+      const int t = n_sel < 0 ? (int)(q % nt) : sel[2 * q + 1];                                 \
+      const int tx = t % TX, ty = t / TX;                                                       \
+      std::vector<std::pair<int, R>> wts;                                                       \
+      std::vector<R> F(C);                                                                      \
+      for (int j = ty * TILE; j < std::min(H, ty * TILE + TILE); ++j)                           \
+        for (int i = tx * TILE; i < std::min(W, tx * TILE + TILE); ++i) {                       \
+          const long long p = ((long long)v * H + j) * W + i;                                   \
+          pixel_weights<R>(rec + (long long)v * G * F_NFIELDS, L, (long long)v * (nt + 1), t,  \
+                           i, j, last[p], wts);                                                 \
+          for (int c = 0; c < C; ++c) F[c] = (R)0;                                              \
+          for (const auto& e : wts)                                                             \
+            for (int c = 0; c < C; ++c)                                                         \
+              F[c] = F[c] + e.second * (R)feats[(long long)e.first * C + c];                    \
+          for (int c = 0; c < C; ++c) out[p * C + c] = (double)F[c];                            \
+        }                                                                                       \
+    }                                                                                           \
+  }                                                                                             \
+  void orc_scatter_##SUF(const double* rec, const long long* off, const int* ids, int G, int V, \
+                         int H, int W, const int* last, const float* map, int C,               \
+                         const int* sel, int n_sel, double* out) {                              \
+    const int TX = (W + TILE - 1) / TILE, TY = (H + TILE - 1) / TILE, nt = TX * TY;            \
+    const long long nsel = n_sel < 0 ? (long long)V * nt : n_sel;                               \
+    Lists L{off, ids};                                                                          \
+    _Pragma("omp parallel for schedule(dynamic, 1)")                                           \
+    for (long long q = 0; q < nsel; ++q) {                                                      \
+      const int v = n_sel < 0 ? (int)(q / nt) : sel[2 * q];                                     \
+      const int t = n_sel < 0 ? (int)(q % nt) : sel[2 * q + 1];                                 \
+      const int tx = t % TX, ty = t / TX;                                                       \
+      std::vector<std::pair<int, R>> wts;                                                       \
+      for (int j = ty * TILE; j < std::min(H, ty * TILE + TILE); ++j)                           \
+        for (int i = tx * TILE; i < std::min(W, tx * TILE + TILE); ++i) {                       \
+          const long long p = ((long long)v * H + j) * W + i;                                   \
+          pixel_weights<R>(rec + (long long)v * G * F_NFIELDS, L, (long long)v * (nt + 1), t,  \
+                           i, j, last[p], wts);                                                 \
+          for (const auto& e : wts)                                                             \
+            for (int c = 0; c < C; ++c) {                                                       \
+              const double add = (double)e.second * (double)map[p * C + c];                     \
+              _Pragma("omp atomic")                                                             \
+              out[(long long)e.first * C + c] += add;                                           \
+            }                                                                                   \
+        }                                                                                       \
+    }                                                                                           \
+  }
+ORC_FEATURES(f, float)
+ORC_FEATURES(d, double)
 
 }  // extern "C"
