@@ -27,11 +27,11 @@ EXPORTS = [
     "splat_copy_tile_lists", "splat_copy_last", "splat_copy_accumulators", "splat_pair_count",
     "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
     "splat_sort_depths_noalloc", "splat_score_partials", "splat_finalize_partials",
-    "splat_backward",
+    "splat_backward", "splat_render_features", "splat_scatter", "splat_attribution",
 ]
 
 
-KERNEL_GROUPS = 14  # SPLAT_NUM_KERNELS
+KERNEL_GROUPS = 16  # SPLAT_NUM_KERNELS
 
 
 class SplatError(RuntimeError):
@@ -91,6 +91,12 @@ def load_library(path: str | None = None):
     L.splat_finalize_partials.restype = I
     L.splat_backward.argtypes = [V, V, V, V, V, V, V, V, V, V]
     L.splat_backward.restype = I
+    L.splat_render_features.argtypes = [V, V, I, V, V]
+    L.splat_render_features.restype = I
+    L.splat_scatter.argtypes = [V, V, I, V, V]
+    L.splat_scatter.restype = I
+    L.splat_attribution.argtypes = [V, V, V, V]
+    L.splat_attribution.restype = I
     if path is None:
         _lib = L
     return L
@@ -235,6 +241,31 @@ class Workspace:
             self._h, _ptr(obs, "obs", f, (self.V, self.H, self.W, 3)),
             _ptr(log_scales, "log_scales", f, (G, 3)), _ptr(quats, "quats", f, (G, 4)),
             _ptr(sh, "sh", f, (G, d, 3)), *outs, _stream(stream)))
+
+    def render_features(self, feats, out, stream=None):
+        """Composite per-Gaussian attributes feats [G, C] with the last render's weights into
+        out [V, H, W, C]."""
+        import torch
+        C = feats.shape[1] if feats.dim() == 2 else 0
+        self._check(self._L.splat_render_features(
+            self._h, _ptr(feats, "feats", torch.float32, (self.G, C)), C,
+            _ptr(out, "out", torch.float32, (self.V, self.H, self.W, C)), _stream(stream)))
+
+    def scatter(self, pixel_map, out, stream=None):
+        """Scatter a per-pixel map [V, H, W, C] to the Gaussians with the last render's weights
+        into out [G, C] (the adjoint of render_features)."""
+        import torch
+        C = pixel_map.shape[3] if pixel_map.dim() == 4 else 0
+        self._check(self._L.splat_scatter(
+            self._h, _ptr(pixel_map, "map", torch.float32, (self.V, self.H, self.W, C)), C,
+            _ptr(out, "out", torch.float32, (self.G, C)), _stream(stream)))
+
+    def attribution(self, obs, out, stream=None):
+        """Scalar attribution [G, 3]: alphaT coverage, PRIMU-style error, error per coverage."""
+        import torch
+        self._check(self._L.splat_attribution(
+            self._h, _ptr(obs, "obs", torch.float32, (self.V, self.H, self.W, 3)),
+            _ptr(out, "out", torch.float32, (self.G, 3)), _stream(stream)))
 
     # -- inspection -----------------------------------------------------------------------------
     def copy_projection(self, rec, rect, stream=None):

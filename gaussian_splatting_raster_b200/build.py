@@ -9,7 +9,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsplat.so")
 SOURCES = ["capi.cu", "project.cu", "binning.cu", "raster.cu", "finalize.cu", "backward.cu",
-           "noalloc.cu"]
+           "attributes.cu", "noalloc.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -35,7 +35,8 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    deps = sources() + [os.path.join(CSRC, "common.cuh"), os.path.join(ROOT, "include", "splat.h")]
+    deps = sources() + [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "traverse.cuh"),
+                        os.path.join(ROOT, "include", "splat.h")]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 

@@ -66,7 +66,7 @@ int alloc(Workspace& w, T** p, size_t n, const char* what) {
 void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
-                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.accb};
+                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.accb, w.sacc};
   for (void* p : dev)
     if (p) cudaFree(p);
   if (w.h_vstart) cudaFreeHost(w.h_vstart);
@@ -80,7 +80,8 @@ void free_all(Workspace& w) {
 
 const char* const kKernelNames[SPLAT_NUM_KERNELS] = {
     "project", "depth_hist", "depth_scatter", "emit", "tile_hist", "hist_scan",
-    "tile_scatter", "tile_ranges", "render", "replay", "finalize", "backward", "grad", "other"};
+    "tile_scatter", "tile_ranges", "render", "replay", "finalize", "backward", "grad", "features", "scatter",
+    "other"};
 
 // fold every recorded (start, end) pair into the per-kernel sums
 int fold_events(Workspace& w) {
@@ -311,6 +312,47 @@ int splat_backward(splat_ws* ws, const float* obs, const float* log_scales, cons
   if ((rc = splat::launch_backward(w, obs, st))) return rc;
   return splat::launch_grad(w, log_scales, quats, sh, grad_raw, grad_detached, grad_support,
                             grad_pscale, st);
+}
+
+constexpr int kMaxAttributeChannels = 64;
+
+int splat_render_features(splat_ws* ws, const float* feats, int C, float* out, void* stream) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  Workspace& w = ws->w;
+  w.err.clear();
+  if (w.stage < 3) return fail(w, SPLAT_ERR_STATE, "splat_render_features before splat_render");
+  if (C < 1 || C > kMaxAttributeChannels)
+    return fail(w, SPLAT_ERR_INVALID_ARG, "splat_render_features: C must be in [1, %d]",
+                kMaxAttributeChannels);
+  int rc;
+  if ((rc = check_dev_ptr(w, feats, "feats", w.G == 0))) return rc;
+  if ((rc = check_dev_ptr(w, out, "out"))) return rc;
+  return splat::launch_features(w, feats, C, out, (cudaStream_t)stream);
+}
+
+int splat_scatter(splat_ws* ws, const float* map, int C, float* out, void* stream) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  Workspace& w = ws->w;
+  w.err.clear();
+  if (w.stage < 3) return fail(w, SPLAT_ERR_STATE, "splat_scatter before splat_render");
+  if (C < 1 || C > kMaxAttributeChannels)
+    return fail(w, SPLAT_ERR_INVALID_ARG, "splat_scatter: C must be in [1, %d]",
+                kMaxAttributeChannels);
+  int rc;
+  if ((rc = check_dev_ptr(w, map, "map"))) return rc;
+  if ((rc = check_dev_ptr(w, out, "out", w.G == 0))) return rc;
+  return splat::launch_scatter(w, map, nullptr, C, out, (cudaStream_t)stream);
+}
+
+int splat_attribution(splat_ws* ws, const float* obs, float* out, void* stream) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  Workspace& w = ws->w;
+  w.err.clear();
+  if (w.stage < 3) return fail(w, SPLAT_ERR_STATE, "splat_attribution before splat_render");
+  int rc;
+  if ((rc = check_dev_ptr(w, obs, "obs"))) return rc;
+  if ((rc = check_dev_ptr(w, out, "out", w.G == 0))) return rc;
+  return splat::launch_scatter(w, nullptr, obs, 2, out, (cudaStream_t)stream);
 }
 
 int splat_score_partials(splat_ws* ws, const float* obs, float* partials, void* stream) {

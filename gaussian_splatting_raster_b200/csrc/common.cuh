@@ -123,6 +123,8 @@ struct Workspace {
   long long* offs = nullptr; // [V*G + 1] exclusive scan of counts
   double* acc = nullptr;     // [V*G*8]
   double* accb = nullptr;    // [max_V*max_G*10] renderer-backward sums, allocated on first use
+  double* sacc = nullptr;    // [G*C] scatter sums, grown on demand
+  size_t sacc_cap = 0;
   float* views = nullptr;    // [V*20]: viewmat (16) + intrinsics (4)
   int* last = nullptr;       // [V*H*W]
   const float* img = nullptr;   // C_hat written by the last render (caller-owned)
@@ -237,6 +239,9 @@ cudaError_t launch_finalize_partials(const float* partials, int G, int deg, doub
 int launch_backward(Workspace& w, const float* obs, cudaStream_t st);
 int launch_grad(Workspace& w, const float* lsc, const float* quats, const float* sh, float* raw,
                 float* det, float* sup, float* psc, cudaStream_t st);
+int launch_features(Workspace& w, const float* feats, int C, float* out, cudaStream_t st);
+int launch_scatter(Workspace& w, const float* map, const float* obs, int C, float* out,
+                   cudaStream_t st);
 int launch_pair_count(Workspace& w, cudaStream_t st);
 int binning_configure(Workspace& w);
 

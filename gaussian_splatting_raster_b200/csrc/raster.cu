@@ -35,51 +35,10 @@
 // atomics per (Gaussian, warp-strip). The SH block never enters the pixel loop: M_color w (B (x) r)
 // factors into M_color B (x) (sum w r); the mean block Sigma^-1 (sum w rho d) is formed once per
 // (Gaussian, view) in finalisation.
-#include "common.cuh"
+#include "traverse.cuh"
 
 namespace splat {
 namespace {
-
-constexpr int kThreads = 256;
-constexpr float kAlphaMin = 1.0f / 255.0f;
-
-struct Entry {
-  bool use;
-  float alpha, dx, dy;
-};
-
-// Can the entry's ellipse {exponent >= cut} (centre A.xy, half-extents ex, ey precomputed by the
-// projection, conservatively widened) reach a pixel centre of the warp's strip: columns
-// x0 + 0.5 .. x0 + 15.5, rows y0 + 0.5 .. y0 + 1.5? Entries outside would only be skipped, so
-// leaving them out changes no decision.
-__device__ __forceinline__ bool reaches_strip(float4 A, float ex, float ey, float x0, float y0) {
-  return A.x + ex >= x0 + 0.5f && A.x - ex <= x0 + 15.5f && A.y + ey >= y0 + 0.5f &&
-         A.y - ey <= y0 + 1.5f;
-}
-
-// position of the composited-entry mask of (global tile gt, chunk starting at list position p):
-// distinct for every chunk of every tile, at most N / 32 + V * nt
-__device__ __forceinline__ long long chunk_index(long long p, int gt) { return (p >> 5) + gt; }
-
-// alpha of one list entry at pixel centre (px, py), with the rasteriser's skip rules
-__device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
-                                            float py) {
-  Entry e;
-  e.dx = px - A.x;
-  e.dy = py - A.y;
-  const float t1 = A.z * e.dx * e.dx;
-  const float t2 = Bq.x * e.dy * e.dy;
-  const float t3 = A.w * e.dx * e.dy;
-  const float pw = -0.5f * (t1 + t2) - t3;
-  e.use = false;
-  e.alpha = 0.0f;
-  if (pw > 0.0f || pw < cut) return e;
-  const float al = fminf(0.99f, Bq.y * exp_cw(pw));
-  if (al < kAlphaMin) return e;
-  e.alpha = al;
-  e.use = true;
-  return e;
-}
 
 __global__ void __launch_bounds__(kThreads)
 k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
@@ -163,18 +122,6 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     Tout[p] = T;
     ncout[p] = n;
     last[p] = lst;
-  }
-}
-
-// one butterfly step of the transpose-reduction: lanes with `hi` keep the upper half of their
-// values and send the lower half, the others the reverse; the received half is added
-template <int HALF>
-__device__ __forceinline__ void tr_step(float* x, bool hi, int off) {
-#pragma unroll
-  for (int k = 0; k < HALF; ++k) {
-    const float send = hi ? x[k] : x[k + HALF];
-    const float keep = hi ? x[k + HALF] : x[k];
-    x[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
   }
 }
 

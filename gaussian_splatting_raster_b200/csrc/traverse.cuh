@@ -1,0 +1,90 @@
+// Device helpers shared by the kernels that traverse the per-tile contributor lists (render,
+// score replay, renderer backward, attribute render and scatter): the rasteriser's per-entry alpha
+// with its skip rules, the warp-strip reach test, the composited-entry mask index, and the
+// transpose-reduction that sums per-entry values over a warp's 32 pixels.
+//
+// Source: "Research Proposal: Renderer Score Tokens for Recurrent Gaussian Splatting",
+// "Two-Stage Algorithm" (both passes walk the same tile bins in the same order with the same
+// decisions; per-Gaussian contributions are reduced within a tile before global atomics).
+#pragma once
+#include "common.cuh"
+
+namespace splat {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr float kAlphaMin = 1.0f / 255.0f;
+
+struct Entry {
+  bool use;
+  float alpha, dx, dy;
+};
+
+// Can the entry's ellipse {exponent >= cut} (centre A.xy, half-extents ex, ey precomputed by the
+// projection, conservatively widened) reach a pixel centre of the warp's strip: columns
+// x0 + 0.5 .. x0 + 15.5, rows y0 + 0.5 .. y0 + 1.5? Entries outside would only be skipped, so
+// leaving them out changes no decision.
+__device__ __forceinline__ bool reaches_strip(float4 A, float ex, float ey, float x0, float y0) {
+  return A.x + ex >= x0 + 0.5f && A.x - ex <= x0 + 15.5f && A.y + ey >= y0 + 0.5f &&
+         A.y - ey <= y0 + 1.5f;
+}
+
+// position of the composited-entry mask of (global tile gt, chunk starting at list position p):
+// distinct for every chunk of every tile, at most N / 32 + V * nt
+__device__ __forceinline__ long long chunk_index(long long p, int gt) { return (p >> 5) + gt; }
+
+// alpha of one list entry at pixel centre (px, py), with the rasteriser's skip rules
+__device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
+                                            float py) {
+  Entry e;
+  e.dx = px - A.x;
+  e.dy = py - A.y;
+  const float t1 = A.z * e.dx * e.dx;
+  const float t2 = Bq.x * e.dy * e.dy;
+  const float t3 = A.w * e.dx * e.dy;
+  const float pw = -0.5f * (t1 + t2) - t3;
+  e.use = false;
+  e.alpha = 0.0f;
+  if (pw > 0.0f || pw < cut) return e;
+  const float al = fminf(0.99f, Bq.y * exp_cw(pw));
+  if (al < kAlphaMin) return e;
+  e.alpha = al;
+  e.use = true;
+  return e;
+}
+
+// one butterfly step of the transpose-reduction: lanes with `hi` keep the upper half of their
+// values and send the lower half, the others the reverse; the received half is added
+template <int HALF>
+__device__ __forceinline__ void tr_step(float* x, bool hi, int off) {
+#pragma unroll
+  for (int k = 0; k < HALF; ++k) {
+    const float send = hi ? x[k] : x[k + HALF];
+    const float keep = hi ? x[k + HALF] : x[k];
+    x[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+  }
+}
+
+// Sum NV per-lane values over the warp so that value k ends in the lanes whose `slot` is k:
+// log2(NV) transpose steps (each lane keeps half of what it holds and sends the other half), then
+// a plain butterfly over the remaining lane bits. After it, lane l holds the warp sum of value
+// (l >> (5 - log2 NV)) & (NV - 1) in x[0] when (l & (32 / NV - 1)) == 0.
+template <int NV>
+__device__ __forceinline__ void slot_reduce(float* x, int lane) {
+  if constexpr (NV >= 16) tr_step<8>(x, lane & 16, 16);
+  if constexpr (NV >= 8) tr_step<4>(x, lane & (NV >= 16 ? 8 : 16), NV >= 16 ? 8 : 16);
+  if constexpr (NV >= 4) tr_step<2>(x, lane & (32 / NV * 2), 32 / NV * 2);
+  if constexpr (NV >= 2) tr_step<1>(x, lane & (32 / NV), 32 / NV);
+#pragma unroll
+  for (int o = 32 / NV / 2; o >= 1; o >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], o);
+}
+template <int NV>
+__device__ __forceinline__ int slot_of(int lane) {
+  constexpr int sh = NV == 1 ? 5 : NV == 2 ? 4 : NV == 4 ? 3 : NV == 8 ? 2 : 1;
+  return NV == 1 ? 0 : (lane >> sh) & (NV - 1);
+}
+template <int NV>
+__device__ __forceinline__ bool slot_holder(int lane) { return (lane & (32 / NV - 1)) == 0; }
+
+}  // namespace
+}  // namespace splat

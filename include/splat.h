@@ -186,6 +186,29 @@ int splat_backward(splat_ws* ws, const float* obs, const float* log_scales, cons
                    const float* sh, float* grad_raw, float* grad_detached, float* grad_support,
                    float* grad_pscale, void* stream);
 
+/*
+ * Attribute compositing and its transpose, over the entries the last splat_render composited
+ * (same order and decisions; w = T alpha; no background term). Sources: "ReCoSplat" 2.1 (learned
+ * feature channels rendered beside RGB), "ATSplat" core method (a per-Gaussian uncertainty score
+ * rendered by alpha compositing), "L2D2-GS" method (a 2D gain back-projected to Gaussians through
+ * the rasteriser's mask channel), [P1] "Novelty Boundary" / Block 3 (alphaT scatter, PRIMU-style
+ * scalar error/coverage).
+ *
+ * splat_render_features: feats [G, C] per-Gaussian attributes -> out [V, H, W, C],
+ *   out_p = sum over composited entries of w f_g. Channels are composited 16 per pass.
+ * splat_scatter: map [V, H, W, C] per-pixel values -> out [G, C], out_g = sum over views and
+ *   pixels of w m_p (the adjoint of splat_render_features; with m = dL/dF it is the gradient
+ *   with respect to the attributes with the Gaussians' other parameters held, as in ATSplat's
+ *   stop-gradient uncertainty loss). Sums in fp64, rounded to fp32 at the end.
+ * splat_attribution: obs [V, H, W, 3] -> out [G, 3] = [sum w (alphaT coverage),
+ *   sum w |C_hat - C_obs| (PRIMU-style error), error / (coverage + 1e-6)].
+ * 1 <= C <= 64. Need splat_render (img, T_final, bg unchanged since). The scatter calls grow a
+ * workspace buffer of 8 G C bytes when needed (cudaMalloc; SPLAT_ERR_OOM when that fails).
+ */
+int splat_render_features(splat_ws* ws, const float* feats, int C, float* out, void* stream);
+int splat_scatter(splat_ws* ws, const float* map, int C, float* out, void* stream);
+int splat_attribution(splat_ws* ws, const float* obs, float* out, void* stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Inspection calls (tests and benchmarks; not part of the render/replay path). They copy
  * workspace state into caller-owned DEVICE buffers on `stream`, or report host-side counters.
@@ -223,7 +246,7 @@ enum {
   SPLAT_K_PROJECT = 0, SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER,
   SPLAT_K_EMIT, SPLAT_K_TILE_HIST, SPLAT_K_HIST_SCAN, SPLAT_K_TILE_SCATTER, SPLAT_K_TILE_RANGES,
   SPLAT_K_RENDER, SPLAT_K_REPLAY, SPLAT_K_FINALIZE, SPLAT_K_BACKWARD, SPLAT_K_GRAD,
-  SPLAT_K_OTHER, SPLAT_NUM_KERNELS
+  SPLAT_K_FEATURES, SPLAT_K_SCATTER, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
 };
 int splat_profile_enable(splat_ws* ws, int enable);
 int splat_profile_read(splat_ws* ws, double* ms, long long* launches, int reset);
