@@ -11,6 +11,8 @@ target views. Default workload: the DepthSplat-scale dense scene (5,898,240 Gaus
 
 --path backward times the renderer backward instead of the score replay (the gradient comparators:
 raw, detached, support- and parameter-scale-normalised gradients, all four per step).
+--path attributes times the attribute path instead: a 9-channel attribute render, the scatter of
+a 9-channel per-pixel map back to the Gaussians, and the scalar attribution (coverage, error).
 
 Multi-GPU: one process per GPU (torchrun); every rank renders and scores its own replica of the
 workload (no data-path collective); value = all ranks' pixels / the slowest rank's time.
@@ -31,9 +33,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "render+score-replay Mpix/s & Gaussian-pixel pairs/s; % of FP32/HBM roofline"
 METRICS = {"score": METRIC,
-           "backward": "render+backward Mpix/s & Gaussian-pixel pairs/s; % of FP32/HBM roofline"}
+           "backward": "render+backward Mpix/s & Gaussian-pixel pairs/s; % of FP32/HBM roofline",
+           "attributes": "render+attributes Mpix/s & Gaussian-pixel pairs/s; % of FP32/HBM roofline"}
+N_ATTR = 9  # attribute channels of the attributes path (learned feature channels beside RGB)
 PATHS = {"score": "render+score_replay+tokens",
-         "backward": "render+backward+gradients(raw,detached,support,pscale)"}
+         "backward": "render+backward+gradients(raw,detached,support,pscale)",
+         "attributes": "render+attribute_render(9ch)+scatter(9ch)+attribution"}
 WORKLOADS = {
     1: "two_plane_occlusion_64x64_1v_256g",
     2: "three_layer_occlusion_128x128_4v_4096g",
@@ -50,7 +55,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--path", choices=["score", "backward"], default="score")
+    ap.add_argument("--path", choices=["score", "backward", "attributes"], default="score")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=0,
@@ -186,6 +191,11 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
         # parameters, and writes four gradient rows
         "backward": n_inst * (4 + 36) + px * (12 + 12 + 4 + 4) + V * G * 80,
         "grad": V * G * (48 + 80) + G * (12 + 16 + 12 * d) + 4 * G * 4 * (11 + 3 * d),
+        # attributes: list entries as the replay; per pixel the list bound and 9 channels out
+        # (render) or in (scatter) or C_hat, C_obs in (attribution); 9 attributes read per
+        # composited entry (from cache: per (v, g) counted once), 9 / 2 fp64 sums per Gaussian
+        "features": n_inst * (4 + 36) + px * (4 + 4 * N_ATTR) + V * G * 4 * N_ATTR,
+        "scatter": 2 * n_inst * (4 + 36) + px * (4 + 4 * N_ATTR + 4 + 24) + G * 8 * (N_ATTR + 2),
         "tiles": V * TX * TY,
     }
 
@@ -195,8 +205,10 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
 # clamp/threshold tests) + transmittance + colour = 17 fp32 + 1 transcendental; replay = the same
 # alpha + suffix recovery (3 channels) + rho + masks + 7 weighted terms = 45 fp32 + 2 special;
 # backward = the same alpha + transmittance recovery + d C_hat / d alpha (two 3-channel dot
-# products) + 10 weighted terms + suffix update = 49 fp32 + 2 special
-ALU_OPS_PER_PAIR = {"render": 18, "replay": 47, "backward": 51}
+# products) + 10 weighted terms + suffix update = 49 fp32 + 2 special; features = alpha (13 fp32 +
+# 1 special) + w + 9 channels x (mul, add) + transmittance = 35; scatter = two traversals (the
+# 9-channel map scatter, 26, and the attribution, 19) = 45
+ALU_OPS_PER_PAIR = {"render": 18, "replay": 47, "backward": 51, "features": 35, "scatter": 45}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -219,17 +231,26 @@ def cpu_oracle_sample(sc, obs_np, seconds_hint=15.0, tiles=0, path="score"):
     r = O.render(p, L, one.H, one.W, one.bg, "f", sel=sel)
     if path == "backward":
         accb = O.backward(p, L, r, obs_np[:1], one.bg, one.H, one.W, "f", sel=sel)
+    elif path == "attributes":
+        rng2 = np.random.default_rng(1)
+        f = rng2.uniform(0, 1, (one.G, N_ATTR)).astype(np.float32)
+        m = rng2.uniform(0, 1, (1, one.H, one.W, N_ATTR)).astype(np.float32)
+        O.render_features(p, L, r, f, one.H, one.W, "f", sel=sel)
+        O.scatter(p, L, r, m, one.H, one.W, "f", sel=sel)
+        O.attribution(p, L, r, obs_np[:1], one.H, one.W, "f", sel=sel)
     else:
         O.replay(p, L, r, obs_np[:1], one.sh_degree, one.H, one.W, "f", sel=sel)
     t_rr = time.perf_counter() - t1
     t2 = time.perf_counter()
     if path == "backward":
         O.gradients(p, accb, one, "f")
-    else:
+    elif path == "score":
         O.finalize(p, np.zeros((1, one.G, 8)), one)
     t_fin = time.perf_counter() - t2
-    second = "backward" if path == "backward" else "replay"
-    last = "gradient chain" if path == "backward" else "finalisation"
+    second = {"backward": "backward", "attributes": "attribute render + scatters",
+              "score": "replay"}[path]
+    last = {"backward": "gradient chain", "attributes": "nothing further",
+            "score": "finalisation"}[path]
     t_view = t_pb + t_rr * nt / n_s + t_fin
     return {"value": one.H * one.W / t_view / 1e6, "unit": "Mpix/s",
             "cores": int(O.lib().orc_num_threads()), "kind": "oracle",
@@ -350,14 +371,31 @@ def main():
                 for k in ("raw", "detached", "support", "pscale")}
 
     grads = alloc_grads() if args.path == "backward" else None
+    if args.path == "attributes":
+        gen = torch.Generator(device=dev).manual_seed(1)
+        feats = torch.rand((ds.G, N_ATTR), generator=gen, device=dev)
+        pmap = torch.rand((ds.V, ds.H, ds.W, N_ATTR), generator=gen, device=dev)
 
-    def run(ds_, obs_, out_, grads_):
+    def alloc_attr():
+        return {"F": torch.empty((ds.V, ds.H, ds.W, N_ATTR), device=dev),
+                "S": torch.empty((ds.G, N_ATTR), device=dev),
+                "A": torch.empty((ds.G, 3), device=dev)}
+
+    attr_out = alloc_attr() if args.path == "attributes" else None
+
+    def run(ds_, obs_, out_, grads_, attr_):
         if args.path == "backward":
             return runner.render_and_backward(ws, ds_, obs_, out_, grads_)
+        if args.path == "attributes":
+            n = runner.render(ws, ds_, out_)
+            ws.render_features(feats, attr_["F"])
+            ws.scatter(pmap, attr_["S"])
+            ws.attribution(obs_, attr_["A"])
+            return n
         return runner.render_and_score(ws, ds_, obs_, out_)
 
     def step():
-        return run(ds, obs, out, grads)
+        return run(ds, obs, out, grads, attr_out)
 
     for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
         n_inst = step()
@@ -412,11 +450,14 @@ def main():
         dobs = [obs, obs.clone()]
         outs = [out, runner.alloc_outputs(ds)]
         dgrads = [grads, alloc_grads()] if args.path == "backward" else [None, None]
+        dattr = [attr_out, alloc_attr()] if args.path == "attributes" else [None, None]
 
         def d_outputs(b):
             o = {"img": outs[b].img, "T": outs[b].T, "n_contrib": outs[b].n_contrib}
             if args.path == "backward":
                 o.update(dgrads[b])
+            elif args.path == "attributes":
+                o.update(dattr[b])
             else:
                 o["tokens"] = outs[b].tokens
             return o
@@ -454,7 +495,7 @@ def main():
             stream.wait_event(in_ready[b])
             if k >= 2:
                 stream.wait_event(out_free[b])  # step k-2's outputs have been copied out
-            run(dsets[b], dobs[b], outs[b], dgrads[b])
+            run(dsets[b], dobs[b], outs[b], dgrads[b], dattr[b])
             comp_done[b].record(stream)
             s_out.wait_event(comp_done[b])
             with torch.cuda.stream(s_out):
@@ -468,7 +509,7 @@ def main():
         e2e = {"value": px_step * args.steps * world / (e2e_total * 1e-3) / 1e6,
                "unit": "Mpix/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_total / args.steps, "pipelined": True}
-        del dsets, dobs, outs, h_out, dgrads
+        del dsets, dobs, outs, h_out, dgrads, dattr
 
     # ---- roofline of the dominant kernel ------------------------------------------------------
     peaks = load_peaks()
@@ -499,7 +540,8 @@ def main():
     render_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in
                     ("project", "depth_hist", "depth_scatter", "emit", "tile_hist",
                      "hist_scan", "tile_scatter", "tile_ranges", "render", "other"))
-    second = ("backward", "grad") if args.path == "backward" else ("replay", "finalize")
+    second = {"backward": ("backward", "grad"), "attributes": ("features", "scatter"),
+              "score": ("replay", "finalize")}[args.path]
     replay_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in second)
 
     cpu = None

@@ -15,9 +15,10 @@
 //      depths) and 3 (depth order inside each tile) gives exactly (depth, index) per tile, and the
 //      scanned (tile, block) histogram yields every tile's [start, end).
 // Every pass -- each depth digit and the tile pass -- is the same stable counting sort: per block
-// of 16K items, per-warp shared-memory histograms (ranks of equal buckets inside a warp from
-// match.any), an int32 exclusive scan of the (bucket, block) counts, and a scatter that replays
-// the ranking. Uniform, bandwidth-shaped work; no decoupled look-back, so no device-side waits.
+// of 16K items, per-warp shared-memory histograms (shared-memory atomics), an int32 exclusive scan
+// of the (bucket, block) counts, and a scatter that ranks equal buckets inside each 32-item batch
+// with match.any (stable: earlier items first). Uniform, bandwidth-shaped work; no decoupled
+// look-back, so no device-side waits.
 #include "common.cuh"
 
 namespace splat {
@@ -130,10 +131,10 @@ int ensure_part(Workspace& w, long long nb) {
 // the stable counting-sort pass
 constexpr int kBinWarps = 8;
 constexpr int kBinThreads = kBinWarps * 32;
-constexpr int kBinChunk = 16384;  // items per block
-constexpr int kBinPerWarp = kBinChunk / kBinWarps;
+constexpr int kDepthChunk = 16384;  // items per block, depth-key passes
+constexpr int kTileChunk = 16384;   // items per block, tile pass
 
-// Items of view v are [start(v), start(v + 1)); each view is cut into blocks of kBinChunk.
+// Items of view v are [start(v), start(v + 1)); each view is cut into blocks of `chunk` items.
 // Uniform layout (every view holds `per_view` items, blocks_per_view blocks) or tables.
 struct Segs {
   long long per_view;        // >= 0: uniform layout
@@ -141,6 +142,7 @@ struct Segs {
   const long long* vstart;   // tables (per_view < 0): [V + 1] item starts
   const int* bstart;         // [V + 1] block starts
   int V;
+  int chunk;                 // items per block (a multiple of 32 * kBinWarps)
 };
 
 struct BlockRange {
@@ -156,8 +158,8 @@ __device__ __forceinline__ BlockRange block_range(const Segs& sg, int b) {
     r.lb = b - r.v * r.nbv;
     r.b0 = r.v * r.nbv;
     r.vbeg = (long long)r.v * sg.per_view;
-    r.beg = r.vbeg + (long long)r.lb * kBinChunk;
-    r.end = min(r.beg + (long long)kBinChunk, r.vbeg + sg.per_view);
+    r.beg = r.vbeg + (long long)r.lb * sg.chunk;
+    r.end = min(r.beg + (long long)sg.chunk, r.vbeg + sg.per_view);
   } else {
     int v = 0;
     while (v + 1 < sg.V && sg.bstart[v + 1] <= b) ++v;
@@ -166,8 +168,8 @@ __device__ __forceinline__ BlockRange block_range(const Segs& sg, int b) {
     r.lb = b - r.b0;
     r.nbv = sg.bstart[v + 1] - r.b0;
     r.vbeg = sg.vstart[v];
-    r.beg = r.vbeg + (long long)r.lb * kBinChunk;
-    r.end = min(r.beg + (long long)kBinChunk, sg.vstart[v + 1]);
+    r.beg = r.vbeg + (long long)r.lb * sg.chunk;
+    r.end = min(r.beg + (long long)sg.chunk, sg.vstart[v + 1]);
   }
   return r;
 }
@@ -178,28 +180,26 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-constexpr int kUnroll = 4;  // 32-item batches whose loads are issued together
+constexpr int kUnroll = 4;       // 32-item batches whose loads are issued together (ranking)
+constexpr int kCountUnroll = 8;  // 32-item batches whose loads are issued together (counting)
 
-// per-warp bucket counts of this block's items into cnt[nbk]; the loads of kUnroll batches are
-// issued before the first is ranked, so each warp keeps several requests in flight
+// per-warp bucket counts of the items [wb, we) into cnt (shared memory): the loads of
+// kCountUnroll batches are issued together, then each lane adds its items with shared-memory
+// atomics (counts do not depend on the order of the adds)
 __device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, int shift,
                                             uint32_t mask, long long wb, long long we,
                                             uint32_t* cnt) {
   const int lane = threadIdx.x & 31;
-  for (long long base = wb; base < we; base += 32 * kUnroll) {
-    uint32_t bk[kUnroll];
+  for (long long base = wb; base < we; base += 32 * kCountUnroll) {
+    uint32_t bk[kCountUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < kCountUnroll; ++u) {
       const long long i = base + 32 * u + lane;
-      bk[u] = i < we ? (keys[i] >> shift) & mask : (0x80000000u | lane);
+      bk[u] = i < we ? (keys[i] >> shift) & mask : 0xffffffffu;
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const bool ok = base + 32 * u + lane < we;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bk[u]);
-      if (ok && lane == __ffs(peers) - 1) cnt[bk[u]] += __popc(peers);
-      __syncwarp();
-    }
+    for (int u = 0; u < kCountUnroll; ++u)
+      if (bk[u] != 0xffffffffu) atomicAdd(cnt + bk[u], 1u);
   }
 }
 
@@ -212,8 +212,8 @@ k_count_hist(const uint32_t* __restrict__ keys, int shift, uint32_t mask, int nb
   for (int t = threadIdx.x; t < kBinWarps * nbk; t += blockDim.x) s_cnt[t] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5;
-  const long long wb = r.beg + (long long)warp * kBinPerWarp;
-  const long long we = min(wb + (long long)kBinPerWarp, r.end);
+  const long long wb = r.beg + (long long)warp * (sg.chunk / kBinWarps);
+  const long long we = min(wb + (long long)(sg.chunk / kBinWarps), r.end);
   warp_counts(keys, shift, mask, wb, we, s_cnt + warp * nbk);
   __syncthreads();
   int* h = hist + (size_t)nbk * r.b0;
@@ -237,8 +237,8 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t* cnt = s_cnt + warp * nbk;
-  const long long wb = r.beg + (long long)warp * kBinPerWarp;
-  const long long we = min(wb + (long long)kBinPerWarp, r.end);
+  const long long wb = r.beg + (long long)warp * (sg.chunk / kBinWarps);
+  const long long we = min(wb + (long long)(sg.chunk / kBinWarps), r.end);
   warp_counts(keys, shift, mask, wb, we, cnt);
   __syncthreads();
   // per bucket: global start of this block's run, then one sub-run per warp in warp order
@@ -440,7 +440,7 @@ int launch_binning(Workspace& w, cudaStream_t st) {
   const int dbits = passes ? (bits + passes - 1) / passes : 0;
   const uint32_t* order = nullptr;  // sorted Gaussian indices per view (nullptr: index order)
   if (passes > 0 && VG > 0) {
-    Segs sg{w.G, (int)((w.G + kBinChunk - 1) / kBinChunk), nullptr, nullptr, w.V};
+    Segs sg{w.G, (int)((w.G + kDepthChunk - 1) / kDepthChunk), nullptr, nullptr, w.V, kDepthChunk};
     const int nblocks = sg.blocks_per_view * w.V;
     const uint32_t* kin = w.dkey;
     const uint32_t* vin = nullptr;
@@ -475,14 +475,14 @@ int launch_binning(Workspace& w, cudaStream_t st) {
   w.h_bstart[0] = 0;
   for (int v = 0; v < w.V; ++v) {
     const long long nv = w.h_vstart[v + 1] - w.h_vstart[v];
-    w.h_bstart[v + 1] = w.h_bstart[v] + (int)((nv + kBinChunk - 1) / kBinChunk);
+    w.h_bstart[v + 1] = w.h_bstart[v] + (int)((nv + kTileChunk - 1) / kTileChunk);
   }
   w.n_blocks = w.h_bstart[w.V];
   cudaMemcpyAsync(w.d_vstart, w.h_vstart, (w.V + 1) * sizeof(long long),
                   cudaMemcpyHostToDevice, st);
   cudaMemcpyAsync(w.d_bstart, w.h_bstart, (w.V + 1) * sizeof(int), cudaMemcpyHostToDevice, st);
   if (N > 0) {
-    Segs sg{-1, 0, w.d_vstart, w.d_bstart, w.V};
+    Segs sg{-1, 0, w.d_vstart, w.d_bstart, w.V, kTileChunk};
     if ((rc = count_pass(w, st, w.inst_tile, w.inst_g, 0, 0xffffffffu, w.nt, sg, w.n_blocks,
                          nullptr, w.sval, SPLAT_K_TILE_HIST, SPLAT_K_TILE_SCATTER)))
       return rc;
