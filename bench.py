@@ -48,6 +48,17 @@ WORKLOADS = {
 }
 
 
+def make_scene(args):
+    from synth import scenes
+    return scenes.resplat_views(args.views) if args.views else scenes.make(args.config)
+
+
+def workload_name(args, sc) -> str:
+    if args.views:
+        return f"resplat_pixel_aligned_256x448_{sc.V}v_{sc.G}g_sh2"
+    return WORKLOADS[args.config]
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -56,6 +67,13 @@ def parse():
     ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--path", choices=["score", "backward", "attributes"], default="score")
+    ap.add_argument("--shard", choices=["replicas", "views"], default="replicas",
+                    help="views: each rank renders and replays its block of the views and one "
+                         "reduce-scatter of the per-Gaussian partial sums gives every rank its "
+                         "slice of tokens (strong scaling over views; score path only)")
+    ap.add_argument("--views", type=int, default=0,
+                    help="view-count scaling: the ReSplat-scale layout with this many context and "
+                         "target views at 256x448 (overrides --config)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=0,
@@ -291,6 +309,16 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
+def pairs_sum_over_ranks(x: int, world: int) -> int:
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return int(t.item())
+
+
 def max_over_ranks(x: float, world: int) -> float:
     import torch
     import torch.distributed as dist
@@ -309,7 +337,7 @@ def run_reference(args):
     import numpy as np
     from oracle import oracle as O
     from synth import scenes
-    sc = scenes.make(args.config)
+    sc = make_scene(args)
     obs = scenes.smooth_observation(99, 1, sc.H, sc.W)
     times, samples = [], []
     for it in range(args.warmup + args.steps):
@@ -323,7 +351,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOADS[args.config], "views_per_step": 1,
+            "config": {"workload": workload_name(args, sc), "views_per_step": 1,
                        "path": PATHS[args.path], "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": val, "unit": "Mpix/s", "cores": samples[0]["cores"],
                              "kind": "oracle", "sample": samples[0]["sample"]},
@@ -336,6 +364,11 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    # Libraries (NCCL's version banner, for one) may write to stdout; the contract is one JSON
+    # line there, so everything else goes to stderr and the line is written to the saved stdout.
+    sys.stdout.flush()
+    json_fd = os.dup(1)
+    os.dup2(2, 1)
     import numpy as np
     import torch
 
@@ -346,20 +379,38 @@ def main():
     rank, world, local = dist_setup()
     dev = torch.device("cuda", torch.cuda.current_device())
     P.load_library()  # built in-tree by __graft_entry__.build(); fails loudly when missing
-    sc = scenes.make(args.config)
+    sc = make_scene(args)
     ds = runner.to_device(sc)
-    ws = runner.workspace_for(ds)
-    out = runner.alloc_outputs(ds)
-
+    shard = args.shard == "views"
+    if shard and args.path != "score":
+        raise SystemExit("--shard views times the score path only")
+    if shard and world == 1:
+        import socket
+        import torch.distributed as dist
+        s_ = socket.socket()
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+        s_.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, device_id=dev)
     # observation: render of the perturbed scene (+ pixel noise), made by the same path, untimed
     obs_scene = runner.to_device(sc.observed_scene())
     obs_out = runner.alloc_outputs(obs_scene)
-    runner.render(ws, obs_scene, obs_out)
+    ws_obs = runner.workspace_for(obs_scene)
+    runner.render(ws_obs, obs_scene, obs_out)
     obs = obs_out.img.clone()
     if sc.obs_noise_sigma > 0:
         obs += torch.from_numpy(sc.pixel_noise()).to(dev)
-    del obs_scene, obs_out
     torch.cuda.synchronize()
+    ws_obs.close()
+    del obs_scene, obs_out, ws_obs
+    if shard:
+        from gaussian_splatting_raster_b200 import sharding
+        vlo, vhi = sharding.view_ranges(sc.V, world)[rank]
+        ws = P.Workspace(max(ds.G, 1), max(vhi - vlo, 1), ds.H, ds.W, ds.deg)
+    else:
+        ws = runner.workspace_for(ds)
+    out = runner.alloc_outputs(ds)
 
     stream = torch.cuda.current_stream()
     l2_flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -395,6 +446,8 @@ def main():
         return runner.render_and_score(ws, ds_, obs_, out_)
 
     def step():
+        if shard:
+            return sharding.sharded_tokens(ws, ds, obs, 1.0)[3]
         return run(ds, obs, out, grads, attr_out)
 
     for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
@@ -432,8 +485,12 @@ def main():
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     px_step = sc.V * sc.H * sc.W
-    value = px_step * args.steps * world / (total_ms * 1e-3) / 1e6
-    pairs_per_s = pairs * args.steps * world / (total_ms * 1e-3)
+    # replicas: every rank does the whole workload; views: the ranks split one workload
+    units = 1 if shard else world
+    value = px_step * args.steps * units / (total_ms * 1e-3) / 1e6
+    pairs_per_s = pairs * args.steps * (world if not shard else 1) / (total_ms * 1e-3)
+    if shard:  # pairs of all ranks' views
+        pairs_per_s = pairs_sum_over_ranks(pairs, world) * args.steps / (total_ms * 1e-3)
 
     # ---- end to end through the public API with host buffers ----------------------------------
     # Every step copies its inputs from pinned host memory and its outputs (tokens, image, final
@@ -441,7 +498,7 @@ def main():
     # pipelined with double-buffered device inputs/outputs: step k+1's host->device copy and step
     # k-1's device->host copy run on two copy streams while step k computes.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not shard:
         names = ("means", "log_scales", "quats", "opac", "sh", "viewmats", "intrin", "bg")
         host = {k: torch.from_numpy(np.ascontiguousarray(getattr(sc, k))).pin_memory()
                 for k in names}
@@ -525,14 +582,14 @@ def main():
         peak = lanes * peaks["sm_max_mhz"] * 1e6 / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "Tops/s (fp32 pipe)", "frac": achieved / peak,
-                "traffic": recorded_traffic(dom, WORKLOADS[args.config]),
+                "traffic": recorded_traffic(dom, workload_name(args, sc)),
                 "peak_source": f"{lanes} fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz "
                                f"({peaks['source']} max clock)"}
     else:
         achieved = ab.get(dom, 0) / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "traffic": recorded_traffic(dom, WORKLOADS[args.config]),
+                "traffic": recorded_traffic(dom, workload_name(args, sc)),
                 "peak_source": f"{peaks['source']} copy bandwidth"}
     for k, v in per_kernel.items():
         if k in ab:
@@ -553,14 +610,15 @@ def main():
         line = {
             "metric": METRICS[args.path], "value": value, "unit": "Mpix/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.config], "gaussians": sc.G, "views": sc.V,
+            "higher_is_better": True, "scaling": "strong" if shard else "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_name(args, sc), "gaussians": sc.G, "views": sc.V,
                        "height": sc.H, "width": sc.W, "sh_degree": sc.sh_degree,
                        "path": PATHS[args.path],
                        "instances_per_step": n_total, "pairs_per_step": pairs,
                        "l2": "256 MiB buffer written between timed steps",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": (f"views x{world} (reduce-scatter of per-Gaussian partials)"
+                                       if shard else f"replicas x{world}")},
             "pairs_per_s": pairs_per_s,
             "ms_view": ms_per_step / sc.V,
             "render_ms_per_step": render_ms, f"{second[0]}_ms_per_step": replay_ms,
@@ -568,10 +626,10 @@ def main():
             "gpu_launches": int(launches), "per_kernel": per_kernel,
             "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
         }
-        print(json.dumps(line), flush=True)
+        os.write(json_fd, (json.dumps(line) + "\n").encode())
     ws.close()
-    if world > 1:
-        import torch.distributed as dist
+    import torch.distributed as dist
+    if dist.is_initialized():
         dist.destroy_process_group()
 
 

@@ -57,7 +57,8 @@ def sharded_tokens(ws, ds, obs, lam: float = 1.0, group=None):
 
     ws: a Workspace sized for all Gaussians and this rank's views; ds: the full DeviceScene;
     obs: [V, H, W, 3] observations of all views. Returns (tokens [hi - lo, 9 + 3d], (lo, hi),
-    per-view render outputs of this rank's views or None when it holds no view)."""
+    per-view render outputs of this rank's views or None when it holds no view, list instances
+    per local view)."""
     import torch
     import torch.distributed as dist
     from . import runner
@@ -67,16 +68,16 @@ def sharded_tokens(ws, ds, obs, lam: float = 1.0, group=None):
     vlo, vhi = view_ranges(ds.V, world)[rank]
     Gp = padded_rows(G, world)
     partials = torch.zeros((Gp, partials_dim(deg)), dtype=torch.float32, device=ds.means.device)
-    out = None
+    out, n = None, []
     if vhi > vlo:
         local = dataclasses.replace(ds, viewmats=ds.viewmats[vlo:vhi].contiguous(),
                                     intrin=ds.intrin[vlo:vhi].contiguous())
         out = runner.alloc_outputs(local)
-        runner.render(ws, local, out)
+        n = runner.render(ws, local, out)
         ws.score_partials(obs[vlo:vhi].contiguous(), partials[:G])
     shard = reduce_partials(partials, group)
     lo, hi = row_range(G, world, rank)
     tokens = torch.empty((hi - lo, token_dim(deg)), dtype=torch.float32, device=shard.device)
     if hi > lo:
         finalize_partials(shard[: hi - lo].contiguous(), deg, tokens, lam)
-    return tokens, (lo, hi), out
+    return tokens, (lo, hi), out, n

@@ -244,6 +244,14 @@ def resplat_pixel_aligned(seed: int = 1003) -> Scene:
     return _pixel_aligned("resplat_256x448_8v", seed, 8, 8, 256, 448, 2, 0.1, 0.0)
 
 
+def resplat_views(n_views: int, seed: int = 1003) -> Scene:
+    """The ReSplat-scale layout with n_views context views backprojected (n_views x 114,688
+    Gaussians) scored in the same number of target views: the view-count scaling workloads
+    (4/8/16/32 views at 256x448)."""
+    return _pixel_aligned(f"resplat_256x448_{n_views}v", seed, n_views, n_views, 256, 448, 2, 0.1,
+                          0.0)
+
+
 def atsplat_anchor(seed: int = 1004) -> Scene:
     """19,456 anchors x 16 offsets = 311,296 Gaussians, SH degree 2, 4 target views 512x960."""
     rng = np.random.default_rng(seed)

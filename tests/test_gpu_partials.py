@@ -122,12 +122,12 @@ def test_sharded_tokens_single_rank_nccl():
                             world_size=1, device_id=torch.device("cuda:0"))
     try:
         ws = runner.workspace_for(ds)
-        z, (lo, hi), out = sharding.sharded_tokens(ws, ds, obs_t, 0.9)
+        z, (lo, hi), out, n = sharding.sharded_tokens(ws, ds, obs_t, 0.9)
         torch.cuda.synchronize()
         ws.close()
     finally:
         dist.destroy_process_group()
-    assert (lo, hi) == (0, sc.G)
+    assert (lo, hi) == (0, sc.G) and len(n) == sc.V
     o = O.run(sc, obs, "f", lam=0.9)
     PU.compare_tokens(z.cpu().numpy(), o["tokens"])
     PU.compare_render({"img": out.img.cpu().numpy(), "T": out.T.cpu().numpy(),
