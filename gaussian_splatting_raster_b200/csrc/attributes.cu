@@ -11,8 +11,8 @@
 //   attribution        [sum w, sum w |r|, sum w |r| / (sum w + 1e-6)] per Gaussian, r = C_hat - C_obs
 // with w = T alpha of the composited entries (the render's decisions; no background term).
 //
-// Same traversal as the score replay: one CTA per (tile, view); each warp walks its two pixel
-// rows' list on its own in 32-entry chunks, staging only the entries the render marked as
+// Same traversal as the score replay: one CTA per (tile, view); each warp walks the list for its
+// 8x4 pixel block on its own in 32-entry chunks, staging only the entries the render marked as
 // composited by some pixel of the warp. The attribute render keeps up to 16 channels per pixel in
 // registers (more channels take further passes); the scatter reduces each entry's per-pixel
 // values over the warp (transpose-reduction) and adds them with fp64 atomics into a workspace
@@ -33,7 +33,8 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
            const float* __restrict__ feats, int C, int c0, float* __restrict__ out) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
-  const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;
@@ -102,7 +103,8 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
           const float* __restrict__ obs, int C, int c0, double* __restrict__ acc) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
-  const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;

@@ -8,10 +8,10 @@
 // (o = sigmoid(a), alpha = o G, w = T alpha, rho = <r, c - C+>, q = sum w; the opacity-logit,
 // SH and projected-centre scores).
 //
-// One CTA per (tile, view), one thread per pixel of the 16x16 tile; the eight warps (two pixel
-// rows each) walk the tile's list independently, with no CTA barrier: each warp stages 32-entry
+// One CTA per (tile, view), one thread per pixel of the 16x16 tile; the eight warps (an 8x4 pixel
+// block each) walk the tile's list independently, with no CTA barrier: each warp stages 32-entry
 // chunks of records in its own shared-memory slice, keeps by ballot the entries whose precomputed
-// box reaches its rows, and stops when all its pixels are saturated. Both passes evaluate alpha
+// box reaches its block, and stops when all its pixels are saturated. Both passes evaluate alpha
 // through the same device function, so the replay takes exactly the render's decisions; the
 // render also leaves, per (tile, warp, chunk), the mask of entries that composited some pixel of
 // the warp, and the replay visits only those.
@@ -21,8 +21,9 @@
 // gives o exp(pw) < (1/255) exp(-1e-3), far below 1/255 even after the few-ulp errors of the
 // exp and of the product, so the entry is skipped without evaluating exp -- the same decision the
 // full evaluation takes, never a different one. The record also holds the half-extents of the
-// ellipse {exponent >= cut}; a warp (two pixel rows) only evaluates the entries whose box reaches
-// its rows.
+// ellipse {exponent >= cut}; a warp only evaluates the entries whose box reaches its block. (8x4
+// blocks meet ~17 % fewer entries than 16x2 strips of the same area: a squarer block has a
+// shorter perimeter for footprints to overlap.)
 //
 // Replay arithmetic. The suffix numerators C_hat - P - T alpha c are formed per channel exactly
 // as the recovery equation writes them (their cancellation dominates the fp32 error of C+), then
@@ -47,13 +48,14 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
          int* __restrict__ ncout, int* __restrict__ last, uint32_t* __restrict__ umask) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
-  const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const long long e = tile_off[(size_t)v * (nt + 1) + t + 1];
   const int gt = v * nt + t;
   // Each warp walks the whole list on its own (no CTA barriers): it stages 32 entries into its
-  // slice of shared memory, ballots which of them can reach its two pixel rows, evaluates only
+  // slice of shared memory, ballots which of them can reach its pixel block, evaluates only
   // those, and leaves as soon as its 32 pixels are done. Per 32-entry chunk it records which
   // entries some pixel of the warp composited: the replay visits exactly those.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -62,7 +64,7 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   float4* wa = s_a + warp * 32;
   float4* wb = s_b + warp * 32;
   float2* wc = s_c + warp * 32;
-  const float x0f = (float)(tx * kTile), y0f = (float)(ty * kTile + 2 * warp);
+  const float x0f = (float)bx, y0f = (float)by;
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int n = 0, lst = 0;
@@ -78,7 +80,7 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       wa[lane] = a;
       wb[lane] = b;
       wc[lane] = make_float2(c.x, c.y);
-      hit = reaches_strip(a, c.z, c.w, x0f, y0f);
+      hit = reaches_block(a, c.z, c.w, x0f, y0f);
     }
     uint32_t bits = __ballot_sync(0xffffffffu, hit);
     uint32_t ubits = 0u;
@@ -133,7 +135,8 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
          double* __restrict__ acc) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
-  const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;
@@ -254,7 +257,8 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
            double* __restrict__ accb) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
-  const int i = tx * kTile + (threadIdx.x & 15), j = ty * kTile + (threadIdx.x >> 4);
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;

@@ -20,13 +20,34 @@ struct Entry {
   float alpha, dx, dy;
 };
 
+// Pixel blocks of the warps. A tile's CTA has eight warps; warp w covers a kWarpW x kWarpH block
+// of the 16x16 tile (blocks in row-major order), lane l the pixel (l % kWarpW, l / kWarpW) of its
+// block. Every kernel that walks the lists uses this one mapping: the render records per warp
+// which entries some pixel of the block composited, and the later passes read those masks.
+#ifndef SPLAT_WARP_W
+#define SPLAT_WARP_W 8
+#endif
+constexpr int kWarpW = SPLAT_WARP_W;
+constexpr int kWarpH = 32 / kWarpW;
+static_assert(kTile % kWarpW == 0 && kTile % kWarpH == 0 &&
+              (kTile / kWarpW) * (kTile / kWarpH) == 8, "eight warp blocks per tile");
+
+// pixel of this thread in tile (tx, ty), and the top-left corner of its warp's block
+__device__ __forceinline__ void tile_pixel(int tx, int ty, int& i, int& j, int& bx, int& by) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  bx = tx * kTile + (warp % (kTile / kWarpW)) * kWarpW;
+  by = ty * kTile + (warp / (kTile / kWarpW)) * kWarpH;
+  i = bx + lane % kWarpW;
+  j = by + lane / kWarpW;
+}
+
 // Can the entry's ellipse {exponent >= cut} (centre A.xy, half-extents ex, ey precomputed by the
-// projection, conservatively widened) reach a pixel centre of the warp's strip: columns
-// x0 + 0.5 .. x0 + 15.5, rows y0 + 0.5 .. y0 + 1.5? Entries outside would only be skipped, so
-// leaving them out changes no decision.
-__device__ __forceinline__ bool reaches_strip(float4 A, float ex, float ey, float x0, float y0) {
-  return A.x + ex >= x0 + 0.5f && A.x - ex <= x0 + 15.5f && A.y + ey >= y0 + 0.5f &&
-         A.y - ey <= y0 + 1.5f;
+// projection, conservatively widened) reach a pixel centre of the warp's block: columns
+// x0 + 0.5 .. x0 + kWarpW - 0.5, rows y0 + 0.5 .. y0 + kWarpH - 0.5? Entries outside would only
+// be skipped, so leaving them out changes no decision.
+__device__ __forceinline__ bool reaches_block(float4 A, float ex, float ey, float x0, float y0) {
+  return A.x + ex >= x0 + 0.5f && A.x - ex <= x0 + ((float)kWarpW - 0.5f) &&
+         A.y + ey >= y0 + 0.5f && A.y - ey <= y0 + ((float)kWarpH - 0.5f);
 }
 
 // position of the composited-entry mask of (global tile gt, chunk starting at list position p):

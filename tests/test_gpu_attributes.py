@@ -1,7 +1,8 @@
 """Attribute render, map scatter and scalar attribution on the GPU (through the C ABI) against
 the oracle (fp32 decisions). The attribute render takes the render's fp32 weights in the same
 order as the oracle's fp32 mode, so it must agree bit for bit; the scatters add fp32 products in
-fp64 in another order: 1e-5 relative per Gaussian (floor 1e-6 x the largest row)."""
+fp64 in another order: 1e-5 relative per Gaussian (floor 1e-6 x the largest row) for non-negative
+maps, 1e-5 of the scatter of |m| for signed ones."""
 import numpy as np
 import pytest
 
@@ -85,7 +86,12 @@ def test_scatter_matches_oracle_and_is_the_adjoint(C):
     f = rng.normal(size=(sc.G, C)).astype(np.float32)
     g = _gpu(sc, None, feats=f, pixel_map=m)
     p, L, r = _oracle(sc)
-    _rows_close(g["S"], O.scatter(p, L, r, m, sc.H, sc.W, "f"))
+    S = O.scatter(p, L, r, m, sc.H, sc.W, "f")
+    # a signed map's sum can be far smaller than its terms; the fp32 products and the warp's fp32
+    # partial sums round relative to the terms, so the bar is relative to the scatter of |m|
+    S_abs = O.scatter(p, L, r, np.abs(m), sc.H, sc.W, "f")
+    err = np.abs(g["S"].astype(np.float64) - S) / np.maximum(S_abs, 1e-30)
+    assert err.max(initial=0) <= 1e-5, (err.max(), np.unravel_index(err.argmax(), err.shape))
     lhs = float((m.astype(np.float64) * g["F"]).sum())
     rhs = float((g["S"].astype(np.float64) * f).sum())
     assert abs(lhs - rhs) <= 1e-5 * float(np.abs(m * g["F"]).sum())
