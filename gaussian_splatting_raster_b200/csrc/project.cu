@@ -33,11 +33,22 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
           unsigned long long* __restrict__ ntot) {
   constexpr int D = (DEG + 1) * (DEG + 1);
   constexpr int NSH = D * 3;
-  // shared memory: the block's SH coefficients [kProjThreads][NSH], then the views [V][20]
+  // shared memory: the block's SH coefficients [kProjThreads][NSH], the views [V][20], then per
+  // view the tangent-clamp limits and the camera centre [V][5] (view constants, computed once)
   extern __shared__ float s_dyn[];
   float* s_sh = s_dyn;
   float* s_views = s_dyn + kProjThreads * NSH;
+  float* s_vc = s_views + V * 20;
   for (int i = threadIdx.x; i < V * 20; i += blockDim.x) s_views[i] = views_in[i];
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    const float* vw = views_in + 20 * v;
+    s_vc[5 * v] = 1.3f * ((0.5f * (float)W) / vw[16]);
+    s_vc[5 * v + 1] = 1.3f * ((0.5f * (float)H) / vw[17]);
+    // camera centre -R^T t
+    s_vc[5 * v + 2] = -(vw[0] * vw[3] + vw[4] * vw[7] + vw[8] * vw[11]);
+    s_vc[5 * v + 3] = -(vw[1] * vw[3] + vw[5] * vw[7] + vw[9] * vw[11]);
+    s_vc[5 * v + 4] = -(vw[2] * vw[3] + vw[6] * vw[7] + vw[10] * vw[11]);
+  }
   // coalesced staging of the block's contiguous SH rows (they dominate the input bytes)
   {
     const long long g0 = (long long)blockIdx.x * kProjThreads;
@@ -98,6 +109,8 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
       for (int j = 0; j < 3; ++j) Sw[i][j] = M[i][0] * M[j][0] + M[i][1] * M[j][1] + M[i][2] * M[j][2];
     o = 1.0f / (1.0f + exp_cw(-a_logit));
   }
+  // the render's early-skip bound: exponents below it give alpha < 1/255 (per Gaussian)
+  const float cut = logf((1.0f / 255.0f) / o) - 1e-3f;
 
   for (int v = 0; v < V; ++v) {
     const size_t i = (size_t)v * G + g;
@@ -129,8 +142,7 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
 #pragma unroll
         for (int b = 0; b < 3; ++b) Sc[a][b] = T1[a][0] * Rv[b][0] + T1[a][1] * Rv[b][1] + T1[a][2] * Rv[b][2];
       const float u = x / z, vv = y / z;
-      const float limx = 1.3f * ((0.5f * (float)W) / fx);
-      const float limy = 1.3f * ((0.5f * (float)H) / fy);
+      const float limx = s_vc[5 * v], limy = s_vc[5 * v + 1];
       const float uc = fminf(limx, fmaxf(-limx, u));
       const float vc = fminf(limy, fmaxf(-limy, vv));
       const float J00 = fx / z, J02 = -(fx * uc) / z;
@@ -160,13 +172,11 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
       const int y1 = clamp_tile(floorf((my + rr) / 16.0f) + 1.0f, TY);
       if (x1 <= x0 || y1 <= y0) vis = false;
       if (vis) {
-        // view direction (world) from the camera centre -R^T t
-        const float cam0 = -(Rv[0][0] * t[0] + Rv[1][0] * t[1] + Rv[2][0] * t[2]);
-        const float cam1 = -(Rv[0][1] * t[0] + Rv[1][1] * t[1] + Rv[2][1] * t[2]);
-        const float cam2 = -(Rv[0][2] * t[0] + Rv[1][2] * t[1] + Rv[2][2] * t[2]);
-        const float d0 = m0 - cam0, d1 = m1 - cam1, d2 = m2 - cam2;
-        const float len = sqrtf(d0 * d0 + d1 * d1 + d2 * d2);
-        const float dx = d0 / len, dy = d1 / len, dz = d2 / len;
+        // view direction (world) from the camera centre; the SH colour only has to agree with
+        // the oracle's to a few ulp, so one reciprocal square root instead of three divisions
+        const float d0 = m0 - s_vc[5 * v + 2], d1 = m1 - s_vc[5 * v + 3], d2 = m2 - s_vc[5 * v + 4];
+        const float il = rsqrtf(d0 * d0 + d1 * d1 + d2 * d2);
+        const float dx = d0 * il, dy = d1 * il, dz = d2 * il;
         float B[16];
         sh_poly<DEG>(dx, dy, dz, B);
         float col[3];
@@ -184,7 +194,6 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
         // (bounding box of every pixel centre that can reach alpha >= 1/255), widened by
         // 1 % + 0.05 px -- far more than fp32 rounding of the exponent (or of det Q when
         // det Q > 1e-4 qa qc) can move its boundary; nearly singular conics get an unbounded box
-        const float cut = logf((1.0f / 255.0f) / o) - 1e-3f;
         float ex = -1.0f, ey = -1.0f;
         if (cut < 0.0f) {
           const float dq = qa * qc - qb * qb;
@@ -247,7 +256,7 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
   const int tok = prof_begin(w, st, SPLAT_K_PROJECT);
 #define SPLAT_PROJ(DEG)                                                                          \
   {                                                                                              \
-    const size_t smem = ((size_t)kProjThreads * 3 * (DEG + 1) * (DEG + 1) + (size_t)w.V * 20) * \
+    const size_t smem = ((size_t)kProjThreads * 3 * (DEG + 1) * (DEG + 1) + (size_t)w.V * 25) * \
                         sizeof(float);                                                           \
     if (smem > 48 * 1024 &&                                                                      \
         cudaFuncSetAttribute(k_project<DEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
