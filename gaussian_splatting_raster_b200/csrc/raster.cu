@@ -199,14 +199,17 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
           const float den = T * (1.0f - al);
           const float w = al * T;
           const float c0 = Bq.z, c1 = Bq.w, c2 = Cq.x;
-          // suffix numerators C_hat - P - w c per channel, in the recovery equation's order
-          // (their cancellation dominates the fp32 error of C+, so they are formed exactly as
-          // written), then one correctly rounded reciprocal of the denominator
+          // suffix numerators C_hat - P - w c per channel, in the recovery equation's order and
+          // unfused like the render's colour sum, so that at the last entry C_hat - P - w c is
+          // exactly the background term (their cancellation dominates the fp32 error of C+);
+          // then one reciprocal of the denominator (T (1 - alpha) >= 1e-6 here, so the fast
+          // reciprocal's relative error of a few 1e-8 is far inside the tokens' bar)
           const float n0 = (Ch0 - P0) - w * c0;
           const float n1 = (Ch1 - P1) - w * c1;
           const float n2 = (Ch2 - P2) - w * c2;
-          const float inv = __frcp_rn(den + 1e-12f);
-          const float rho = r0 * (c0 - n0 * inv) + r1 * (c1 - n1 * inv) + r2 * (c2 - n2 * inv);
+          const float inv = __fdividef(1.0f, den + 1e-12f);
+          const float rho = fmaf(r0, fmaf(-n0, inv, c0),
+                                 fmaf(r1, fmaf(-n1, inv, c1), r2 * fmaf(-n2, inv, c2)));
           const bool Ma = (den >= 1e-4f) && (al < 0.99f);
           x[0] = w;
           x[1] = w * r0;
