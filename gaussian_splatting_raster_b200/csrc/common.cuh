@@ -54,6 +54,28 @@ constexpr float kC6 = (float)(1.0 / 720.0);
 constexpr float kC7 = (float)(1.0 / 5040.0);
 }  // namespace cw
 
+// exp of x in [-87, 88] without range checks (exp_cw below adds them), bit-identical to exp_cw
+// there. k = round-half-even(x log2e) is taken by adding and subtracting 1.5 * 2^23 (exact for
+// |x log2e| < 2^22; the addition itself rounds half to even), whose bits also hold k as an
+// integer: no float-to-integer conversions.
+__device__ __forceinline__ float exp_cw_core(float x) {
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23, bits 0x4B400000
+  const float t = x * cw::kLog2e + kMagic;
+  const float k = t - kMagic;
+  const int ki = __float_as_int(t) - 0x4B400000;
+  // k * ln2_hi is exact (16-bit ln2_hi, |k| < 2^8), so one fused step rounds as x - k ln2_hi does
+  const float r = fmaf(-k, cw::kLn2Hi, x) - k * cw::kLn2Lo;
+  float p = cw::kC7;
+  p = fmaf(p, r, cw::kC6);
+  p = fmaf(p, r, cw::kC5);
+  p = fmaf(p, r, cw::kC4);
+  p = fmaf(p, r, cw::kC3);
+  p = fmaf(p, r, cw::kC2);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  return p * __int_as_float((ki + 127) << 23);
+}
+
 __device__ __forceinline__ float exp_cw(float x) {
   if (x != x) return x;
   if (!(x > -87.0f)) return 0.0f;

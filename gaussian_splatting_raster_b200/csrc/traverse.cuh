@@ -67,7 +67,8 @@ __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, flo
   e.use = false;
   e.alpha = 0.0f;
   if (pw > 0.0f || pw < cut) return e;
-  const float al = fminf(0.99f, Bq.y * exp_cw(pw));
+  // here cut <= pw <= 0 and cut >= log(1/255) - 1e-3 (opacity <= 1), inside exp_cw_core's range
+  const float al = fminf(0.99f, Bq.y * exp_cw_core(pw));
   if (al < kAlphaMin) return e;
   e.alpha = al;
   e.use = true;
