@@ -182,8 +182,9 @@ def recorded_traffic(kernel: str, workload: str):
     return int(d["dram_read_bytes"]) + int(d["dram_write_bytes"])
 
 
-def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
-    """Bytes each kernel group must move by its definition (unique inputs + outputs)."""
+def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dict:
+    """Bytes each kernel group must move by its definition (unique inputs + outputs), per step;
+    depth_passes = the number of depth-digit passes the binning ran."""
     G, V, H, W, d = sc.G, sc.V, sc.H, sc.W, sc.d
     px = V * H * W
     TX, TY = (W + 15) // 16, (H + 15) // 16
@@ -193,11 +194,13 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int) -> dict:
 
         # one depth-digit pass per launch over every (v, g): histogram reads the keys, the
         # scatter reads key + index and writes both
-        "depth_hist": V * G * 4,
-        "depth_scatter": V * G * 16,
-        # rectangles gathered into depth order (16 B in, 16 B + count out), the counts scanned
-        # (4 B in, 8 B out), instances (tile, g) emitted (rectangle, index, offset in; 8 B out)
-        "emit": V * G * (16 + 20 + 12 + 28) + n_inst * 8,
+        "depth_hist": depth_passes * V * G * 4,
+        # per pass keys and values in and out (the last writes no keys)
+        "depth_scatter": depth_passes * V * G * 16 - V * G * 4,
+        # rectangles gathered into depth order (order 4 B + rectangle 16 B in, 16 B + count out),
+        # the counts scanned (4 B in, 8 B out), instances (tile, g) emitted (rectangle, index,
+        # offset in; 8 B out)
+        "emit": V * G * (20 + 20 + 12 + 28) + n_inst * 8,
         "tile_hist": n_inst * 4,
         "tile_scatter": n_inst * (4 + 4 + 4),
         # gather 36 B per list entry staged, write C_hat, T, n, last
@@ -570,7 +573,9 @@ def main():
 
     # ---- roofline of the dominant kernel ------------------------------------------------------
     peaks = load_peaks()
-    ab = algorithmic_bytes(sc, n_total, pairs)
+    per_kernel0 = {k: v for k, v in kern.items() if v[1] > 0}
+    dp = per_kernel0.get("depth_scatter", (0.0, 0))[1] // max(args.steps, 1)
+    ab = algorithmic_bytes(sc, n_total, pairs, dp)
     per_kernel = {k: {"ms_per_step": v[0] / args.steps, "launches": v[1]}
                   for k, v in kern.items() if v[1] > 0}
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms_per_step"])
