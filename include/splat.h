@@ -27,8 +27,10 @@
  *     On error, splat_last_error(ws) returns a NUL-terminated message owned by the workspace,
  *     valid until the next call on it. Argument errors are detected before any work is
  *     enqueued. A workspace is not thread-safe: one host thread at a time.
- *   - Call order per problem: splat_project -> splat_bin_sort -> splat_render ->
- *     splat_score_replay. A call made out of order returns SPLAT_ERR_STATE.
+ *   - Call order per problem: splat_project -> splat_bin_sort -> splat_render, then any of
+ *     splat_score_replay, splat_score_partials, splat_backward, splat_render_features,
+ *     splat_scatter, splat_attribution (each reads the last render). A call made out of order
+ *     returns SPLAT_ERR_STATE.
  */
 #ifndef SPLAT_H
 #define SPLAT_H
@@ -89,8 +91,9 @@ int splat_project(splat_ws* ws, const float* means, const float* log_scales, con
 /*
  * Stage 1 tile binning and contributor sort ([P1] Stage 1 step 1): every visible (g, v) emits one
  * instance per tile of its rectangle; each tile's list is ordered by (camera depth z, Gaussian
- * index) -- a stable counting sort by tile followed by a per-tile radix sort of the fp32 depth
- * bits. The lists stay in the workspace ([P1] Stage 1: not exposed as a per-pixel tensor).
+ * index) -- a stable radix sort of one fp32 depth key per (view, Gaussian) over the key bits
+ * that vary, emission of the instances in that order, and one stable counting sort by tile.
+ * The lists stay in the workspace ([P1] Stage 1: not exposed as a per-pixel tensor).
  * n_instances_out (HOST pointer, may be NULL) receives V counts. Synchronises with the stream
  * once (the counts size the sort).
  */
@@ -118,7 +121,7 @@ int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int*
  * masks with M_alpha = (T (1 - alpha) >= 1e-4 and alpha < 0.99) and M_color (colour clamp
  * inactive), forms r = C_hat - C_obs, rho = <r, c - C+>, w = T alpha and accumulates per (g, v)
  *   q = sum w, sum w r, sum M_alpha w rho, sum M_alpha w rho (p - mu2D)
- * (CTA-level reduction per tile, then fp64 atomics). Then, per Gaussian over the views where it
+ * (reduction over each warp's pixels, then fp64 atomics). Then, per Gaussian over the views where it
  * is visible: q_gv = 1e-6 + q, q_g = 1e-6 + sum_v q_gv, gamma = q_gv / q_g, and
  *   tokens[g] = [ b_mu (3) = sum_v gamma J^T Sigma2D^-1 Sd / q_gv,
  *                 s_alpha (1) = sum_v gamma (1 - o) Sa / q_gv,
