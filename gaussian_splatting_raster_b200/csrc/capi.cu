@@ -293,7 +293,7 @@ int splat_backward(splat_ws* ws, const float* obs, const float* log_scales, cons
   Workspace& w = ws->w;
   w.err.clear();
   if (w.stage < 3) return fail(w, SPLAT_ERR_STATE, "splat_backward before splat_render");
-  if (!grad_raw && !grad_detached && !grad_support && !grad_pscale)
+  if (w.G > 0 && !grad_raw && !grad_detached && !grad_support && !grad_pscale)
     return fail(w, SPLAT_ERR_INVALID_ARG, "splat_backward: no output requested");
   int rc;
   const bool none = w.G == 0;

@@ -171,7 +171,7 @@ int splat_finalize_partials(const float* partials, int G, int sh_degree, float l
  * S = diag(exp(log_scale)) and R from the normalised quaternion. Output rows, fp32 [G, 11 + 3d]:
  *   [dL/dmean (3), dL/dlog_scale (3), dL/dquat (w, x, y, z), dL/dopacity_logit,
  *    dL/dsh (3d, index k*3 + channel)]
- * for the variants (each pointer may be NULL; at least one must be given):
+ * for the variants (each pointer may be NULL; at least one must be given when G > 0):
  *   grad_raw      the derivative itself;
  *   grad_detached the derivative with the paths the score operators stop cut (Sigma2D and the
  *                 view direction): mean through the projected centre only, zero scale and

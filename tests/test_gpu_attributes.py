@@ -160,3 +160,19 @@ def test_call_errors():
                            torch.zeros((1, 32, 32, 65), device="cuda"))
     assert e.value.code == -1
     ws.close()
+
+
+def test_all_culled_and_empty():
+    """Nothing composited: attributes render 0 and scatter 0; G = 0 works."""
+    sc = scenes.tiny_scene(3, 5, 20, 24, V=2)
+    sc.means[:, 2] = -1.0
+    m = np.ones((2, 20, 24, 2), np.float32)
+    g = _gpu(sc, np.zeros((2, 20, 24, 3), np.float32), feats=np.ones((5, 3), np.float32),
+             pixel_map=m)
+    assert (g["F"] == 0).all() and (g["S"] == 0).all() and (g["A"][:, :2] == 0).all()
+    sc0 = scenes.tiny_scene(3, 1, 20, 24, V=1)
+    for name in ("means", "log_scales", "quats", "opac", "sh"):
+        setattr(sc0, name, getattr(sc0, name)[:0])
+    g0 = _gpu(sc0, np.zeros((1, 20, 24, 3), np.float32), feats=np.zeros((0, 4), np.float32),
+              pixel_map=np.ones((1, 20, 24, 4), np.float32))
+    assert (g0["F"] == 0).all() and g0["S"].shape == (0, 4) and g0["A"].shape == (0, 3)

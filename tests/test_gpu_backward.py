@@ -143,3 +143,18 @@ def test_backward_call_errors():
         ws.backward(obs, ds.log_scales, ds.quats, ds.sh)
     assert e.value.code == -1
     ws.close()
+
+
+def test_backward_all_culled_and_empty():
+    """Every Gaussian behind the cameras: zero gradients; G = 0: empty outputs, no error."""
+    sc = scenes.tiny_scene(3, 5, 20, 24, V=2)
+    sc.means[:, 2] = -1.0
+    obs = np.random.default_rng(1).uniform(0, 1, (2, 20, 24, 3)).astype(np.float32)
+    g = PU.gpu_backward(sc, obs)
+    for k in PU.GRAD_VARIANTS:
+        assert (g[k] == 0).all()
+    sc0 = scenes.tiny_scene(3, 1, 20, 24, V=1)
+    for name in ("means", "log_scales", "quats", "opac", "sh"):
+        setattr(sc0, name, getattr(sc0, name)[:0])
+    g0 = PU.gpu_backward(sc0, np.zeros((1, 20, 24, 3), np.float32))
+    assert g0["raw"].shape == (0, 23)
