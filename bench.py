@@ -482,6 +482,12 @@ def main():
     barrier(world)
     clocks = sampler.stop() if sampler else None
     launches = ws.launch_count - launches_before
+    # device memory in use after the timed steps (the workspace grows only during warm-up, so
+    # this is the steady-state peak): library workspace + torch tensors + CUDA context
+    free_b, total_b = torch.cuda.mem_get_info(dev)
+    vram = {"device_used_gb": (total_b - free_b) / 1e9,
+            "torch_reserved_gb": torch.cuda.memory_reserved(dev) / 1e9,
+            "device_total_gb": total_b / 1e9}
     kern = ws.profile_read(reset=True)
     ws.profile(False)
 
@@ -629,7 +635,7 @@ def main():
             "render_ms_per_step": render_ms, f"{second[0]}_ms_per_step": replay_ms,
             f"{second[0]}_over_render": replay_ms / render_ms if render_ms else None,
             "gpu_launches": int(launches), "per_kernel": per_kernel,
-            "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "vram": vram,
         }
         os.write(json_fd, (json.dumps(line) + "\n").encode())
     ws.close()
