@@ -71,6 +71,8 @@ def parse():
                     help="views: each rank renders and replays its block of the views and one "
                          "reduce-scatter of the per-Gaussian partial sums gives every rank its "
                          "slice of tokens (strong scaling over views; score path only)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="fixed-point integer accumulation (bitwise reproducible sums)")
     ap.add_argument("--views", type=int, default=0,
                     help="view-count scaling: the ReSplat-scale layout with this many context and "
                          "target views at 256x448 (overrides --config)")
@@ -414,6 +416,8 @@ def main():
     else:
         ws = runner.workspace_for(ds)
     out = runner.alloc_outputs(ds)
+    if args.deterministic:
+        ws.deterministic(True)
 
     stream = torch.cuda.current_stream()
     l2_flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -626,6 +630,8 @@ def main():
             "config": {"workload": workload_name(args, sc), "gaussians": sc.G, "views": sc.V,
                        "height": sc.H, "width": sc.W, "sh_degree": sc.sh_degree,
                        "path": PATHS[args.path],
+                       "accumulation": "fixed-point (deterministic)" if args.deterministic
+                       else "fp64 atomics",
                        "instances_per_step": n_total, "pairs_per_step": pairs,
                        "l2": "256 MiB buffer written between timed steps",
                        "parallelism": (f"views x{world} (reduce-scatter of per-Gaussian partials)"

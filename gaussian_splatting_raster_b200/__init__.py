@@ -28,6 +28,7 @@ EXPORTS = [
     "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
     "splat_sort_depths_noalloc", "splat_score_partials", "splat_finalize_partials",
     "splat_backward", "splat_render_features", "splat_scatter", "splat_attribution",
+    "splat_set_deterministic",
 ]
 
 
@@ -97,6 +98,8 @@ def load_library(path: str | None = None):
     L.splat_scatter.restype = I
     L.splat_attribution.argtypes = [V, V, V, V]
     L.splat_attribution.restype = I
+    L.splat_set_deterministic.argtypes = [V, I]
+    L.splat_set_deterministic.restype = I
     if path is None:
         _lib = L
     return L
@@ -298,6 +301,11 @@ class Workspace:
     @property
     def launch_count(self) -> int:
         return int(self._L.splat_launch_count(self._h))
+
+    def deterministic(self, enable: bool = True):
+        """Fixed-point integer accumulation in the replay and the backward: bitwise reproducible
+        tokens and gradients (off by default)."""
+        self._check(self._L.splat_set_deterministic(self._h, 1 if enable else 0))
 
     def profile(self, enable: bool = True):
         """Bracket every kernel with CUDA events (per-kernel device time)."""

@@ -66,7 +66,8 @@ int alloc(Workspace& w, T** p, size_t n, const char* what) {
 void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
-                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.accb, w.sacc};
+                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.accb, w.sacc,
+                 w.acc_fix, w.accb_fix};
   for (void* p : dev)
     if (p) cudaFree(p);
   if (w.h_vstart) cudaFreeHost(w.h_vstart);
@@ -452,6 +453,12 @@ int splat_pair_count(splat_ws* ws, long long* pairs, void* stream) {
 }
 
 long long splat_launch_count(const splat_ws* ws) { return ws ? ws->w.launches : 0; }
+
+int splat_set_deterministic(splat_ws* ws, int enable) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  ws->w.det = enable != 0;
+  return SPLAT_OK;
+}
 
 int splat_profile_enable(splat_ws* ws, int enable) {
   if (!ws) return SPLAT_ERR_INVALID_ARG;

@@ -136,6 +136,7 @@ struct Workspace {
   // current problem
   int G = 0, V = 0, H = 0, W = 0, deg = 0, TX = 0, TY = 0, nt = 0;
   int stage = 0;  // 0 empty, 1 projected, 2 binned, 3 rendered, 4 replayed
+  bool det = false;  // fixed-point integer accumulation (bitwise reproducible sums)
   long long launches = 0;
 
   // per (v, g)
@@ -146,6 +147,11 @@ struct Workspace {
   double* acc = nullptr;     // [V*G*8]
   double* accb = nullptr;    // [max_V*max_G*10] renderer-backward sums, allocated on first use
   double* sacc = nullptr;    // [G*C] scatter sums, grown on demand
+  // deterministic mode: 128-bit fixed-point (low, high) words of the replay / backward sums
+  unsigned long long* acc_fix = nullptr;
+  size_t acc_fix_cap = 0;
+  unsigned long long* accb_fix = nullptr;
+  size_t accb_fix_cap = 0;
   size_t sacc_cap = 0;
   float* views = nullptr;    // [V*20]: viewmat (16) + intrinsics (4)
   int* last = nullptr;       // [V*H*W]

@@ -36,6 +36,8 @@
 // atomics per (Gaussian, warp-strip). The SH block never enters the pixel loop: M_color w (B (x) r)
 // factors into M_color B (x) (sum w r); the mean block Sigma^-1 (sum w rho d) is formed once per
 // (Gaussian, view) in finalisation.
+#include <algorithm>
+
 #include "traverse.cuh"
 
 namespace splat {
@@ -127,12 +129,62 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   }
 }
 
+// Deterministic accumulation: each warp's partial sum x (fp32) is turned into the signed 128-bit
+// fixed-point integer X = x 2^60 (exact for |x| >= 2^-37; smaller values are truncated toward
+// zero, the same way every run) and added with two 64-bit integer atomics -- the low word, then
+// the high word plus the carry out of this particular low-word add. Integer addition does not
+// depend on order, so the sums are the same bits on every run; the total of the carries is exactly
+// the number of times the low word wrapped. A last pass turns (high, low) into a double.
+constexpr int kFixShift = 60;
+
+__device__ __forceinline__ void add_fixed(unsigned long long* lohi, float x) {
+  const unsigned int bits = __float_as_uint(x);
+  const int ex = (int)((bits >> 23) & 0xffu);
+  if (ex == 0 || ex == 0xff) return;  // zero, subnormal (below 2^-126) or not finite
+  const unsigned long long m = (bits & 0x7fffffu) | 0x800000u;  // x = +-m 2^(ex - 150)
+  const int sh = ex - 150 + kFixShift;                           // X = m 2^sh
+  unsigned long long lo, hi;
+  if (sh >= 64) {
+    lo = 0ull;
+    hi = sh - 64 < 40 ? m << (sh - 64) : 0ull;  // |x| >= 2^67 does not occur here
+  } else if (sh > 40) {
+    lo = m << sh;
+    hi = m >> (64 - sh);
+  } else if (sh >= 0) {
+    lo = m << sh;
+    hi = 0ull;
+  } else {
+    lo = -sh < 24 ? m >> (-sh) : 0ull;
+    hi = 0ull;
+  }
+  if (bits >> 31) {  // two's complement of the 128-bit value
+    lo = ~lo + 1ull;
+    hi = ~hi + (lo == 0ull ? 1ull : 0ull);
+  }
+  if (lo) {
+    const unsigned long long old = atomicAdd(lohi, lo);
+    if (old + lo < old) hi += 1ull;  // carry out of this add
+  }
+  if (hi) atomicAdd(lohi + 1, hi);
+}
+
+// (high, low) pairs -> doubles: dst[k] = (hi 2^64 + lo) 2^-60
+__global__ void k_fixed_to_double(const unsigned long long* __restrict__ src,
+                                  double* __restrict__ dst, long long n) {
+  for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
+       k += (long long)gridDim.x * blockDim.x) {
+    const unsigned long long lo = src[2 * k], hi = src[2 * k + 1];
+    dst[k] = ldexp((double)(long long)hi, 64 - kFixShift) + ldexp((double)lo, -kFixShift);
+  }
+}
+
+template <bool kDet>
 __global__ void __launch_bounds__(kThreads)
 k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
          const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
          const float* __restrict__ img, const float* __restrict__ obs,
          const int* __restrict__ last, const uint32_t* __restrict__ umask,
-         double* __restrict__ acc) {
+         double* __restrict__ acc, unsigned long long* __restrict__ acc_fix) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
@@ -234,7 +286,12 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
         x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
         if ((lane & 3) == 0 && slot < 7 && x[0] != 0.0f)
-          atomicAdd(accv + (size_t)wg[q] * kAccN + slot, (double)x[0]);
+        {
+          if constexpr (kDet)
+            add_fixed(acc_fix + 2 * (((size_t)v * G + wg[q]) * kAccN + slot), x[0]);
+          else
+            atomicAdd(accv + (size_t)wg[q] * kAccN + slot, (double)x[0]);
+        }
       }
     }
     __syncwarp();
@@ -251,13 +308,14 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
 // and, where alpha = o G is not clamped, h = ga alpha, the pixel adds to its (view, Gaussian)
 //   q += w, w r (3), h, h (dx, dy), h (dx^2, dx dy, dy^2)     (w = T alpha)
 // by a 16-slot transpose-reduction per entry and fp64 atomics from the ten lanes holding sums.
+template <bool kDet>
 __global__ void __launch_bounds__(kThreads)
 k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
            const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
            const float* __restrict__ img, const float* __restrict__ Tfin,
            const float* __restrict__ bgp, const float* __restrict__ obs,
            const int* __restrict__ last, const uint32_t* __restrict__ umask,
-           double* __restrict__ accb) {
+           double* __restrict__ accb, unsigned long long* __restrict__ accb_fix) {
   const int t = blockIdx.x, v = blockIdx.y;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
@@ -349,7 +407,12 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         tr_step<1>(x, lane & 2, 2);
         x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
         if ((lane & 1) == 0 && slot < kAccBN && x[0] != 0.0f)
-          atomicAdd(accv + (size_t)wg[q] * kAccBN + slot, (double)x[0]);
+        {
+          if constexpr (kDet)
+            add_fixed(accb_fix + 2 * (((size_t)v * G + wg[q]) * kAccBN + slot), x[0]);
+          else
+            atomicAdd(accv + (size_t)wg[q] * kAccBN + slot, (double)x[0]);
+        }
       }
     }
     __syncwarp();
@@ -377,32 +440,93 @@ int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int
   return check_launch(w, "render kernel");
 }
 
+// the fixed-point (high, low) words of deterministic mode: allocated on first use, sized for the
+// workspace maxima, cleared before every pass
+static int fix_buffer(Workspace& w, unsigned long long** buf, size_t& cap, int nslot,
+                      cudaStream_t st) {
+  const size_t need = (size_t)w.max_V * w.max_G * nslot * 2;
+  if (cap < need) {
+    if (*buf) cudaFree(*buf);
+    *buf = nullptr;
+    cap = 0;
+    if (cudaMalloc(buf, need * sizeof(unsigned long long)) != cudaSuccess) {
+      *buf = nullptr;
+      cudaGetLastError();
+      return set_err(w, SPLAT_ERR_OOM, "deterministic sums: device allocation failed");
+    }
+    cap = need;
+  }
+  const cudaError_t e =
+      cudaMemsetAsync(*buf, 0, (size_t)w.V * w.G * nslot * 2 * sizeof(unsigned long long), st);
+  if (e != cudaSuccess)
+    return set_err(w, SPLAT_ERR_CUDA, std::string("deterministic sums clear: ") +
+                                          cudaGetErrorString(e));
+  return SPLAT_OK;
+}
+
+static int fix_to_double(Workspace& w, const unsigned long long* src, double* dst, int nslot,
+                         cudaStream_t st) {
+  const long long n = (long long)w.V * w.G * nslot;
+  k_fixed_to_double<<<(unsigned)std::min<long long>((n + 255) / 256, 8 * 148), 256, 0, st>>>(
+      src, dst, n);
+  return check_launch(w, "fixed-point conversion kernel");
+}
+
 int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
   const int tok = prof_begin(w, st, SPLAT_K_REPLAY);
-  if (w.G > 0) {
+  int rc = SPLAT_OK;
+  const bool det = w.det && w.G > 0;
+  if (det) {
+    rc = fix_buffer(w, &w.acc_fix, w.acc_fix_cap, kAccN, st);
+  } else if (w.G > 0) {
     cudaError_t e = cudaMemsetAsync(w.acc, 0, (size_t)w.V * w.G * kAccN * sizeof(double), st);
     if (e != cudaSuccess)
-      return set_err(w, SPLAT_ERR_CUDA, std::string("accumulator clear: ") + cudaGetErrorString(e));
+      rc = set_err(w, SPLAT_ERR_CUDA, std::string("accumulator clear: ") + cudaGetErrorString(e));
   }
-  dim3 grid(w.nt, w.V);
-  k_replay<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX, w.nt,
-                                      w.img, obs, w.last, w.umask, w.acc);
+  if (!rc) {
+    dim3 grid(w.nt, w.V);
+    if (det)
+      k_replay<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,
+                                                w.nt, w.img, obs, w.last, w.umask, w.acc,
+                                                w.acc_fix);
+    else
+      k_replay<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,
+                                                 w.nt, w.img, obs, w.last, w.umask, w.acc,
+                                                 nullptr);
+    rc = check_launch(w, "replay kernel");
+  }
+  if (!rc && det) rc = fix_to_double(w, w.acc_fix, w.acc, kAccN, st);
   prof_end(w, st, tok);
-  return check_launch(w, "replay kernel");
+  return rc;
 }
 
 int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {
   const int tok = prof_begin(w, st, SPLAT_K_BACKWARD);
-  if (w.G > 0) {
+  int rc = SPLAT_OK;
+  const bool det = w.det && w.G > 0;
+  if (det) {
+    rc = fix_buffer(w, &w.accb_fix, w.accb_fix_cap, kAccBN, st);
+  } else if (w.G > 0) {
     cudaError_t e = cudaMemsetAsync(w.accb, 0, (size_t)w.V * w.G * kAccBN * sizeof(double), st);
     if (e != cudaSuccess)
-      return set_err(w, SPLAT_ERR_CUDA, std::string("backward sums clear: ") + cudaGetErrorString(e));
+      rc = set_err(w, SPLAT_ERR_CUDA, std::string("backward sums clear: ") +
+                                          cudaGetErrorString(e));
   }
-  dim3 grid(w.nt, w.V);
-  k_backward<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX, w.nt,
-                                        w.img, w.Tfin, w.bg, obs, w.last, w.umask, w.accb);
+  if (!rc) {
+    dim3 grid(w.nt, w.V);
+    if (det)
+      k_backward<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,
+                                                  w.nt, w.img, w.Tfin, w.bg, obs, w.last,
+                                                  w.umask, w.accb, w.accb_fix);
+    else
+      k_backward<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W,
+                                                   w.TX, w.nt, w.img, w.Tfin, w.bg, obs, w.last,
+                                                   w.umask, w.accb, nullptr);
+    rc = check_launch(w, "backward kernel");
+  }
+  if (!rc && det) rc = fix_to_double(w, w.accb_fix, w.accb, kAccBN, st);
   prof_end(w, st, tok);
-  return check_launch(w, "backward kernel");
+  return rc;
 }
 
 int launch_pair_count(Workspace& w, cudaStream_t st) {

@@ -212,6 +212,18 @@ int splat_render_features(splat_ws* ws, const float* feats, int C, float* out, v
 int splat_scatter(splat_ws* ws, const float* map, int C, float* out, void* stream);
 int splat_attribution(splat_ws* ws, const float* obs, float* out, void* stream);
 
+/*
+ * Deterministic accumulation (a library option; the pages have none). With enable != 0 the score
+ * replay (splat_score_replay, splat_score_partials) and the renderer backward add their per-(view,
+ * Gaussian) sums as 128-bit fixed-point integers (units of 2^-60; two 64-bit integer atomics with
+ * an exact carry), which do not depend on the order of the adds: tokens and gradients are then
+ * the same bits on every run, which exposes any race between runs. Off by default (fp64 atomics:
+ * results agree to rounding order). The first deterministic call allocates 16 bytes per sum of
+ * the workspace maxima (SPLAT_ERR_OOM when that fails); each call then clears them and adds one
+ * conversion pass. Takes effect from the next call.
+ */
+int splat_set_deterministic(splat_ws* ws, int enable);
+
 /* ---------------------------------------------------------------------------------------------
  * Inspection calls (tests and benchmarks; not part of the render/replay path). They copy
  * workspace state into caller-owned DEVICE buffers on `stream`, or report host-side counters.
