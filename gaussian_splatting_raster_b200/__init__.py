@@ -10,7 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-from .build import LIB, build  # noqa: F401
+from .build import LIB, LIB_CHECKED, build  # noqa: F401
 
 __all__ = ["Workspace", "SplatError", "load_library", "LIB", "build", "token_dim",
            "partials_dim", "grad_dim", "finalize_partials"]
@@ -28,7 +28,7 @@ EXPORTS = [
     "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
     "splat_sort_depths_noalloc", "splat_score_partials", "splat_finalize_partials",
     "splat_backward", "splat_render_features", "splat_scatter", "splat_attribution",
-    "splat_set_deterministic",
+    "splat_set_deterministic", "splat_check_status", "splat_checked_build",
 ]
 
 
@@ -100,6 +100,10 @@ def load_library(path: str | None = None):
     L.splat_attribution.restype = I
     L.splat_set_deterministic.argtypes = [V, I]
     L.splat_set_deterministic.restype = I
+    L.splat_check_status.argtypes = [V, V]
+    L.splat_check_status.restype = I
+    L.splat_checked_build.argtypes = []
+    L.splat_checked_build.restype = I
     if path is None:
         _lib = L
     return L
@@ -156,8 +160,11 @@ class Workspace:
     """Library-owned workspace (records, tile lists, accumulators) for problems up to the given
     maxima. Calls enqueue on the current torch CUDA stream unless one is passed."""
 
-    def __init__(self, max_G: int, max_V: int, max_H: int, max_W: int, max_sh_degree: int = 3):
-        self._L = load_library()
+    def __init__(self, max_G: int, max_V: int, max_H: int, max_W: int, max_sh_degree: int = 3,
+                 lib=None):
+        """lib: a loaded library to use instead of the default one (e.g. the checked build,
+        load_library(LIB_CHECKED))."""
+        self._L = lib if lib is not None else load_library()
         h = ctypes.c_void_p()
         rc = self._L.splat_ws_create(ctypes.byref(h), max_G, max_V, max_H, max_W, max_sh_degree)
         if rc != 0:
@@ -301,6 +308,11 @@ class Workspace:
     @property
     def launch_count(self) -> int:
         return int(self._L.splat_launch_count(self._h))
+
+    def check_status(self, stream=None):
+        """Raise SplatError(BOUNDS) when a bounds check of the checked build failed since the
+        last call (synchronises the stream; a no-op check in the release build)."""
+        self._check(self._L.splat_check_status(self._h, _stream(stream)))
 
     def deterministic(self, enable: bool = True):
         """Fixed-point integer accumulation in the replay and the backward: bitwise reproducible

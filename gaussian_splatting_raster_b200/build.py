@@ -8,6 +8,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsplat.so")
+LIB_CHECKED = os.path.join(PKG, "libsplat_checked.so")  # bounds-checked build (-DSPLAT_CHECKED)
 SOURCES = ["capi.cu", "project.cu", "binning.cu", "raster.cu", "finalize.cu", "backward.cu",
            "attributes.cu", "noalloc.cu"]
 
@@ -31,27 +32,30 @@ def sources() -> list[str]:
     return [os.path.join(CSRC, s) for s in SOURCES]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "traverse.cuh"),
                         os.path.join(ROOT, "include", "splat.h")]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *sources(), "-o", LIB + ".tmp"]
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Compile libsplat.so (or, with checked=True, the bounds-checked libsplat_checked.so)."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(lib):
+        return lib
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *sources(), "-o", lib + ".tmp"]
+    if checked:
+        cmd.insert(1, "-DSPLAT_CHECKED")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
     import sys
-    build(force=True, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force=True, verbose="-v" in sys.argv, checked="--checked" in sys.argv))

@@ -20,6 +20,9 @@
 #include "traverse.cuh"
 
 namespace splat {
+
+SPLAT_BOUNDS_WORD(bounds_word_attributes)
+
 namespace {
 
 constexpr int kMaxPass = 16;  // channels per traversal
@@ -59,16 +62,21 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   for (int base = 0; base < wmax; base += 32) {
     uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
     if (!bits) continue;  // warp-uniform
+    bool bad = false;
     if ((bits >> lane) & 1u) {
       const uint32_t g = ids[s + base + lane];
-      const float4* r = recv + (size_t)g * kRecF4;
-      wa[lane] = r[0];
-      wb[lane] = r[1];
-      wc[lane] = r[2].y;
-      const float* fg = feats + (size_t)g * C + c0;
+      bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
+      if (!bad) {
+        const float4* r = recv + (size_t)g * kRecF4;
+        wa[lane] = r[0];
+        wb[lane] = r[1];
+        wc[lane] = r[2].y;
+        const float* fg = feats + (size_t)g * C + c0;
 #pragma unroll
-      for (int k = 0; k < CB; ++k) wf[lane * CB + k] = k < nc ? fg[k] : 0.0f;
+        for (int k = 0; k < CB; ++k) wf[lane * CB + k] = k < nc ? fg[k] : 0.0f;
+      }
     }
+    if (kChecked) bits &= ~__ballot_sync(0xffffffffu, bad);
     __syncwarp();
     while (bits) {
       const int q = __ffs(bits) - 1;
@@ -144,14 +152,19 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   for (int base = 0; base < wmax; base += 32) {
     uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
     if (!bits) continue;  // warp-uniform
+    bool bad = false;
     if ((bits >> lane) & 1u) {
       const uint32_t g = ids[s + base + lane];
-      const float4* r = recv + (size_t)g * kRecF4;
-      wa[lane] = r[0];
-      wb[lane] = r[1];
-      wc[lane] = r[2].y;
-      wg[lane] = g;
+      bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
+      if (!bad) {
+        const float4* r = recv + (size_t)g * kRecF4;
+        wa[lane] = r[0];
+        wb[lane] = r[1];
+        wc[lane] = r[2].y;
+        wg[lane] = g;
+      }
     }
+    if (kChecked) bits &= ~__ballot_sync(0xffffffffu, bad);
     __syncwarp();
     while (bits) {
       const int q = __ffs(bits) - 1;

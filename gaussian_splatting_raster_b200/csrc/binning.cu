@@ -22,6 +22,9 @@
 #include "common.cuh"
 
 namespace splat {
+
+SPLAT_BOUNDS_WORD(bounds_word_binning)
+
 namespace {
 
 // ---------------------------------------------------------------------------------------------
@@ -254,6 +257,8 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
   }
   __syncthreads();
   const uint32_t lt = lanemask_lt();
+  const unsigned long long lim =
+      sg.per_view >= 0 ? (unsigned long long)sg.per_view * sg.V : (unsigned long long)sg.vstart[sg.V];
   for (long long base = wb; base < we; base += 32 * kUnroll) {
     uint32_t key[kUnroll], val[kUnroll];
 #pragma unroll
@@ -270,8 +275,10 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
       const uint32_t peers = __match_any_sync(0xffffffffu, bk);
       if (ok) {
         const uint32_t pos = cnt[bk] + __popc(peers & lt);
-        if (kout) kout[pos] = key[u];
-        vout[pos] = val[u];
+        if (in_bounds(pos, lim, &g_bounds_word)) {
+          if (kout) kout[pos] = key[u];
+          vout[pos] = val[u];
+        }
       }
       __syncwarp();
       if (ok && lane == __ffs(peers) - 1) cnt[bk] += __popc(peers);
@@ -304,10 +311,13 @@ __global__ void k_emit(const int4* __restrict__ rect_s, const uint32_t* __restri
   const long long v = k / G;
   const uint32_t g = order ? order[k] : (uint32_t)(k - v * G);
   long long pos = offs[k];
+  const unsigned long long lim = kChecked ? (unsigned long long)offs[VG] : 0ull;
   for (int ty = rc.y; ty < rc.w; ++ty)
     for (int tx = rc.x; tx < rc.z; ++tx) {
-      inst_tile[pos] = (uint32_t)(ty * TX + tx);
-      inst_g[pos] = g;
+      if (in_bounds(pos, lim, &g_bounds_word)) {
+        inst_tile[pos] = (uint32_t)(ty * TX + tx);
+        inst_g[pos] = g;
+      }
       ++pos;
     }
 }

@@ -454,6 +454,20 @@ int splat_pair_count(splat_ws* ws, long long* pairs, void* stream) {
 
 long long splat_launch_count(const splat_ws* ws) { return ws ? ws->w.launches : 0; }
 
+int splat_check_status(splat_ws* ws, void* stream) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  Workspace& w = ws->w;
+  w.err.clear();
+  cudaStream_t st = (cudaStream_t)stream;
+  const unsigned int bad = splat::bounds_word_raster(st) | splat::bounds_word_binning(st) |
+                           splat::bounds_word_attributes(st);
+  if (bad & 0x80000000u) return fail(w, SPLAT_ERR_CUDA, "reading the bounds-check words failed");
+  if (bad) return fail(w, SPLAT_ERR_BOUNDS, "a device-side bounds check failed (access skipped)");
+  return SPLAT_OK;
+}
+
+int splat_checked_build(void) { return splat::kChecked ? 1 : 0; }
+
 int splat_set_deterministic(splat_ws* ws, int enable) {
   if (!ws) return SPLAT_ERR_INVALID_ARG;
   ws->w.det = enable != 0;

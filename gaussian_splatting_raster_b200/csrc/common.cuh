@@ -128,6 +128,40 @@ __device__ __forceinline__ void sh_poly(float x, float y, float z, float* B) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Checked build (-DSPLAT_CHECKED): the kernels bounds-check every index that comes from data
+// (list entries, scatter positions); a failed check sets a bit in the error word of its source
+// file and the access is skipped; splat_check_status reads and clears the words. In the release
+// build the checks compile to nothing.
+// ---------------------------------------------------------------------------------------------
+#ifdef SPLAT_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+__device__ __forceinline__ bool in_bounds(unsigned long long i, unsigned long long n,
+                                          unsigned int* word) {
+  if (!kChecked || i < n) return true;
+  atomicOr(word, 1u);
+  return false;
+}
+
+// one error word per source file, with a host accessor that reads and clears it (stream-ordered)
+#define SPLAT_BOUNDS_WORD(accessor)                                                         \
+  static __device__ unsigned int g_bounds_word;                                             \
+  unsigned int accessor(cudaStream_t st) {                                                   \
+    unsigned int v = 0, z = 0;                                                               \
+    if (!kChecked) return 0;                                                                 \
+    if (cudaMemcpyFromSymbolAsync(&v, g_bounds_word, sizeof v, 0, cudaMemcpyDeviceToHost,   \
+                                  st) != cudaSuccess ||                                      \
+        cudaMemcpyToSymbolAsync(g_bounds_word, &z, sizeof z, 0, cudaMemcpyHostToDevice,     \
+                                st) != cudaSuccess ||                                        \
+        cudaStreamSynchronize(st) != cudaSuccess)                                           \
+      return 0x80000000u;                                                                    \
+    return v;                                                                                \
+  }
+
+// ---------------------------------------------------------------------------------------------
 // workspace
 // ---------------------------------------------------------------------------------------------
 struct Workspace {
@@ -271,6 +305,9 @@ int launch_features(Workspace& w, const float* feats, int C, float* out, cudaStr
 int launch_scatter(Workspace& w, const float* map, const float* obs, int C, float* out,
                    cudaStream_t st);
 int launch_pair_count(Workspace& w, cudaStream_t st);
+unsigned int bounds_word_raster(cudaStream_t st);
+unsigned int bounds_word_binning(cudaStream_t st);
+unsigned int bounds_word_attributes(cudaStream_t st);
 int binning_configure(Workspace& w);
 
 // reduce-then-scan over n int32 values into int64 exclusive prefixes (out has n + 1 entries; the

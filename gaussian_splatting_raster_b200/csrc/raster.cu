@@ -41,6 +41,9 @@
 #include "traverse.cuh"
 
 namespace splat {
+
+SPLAT_BOUNDS_WORD(bounds_word_raster)
+
 namespace {
 
 __global__ void __launch_bounds__(kThreads)
@@ -77,12 +80,15 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     const long long k = base + lane;
     bool hit = false;
     if (k < e) {
-      const float4* r = recv + (size_t)ids[k] * kRecF4;
-      const float4 a = r[0], b = r[1], c = r[2];  // c = (colour b, cut, ex, ey)
-      wa[lane] = a;
-      wb[lane] = b;
-      wc[lane] = make_float2(c.x, c.y);
-      hit = reaches_block(a, c.z, c.w, x0f, y0f);
+      const uint32_t gi = ids[k];
+      if (in_bounds(gi, (unsigned)G, &g_bounds_word)) {
+        const float4* r = recv + (size_t)gi * kRecF4;
+        const float4 a = r[0], b = r[1], c = r[2];  // c = (colour b, cut, ex, ey)
+        wa[lane] = a;
+        wb[lane] = b;
+        wc[lane] = make_float2(c.x, c.y);
+        hit = reaches_block(a, c.z, c.w, x0f, y0f);
+      }
     }
     uint32_t bits = __ballot_sync(0xffffffffu, hit);
     uint32_t ubits = 0u;
@@ -226,15 +232,20 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   for (int base = 0; base < wmax; base += 32) {
     uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
     if (!bits) continue;  // warp-uniform
+    bool bad = false;
     if ((bits >> lane) & 1u) {
       const uint32_t g = ids[s + base + lane];
-      const float4* r = recv + (size_t)g * kRecF4;
-      const float4 c = r[2];
-      wa[lane] = r[0];
-      wb[lane] = r[1];
-      wc[lane] = make_float2(c.x, c.y);
-      wg[lane] = g;
+      bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
+      if (!bad) {
+        const float4* r = recv + (size_t)g * kRecF4;
+        const float4 c = r[2];
+        wa[lane] = r[0];
+        wb[lane] = r[1];
+        wc[lane] = make_float2(c.x, c.y);
+        wg[lane] = g;
+      }
     }
+    if (kChecked) bits &= ~__ballot_sync(0xffffffffu, bad);
     __syncwarp();
     while (bits) {  // warp-uniform: entries some pixel of this warp composited, in list order
       const int q = __ffs(bits) - 1;
@@ -352,15 +363,20 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   for (int base = (wmax - 1) & ~31; base >= 0; base -= 32) {
     uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
     if (!bits) continue;  // warp-uniform
+    bool bad = false;
     if ((bits >> lane) & 1u) {
       const uint32_t g = ids[s + base + lane];
-      const float4* r = recv + (size_t)g * kRecF4;
-      const float4 c = r[2];
-      wa[lane] = r[0];
-      wb[lane] = r[1];
-      wc[lane] = make_float2(c.x, c.y);
-      wg[lane] = g;
+      bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
+      if (!bad) {
+        const float4* r = recv + (size_t)g * kRecF4;
+        const float4 c = r[2];
+        wa[lane] = r[0];
+        wb[lane] = r[1];
+        wc[lane] = make_float2(c.x, c.y);
+        wg[lane] = g;
+      }
     }
+    if (kChecked) bits &= ~__ballot_sync(0xffffffffu, bad);
     __syncwarp();
     while (bits) {  // warp-uniform, from the highest list position down
       const int q = 31 - __clz(bits);

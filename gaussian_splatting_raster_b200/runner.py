@@ -84,5 +84,5 @@ def render_and_backward(ws: Workspace, ds: DeviceScene, obs, out: Outputs, grads
     return n
 
 
-def workspace_for(ds: DeviceScene) -> Workspace:
-    return Workspace(max(ds.G, 1), ds.V, ds.H, ds.W, ds.deg)
+def workspace_for(ds: DeviceScene, lib=None) -> Workspace:
+    return Workspace(max(ds.G, 1), ds.V, ds.H, ds.W, ds.deg, lib=lib)

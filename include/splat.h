@@ -224,6 +224,17 @@ int splat_attribution(splat_ws* ws, const float* obs, float* out, void* stream);
  */
 int splat_set_deterministic(splat_ws* ws, int enable);
 
+/*
+ * Checked build (the library compiled with -DSPLAT_CHECKED, libsplat_checked.so; a library option,
+ * the pages have none): every index the kernels take from data -- tile-list entries, scatter and
+ * emission positions -- is bounds-checked; a failed check skips the access and sets a device
+ * error word. splat_check_status synchronises `stream`, reads and clears the words and returns
+ * SPLAT_ERR_BOUNDS when any check failed since the last call (always SPLAT_OK in the release
+ * build). splat_checked_build returns 1 in the checked build, 0 otherwise.
+ */
+int splat_check_status(splat_ws* ws, void* stream);
+int splat_checked_build(void);
+
 /* ---------------------------------------------------------------------------------------------
  * Inspection calls (tests and benchmarks; not part of the render/replay path). They copy
  * workspace state into caller-owned DEVICE buffers on `stream`, or report host-side counters.
