@@ -1,11 +1,12 @@
 // Device helpers shared by the kernels that traverse the per-tile contributor lists (render,
 // score replay, renderer backward, attribute render and scatter): the rasteriser's per-entry alpha
-// with its skip rules, the warp-strip reach test, the composited-entry mask index, and the
+// with its skip rules, the warp-block reach test, the composited-entry mask index, and the
 // transpose-reduction that sums per-entry values over a warp's 32 pixels.
 //
 // Source: "Research Proposal: Renderer Score Tokens for Recurrent Gaussian Splatting",
 // "Two-Stage Algorithm" (both passes walk the same tile bins in the same order with the same
-// decisions; per-Gaussian contributions are reduced within a tile before global atomics).
+// decisions; per-Gaussian contributions are reduced on chip -- here over each warp of a tile --
+// before global atomics).
 #pragma once
 #include "common.cuh"
 
