@@ -259,31 +259,51 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
   const uint32_t lt = lanemask_lt();
   const unsigned long long lim =
       sg.per_view >= 0 ? (unsigned long long)sg.per_view * sg.V : (unsigned long long)sg.vstart[sg.V];
-  for (long long base = wb; base < we; base += 32 * kUnroll) {
+  // 32-bit offsets from the warp's first item; whole groups without tail checks, then the tail
+  const uint32_t* kp = keys + wb;
+  const uint32_t* vp = vals ? vals + wb : nullptr;
+  const int n = we > wb ? (int)(we - wb) : 0;
+  const uint32_t vbase = (uint32_t)(wb - r.vbeg);
+  const int nfull = n / (32 * kUnroll) * (32 * kUnroll);
+  for (int b = 0; b < nfull; b += 32 * kUnroll) {
     uint32_t key[kUnroll], val[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const long long i = base + 32 * u + lane;
-      const bool ok = i < we;
-      key[u] = ok ? keys[i] : 0u;
-      val[u] = ok ? (vals ? vals[i] : (uint32_t)(i - r.vbeg)) : 0u;
+      const int o = b + 32 * u + lane;
+      key[u] = kp[o];
+      val[u] = vp ? vp[o] : vbase + (uint32_t)o;
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const bool ok = base + 32 * u + lane < we;
-      const uint32_t bk = ok ? (key[u] >> shift) & mask : (0x80000000u | lane);
+      const uint32_t bk = (key[u] >> shift) & mask;
       const uint32_t peers = __match_any_sync(0xffffffffu, bk);
-      if (ok) {
-        const uint32_t pos = cnt[bk] + __popc(peers & lt);
-        if (in_bounds(pos, lim, &g_bounds_word)) {
-          if (kout) kout[pos] = key[u];
-          vout[pos] = val[u];
-        }
+      const uint32_t pos = cnt[bk] + __popc(peers & lt);
+      if (in_bounds(pos, lim, &g_bounds_word)) {
+        if (kout) kout[pos] = key[u];
+        vout[pos] = val[u];
       }
       __syncwarp();
-      if (ok && lane == __ffs(peers) - 1) cnt[bk] += __popc(peers);
+      if (lane == __ffs(peers) - 1) cnt[bk] += __popc(peers);
       __syncwarp();
     }
+  }
+  for (int b = nfull; b < n; b += 32) {
+    const int o = b + lane;
+    const bool ok = o < n;
+    const uint32_t key = ok ? kp[o] : 0u;
+    const uint32_t val = ok ? (vp ? vp[o] : vbase + (uint32_t)o) : 0u;
+    const uint32_t bk = ok ? (key >> shift) & mask : (0x80000000u | lane);
+    const uint32_t peers = __match_any_sync(0xffffffffu, bk);
+    if (ok) {
+      const uint32_t pos = cnt[bk] + __popc(peers & lt);
+      if (in_bounds(pos, lim, &g_bounds_word)) {
+        if (kout) kout[pos] = key;
+        vout[pos] = val;
+      }
+    }
+    __syncwarp();
+    if (ok && lane == __ffs(peers) - 1) cnt[bk] += __popc(peers);
+    __syncwarp();
   }
 }
 
