@@ -183,25 +183,37 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-constexpr int kUnroll = 4;       // 32-item batches whose loads are issued together (ranking)
-constexpr int kCountUnroll = 8;  // 32-item batches whose loads are issued together (counting)
+constexpr int kUnroll = 16;      // 32-item batches whose loads are issued together (ranking)
+constexpr int kCountUnroll = 32; // 32-item batches whose loads are issued together (counting)
+constexpr int kHistUnroll = 32;  // the same for the histogram kernel
 
-// per-warp bucket counts of the items [wb, we) into cnt (shared memory): the loads of
-// kCountUnroll batches are issued together, then each lane adds its items with shared-memory
-// atomics (counts do not depend on the order of the adds)
+// per-warp bucket counts of the items [wb, we) into cnt (shared memory): the loads of UNR
+// batches are issued together, then each lane adds its items with shared-memory atomics (counts
+// do not depend on the order of the adds); whole groups without tail checks, then the tail
+template <int UNR>
 __device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, int shift,
                                             uint32_t mask, long long wb, long long we,
                                             uint32_t* cnt) {
   const int lane = threadIdx.x & 31;
-  for (long long base = wb; base < we; base += 32 * kCountUnroll) {
-    uint32_t bk[kCountUnroll];
+  const uint32_t* kp = keys + wb;
+  const int n = we > wb ? (int)(we - wb) : 0;
+  const int nfull = n / (32 * UNR) * (32 * UNR);
+  for (int b = 0; b < nfull; b += 32 * UNR) {
+    uint32_t bk[UNR];
 #pragma unroll
-    for (int u = 0; u < kCountUnroll; ++u) {
-      const long long i = base + 32 * u + lane;
-      bk[u] = i < we ? (keys[i] >> shift) & mask : 0xffffffffu;
+    for (int u = 0; u < UNR; ++u) bk[u] = (kp[b + 32 * u + lane] >> shift) & mask;
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) atomicAdd(cnt + bk[u], 1u);
+  }
+  if (nfull < n) {
+    uint32_t bk[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int o = nfull + 32 * u + lane;
+      bk[u] = o < n ? (kp[o] >> shift) & mask : 0xffffffffu;
     }
 #pragma unroll
-    for (int u = 0; u < kCountUnroll; ++u)
+    for (int u = 0; u < UNR; ++u)
       if (bk[u] != 0xffffffffu) atomicAdd(cnt + bk[u], 1u);
   }
 }
@@ -217,7 +229,7 @@ k_count_hist(const uint32_t* __restrict__ keys, int shift, uint32_t mask, int nb
   const int warp = threadIdx.x >> 5;
   const long long wb = r.beg + (long long)warp * (sg.chunk / kBinWarps);
   const long long we = min(wb + (long long)(sg.chunk / kBinWarps), r.end);
-  warp_counts(keys, shift, mask, wb, we, s_cnt + warp * nbk);
+  warp_counts<kHistUnroll>(keys, shift, mask, wb, we, s_cnt + warp * nbk);
   __syncthreads();
   int* h = hist + (size_t)nbk * r.b0;
   for (int t = threadIdx.x; t < nbk; t += blockDim.x) {
@@ -242,7 +254,7 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
   uint32_t* cnt = s_cnt + warp * nbk;
   const long long wb = r.beg + (long long)warp * (sg.chunk / kBinWarps);
   const long long we = min(wb + (long long)(sg.chunk / kBinWarps), r.end);
-  warp_counts(keys, shift, mask, wb, we, cnt);
+  warp_counts<kCountUnroll>(keys, shift, mask, wb, we, cnt);
   __syncthreads();
   // per bucket: global start of this block's run, then one sub-run per warp in warp order
   const int* h = hist_scan + (size_t)nbk * r.b0;

@@ -36,8 +36,9 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
   // shared memory: the block's SH coefficients [kProjThreads][NSH], the views [V][20], then per
   // view the tangent-clamp limits and the camera centre [V][5] (view constants, computed once)
   extern __shared__ float s_dyn[];
+  constexpr int SP = NSH | 1;  // odd per-thread stride: conflict-free shared-memory reads
   float* s_sh = s_dyn;
-  float* s_views = s_dyn + kProjThreads * NSH;
+  float* s_views = s_dyn + kProjThreads * SP;
   float* s_vc = s_views + V * 20;
   for (int i = threadIdx.x; i < V * 20; i += blockDim.x) s_views[i] = views_in[i];
   for (int v = threadIdx.x; v < V; v += blockDim.x) {
@@ -57,11 +58,24 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
     const float* src = sh + g0 * NSH;
     if ((((uintptr_t)src) & 15) == 0) {
       const float4* s4 = reinterpret_cast<const float4*>(src);
-      for (int k = threadIdx.x; k < nf / 4; k += blockDim.x)
-        reinterpret_cast<float4*>(s_sh)[k] = s4[k];
-      for (int k = (nf / 4) * 4 + threadIdx.x; k < nf; k += blockDim.x) s_sh[k] = src[k];
+      for (int k = threadIdx.x; k < nf / 4; k += blockDim.x) {
+        const float4 f = s4[k];
+        const float e[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int L = 4 * k + c, t = L / NSH;
+          s_sh[t * SP + (L - t * NSH)] = e[c];
+        }
+      }
+      for (int L = (nf / 4) * 4 + threadIdx.x; L < nf; L += blockDim.x) {
+        const int t = L / NSH;
+        s_sh[t * SP + (L - t * NSH)] = src[L];
+      }
     } else {
-      for (int k = threadIdx.x; k < nf; k += blockDim.x) s_sh[k] = src[k];
+      for (int L = threadIdx.x; L < nf; L += blockDim.x) {
+        const int t = L / NSH;
+        s_sh[t * SP + (L - t * NSH)] = src[L];
+      }
     }
   }
   __syncthreads();
@@ -73,7 +87,7 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
   const float q0 = quats[4 * g], q1 = quats[4 * g + 1], q2 = quats[4 * g + 2],
               q3 = quats[4 * g + 3];
   const float a_logit = opac[g];
-  const float* shc = s_sh + threadIdx.x * NSH;
+  const float* shc = s_sh + threadIdx.x * SP;
 
   bool ok = isfinite(m0) && isfinite(m1) && isfinite(m2) && isfinite(l0) && isfinite(l1) &&
             isfinite(l2) && isfinite(q0) && isfinite(q1) && isfinite(q2) && isfinite(q3) &&
@@ -256,7 +270,7 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
   const int tok = prof_begin(w, st, SPLAT_K_PROJECT);
 #define SPLAT_PROJ(DEG)                                                                          \
   {                                                                                              \
-    const size_t smem = ((size_t)kProjThreads * 3 * (DEG + 1) * (DEG + 1) + (size_t)w.V * 25) * \
+    const size_t smem = ((size_t)kProjThreads * ((3 * (DEG + 1) * (DEG + 1)) | 1) + (size_t)w.V * 25) * \
                         sizeof(float);                                                           \
     if (smem > 48 * 1024 &&                                                                      \
         cudaFuncSetAttribute(k_project<DEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \

@@ -91,12 +91,11 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       }
     }
     uint32_t bits = __ballot_sync(0xffffffffu, hit);
-    uint32_t ubits = 0u;
+    uint32_t lbits = 0u;  // entries of this chunk this lane composited
     __syncwarp();
     while (bits) {  // warp-uniform: entries that can reach this warp's rows, in list order
       const int q = __ffs(bits) - 1;
       bits &= bits - 1;
-      bool comp = false;
       if (!done) {
         const float4 A = wa[q], Bq = wb[q];
         const float2 Cq = wc[q];
@@ -115,12 +114,12 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
             T = Tn;
             ++n;
             lst = (int)(base - s) + q + 1;
-            comp = true;
+            lbits |= 1u << q;
           }
         }
       }
-      if (__any_sync(0xffffffffu, comp)) ubits |= 1u << q;
     }
+    const uint32_t ubits = __reduce_or_sync(0xffffffffu, lbits);
     if (lane == 0) umask[chunk_index(base, gt) * 8 + warp] = ubits;
     __syncwarp();
   }
