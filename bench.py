@@ -452,9 +452,14 @@ def main():
             return n
         return runner.render_and_score(ws, ds_, obs_, out_)
 
+    last_out = {}
+
     def step():
         if shard:
-            return sharding.sharded_tokens(ws, ds, obs, 1.0)[3]
+            r = sharding.sharded_tokens(ws, ds, obs, 1.0)
+            last_out["o"] = r[2]
+            return r[3]
+        last_out["o"] = out
         return run(ds, obs, out, grads, attr_out)
 
     for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
@@ -463,6 +468,8 @@ def main():
         n_inst = step()
     torch.cuda.synchronize()
     pairs = ws.pair_count()
+    # composited pairs: sum over this rank's pixels of the entries that contributed (n_contrib)
+    composited = int(last_out["o"].n_contrib.sum(dtype=torch.int64).item())
     n_total = int(sum(n_inst))
 
     # ---- timed region: device time per step (CUDA events), L2 flushed between steps ----------
@@ -504,6 +511,7 @@ def main():
     pairs_per_s = pairs * args.steps * (world if not shard else 1) / (total_ms * 1e-3)
     if shard:  # pairs of all ranks' views
         pairs_per_s = pairs_sum_over_ranks(pairs, world) * args.steps / (total_ms * 1e-3)
+        composited = pairs_sum_over_ranks(composited, world)
 
     # ---- end to end through the public API with host buffers ----------------------------------
     # Every step copies its inputs from pinned host memory and its outputs (tokens, image, final
@@ -633,12 +641,14 @@ def main():
                        "accumulation": "fixed-point (deterministic)" if args.deterministic
                        else "fp64 atomics",
                        "instances_per_step": n_total, "pairs_per_step": pairs,
+                       "composited_pairs_per_step": composited,
                        "l2": "256 MiB buffer written between timed steps",
                        "parallelism": (f"views x{world} (reduce-scatter of per-Gaussian partials)"
                                        if shard else f"replicas x{world}")},
             "pairs_per_s": pairs_per_s,
             "ms_view": ms_per_step / sc.V,
             "render_ms_per_step": render_ms, f"{second[0]}_ms_per_step": replay_ms,
+            "render_ms_per_view": render_ms / sc.V, f"{second[0]}_ms_per_view": replay_ms / sc.V,
             f"{second[0]}_over_render": replay_ms / render_ms if render_ms else None,
             "gpu_launches": int(launches), "per_kernel": per_kernel,
             "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "vram": vram,

@@ -332,26 +332,54 @@ __global__ void k_gather_rects(const int4* __restrict__ rect, const uint32_t* __
   cnt_s[k] = (rc.z - rc.x) * (rc.w - rc.y);
 }
 
-// instances (tile, g) in depth order
-__global__ void k_emit(const int4* __restrict__ rect_s, const uint32_t* __restrict__ order,
-                       const long long* __restrict__ offs, long long VG, int G, int TX,
-                       uint32_t* __restrict__ inst_tile, uint32_t* __restrict__ inst_g) {
-  const long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= VG) return;
-  const int4 rc = rect_s[k];
-  if (rc.z <= rc.x || rc.w <= rc.y) return;
-  const long long v = k / G;
-  const uint32_t g = order ? order[k] : (uint32_t)(k - v * G);
-  long long pos = offs[k];
+// instances (tile, g) in depth order. One warp per 32 consecutive entries: the lanes write the
+// warp's output range in order, 32 consecutive positions at a time (coalesced, and balanced
+// however many tiles each entry covers); each position finds its entry by a binary search over
+// the 32 entry offsets, then its tile from its index inside the entry's rectangle (row-major).
+__global__ void __launch_bounds__(256)
+k_emit(const int4* __restrict__ rect_s, const uint32_t* __restrict__ order,
+       const long long* __restrict__ offs, long long VG, int G, int TX,
+       uint32_t* __restrict__ inst_tile, uint32_t* __restrict__ inst_g) {
+  const int lane = threadIdx.x & 31;
+  const long long k0 = (long long)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  if (k0 >= VG) return;  // warp-uniform
+  const long long k = k0 + lane;
+  const bool ok = k < VG;
+  int4 rc = make_int4(0, 0, 0, 0);
+  uint32_t g = 0;
+  if (ok) {
+    rc = rect_s[k];
+    const long long v = k / G;
+    g = order ? order[k] : (uint32_t)(k - v * G);
+  }
+  const long long start = offs[k0];
+  const int total = (int)(offs[min(k0 + 32, VG)] - start);
+  // entry start relative to the warp's range; lanes past the end sit at the end (never chosen)
+  const int rel = ok ? (int)(offs[k] - start) : total;
+  const int wdt = rc.z - rc.x;
   const unsigned long long lim = kChecked ? (unsigned long long)offs[VG] : 0ull;
-  for (int ty = rc.y; ty < rc.w; ++ty)
-    for (int tx = rc.x; tx < rc.z; ++tx) {
+  for (int b = 0; b < total; b += 32) {
+    const int p = b + lane;
+    // the last entry whose start is <= p (starts are non-decreasing; entry 0 starts at 0)
+    int j = 0;
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1)
+      if (__shfl_sync(0xffffffffu, rel, j + s) <= p) j += s;
+    const int x0 = __shfl_sync(0xffffffffu, rc.x, j);
+    const int y0 = __shfl_sync(0xffffffffu, rc.y, j);
+    const int wj = __shfl_sync(0xffffffffu, wdt, j);
+    const int rj = __shfl_sync(0xffffffffu, rel, j);
+    const uint32_t gj = __shfl_sync(0xffffffffu, g, j);
+    if (p < total) {
+      const int li = p - rj;  // wj > 0: an entry with an empty rectangle owns no position
+      const int dy = (int)((unsigned)li / (unsigned)wj);
+      const long long pos = start + p;
       if (in_bounds(pos, lim, &g_bounds_word)) {
-        inst_tile[pos] = (uint32_t)(ty * TX + tx);
-        inst_g[pos] = g;
+        inst_tile[pos] = (uint32_t)((y0 + dy) * TX + x0 + (li - dy * wj));
+        inst_g[pos] = gj;
       }
-      ++pos;
     }
+  }
 }
 
 __global__ void k_tile_ranges(const int* __restrict__ hist_scan, const long long* __restrict__ vstart,

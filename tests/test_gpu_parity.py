@@ -78,6 +78,23 @@ def test_long_tile_list_uses_global_sort():
     assert o["lists"]["n"] > 8192
 
 
+def test_mixed_footprints_in_one_warp():
+    """Instance emission with very uneven rectangles side by side in depth order: Gaussians that
+    cover every tile of a ragged 7 x 10 tile grid, culled ones (no instance) and small ones,
+    G not a multiple of 32."""
+    sc = scenes.tiny_scene(21, 1061, 100, 150, V=2, deg=1, log_scale_mean=math.log(0.02))
+    rng = np.random.default_rng(5)
+    big = rng.choice(sc.G, 90, replace=False)
+    sc.log_scales[big] = math.log(3.0)  # footprint larger than the image
+    culled = rng.choice(np.setdiff1d(np.arange(sc.G), big), 200, replace=False)
+    sc.means[culled, 2] = -1.0
+    obs = np.random.default_rng(2).uniform(0, 1, (2, 100, 150, 3)).astype(np.float32)
+    g, o = _full_check(sc, obs)
+    rect = o["proj"]["rect"]
+    counts = (rect[..., 2] - rect[..., 0]) * (rect[..., 3] - rect[..., 1])
+    assert counts.max() == 70 and (counts == 0).sum() >= 2 * 200
+
+
 def test_empty_scene_and_all_culled():
     sc = scenes.tiny_scene(3, 5, 20, 24, V=2)
     sc.means[:, 2] = -1.0  # all behind the cameras
