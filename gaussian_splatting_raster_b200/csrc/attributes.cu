@@ -44,7 +44,7 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float s_cut[kThreads];
-  __shared__ float s_f[kThreads * CB];
+  __shared__ __align__(16) float s_f[kThreads * CB];
   float4* wa = s_a + warp * 32;
   float4* wb = s_b + warp * 32;
   float* wc = s_cut + warp * 32;
@@ -85,8 +85,19 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         const Entry E = eval_entry(wa[q], wb[q], wc[q], px, py);
         if (E.use) {
           const float w = E.alpha * T;
+          if constexpr (CB % 2 == 0) {  // two products per packed multiply, scalar sums
+            const float2 ww = make_float2(w, w);
+            const float2* f2 = reinterpret_cast<const float2*>(wf + q * CB);
 #pragma unroll
-          for (int k = 0; k < CB; ++k) F[k] = F[k] + w * wf[q * CB + k];
+            for (int k = 0; k < CB; k += 2) {
+              const float2 p = __fmul2_rn(ww, f2[k / 2]);
+              F[k] = F[k] + p.x;
+              F[k + 1] = F[k + 1] + p.y;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < CB; ++k) F[k] = F[k] + w * wf[q * CB + k];
+          }
           T = T * (1.0f - E.alpha);
         }
       }

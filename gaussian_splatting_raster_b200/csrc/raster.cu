@@ -108,8 +108,9 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
             const float wgt = E.alpha * T;
             // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is
             // then exactly the background term, and the suffix recovery sees no rounding mismatch
-            C0 = C0 + wgt * Bq.z;
-            C1 = C1 + wgt * Bq.w;
+            const float2 wc01 = __fmul2_rn(make_float2(wgt, wgt), make_float2(Bq.z, Bq.w));
+            C0 = C0 + wc01.x;
+            C1 = C1 + wc01.y;
             C2 = C2 + wgt * Cq.x;
             T = Tn;
             ++n;
@@ -225,7 +226,10 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const int wmax = __reduce_max_sync(0xffffffffu, lst);  // entries this warp must traverse
   const float4* recv = rec + (size_t)v * G * kRecF4;
   double* accv = acc + (size_t)v * G * kAccN;
-  float T = 1.0f, P0 = 0.0f, P1 = 0.0f, P2 = 0.0f;  // transmittance, prefix colour
+  float T = 1.0f, P2 = 0.0f;  // transmittance, prefix colour (channels 0 and 1 packed)
+  float2 P01 = make_float2(0.0f, 0.0f);
+  const float2 Ch01 = make_float2(Ch0, Ch1), r01 = make_float2(r0, r1);
+  const float2 m1 = make_float2(-1.0f, -1.0f);
   const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
   const int slot = (lane >> 2) & 7;  // value index this lane holds after the reduction
   for (int base = 0; base < wmax; base += 32) {
@@ -266,26 +270,35 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
           // exactly the background term (their cancellation dominates the fp32 error of C+);
           // then one reciprocal of the denominator (T (1 - alpha) >= 1e-6 here, so the fast
           // reciprocal's relative error of a few 1e-8 is far inside the tokens' bar)
-          const float n0 = (Ch0 - P0) - w * c0;
-          const float n1 = (Ch1 - P1) - w * c1;
-          const float n2 = (Ch2 - P2) - w * c2;
+          const float2 ww = make_float2(w, w);
+          const float2 c01 = make_float2(c0, c1);
+          const float2 wc01 = __fmul2_rn(ww, c01);
+          const float wc2 = w * c2;
+          // C_hat - P for channels 0 and 1 in one op (fma(P, -1, C_hat) rounds the difference
+          // once); the products w c are subtracted by scalar ops
+          const float2 cp01 = __ffma2_rn(P01, m1, Ch01);
+          const float n0 = cp01.x - wc01.x;
+          const float n1 = cp01.y - wc01.y;
+          const float n2 = (Ch2 - P2) - wc2;
           const float inv = __fdividef(1.0f, den + 1e-12f);
-          const float rho = fmaf(r0, fmaf(-n0, inv, c0),
-                                 fmaf(r1, fmaf(-n1, inv, c1), r2 * fmaf(-n2, inv, c2)));
+          const float2 a01 = __ffma2_rn(make_float2(n0, n1), make_float2(-inv, -inv), c01);
+          const float rho = fmaf(r0, a01.x, fmaf(r1, a01.y, r2 * fmaf(-n2, inv, c2)));
           const bool Ma = (den >= 1e-4f) && (al < 0.99f);
+          const float2 wr01 = __fmul2_rn(ww, r01);
           x[0] = w;
-          x[1] = w * r0;
-          x[2] = w * r1;
+          x[1] = wr01.x;
+          x[2] = wr01.y;
           x[3] = w * r2;
           if (Ma) {
             const float wr = w * rho;
+            const float2 wd = __fmul2_rn(make_float2(wr, wr), make_float2(E.dx, E.dy));
             x[4] = wr;
-            x[5] = wr * E.dx;
-            x[6] = wr * E.dy;
+            x[5] = wd.x;
+            x[6] = wd.y;
           }
-          P0 = P0 + w * c0;
-          P1 = P1 + w * c1;
-          P2 = P2 + w * c2;
+          P01.x = P01.x + wc01.x;
+          P01.y = P01.y + wc01.y;
+          P2 = P2 + wc2;
           T = den;
         }
       }

@@ -7,6 +7,15 @@
 // "Two-Stage Algorithm" (both passes walk the same tile bins in the same order with the same
 // decisions; per-Gaussian contributions are reduced on chip -- here over each warp of a tile --
 // before global atomics).
+//
+// Packed fp32 pairs (__fmul2_rn, __fadd2_rn, __ffma2_rn: one instruction for two lanes' worth of
+// work) round each element exactly like the scalar operation, and the pair loops here are
+// issue-bound, so they use them where two independent operations of one kind meet. One rule
+// keeps the results bit-identical to the scalar arithmetic: the compiler fuses a packed product
+// whose only consumer is a packed add into one fma (also when both are written as PTX with an
+// explicit rounding mode, and -fmad=false does not stop it), so a packed product only ever feeds
+// scalar adds (which -fmad=false keeps unfused), packed adds take no products, and a packed fma
+// stands only where one rounding is meant (fma(a, -1, b) is b - a rounded once).
 #pragma once
 #include "common.cuh"
 
@@ -59,8 +68,10 @@ __device__ __forceinline__ long long chunk_index(long long p, int gt) { return (
 __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
                                             float py) {
   Entry e;
-  e.dx = px - A.x;
-  e.dy = py - A.y;
+  // (px - A.x, py - A.y) in one packed op: fma(a, -1, p) rounds p - a exactly once
+  const float2 d = __ffma2_rn(make_float2(A.x, A.y), make_float2(-1.0f, -1.0f), make_float2(px, py));
+  e.dx = d.x;
+  e.dy = d.y;
   const float t1 = A.z * e.dx * e.dx;
   const float t2 = Bq.x * e.dy * e.dy;
   const float t3 = A.w * e.dx * e.dy;
@@ -80,11 +91,21 @@ __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, flo
 // values and send the lower half, the others the reverse; the received half is added
 template <int HALF>
 __device__ __forceinline__ void tr_step(float* x, bool hi, int off) {
+  if constexpr (HALF == 1) {
+    const float send = hi ? x[0] : x[1];
+    const float keep = hi ? x[1] : x[0];
+    x[0] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+  } else {
 #pragma unroll
-  for (int k = 0; k < HALF; ++k) {
-    const float send = hi ? x[k] : x[k + HALF];
-    const float keep = hi ? x[k + HALF] : x[k];
-    x[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    for (int k = 0; k < HALF; k += 2) {  // two values per packed add (keep + received)
+      const float s0 = hi ? x[k] : x[k + HALF], k0 = hi ? x[k + HALF] : x[k];
+      const float s1 = hi ? x[k + 1] : x[k + 1 + HALF], k1 = hi ? x[k + 1 + HALF] : x[k + 1];
+      const float2 rv = make_float2(__shfl_xor_sync(0xffffffffu, s0, off),
+                                    __shfl_xor_sync(0xffffffffu, s1, off));
+      const float2 sum = __fadd2_rn(make_float2(k0, k1), rv);
+      x[k] = sum.x;
+      x[k + 1] = sum.y;
+    }
   }
 }
 
