@@ -11,10 +11,12 @@
 // log q_g, e~(3), l], 9 + 3 d_SH entries).
 //
 // Because gamma_gv / q_gv = 1 / q_g for every view, each block is a plain sum over views divided
-// once by q_g (the linear rewrite; no second pass over the views). Sums and the eigenvalues are
-// evaluated in double; the SH block's per-view products in fp32, accumulated in a shared-memory
-// tile of the block's token rows (keeps registers, hence occupancy, low) that is then written out
-// with coalesced stores.
+// once by q_g (the linear rewrite; no second pass over the views). The per-view terms (Jacobian,
+// pullback, J^T J, SH products) are fp32 products (~6e-8 relative rounding each; fewer registers,
+// so more Gaussians in flight in this latency-bound loop); the sums over views, the division by
+// q_g and the eigenvalues are double. The SH block is accumulated in a shared-memory tile of the
+// block's token rows (keeps registers, hence occupancy, low) that is then written out with
+// coalesced stores.
 #include "common.cuh"
 
 namespace splat {
@@ -78,30 +80,32 @@ __device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
     const double qgv = eps + a01.x;
     qsum += qgv;
     sa += (1.0 - (double)r1.y) * a45.x;
-    const double qa = r0.z, qb = r0.w, qc = r1.x;
-    const double sm0 = qa * a45.y + qb * a67.x;
-    const double sm1 = qb * a45.y + qc * a67.x;
+    // per-view products in fp32 (rounding ~1e-7 relative), sums over views in double
+    const float sd0 = (float)a45.y, sd1 = (float)a67.x;
+    const float sm0 = r0.z * sd0 + r0.w * sd1;
+    const float sm1 = r0.w * sd0 + r1.x * sd1;
     // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
     const float* vw = views + 20 * v;
-    const double fx = vw[16], fy = vw[17];
-    const double x = r3.y, y = r3.z, z = r3.x;
-    const double j00 = fx / z, j02 = -fx * x / (z * z);
-    const double j11 = fy / z, j12 = -fy * y / (z * z);
-    double J0[3], J1[3];
+    const float fx = vw[16], fy = vw[17];
+    const float x = r3.y, y = r3.z, iz = 1.0f / r3.x;
+    const float j00 = fx * iz, j02 = -fx * x * iz * iz;
+    const float j11 = fy * iz, j12 = -fy * y * iz * iz;
+    float J0[3], J1[3];
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
-      J0[c] = j00 * (double)vw[c] + j02 * (double)vw[8 + c];
-      J1[c] = j11 * (double)vw[4 + c] + j12 * (double)vw[8 + c];
+      J0[c] = j00 * vw[c] + j02 * vw[8 + c];
+      J1[c] = j11 * vw[4 + c] + j12 * vw[8 + c];
     }
-    b[0] += J0[0] * sm0 + J1[0] * sm1;
-    b[1] += J0[1] * sm0 + J1[1] * sm1;
-    b[2] += J0[2] * sm0 + J1[2] * sm1;
-    A[0] += qgv * (J0[0] * J0[0] + J1[0] * J1[0]);
-    A[1] += qgv * (J0[0] * J0[1] + J1[0] * J1[1]);
-    A[2] += qgv * (J0[0] * J0[2] + J1[0] * J1[2]);
-    A[3] += qgv * (J0[1] * J0[1] + J1[1] * J1[1]);
-    A[4] += qgv * (J0[1] * J0[2] + J1[1] * J1[2]);
-    A[5] += qgv * (J0[2] * J0[2] + J1[2] * J1[2]);
+    b[0] += (double)(J0[0] * sm0 + J1[0] * sm1);
+    b[1] += (double)(J0[1] * sm0 + J1[1] * sm1);
+    b[2] += (double)(J0[2] * sm0 + J1[2] * sm1);
+    const float qf = (float)qgv;
+    A[0] += (double)(qf * (J0[0] * J0[0] + J1[0] * J1[0]));
+    A[1] += (double)(qf * (J0[0] * J0[1] + J1[0] * J1[1]));
+    A[2] += (double)(qf * (J0[0] * J0[2] + J1[0] * J1[2]));
+    A[3] += (double)(qf * (J0[1] * J0[1] + J1[1] * J1[1]));
+    A[4] += (double)(qf * (J0[1] * J0[2] + J1[1] * J1[2]));
+    A[5] += (double)(qf * (J0[2] * J0[2] + J1[2] * J1[2]));
     // view direction (mu - camera centre) / |.| = R_v^T x_c / |x_c|
     float B[16];
     {
