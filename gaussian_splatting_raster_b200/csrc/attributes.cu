@@ -31,10 +31,12 @@ constexpr int kMaxPass = 16;  // channels per traversal
 template <int CB>
 __global__ void __launch_bounds__(kThreads)
 k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-           const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
+           const long long* __restrict__ tile_off, const int* __restrict__ order,
+           int G, int H, int W, int TX, int nt,
            const int* __restrict__ last, const uint32_t* __restrict__ umask,
            const float* __restrict__ feats, int C, int c0, float* __restrict__ out) {
-  const int t = blockIdx.x, v = blockIdx.y;
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
   tile_pixel(tx, ty, i, j, bx, by);
@@ -116,11 +118,13 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
 template <int NV, bool RESID>
 __global__ void __launch_bounds__(kThreads)
 k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-          const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
+          const long long* __restrict__ tile_off, const int* __restrict__ order,
+          int G, int H, int W, int TX, int nt,
           const int* __restrict__ last, const uint32_t* __restrict__ umask,
           const float* __restrict__ map, const float* __restrict__ img,
           const float* __restrict__ obs, int C, int c0, double* __restrict__ acc) {
-  const int t = blockIdx.x, v = blockIdx.y;
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
   tile_pixel(tx, ty, i, j, bx, by);
@@ -242,7 +246,7 @@ int launch_features(Workspace& w, const float* feats, int C, float* out, cudaStr
   for (int c0 = 0; c0 < C; c0 += kMaxPass) {
     const int nc = C - c0 < kMaxPass ? C - c0 : kMaxPass;
 #define SPLAT_FEAT(CB)                                                                          \
-  k_features<CB><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,    \
+  k_features<CB><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,    \
                                            w.nt, w.last, w.umask, feats, C, c0, out)
     if (nc == 1) SPLAT_FEAT(1);
     else if (nc <= 4) SPLAT_FEAT(4);
@@ -278,7 +282,7 @@ int launch_scatter(Workspace& w, const float* map, const float* obs, int C, floa
   } end_tok{w, st, tok};
   dim3 grid(w.nt, w.V);
   if (attr) {
-    k_scatter<2, true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,
+    k_scatter<2, true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                                   w.nt, w.last, w.umask, nullptr, w.img, obs, 2,
                                                   0, w.sacc);
     if ((rc = check_launch(w, "attribution kernel"))) return rc;
@@ -286,7 +290,7 @@ int launch_scatter(Workspace& w, const float* map, const float* obs, int C, floa
     for (int c0 = 0; c0 < C; c0 += kMaxPass) {
       const int nc = C - c0 < kMaxPass ? C - c0 : kMaxPass;
 #define SPLAT_SCAT(NV)                                                                          \
-  k_scatter<NV, false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W,    \
+  k_scatter<NV, false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W,    \
                                                   w.TX, w.nt, w.last, w.umask, map, nullptr,   \
                                                   nullptr, C, c0, w.sacc)
       if (nc == 1) SPLAT_SCAT(1);

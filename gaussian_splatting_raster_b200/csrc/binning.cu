@@ -396,6 +396,76 @@ __global__ void k_tile_ranges(const int* __restrict__ hist_scan, const long long
   tile_off[idx] = o;
 }
 
+// Launch order of the (tile, view) CTAs of the kernels that walk the lists: longest list first.
+// The CTAs of a launch start in block-index order, so the long lists start in the first waves and
+// the last wave holds short ones instead of leaving SMs idle behind one long list. Length classes
+// of eight per octave (the leading bit and the next three, monotone in the length); inside a class
+// the tiles keep their (view, row, column) order, so neighbouring tiles, which share Gaussians,
+// still run close together. One block: a stable counting sort over 32 warp segments, the same
+// scheme as the binning passes (per-warp class counts, a scan over (class, warp), match.any
+// ranking).
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderWarps = kOrderThreads / 32;
+constexpr int kOrderClasses = 256;
+
+__device__ __forceinline__ int len_class(const long long* __restrict__ tile_off, int nt, int k) {
+  const int v = k / nt;
+  const long long* o = tile_off + (size_t)v * (nt + 1) + (k - v * nt);
+  const long long len = o[1] - o[0];
+  if (len <= 0) return kOrderClasses - 1;  // empty lists last
+  const unsigned long long u = (unsigned long long)len;
+  const int msb = 63 - __clzll(u);
+  const int frac = msb >= 3 ? (int)((u >> (msb - 3)) & 7u) : (int)((u << (3 - msb)) & 7u);
+  return kOrderClasses - 2 - (min(msb, 30) * 8 + frac);  // longest lists in the lowest class
+}
+
+__global__ void __launch_bounds__(kOrderThreads)
+k_tile_order(const long long* __restrict__ tile_off, int V, int nt, int* __restrict__ order) {
+  __shared__ int s_cnt[kOrderWarps * kOrderClasses];  // [warp][class]
+  __shared__ int s_warp[32];
+  const int n = V * nt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = (n + kOrderWarps - 1) / kOrderWarps;
+  const int kb = min(n, warp * per), ke = min(n, kb + per);
+  for (int c = threadIdx.x; c < kOrderWarps * kOrderClasses; c += blockDim.x) s_cnt[c] = 0;
+  __syncthreads();
+  for (int k = kb + lane; k < ke; k += 32) atomicAdd(&s_cnt[warp * kOrderClasses + len_class(tile_off, nt, k)], 1);
+  __syncthreads();
+  // exclusive scan in (class, warp) order: thread t owns entries 8t .. 8t + 7 of that order
+  constexpr int kPer = kOrderWarps * kOrderClasses / kOrderThreads;
+  int c[kPer], sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = kPer * threadIdx.x + i;
+    c[i] = s_cnt[(e % kOrderWarps) * kOrderClasses + e / kOrderWarps];
+    sum += c[i];
+  }
+  int run = block_exclusive_scan<int>(sum, s_warp, nullptr);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = kPer * threadIdx.x + i;
+    s_cnt[(e % kOrderWarps) * kOrderClasses + e / kOrderWarps] = run;
+    run += c[i];
+  }
+  __syncthreads();
+  // each warp places its segment in order; equal classes inside a batch of 32 ranked by lane
+  const uint32_t lt = lanemask_lt();
+  int* cnt = s_cnt + warp * kOrderClasses;
+  for (int base = kb; base < ke; base += 32) {
+    const int k = base + lane;
+    const bool ok = k < ke;
+    const int cl = ok ? len_class(tile_off, nt, k) : -1 - lane;  // unique for idle lanes
+    const uint32_t peers = __match_any_sync(0xffffffffu, cl);
+    if (ok) {
+      const int pos = cnt[cl] + __popc(peers & lt);
+      if (in_bounds(pos, (unsigned long long)n, &g_bounds_word)) order[pos] = k;
+    }
+    __syncwarp();
+    if (ok && lane == __ffs(peers) - 1) cnt[cl] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 template <typename T>
 int grow(Workspace& w, T** p, size_t n, const char* what) {
   if (*p) cudaFree(*p);
@@ -563,8 +633,16 @@ int launch_binning(Workspace& w, cudaStream_t st) {
   const int tok_r = prof_begin(w, st, SPLAT_K_TILE_RANGES);
   k_tile_ranges<<<(nr + 255) / 256, 256, 0, st>>>(w.hist, w.d_vstart, w.d_bstart, w.V, w.nt,
                                                   w.tile_off);
+  if ((rc = check_launch(w, "tile ranges kernel"))) {
+    prof_end(w, st, tok_r);
+    return rc;
+  }
+  if (w.V * w.nt > 0) {
+    k_tile_order<<<1, kOrderThreads, 0, st>>>(w.tile_off, w.V, w.nt, w.tile_order);
+    rc = check_launch(w, "tile order kernel");
+  }
   prof_end(w, st, tok_r);
-  return check_launch(w, "tile ranges kernel");
+  return rc;
 }
 
 // shared-memory opt-in for the counting-sort kernels (called once per workspace)

@@ -67,7 +67,7 @@ void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
                  w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.accb, w.sacc,
-                 w.acc_fix, w.accb_fix};
+                 w.acc_fix, w.accb_fix, w.tile_order};
   for (void* p : dev)
     if (p) cudaFree(p);
   if (w.h_vstart) cudaFreeHost(w.h_vstart);
@@ -132,6 +132,7 @@ int splat_ws_create(splat_ws** out, int max_G, int max_V, int max_H, int max_W,
   if (!rc) rc = alloc(w, &w.views, (size_t)max_V * 20, "views");
   if (!rc) rc = alloc(w, &w.last, (size_t)max_V * max_H * max_W, "list bounds");
   if (!rc) rc = alloc(w, &w.tile_off, (size_t)max_V * (w.max_nt + 1), "tile offsets");
+  if (!rc) rc = alloc(w, &w.tile_order, (size_t)max_V * w.max_nt, "tile launch order");
   if (!rc) rc = alloc(w, &w.d_vstart, (size_t)max_V + 1, "view starts");
   if (!rc) rc = alloc(w, &w.d_bstart, (size_t)max_V + 1, "block starts");
   if (!rc) rc = alloc(w, &w.d_scratch, 8, "scratch");

@@ -221,6 +221,7 @@ struct Workspace {
   size_t hist_cap = 0;
   int* hist = nullptr;
   long long* tile_off = nullptr;  // [V*(nt+1)]
+  int* tile_order = nullptr;      // [V*nt] tiles (v*nt + t) in launch order, longest list first
 
   // per-view tables
   long long* d_vstart = nullptr;  // [V+1] first instance of each view

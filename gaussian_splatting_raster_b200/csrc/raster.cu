@@ -48,10 +48,12 @@ namespace {
 
 __global__ void __launch_bounds__(kThreads)
 k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-         const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
+         const long long* __restrict__ tile_off, const int* __restrict__ order,
+         int G, int H, int W, int TX, int nt,
          const float* __restrict__ bgp, float* __restrict__ img, float* __restrict__ Tout,
          int* __restrict__ ncout, int* __restrict__ last, uint32_t* __restrict__ umask) {
-  const int t = blockIdx.x, v = blockIdx.y;
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
   tile_pixel(tx, ty, i, j, bx, by);
@@ -185,13 +187,15 @@ __global__ void k_fixed_to_double(const unsigned long long* __restrict__ src,
 }
 
 template <bool kDet>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 5)  // 48 registers: 5 CTAs per SM
 k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-         const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
+         const long long* __restrict__ tile_off, const int* __restrict__ order,
+         int G, int H, int W, int TX, int nt,
          const float* __restrict__ img, const float* __restrict__ obs,
          const int* __restrict__ last, const uint32_t* __restrict__ umask,
          double* __restrict__ acc, unsigned long long* __restrict__ acc_fix) {
-  const int t = blockIdx.x, v = blockIdx.y;
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
   tile_pixel(tx, ty, i, j, bx, by);
@@ -334,12 +338,14 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
 template <bool kDet>
 __global__ void __launch_bounds__(kThreads)
 k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-           const long long* __restrict__ tile_off, int G, int H, int W, int TX, int nt,
+           const long long* __restrict__ tile_off, const int* __restrict__ order,
+           int G, int H, int W, int TX, int nt,
            const float* __restrict__ img, const float* __restrict__ Tfin,
            const float* __restrict__ bgp, const float* __restrict__ obs,
            const int* __restrict__ last, const uint32_t* __restrict__ umask,
            double* __restrict__ accb, unsigned long long* __restrict__ accb_fix) {
-  const int t = blockIdx.x, v = blockIdx.y;
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
   tile_pixel(tx, ty, i, j, bx, by);
@@ -462,8 +468,8 @@ int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int
                   cudaStream_t st) {
   dim3 grid(w.nt, w.V);
   const int tok = prof_begin(w, st, SPLAT_K_RENDER);
-  k_render<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX, w.nt, bg,
-                                      img, T_final, n_contrib, w.last, w.umask);
+  k_render<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
+                                      w.nt, bg, img, T_final, n_contrib, w.last, w.umask);
   prof_end(w, st, tok);
   return check_launch(w, "render kernel");
 }
@@ -514,11 +520,11 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
   if (!rc) {
     dim3 grid(w.nt, w.V);
     if (det)
-      k_replay<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,
+      k_replay<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                                 w.nt, w.img, obs, w.last, w.umask, w.acc,
                                                 w.acc_fix);
     else
-      k_replay<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,
+      k_replay<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                                  w.nt, w.img, obs, w.last, w.umask, w.acc,
                                                  nullptr);
     rc = check_launch(w, "replay kernel");
@@ -543,11 +549,11 @@ int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {
   if (!rc) {
     dim3 grid(w.nt, w.V);
     if (det)
-      k_backward<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W, w.TX,
+      k_backward<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                                   w.nt, w.img, w.Tfin, w.bg, obs, w.last,
                                                   w.umask, w.accb, w.accb_fix);
     else
-      k_backward<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.G, w.H, w.W,
+      k_backward<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W,
                                                    w.TX, w.nt, w.img, w.Tfin, w.bg, obs, w.last,
                                                    w.umask, w.accb, nullptr);
     rc = check_launch(w, "backward kernel");

@@ -60,6 +60,18 @@ __device__ __forceinline__ bool reaches_block(float4 A, float ex, float ey, floa
          A.y + ey >= y0 + 0.5f && A.y - ey <= y0 + ((float)kWarpH - 0.5f);
 }
 
+// (tile, view) of this CTA: the list-walking kernels launch a (tiles, views) grid and take the
+// tiles in the order the binning wrote (longest list first). False for an order entry outside
+// [0, V nt) (checked build only; the CTA then does nothing).
+__device__ __forceinline__ bool block_tile(const int* __restrict__ order, int nt,
+                                           unsigned int* bounds_word, int& t, int& v) {
+  const int o = order[blockIdx.y * gridDim.x + blockIdx.x];
+  if (!in_bounds((unsigned)o, (unsigned long long)nt * gridDim.y, bounds_word)) return false;
+  v = o / nt;
+  t = o - v * nt;
+  return true;
+}
+
 // position of the composited-entry mask of (global tile gt, chunk starting at list position p):
 // distinct for every chunk of every tile, at most N / 32 + V * nt
 __device__ __forceinline__ long long chunk_index(long long p, int gt) { return (p >> 5) + gt; }
