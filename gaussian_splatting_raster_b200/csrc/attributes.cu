@@ -269,10 +269,8 @@ int launch_scatter(Workspace& w, const float* map, const float* obs, int C, floa
   if (attr) C = 2;
   int rc;
   if ((rc = grow_scratch(w, (size_t)w.G * C))) return rc;
-  cudaError_t e = cudaSuccess;
-  if ((size_t)w.G * C > 0) e = cudaMemsetAsync(w.sacc, 0, (size_t)w.G * C * sizeof(double), st);
-  if (e != cudaSuccess)
-    return set_err(w, SPLAT_ERR_CUDA, std::string("scatter sums clear: ") + cudaGetErrorString(e));
+  if ((rc = zero_async(w, w.sacc, (size_t)w.G * C * sizeof(double), st, "scatter sums clear")))
+    return rc;
   const int tok = prof_begin(w, st, SPLAT_K_SCATTER);
   struct EndTok {  // closes the timing bracket on every return path
     Workspace& w;

@@ -506,6 +506,42 @@ int scan_i32_to_i64(Workspace& w, const int* in, long long* out, long long n, cu
   return check_launch(w, "scan total");
 }
 
+namespace {
+__global__ void k_zero(uint4* __restrict__ p16, size_t n16, uint32_t* __restrict__ p4, size_t n4) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n16; k += stride)
+    p16[k] = make_uint4(0u, 0u, 0u, 0u);
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n4; k += stride) p4[k] = 0u;
+}
+__global__ void k_copy_words(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst, size_t n) {
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n;
+       k += (size_t)gridDim.x * blockDim.x)
+    dst[k] = src[k];
+}
+}  // namespace
+
+int zero_async(Workspace& w, void* p, size_t bytes, cudaStream_t st, const char* what) {
+  if (bytes == 0) return SPLAT_OK;
+  if (((uintptr_t)p & 15) || (bytes & 3))
+    return set_err(w, SPLAT_ERR_INVALID_ARG, std::string(what) + ": clear of an unaligned range");
+  const size_t n16 = bytes / 16, n4 = (bytes - n16 * 16) / 4;
+  const size_t want = (n16 + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 8 ? (want > 0 ? want : 1) : 148 * 8);
+  k_zero<<<blocks, 256, 0, st>>>(reinterpret_cast<uint4*>(p), n16,
+                                 reinterpret_cast<uint32_t*>(static_cast<char*>(p) + n16 * 16), n4);
+  return check_launch(w, what);
+}
+
+int copy_words(Workspace& w, const void* src, void* dst, size_t bytes, cudaStream_t st,
+               const char* what) {
+  if (bytes == 0) return SPLAT_OK;
+  const size_t n = bytes / 4;
+  const unsigned blocks = (unsigned)((n + 255) / 256 < 64 ? (n + 255) / 256 : 64);
+  k_copy_words<<<blocks, 256, 0, st>>>(static_cast<const uint32_t*>(src),
+                                       static_cast<uint32_t*>(dst), n);
+  return check_launch(w, what);
+}
+
 int scan_i32_inplace(Workspace& w, int* data, long long n, cudaStream_t st) {
   const long long nb = (n + kScanTile - 1) / kScanTile;
   int rc = ensure_part(w, nb > 0 ? nb : 1);
@@ -618,9 +654,11 @@ int launch_binning(Workspace& w, cudaStream_t st) {
     w.h_bstart[v + 1] = w.h_bstart[v] + (int)((nv + kTileChunk - 1) / kTileChunk);
   }
   w.n_blocks = w.h_bstart[w.V];
-  cudaMemcpyAsync(w.d_vstart, w.h_vstart, (w.V + 1) * sizeof(long long),
-                  cudaMemcpyHostToDevice, st);
-  cudaMemcpyAsync(w.d_bstart, w.h_bstart, (w.V + 1) * sizeof(int), cudaMemcpyHostToDevice, st);
+  if ((rc = copy_words(w, w.hd_vstart, w.d_vstart, (w.V + 1) * sizeof(long long), st,
+                       "view starts upload")) ||
+      (rc = copy_words(w, w.hd_bstart, w.d_bstart, (w.V + 1) * sizeof(int), st,
+                       "block starts upload")))
+    return rc;
   if (N > 0) {
     Segs sg{-1, 0, w.d_vstart, w.d_bstart, w.V, kTileChunk};
     if ((rc = count_pass(w, st, w.inst_tile, w.inst_g, 0, 0xffffffffu, w.nt, sg, w.n_blocks,

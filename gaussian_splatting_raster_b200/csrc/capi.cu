@@ -63,6 +63,24 @@ int alloc(Workspace& w, T** p, size_t n, const char* what) {
   return SPLAT_OK;
 }
 
+// pinned host memory the kernels read and write directly (mapped): the few words a step exchanges
+// with the host move without a copy engine
+template <typename T>
+int alloc_mapped(Workspace& w, T** h, T** d, size_t n, const char* what) {
+  *h = nullptr;
+  *d = nullptr;
+  if (cudaHostAlloc((void**)h, n * sizeof(T), cudaHostAllocMapped) != cudaSuccess) {
+    cudaGetLastError();
+    *h = nullptr;
+    return fail(w, SPLAT_ERR_OOM, "pinned host allocation of %zu bytes failed (%s)", n * sizeof(T), what);
+  }
+  if (cudaHostGetDevicePointer((void**)d, *h, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(w, SPLAT_ERR_CUDA, "no device address for mapped host memory (%s)", what);
+  }
+  return SPLAT_OK;
+}
+
 void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
@@ -139,21 +157,17 @@ int splat_ws_create(splat_ws** out, int max_G, int max_V, int max_H, int max_W,
   if (!rc) rc = alloc(w, &w.dkey, VG, "depth keys");
   if (!rc) rc = alloc(w, &w.kbits, (size_t)2 * splat::kKeyStripes * max_V, "key statistics");
   if (!rc) rc = alloc(w, &w.ntot, (size_t)splat::kKeyStripes * max_V, "instance counts");
-  if (!rc && cudaMallocHost(&w.h_ntot, (size_t)splat::kKeyStripes * max_V *
-                                           sizeof(unsigned long long)) != cudaSuccess)
-    rc = SPLAT_ERR_OOM;
+  if (!rc) rc = alloc_mapped(w, &w.h_ntot, &w.hd_ntot, (size_t)splat::kKeyStripes * max_V,
+                             "instance counts (host)");
   if (!rc) rc = alloc(w, &w.dk1, VG, "depth keys 2");
   if (!rc) rc = alloc(w, &w.dk2, VG, "depth keys 3");
   if (!rc) rc = alloc(w, &w.dv0, VG, "depth order");
   if (!rc) rc = alloc(w, &w.dv1, VG, "depth order 2");
   if (!rc) rc = alloc(w, &w.rect_s, VG, "rectangles in depth order");
-  if (!rc && cudaMallocHost(&w.h_kbits, (size_t)2 * splat::kKeyStripes * max_V * sizeof(uint32_t)) !=
-                  cudaSuccess)
-    rc = SPLAT_ERR_OOM;
-  if (!rc && cudaMallocHost(&w.h_vstart, (max_V + 1) * sizeof(long long)) != cudaSuccess)
-    rc = SPLAT_ERR_OOM;
-  if (!rc && cudaMallocHost(&w.h_bstart, (max_V + 1) * sizeof(int)) != cudaSuccess)
-    rc = SPLAT_ERR_OOM;
+  if (!rc) rc = alloc_mapped(w, &w.h_kbits, &w.hd_kbits, (size_t)2 * splat::kKeyStripes * max_V,
+                             "key statistics (host)");
+  if (!rc) rc = alloc_mapped(w, &w.h_vstart, &w.hd_vstart, (size_t)max_V + 1, "view starts (host)");
+  if (!rc) rc = alloc_mapped(w, &w.h_bstart, &w.hd_bstart, (size_t)max_V + 1, "block starts (host)");
   if (!rc && cudaMallocHost(&w.h_scratch, 8 * sizeof(long long)) != cudaSuccess)
     rc = SPLAT_ERR_OOM;
   if (!rc) rc = splat::binning_configure(w);
@@ -228,12 +242,14 @@ int splat_bin_sort(splat_ws* ws, long long* n_instances_out, void* stream) {
   // the one synchronisation of the path: per-view instance counts and depth-key statistics,
   // accumulated in striped copies by the projection, folded here
   const int ns = splat::kKeyStripes;
-  cudaError_t e = cudaMemcpyAsync(w.h_ntot, w.ntot, (size_t)ns * w.V * sizeof(unsigned long long),
-                                  cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(w.h_kbits, w.kbits, (size_t)2 * ns * w.V * sizeof(uint32_t),
-                        cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  // (kernels store them into mapped host memory: no copy engine, so the wait is not queued
+  // behind a caller's large transfers on other streams)
+  if ((rc = splat::copy_words(w, w.ntot, w.hd_ntot, (size_t)ns * w.V * sizeof(unsigned long long),
+                              st, "instance counts readback")) ||
+      (rc = splat::copy_words(w, w.kbits, w.hd_kbits, (size_t)2 * ns * w.V * sizeof(uint32_t), st,
+                              "key statistics readback")))
+    return rc;
+  cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(w, "reading the instance counts", e);
   w.h_vstart[0] = 0;
   for (int v = 0; v < w.V; ++v) {

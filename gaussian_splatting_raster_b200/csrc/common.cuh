@@ -201,7 +201,8 @@ struct Workspace {
   uint32_t* dkey = nullptr;    // [V*G] depth sort keys (written by the projection)
   uint32_t* kbits = nullptr;   // [V][kKeyStripes][2]: OR of visible keys, OR of complements
   unsigned long long* ntot = nullptr;  // [V][kKeyStripes] instance counts (striped)
-  unsigned long long* h_ntot = nullptr;  // pinned copy
+  unsigned long long* h_ntot = nullptr;  // pinned, mapped (hd_ntot: its device address)
+  unsigned long long* hd_ntot = nullptr;
   uint32_t* dk1 = nullptr;     // [V*G] radix ping-pong keys (dkey itself is never overwritten)
   uint32_t* dk2 = nullptr;     // [V*G]
   uint32_t* dv0 = nullptr;     // [V*G] radix values (Gaussian index), ping
@@ -226,9 +227,12 @@ struct Workspace {
   // per-view tables
   long long* d_vstart = nullptr;  // [V+1] first instance of each view
   int* d_bstart = nullptr;        // [V+1] first binning block of each view
-  long long* h_vstart = nullptr;  // pinned
-  int* h_bstart = nullptr;        // pinned
-  uint32_t* h_kbits = nullptr;    // pinned [V][kKeyStripes][2]
+  long long* h_vstart = nullptr;  // pinned, mapped (hd_*: device addresses of the same memory)
+  int* h_bstart = nullptr;        // pinned, mapped
+  uint32_t* h_kbits = nullptr;    // pinned, mapped [V][kKeyStripes][2]
+  long long* hd_vstart = nullptr;
+  int* hd_bstart = nullptr;
+  uint32_t* hd_kbits = nullptr;
   long long n_total = 0;
   int n_blocks = 0;
 
@@ -316,5 +320,12 @@ int binning_configure(Workspace& w);
 int scan_i32_to_i64(Workspace& w, const int* in, long long* out, long long n, cudaStream_t st);
 // same, int32 in place (values and total < 2^31)
 int scan_i32_inplace(Workspace& w, int* data, long long n, cudaStream_t st);
+// Stream-ordered clear and word copy done by kernels on the SMs, never by a copy engine: inside a
+// step nothing may queue behind a caller's large host<->device transfers on other streams (a
+// copy engine serves its queue in order). copy_words also moves the few words the host reads or
+// writes each step through mapped pinned memory (sizes in bytes, multiples of 4).
+int zero_async(Workspace& w, void* p, size_t bytes, cudaStream_t st, const char* what);
+int copy_words(Workspace& w, const void* src, void* dst, size_t bytes, cudaStream_t st,
+               const char* what);
 
 }  // namespace splat

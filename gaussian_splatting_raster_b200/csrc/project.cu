@@ -259,12 +259,12 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
 
 int launch_project(Workspace& w, const float* means, const float* lsc, const float* quats,
                    const float* opac, const float* sh, cudaStream_t st) {
-  cudaError_t e =
-      cudaMemsetAsync(w.kbits, 0, (size_t)2 * kKeyStripes * w.V * sizeof(uint32_t), st);
-  if (e == cudaSuccess)
-    e = cudaMemsetAsync(w.ntot, 0, (size_t)kKeyStripes * w.V * sizeof(unsigned long long), st);
-  if (e != cudaSuccess)
-    return set_err(w, SPLAT_ERR_CUDA, std::string("key statistics clear: ") + cudaGetErrorString(e));
+  int rc = zero_async(w, w.kbits, (size_t)2 * kKeyStripes * w.V * sizeof(uint32_t), st,
+                      "key statistics clear");
+  if (!rc)
+    rc = zero_async(w, w.ntot, (size_t)kKeyStripes * w.V * sizeof(unsigned long long), st,
+                    "instance counts clear");
+  if (rc) return rc;
   if (w.G == 0) return SPLAT_OK;
   const int blocks = (w.G + kProjThreads - 1) / kProjThreads;
   const int tok = prof_begin(w, st, SPLAT_K_PROJECT);

@@ -490,12 +490,8 @@ static int fix_buffer(Workspace& w, unsigned long long** buf, size_t& cap, int n
     }
     cap = need;
   }
-  const cudaError_t e =
-      cudaMemsetAsync(*buf, 0, (size_t)w.V * w.G * nslot * 2 * sizeof(unsigned long long), st);
-  if (e != cudaSuccess)
-    return set_err(w, SPLAT_ERR_CUDA, std::string("deterministic sums clear: ") +
-                                          cudaGetErrorString(e));
-  return SPLAT_OK;
+  return zero_async(w, *buf, (size_t)w.V * w.G * nslot * 2 * sizeof(unsigned long long), st,
+                    "deterministic sums clear");
 }
 
 static int fix_to_double(Workspace& w, const unsigned long long* src, double* dst, int nslot,
@@ -513,9 +509,7 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
   if (det) {
     rc = fix_buffer(w, &w.acc_fix, w.acc_fix_cap, kAccN, st);
   } else if (w.G > 0) {
-    cudaError_t e = cudaMemsetAsync(w.acc, 0, (size_t)w.V * w.G * kAccN * sizeof(double), st);
-    if (e != cudaSuccess)
-      rc = set_err(w, SPLAT_ERR_CUDA, std::string("accumulator clear: ") + cudaGetErrorString(e));
+    rc = zero_async(w, w.acc, (size_t)w.V * w.G * kAccN * sizeof(double), st, "accumulator clear");
   }
   if (!rc) {
     dim3 grid(w.nt, w.V);
@@ -541,10 +535,8 @@ int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {
   if (det) {
     rc = fix_buffer(w, &w.accb_fix, w.accb_fix_cap, kAccBN, st);
   } else if (w.G > 0) {
-    cudaError_t e = cudaMemsetAsync(w.accb, 0, (size_t)w.V * w.G * kAccBN * sizeof(double), st);
-    if (e != cudaSuccess)
-      rc = set_err(w, SPLAT_ERR_CUDA, std::string("backward sums clear: ") +
-                                          cudaGetErrorString(e));
+    rc = zero_async(w, w.accb, (size_t)w.V * w.G * kAccBN * sizeof(double), st,
+                    "backward sums clear");
   }
   if (!rc) {
     dim3 grid(w.nt, w.V);
@@ -564,7 +556,8 @@ int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {
 }
 
 int launch_pair_count(Workspace& w, cudaStream_t st) {
-  cudaMemsetAsync(w.d_scratch, 0, sizeof(long long), st);
+  int rc = zero_async(w, w.d_scratch, sizeof(long long), st, "pair count clear");
+  if (rc) return rc;
   const long long n = (long long)w.V * w.H * w.W;
   k_pair_sum<<<296, 256, 0, st>>>(w.last, n, w.d_scratch);
   return check_launch(w, "pair count kernel");

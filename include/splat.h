@@ -22,7 +22,10 @@
  *     except where a call says so.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every call
  *     only enqueues work on that stream and returns; the exception is splat_bin_sort, which
- *     waits for the per-view instance counts (one device-to-host read).
+ *     waits for the per-view instance counts (a few words that kernels store into mapped
+ *     pinned host memory). Nothing a call enqueues uses a copy engine: clears and these small
+ *     exchanges are kernels, so a step never waits behind the caller's large host<->device
+ *     copies on other streams.
  *   - Return value: SPLAT_OK (0) or a negative splat_status. No C++ exception crosses the ABI.
  *     On error, splat_last_error(ws) returns a NUL-terminated message owned by the workspace,
  *     valid until the next call on it. Argument errors are detected before any work is
