@@ -43,7 +43,8 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
+  const int twarp = tile_warp();                                 // block in the tile
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float s_cut[kThreads];
   __shared__ __align__(16) float s_f[kThreads * CB];
@@ -62,7 +63,7 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   for (int k = 0; k < CB; ++k) F[k] = 0.0f;
   float T = 1.0f;
   for (int base = 0; base < wmax; base += 32) {
-    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
+    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + twarp];
     if (!bits) continue;  // warp-uniform
     bool bad = false;
     if ((bits >> lane) & 1u) {
@@ -131,7 +132,8 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
+  const int twarp = tile_warp();                                 // block in the tile
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float s_cut[kThreads];
   __shared__ uint32_t s_g[kThreads];
@@ -165,7 +167,7 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool holder = slot_holder<NV>(lane) && slot < nc;
   float T = 1.0f;
   for (int base = 0; base < wmax; base += 32) {
-    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
+    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + twarp];
     if (!bits) continue;  // warp-uniform
     bool bad = false;
     if ((bits >> lane) & 1u) {
@@ -242,7 +244,7 @@ int grow_scratch(Workspace& w, size_t n) {
 
 int launch_features(Workspace& w, const float* feats, int C, float* out, cudaStream_t st) {
   const int tok = prof_begin(w, st, SPLAT_K_FEATURES);
-  dim3 grid(w.nt, w.V);
+  dim3 grid(w.nt * kCtaPerTile, w.V);
   for (int c0 = 0; c0 < C; c0 += kMaxPass) {
     const int nc = C - c0 < kMaxPass ? C - c0 : kMaxPass;
 #define SPLAT_FEAT(CB)                                                                          \
@@ -278,7 +280,7 @@ int launch_scatter(Workspace& w, const float* map, const float* obs, int C, floa
     int tok;
     ~EndTok() { prof_end(w, st, tok); }
   } end_tok{w, st, tok};
-  dim3 grid(w.nt, w.V);
+  dim3 grid(w.nt * kCtaPerTile, w.V);
   if (attr) {
     k_scatter<2, true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                                   w.nt, w.last, w.umask, nullptr, w.img, obs, 2,

@@ -65,7 +65,8 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   // slice of shared memory, ballots which of them can reach its pixel block, evaluates only
   // those, and leaves as soon as its 32 pixels are done. Per 32-entry chunk it records which
   // entries some pixel of the warp composited: the replay visits exactly those.
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
+  const int twarp = tile_warp();                                 // block in the tile
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];  // (colour b, exponent cut)
   float4* wa = s_a + warp * 32;
@@ -123,7 +124,7 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       }
     }
     const uint32_t ubits = __reduce_or_sync(0xffffffffu, lbits);
-    if (lane == 0) umask[chunk_index(base, gt) * 8 + warp] = ubits;
+    if (lane == 0) umask[chunk_index(base, gt) * 8 + twarp] = ubits;
     __syncwarp();
   }
   if (inside) {
@@ -187,7 +188,7 @@ __global__ void k_fixed_to_double(const unsigned long long* __restrict__ src,
 }
 
 template <bool kDet>
-__global__ void __launch_bounds__(kThreads, 5)  // 48 registers: 5 CTAs per SM
+__global__ void __launch_bounds__(kThreads, 5 * kCtaPerTile)  // 48 registers: 40 warps per SM
 k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
          const long long* __restrict__ tile_off, const int* __restrict__ order,
          int G, int H, int W, int TX, int nt,
@@ -206,7 +207,8 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   // per chunk it stages and evaluates only the entries the render recorded as composited by some
   // pixel of the warp -- every other entry contributes nothing to any of its pixels. Its
   // per-entry sums go straight from the seven lanes holding them to the fp64 accumulators.
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
+  const int twarp = tile_warp();                                 // block in the tile
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];
   __shared__ uint32_t s_g[kThreads];
@@ -237,7 +239,7 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
   const int slot = (lane >> 2) & 7;  // value index this lane holds after the reduction
   for (int base = 0; base < wmax; base += 32) {
-    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
+    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + twarp];
     if (!bits) continue;  // warp-uniform
     bool bad = false;
     if ((bits >> lane) & 1u) {
@@ -352,7 +354,8 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const bool inside = i < W && j < H;
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
+  const int twarp = tile_warp();                                 // block in the tile
   __shared__ float4 s_a[kThreads], s_b[kThreads];
   __shared__ float2 s_c[kThreads];
   __shared__ uint32_t s_g[kThreads];
@@ -379,7 +382,7 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   double* accv = accb + (size_t)v * G * kAccBN;
   const int slot = (lane >> 1) & 15;  // value index this lane holds after the reduction
   for (int base = (wmax - 1) & ~31; base >= 0; base -= 32) {
-    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + warp];
+    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + twarp];
     if (!bits) continue;  // warp-uniform
     bool bad = false;
     if ((bits >> lane) & 1u) {
@@ -466,7 +469,7 @@ __global__ void k_pair_sum(const int* __restrict__ last, long long n, long long*
 
 int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int* n_contrib,
                   cudaStream_t st) {
-  dim3 grid(w.nt, w.V);
+  dim3 grid(w.nt * kCtaPerTile, w.V);
   const int tok = prof_begin(w, st, SPLAT_K_RENDER);
   k_render<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                       w.nt, bg, img, T_final, n_contrib, w.last, w.umask);
@@ -512,7 +515,7 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
     rc = zero_async(w, w.acc, (size_t)w.V * w.G * kAccN * sizeof(double), st, "accumulator clear");
   }
   if (!rc) {
-    dim3 grid(w.nt, w.V);
+    dim3 grid(w.nt * kCtaPerTile, w.V);
     if (det)
       k_replay<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                                 w.nt, w.img, obs, w.last, w.umask, w.acc,
@@ -539,7 +542,7 @@ int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {
                     "backward sums clear");
   }
   if (!rc) {
-    dim3 grid(w.nt, w.V);
+    dim3 grid(w.nt * kCtaPerTile, w.V);
     if (det)
       k_backward<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
                                                   w.nt, w.img, w.Tfin, w.bg, obs, w.last,

@@ -22,7 +22,17 @@
 namespace splat {
 namespace {
 
-constexpr int kThreads = 256;
+// A tile's eight warp blocks run in kCtaPerTile CTAs of kCtaWarps warps each. The warps walk the
+// lists independently (no CTA barriers), so a CTA is only a residency unit: smaller CTAs let the
+// warps of a finished block make room sooner.
+#ifndef SPLAT_CTA_WARPS
+#define SPLAT_CTA_WARPS 8
+#endif
+constexpr int kCtaWarps = SPLAT_CTA_WARPS;
+static_assert(kCtaWarps == 1 || kCtaWarps == 2 || kCtaWarps == 4 || kCtaWarps == 8,
+              "warps per CTA divide the tile's eight warp blocks");
+constexpr int kCtaPerTile = 8 / kCtaWarps;
+constexpr int kThreads = 32 * kCtaWarps;
 constexpr float kAlphaMin = 1.0f / 255.0f;
 
 struct Entry {
@@ -42,9 +52,15 @@ constexpr int kWarpH = 32 / kWarpW;
 static_assert(kTile % kWarpW == 0 && kTile % kWarpH == 0 &&
               (kTile / kWarpW) * (kTile / kWarpH) == 8, "eight warp blocks per tile");
 
+// this warp's block (0 .. 7) in its tile
+__device__ __forceinline__ int tile_warp() {
+  return (int)((blockIdx.y * gridDim.x + blockIdx.x) % kCtaPerTile) * kCtaWarps +
+         (int)(threadIdx.x >> 5);
+}
+
 // pixel of this thread in tile (tx, ty), and the top-left corner of its warp's block
 __device__ __forceinline__ void tile_pixel(int tx, int ty, int& i, int& j, int& bx, int& by) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = tile_warp(), lane = threadIdx.x & 31;
   bx = tx * kTile + (warp % (kTile / kWarpW)) * kWarpW;
   by = ty * kTile + (warp / (kTile / kWarpW)) * kWarpH;
   i = bx + lane % kWarpW;
@@ -60,12 +76,12 @@ __device__ __forceinline__ bool reaches_block(float4 A, float ex, float ey, floa
          A.y + ey >= y0 + 0.5f && A.y - ey <= y0 + ((float)kWarpH - 0.5f);
 }
 
-// (tile, view) of this CTA: the list-walking kernels launch a (tiles, views) grid and take the
-// tiles in the order the binning wrote (longest list first). False for an order entry outside
-// [0, V nt) (checked build only; the CTA then does nothing).
+// (tile, view) of this CTA: the list-walking kernels launch a (tiles x kCtaPerTile, views) grid
+// and take the tiles in the order the binning wrote (longest list first). False for an order
+// entry outside [0, V nt) (checked build only; the CTA then does nothing).
 __device__ __forceinline__ bool block_tile(const int* __restrict__ order, int nt,
                                            unsigned int* bounds_word, int& t, int& v) {
-  const int o = order[blockIdx.y * gridDim.x + blockIdx.x];
+  const int o = order[(blockIdx.y * gridDim.x + blockIdx.x) / kCtaPerTile];
   if (!in_bounds((unsigned)o, (unsigned long long)nt * gridDim.y, bounds_word)) return false;
   v = o / nt;
   t = o - v * nt;
