@@ -4,7 +4,10 @@
 // contraction), IEEE division and square root, and denormals preserved. The preprocess, render
 // and replay decisions that turn floating point into integers (tile rectangle, depth order, the
 // 1/255 and 1e-4 thresholds, the 0.99 clamp) therefore depend only on the stated sequence of
-// correctly rounded fp32 operations; fused multiply-adds appear only where written as fmaf().
+// correctly rounded fp32 operations; fused multiply-adds appear only where written as fmaf() or
+// __ffma2_rn(). (-fmad=false does not cover packed pairs: the compiler fuses a packed product
+// into a packed add that is its only consumer, so packed products only feed scalar adds; see the
+// list-walking helpers.)
 #pragma once
 
 #include <cuda_runtime.h>

@@ -8,8 +8,10 @@
 // (o = sigmoid(a), alpha = o G, w = T alpha, rho = <r, c - C+>, q = sum w; the opacity-logit,
 // SH and projected-centre scores).
 //
-// One CTA per (tile, view), one thread per pixel of the 16x16 tile; the eight warps (an 8x4 pixel
-// block each) walk the tile's list independently, with no CTA barrier: each warp stages 32-entry
+// One CTA per (tile, view), one thread per pixel of the 16x16 tile, the CTAs taking the tiles in
+// the binning's launch order (longest list first, so that no long list starts in the last wave);
+// the eight warps (an 8x4 pixel block each) walk the tile's list independently, with no CTA
+// barrier: each warp stages 32-entry
 // chunks of records in its own shared-memory slice, keeps by ballot the entries whose precomputed
 // box reaches its block, and stops when all its pixels are saturated. Both passes evaluate alpha
 // through the same device function, so the replay takes exactly the render's decisions; the
@@ -27,13 +29,14 @@
 //
 // Replay arithmetic. The suffix numerators C_hat - P - T alpha c are formed per channel exactly
 // as the recovery equation writes them (their cancellation dominates the fp32 error of C+), then
-// multiplied by one correctly rounded reciprocal of T (1 - alpha) + eps. (Rewriting rho through
+// multiplied by one fast reciprocal of T (1 - alpha) + eps (T (1 - alpha) >= 1e-6 wherever the
+// result is used; relative error a few 1e-8). (Rewriting rho through
 // running dot products <r, P> is algebraically the same but moves that cancellation and costs
 // ~4e-4 relative token error.) Per entry and warp the seven per-pixel terms
 // (w, w r (3), w rho, w rho (p - mu2D) (2)) are summed by a transpose-reduction (each exchange
 // step halves the values a lane carries: 9 shuffles instead of 35), and the seven lanes holding a
 // result add it to the (view, Gaussian) accumulator with one fp64 atomic each -- seven global
-// atomics per (Gaussian, warp-strip). The SH block never enters the pixel loop: M_color w (B (x) r)
+// atomics per (Gaussian, warp block). The SH block never enters the pixel loop: M_color w (B (x) r)
 // factors into M_color B (x) (sum w r); the mean block Sigma^-1 (sum w rho d) is formed once per
 // (Gaussian, view) in finalisation.
 #include <algorithm>
