@@ -62,16 +62,19 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* s_warp, T* total) {
   return r;
 }
 
+// tile sums (the order of the adds does not matter: coalesced loads)
 template <typename TI>
 __global__ void __launch_bounds__(kScanThreads)
 k_scan_reduce(const TI* __restrict__ in, long long n, long long* __restrict__ part) {
   __shared__ long long s_warp[32];
   __shared__ long long s_tot;
-  const long long base = (long long)blockIdx.x * kScanTile + (long long)threadIdx.x * kScanIpt;
+  const long long base = (long long)blockIdx.x * kScanTile + threadIdx.x;
   long long s = 0;
 #pragma unroll
-  for (int k = 0; k < kScanIpt; ++k)
-    if (base + k < n) s += (long long)in[base + k];
+  for (int k = 0; k < kScanIpt; ++k) {
+    const long long i = base + (long long)k * kScanThreads;
+    if (i < n) s += (long long)in[i];
+  }
   block_exclusive_scan<long long>(s, s_warp, &s_tot);
   if (threadIdx.x == 0) part[blockIdx.x] = s_tot;
 }
@@ -94,24 +97,40 @@ __global__ void __launch_bounds__(1024) k_scan_partials(long long* part, int nb)
   if (threadIdx.x == 0) part[nb] = carry;
 }
 
+// exclusive scan of one tile plus its partial: coalesced loads into shared memory, a sequential
+// scan of kScanIpt contiguous values per thread, a block scan of the thread sums, coalesced
+// stores. The whole tile is read before any of it is written, so in == out is allowed.
+__device__ __forceinline__ int scan_pad(int i) { return i + (i >> 4); }  // 1 word per 16: banks
+
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(kScanThreads)
 k_scan_down(const TI* in, TO* out, long long n, const long long* __restrict__ part) {
+  __shared__ long long s_buf[kScanTile + kScanTile / 16];
   __shared__ long long s_warp[32];
-  const long long base = (long long)blockIdx.x * kScanTile + (long long)threadIdx.x * kScanIpt;
+  const long long base = (long long)blockIdx.x * kScanTile;
+#pragma unroll
+  for (int k = 0; k < kScanIpt; ++k) {
+    const int i = threadIdx.x + k * kScanThreads;
+    s_buf[scan_pad(i)] = base + i < n ? (long long)in[base + i] : 0;
+  }
+  __syncthreads();
   long long v[kScanIpt];
   long long s = 0;
 #pragma unroll
   for (int k = 0; k < kScanIpt; ++k) {
-    v[k] = base + k < n ? (long long)in[base + k] : 0;
-    const long long t = v[k];
+    const long long t = s_buf[scan_pad(threadIdx.x * kScanIpt + k)];
     v[k] = s;
     s += t;
   }
   const long long ex = block_exclusive_scan<long long>(s, s_warp, nullptr) + part[blockIdx.x];
 #pragma unroll
-  for (int k = 0; k < kScanIpt; ++k)
-    if (base + k < n) out[base + k] = (TO)(ex + v[k]);
+  for (int k = 0; k < kScanIpt; ++k) s_buf[scan_pad(threadIdx.x * kScanIpt + k)] = ex + v[k];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kScanIpt; ++k) {
+    const int i = threadIdx.x + k * kScanThreads;
+    if (base + i < n) out[base + i] = (TO)s_buf[scan_pad(i)];
+  }
 }
 
 __global__ void k_store_total(const long long* part, int nb, long long* dst) { *dst = part[nb]; }
