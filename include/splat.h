@@ -25,7 +25,9 @@
  *     waits for the per-view instance counts (a few words that kernels store into mapped
  *     pinned host memory). Nothing a call enqueues uses a copy engine: clears and these small
  *     exchanges are kernels, so a step never waits behind the caller's large host<->device
- *     copies on other streams.
+ *     copies on other streams. (When splat_bin_sort has to grow the instance lists -- the first
+ *     step of a workspace, or more instances than before -- the device allocation synchronises
+ *     with every stream; steady-state steps allocate nothing.)
  *   - Return value: SPLAT_OK (0) or a negative splat_status. No C++ exception crosses the ABI.
  *     On error, splat_last_error(ws) returns a NUL-terminated message owned by the workspace,
  *     valid until the next call on it. Argument errors are detected before any work is

@@ -95,6 +95,51 @@ def test_mixed_footprints_in_one_warp():
     assert counts.max() == 70 and (counts == 0).sum() >= 2 * 200
 
 
+def test_step_beside_large_copies_on_other_streams():
+    """The step's host exchange (instance counts out, view starts back) goes through mapped
+    memory, not a copy engine: a render + replay enqueued while 1 GiB host->device and
+    device->host copies are in flight on two other streams gives the same bits as a quiet run,
+    and the binning's count readback does not wait for those copies to finish."""
+    import time
+    import torch
+    from gaussian_splatting_raster_b200 import runner
+    sc = scenes.make(2)
+    obs = O.observe(sc, "f")
+    quiet = PU.gpu_run(sc, obs, with_acc=False)
+    n = 256 * 1024 * 1024  # 1 GiB of float32 each way
+    h_src = torch.empty(n, dtype=torch.float32).pin_memory()
+    h_dst = torch.empty(n, dtype=torch.float32).pin_memory()
+    d_dst = torch.empty(n, device="cuda")
+    d_src = torch.zeros(n, device="cuda")
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ds = runner.to_device(sc)
+    ws = runner.workspace_for(ds)
+    out = runner.alloc_outputs(ds)
+    obs_t = torch.as_tensor(obs).cuda()
+    # one step first: a workspace grows its instance lists on first use, and a device allocation
+    # synchronises with every stream (steady-state steps allocate nothing)
+    runner.render_and_score(ws, ds, obs_t, out)
+    torch.cuda.synchronize()
+    copies_done = torch.cuda.Event()
+    with torch.cuda.stream(s_in):
+        d_dst.copy_(h_src, non_blocking=True)
+    with torch.cuda.stream(s_out):
+        h_dst.copy_(d_src, non_blocking=True)
+        copies_done.record(s_out)
+    t0 = time.perf_counter()
+    runner.render_and_score(ws, ds, obs_t, out)  # bin_sort returns once its counts are read
+    t_step = time.perf_counter() - t0
+    in_flight = not copies_done.query()
+    torch.cuda.synchronize()
+    assert (out.img.cpu().numpy() == quiet["img"]).all()
+    assert (out.n_contrib.cpu().numpy() == quiet["n_contrib"]).all()
+    # (the fp64 atomic sums may be added in another order: tokens equal up to that rounding)
+    np.testing.assert_allclose(out.tokens.cpu().numpy(), quiet["tokens"], rtol=1e-6, atol=1e-9)
+    ws.close()
+    # the copies take tens of ms; the readback must not have waited for them
+    assert in_flight, f"the step ({t_step * 1e3:.1f} ms) ended after the copies"
+
+
 def test_empty_scene_and_all_culled():
     sc = scenes.tiny_scene(3, 5, 20, 24, V=2)
     sc.means[:, 2] = -1.0  # all behind the cameras
