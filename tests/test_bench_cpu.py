@@ -1,0 +1,99 @@
+"""Host-side checks of bench.py that need no GPU: the reference arm (the CPU oracle timed on the
+host) prints exactly one JSON line with the contract's keys, a non-zero rank of it prints nothing,
+the DRAM-traffic record is reported only for the workload and sources it was captured on, the
+peaks file falls back when absent, and the algorithmic byte counts split into the parts that
+grow with the instance count and the parts that do not."""
+import importlib.util
+import json
+import os
+import shutil
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CONTRACT = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+            "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config")
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _reference(extra_env=None):
+    env = dict(os.environ, **(extra_env or {}))
+    return subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "1",
+                           "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
+                          capture_output=True, text=True, timeout=600)
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = _reference()
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in CONTRACT + ("impl", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["unit"] == "Mpix/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["data"] == "synthetic"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "Mpix/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == _bench().WORKLOADS[1]
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    r = _reference({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
+
+
+def test_traffic_record_follows_workload_and_sources(tmp_path, monkeypatch):
+    b = _bench()
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    for kernel, e in rec["kernels"].items():
+        total = e["dram_read_bytes"] + e["dram_write_bytes"]
+        assert b.recorded_traffic(kernel, e["workload"]) == total
+        assert b.recorded_traffic(kernel, e["workload"] + "_other") is None
+    assert b.recorded_traffic("no_such_kernel", "any") is None
+    # a copy of the record and its sources answers the same until one source byte changes
+    kernel, e = next(iter(rec["kernels"].items()))
+    for f in e["sources"] + ["profiles/dram_traffic.json"]:
+        (tmp_path / f).parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(ROOT, f), tmp_path / f)
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    assert b.recorded_traffic(kernel, e["workload"]) == e["dram_read_bytes"] + e["dram_write_bytes"]
+    with open(tmp_path / e["sources"][-1], "a") as fh:
+        fh.write("\n")
+    assert b.recorded_traffic(kernel, e["workload"]) is None
+
+
+def test_peaks_file_and_fallback(tmp_path, monkeypatch):
+    b = _bench()
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    assert b.load_peaks()["source"] == "fallback"
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 1234.5, "sm_max_mhz": 1900}))
+    assert b.load_peaks() == {"hbm_gbs": 1234.5, "sm_max_mhz": 1900.0, "source": "measured"}
+
+
+def test_algorithmic_bytes_split_by_what_they_scale_with():
+    b = _bench()
+    sys.path.insert(0, ROOT)
+    from synth import scenes
+    sc = scenes.make(2)
+    a = b.algorithmic_bytes(sc, 1000, 0)
+    a2 = b.algorithmic_bytes(sc, 2000, 0)
+    per_instance = {"emit": 8, "tile_hist": 4, "tile_scatter": 12, "render": 40, "replay": 40,
+                    "backward": 40, "features": 40, "scatter": 80}
+    for k, v in a.items():
+        assert v >= 0, k
+        assert a2[k] - v == 1000 * per_instance.get(k, 0), k
+    # one depth pass more adds one histogram read and one key+index read and write per (v, g)
+    a4 = b.algorithmic_bytes(sc, 1000, 0, depth_passes=4)
+    VG = sc.V * sc.G
+    assert a4["depth_hist"] - a["depth_hist"] == 4 * VG
+    assert a4["depth_scatter"] - a["depth_scatter"] == 16 * VG
