@@ -554,6 +554,8 @@ int zero_async(Workspace& w, void* p, size_t bytes, cudaStream_t st, const char*
 int copy_words(Workspace& w, const void* src, void* dst, size_t bytes, cudaStream_t st,
                const char* what) {
   if (bytes == 0) return SPLAT_OK;
+  if ((bytes & 3) || ((uintptr_t)src & 3) || ((uintptr_t)dst & 3))
+    return set_err(w, SPLAT_ERR_INVALID_ARG, std::string(what) + ": copy of an unaligned range");
   const size_t n = bytes / 4;
   const unsigned blocks = (unsigned)((n + 255) / 256 < 64 ? (n + 255) / 256 : 64);
   k_copy_words<<<blocks, 256, 0, st>>>(static_cast<const uint32_t*>(src),

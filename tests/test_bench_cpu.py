@@ -53,23 +53,28 @@ def test_reference_arm_other_ranks_do_no_work():
 
 
 def test_traffic_record_follows_workload_and_sources(tmp_path, monkeypatch):
+    """A record answers only for its workload and only while its sources hash the same."""
+    import hashlib
     b = _bench()
-    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
-    for kernel, e in rec["kernels"].items():
-        total = e["dram_read_bytes"] + e["dram_write_bytes"]
-        assert b.recorded_traffic(kernel, e["workload"]) == total
-        assert b.recorded_traffic(kernel, e["workload"] + "_other") is None
-    assert b.recorded_traffic("no_such_kernel", "any") is None
-    # a copy of the record and its sources answers the same until one source byte changes
-    kernel, e = next(iter(rec["kernels"].items()))
-    for f in e["sources"] + ["profiles/dram_traffic.json"]:
+    srcs = ["gaussian_splatting_raster_b200/csrc/traverse.cuh",
+            "gaussian_splatting_raster_b200/csrc/raster.cu"]
+    for f in srcs:
         (tmp_path / f).parent.mkdir(parents=True, exist_ok=True)
         shutil.copy(os.path.join(ROOT, f), tmp_path / f)
+    m = hashlib.sha256()
+    for f in srcs:
+        m.update((tmp_path / f).read_bytes())
+    rec = {"kernels": {"replay": {"workload": "w1", "dram_read_bytes": 300, "dram_write_bytes": 45,
+                                  "sources": srcs, "sha256": m.hexdigest()}}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(b, "ROOT", str(tmp_path))
-    assert b.recorded_traffic(kernel, e["workload"]) == e["dram_read_bytes"] + e["dram_write_bytes"]
-    with open(tmp_path / e["sources"][-1], "a") as fh:
+    assert b.recorded_traffic("replay", "w1") == 345
+    assert b.recorded_traffic("replay", "w2") is None
+    assert b.recorded_traffic("render", "w1") is None
+    with open(tmp_path / srcs[0], "a") as fh:  # any change to a source retires the record
         fh.write("\n")
-    assert b.recorded_traffic(kernel, e["workload"]) is None
+    assert b.recorded_traffic("replay", "w1") is None
 
 
 def test_peaks_file_and_fallback(tmp_path, monkeypatch):
