@@ -56,3 +56,46 @@ def test_missing_library_fails_loudly(tmp_path):
     import gaussian_splatting_raster_b200 as P
     with pytest.raises(OSError):
         P.load_library(str(tmp_path / "nope.so"))
+
+
+# entry points whose first argument is the workspace handle (or, for splat_ws_create, the place
+# to store it): a NULL there is an argument error reported before any device work
+_HANDLE_CALLS = [
+    "splat_ws_create", "splat_project", "splat_bin_sort", "splat_render", "splat_score_replay",
+    "splat_score_partials", "splat_backward", "splat_render_features", "splat_scatter",
+    "splat_attribution", "splat_copy_projection", "splat_copy_tile_lists", "splat_copy_last",
+    "splat_copy_accumulators", "splat_pair_count", "splat_check_status", "splat_set_deterministic",
+    "splat_profile_enable", "splat_profile_read",
+]
+
+
+def _zero_args(fn):
+    args = []
+    for t in fn.argtypes:
+        if t in (ctypes.c_int, ctypes.c_longlong):
+            args.append(0)
+        elif t is ctypes.c_float:
+            args.append(ctypes.c_float(0.0))
+        else:  # pointers and handles
+            args.append(None)
+    return args
+
+
+def test_null_handle_is_an_argument_error(lib_path):
+    import gaussian_splatting_raster_b200 as P
+    L = P.load_library()
+    assert set(_HANDLE_CALLS) <= set(P.EXPORTS)
+    for name in _HANDLE_CALLS:
+        fn = getattr(L, name)
+        assert fn(*_zero_args(fn)) == -1, name  # SPLAT_ERR_INVALID_ARG
+    L.splat_ws_destroy(None)  # a no-op
+
+
+def test_kernel_group_names_and_build_flavour(lib_path):
+    import gaussian_splatting_raster_b200 as P
+    L = P.load_library()
+    names = [L.splat_kernel_name(i).decode() for i in range(P.KERNEL_GROUPS)]
+    assert len(set(names)) == P.KERNEL_GROUPS and "?" not in names
+    assert {"project", "render", "replay", "finalize", "backward"} <= set(names)
+    assert L.splat_kernel_name(-1) == b"?" and L.splat_kernel_name(P.KERNEL_GROUPS) == b"?"
+    assert L.splat_checked_build() == 0  # the release library
