@@ -343,3 +343,18 @@ def smooth_observation(seed: int, V: int, H: int, W: int) -> np.ndarray:
             f = _smooth_field(rng, H, W, n_waves=4)
             out[v, :, :, c] = 0.5 + 0.2 * f / 4.0
     return out
+
+
+def clamp_scene(seed: int = 51, G: int = 6, H: int = 24, W: int = 32, V: int = 2) -> Scene:
+    """A tiny scene in which the renderer's two clamps are active: Gaussian 1 is opaque (logit 7)
+    and wide (about 8 px standard deviation in the images) at the back, so alpha = min(0.99, o G)
+    saturates at 0.99 on the pixel centres within about 1 px of its projected centre; Gaussian 2
+    has a DC red coefficient of -3, so its red channel is below zero before the colour clamp in
+    every view. The other Gaussians are drawn as in ``tiny_scene``."""
+    sc = tiny_scene(seed, G, H, W, V=V, deg=1, opac_mean=0.0, opac_sigma=0.5,
+                    log_scale_mean=math.log(0.06))
+    sc.means[1] = [0.02, -0.03, 3.8]
+    sc.log_scales[1] = np.log([0.95, 0.9, 1.0])
+    sc.opac[1] = 7.0
+    sc.sh[2, 0, 0] = -3.0
+    return sc

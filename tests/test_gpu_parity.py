@@ -69,8 +69,31 @@ def test_sh_degrees_and_ragged_image(deg):
     _full_check(sc, obs, lam=0.5)
 
 
-def test_long_tile_list_uses_global_sort():
-    """One 16x16 tile with 12000 overlapping Gaussians: longer than the shared-memory sort."""
+
+def test_clamp_scene_tokens():
+    """Both score masks active: Gaussian 1 saturates at alpha = 0.99 on a few pixel centres
+    (M_alpha removes those pixels from its opacity and centre scores) and the red channel of
+    Gaussian 2 is clamped (M_color removes it from the SH block). The oracle's masks are pinned to
+    finite differences on this scene; the GPU tokens meet the usual bar against them."""
+    sc = scenes.clamp_scene()
+    obs = np.random.default_rng(5).uniform(0.2, 0.8, (sc.V, sc.H, sc.W, 3)).astype(np.float32)
+    g, o = _full_check(sc, obs)
+    flags = g["rec"][:, :, 15].view(np.int32)
+    assert ((flags[:, 2] & 7) == 6).all()  # red clamped in every view, on the GPU side too
+    p, L = o["proj"], o["lists"]
+    n_sat = 0
+    for v in range(sc.V):
+        for j in range(sc.H):
+            for i in range(sc.W):
+                tr = O.trace(p, L, sc.H, sc.W, sc.bg, v, i, j, "f")
+                n_sat += int(((tr[:, 0] == 1) & (tr[:, 1] == np.float32(0.99))).sum())
+    assert n_sat >= 4  # alpha clamp reached with the kernels' fp32 decisions
+    assert np.abs(g["tokens"][2, 4::3][: sc.d]).max() == 0.0  # clamped channel: zero SH score
+
+def test_long_tile_list():
+    """One 16x16 tile with 12000 overlapping Gaussians: a list of more than 8192 entries (many
+    32-entry chunks per warp, several counting-sort blocks for one tile) in bit-exact order, with
+    the render and tokens at their usual bars."""
     sc = scenes.tiny_scene(7, 12000, 16, 16, V=1, deg=1, depth_range=(1.0, 60.0),
                            log_scale_mean=math.log(0.05))
     obs = np.full((1, 16, 16, 3), 0.3, np.float32)

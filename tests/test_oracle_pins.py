@@ -455,6 +455,134 @@ def test_scores_equal_central_finite_differences(seed):
         np.testing.assert_allclose(tokens[g, 3] * qg[g], ga, rtol=1e-10)
 
 
+
+def test_score_masks_equal_central_differences_with_clamps_active():
+    """The replay's masks against the derivative they stand for. "Exact Score Operators" defines
+    M_alpha and M_color as the clamp-aware local VJP: where alpha = min(0.99, o G) sits at 0.99,
+    or a colour channel at its zero clamp, the derivative through that path is zero. On a scene
+    where both clamps are active (Gaussian 1 saturates at alpha = 0.99 on a few pixel centres,
+    the red channel of Gaussian 2 is clamped in every view), central differences of
+    L = 1/2 sum |C_hat - C_obs|^2 (no skip, stop or clamp decision flips within +-h) equal, per
+    Gaussian: the opacity-logit score sum_v (1 - o) Sa, the finalised SH block times q_g
+    (sum_v M_color Swr (x) B), the projected-centre score Sigma2D^{-1} Sd of every view, and the
+    finalised mean block times q_g (3-D mean through the projected centres). The same scores equal
+    the renderer backward's gradient for the opacity logit and the SH coefficients, and the scene
+    is checked to be sensitive: the pixels the masks remove carry far more than the tolerance."""
+    sc = scenes.clamp_scene()
+    p = O.project(sc, "d")
+    assert p["valid"].all()
+    rec = p["rec"]
+    assert (rec[:, 2, 13] == 6).all() and (rec[:, [0, 1, 3, 4, 5], 13] == 7).all()
+    L = O.bin_lists(p, sc.H, sc.W)
+    obs = np.random.default_rng(5).uniform(0.2, 0.8, (sc.V, sc.H, sc.W, 3)).astype(np.float32)
+    r = O.render(p, L, sc.H, sc.W, sc.bg, "d")
+    acc = O.replay(p, L, r, obs, sc.sh_degree, sc.H, sc.W, "d")["acc"]
+    tokens = O.finalize(p, acc, sc, lam=1.0)
+    qg = 1e-6 + sum(1e-6 + acc[v, :, 0] for v in range(sc.V))
+    d = sc.d
+    h = 1e-5
+    tol = 1e-6
+
+    # the alpha clamp is reached, and what the clamped pixels would add to Gaussian 1's opacity
+    # and centre scores is far above the tolerance
+    clamped_sa = np.zeros(sc.V)
+    clamped_sd = np.zeros((sc.V, 2))
+    n_clamped = 0
+    for v in range(sc.V):
+        for j in range(sc.H):
+            for i in range(sc.W):
+                tr = O.trace(p, L, sc.H, sc.W, sc.bg, v, i, j, "d")
+                for row in tr[(tr[:, 0] == 1) & (tr[:, 1] >= 0.99)]:
+                    assert row[1] == 0.99
+                    rr = r["img"][v, j, i] - obs[v, j, i]
+                    wrho = row[2] * row[1] * float(rr @ (row[3:6] - row[6:9]))
+                    clamped_sa[v] += wrho
+                    clamped_sd[v] += wrho * np.array([i + 0.5 - rec[v, 1, 0],
+                                                      j + 0.5 - rec[v, 1, 1]])
+                    n_clamped += 1
+    assert n_clamped >= 4
+
+    def rel(a, b):
+        a, b = np.asarray(a, float), np.asarray(b, float)
+        return np.abs(a - b).max() / max(np.abs(b).max(), 1e-12)
+
+    def L_of_scene(s2):
+        p2 = O.project(s2, "d")
+        assert (p2["rect"] == p["rect"]).all()
+        return _loss(sc, p2["rec"], L, obs, p2["valid"])[0]
+
+    # opacity logit, per Gaussian: sum_v (1 - o) Sa
+    sa = np.array([sum((1 - rec[v, g, 6]) * acc[v, g, 4] for v in range(sc.V))
+                   for g in range(sc.G)])
+    for g in range(sc.G):
+        s_p, s_m = _copy(sc), _copy(sc)
+        s_p.opac[g] += h
+        s_m.opac[g] -= h
+        fd = (L_of_scene(s_p) - L_of_scene(s_m)) / (float(s_p.opac[g]) - float(s_m.opac[g]))
+        assert rel(sa[g], fd) < tol, (g, sa[g], fd)
+        np.testing.assert_allclose(tokens[g, 3] * qg[g], sa[g], rtol=1e-10)
+    without_mask = sa[1] + sum((1 - rec[v, 1, 6]) * clamped_sa[v] for v in range(sc.V))
+    assert rel(without_mask, sa[1]) > 1e3 * tol
+
+    # SH coefficients, per Gaussian: the finalised block times q_g = sum_v M_color Swr (x) B
+    for g in range(sc.G):
+        fd = np.zeros((d, 3))
+        for k in range(d):
+            for ch in range(3):
+                s_p, s_m = _copy(sc), _copy(sc)
+                s_p.sh[g, k, ch] += h
+                s_m.sh[g, k, ch] -= h
+                fd[k, ch] = ((L_of_scene(s_p) - L_of_scene(s_m))
+                             / (float(s_p.sh[g, k, ch]) - float(s_m.sh[g, k, ch])))
+        an = tokens[g, 4:4 + 3 * d].reshape(d, 3) * qg[g]
+        assert rel(an, fd) < tol, (g, an, fd)
+        if g == 2:
+            assert (fd[:, 0] == 0).all() and (an[:, 0] == 0).all()  # clamped channel
+            unmasked_red = sum(acc[v, 2, 1] * p["B"][v, 2, :d] for v in range(sc.V))
+            assert np.abs(unmasked_red).max() > 1e3 * tol * np.abs(fd).max()
+
+    # projected centre, per view and Gaussian: Sigma2D^{-1} Sd (a step of 1e-4 px: at 1e-5 the
+    # rounding of L, ~1e-14, is 1e-6 of the smallest centre score here)
+    hc = 1e-4
+    for v in range(sc.V):
+        for g in range(sc.G):
+            fd = np.zeros(2)
+            for ax in range(2):
+                rp, rm = rec.copy(), rec.copy()
+                rp[v, g, ax] += hc
+                rm[v, g, ax] -= hc
+                fd[ax] = (_loss(sc, rp, L, obs, p["valid"])[0]
+                          - _loss(sc, rm, L, obs, p["valid"])[0]) / (2 * hc)
+            Q = np.array([[rec[v, g, 2], rec[v, g, 3]], [rec[v, g, 3], rec[v, g, 4]]])
+            an = Q @ acc[v, g, 5:7]
+            assert rel(an, fd) < tol, (v, g, an, fd)
+            if g == 1:
+                assert rel(Q @ (acc[v, 1, 5:7] + clamped_sd[v]), an) > 1e3 * tol
+
+    # 3-D mean through the projected centres: the finalised mean block times q_g
+    for g in range(sc.G):
+        fd = np.zeros(3)
+        for ax in range(3):
+            ls, xs = [], []
+            for sgn in (1, -1):
+                s2 = _copy(sc)
+                s2.means[g, ax] += sgn * h
+                xs.append(float(s2.means[g, ax]))
+                p2 = O.project(s2, "d")
+                rr = rec.copy()
+                rr[:, g, 0:2] = p2["rec"][:, g, 0:2]
+                ls.append(_loss(sc, rr, L, obs, p["valid"])[0])
+            fd[ax] = (ls[0] - ls[1]) / (xs[0] - xs[1])
+        assert rel(tokens[g, 0:3] * qg[g], fd) < 2 * tol, (g, tokens[g, 0:3] * qg[g], fd)
+
+    # the renderer backward's raw gradient: the same opacity-logit and SH derivatives
+    raw = O.run_backward(sc, obs, "d")["raw"]
+    np.testing.assert_allclose(raw[:, 10], sa, rtol=1e-9, atol=1e-12 * np.abs(sa).max())
+    sh_an = tokens[:, 4:4 + 3 * d] * qg[:, None]
+    np.testing.assert_allclose(raw[:, 11:11 + 3 * d], sh_an, rtol=1e-9,
+                               atol=1e-12 * np.abs(sh_an).max())
+
+
 def _copy(sc):
     import dataclasses
     return dataclasses.replace(sc, means=sc.means.copy(), opac=sc.opac.copy(), sh=sc.sh.copy())
