@@ -7,7 +7,10 @@ target views. Default workload: the DepthSplat-scale dense scene (5,898,240 Gaus
 3, 4 target views 512x960). Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
-                  [--path score|backward]
+                  [--path score|backward|attributes] [--cpu-threads T]
+
+--impl reference times the CPU oracle instead (one whole view per step, all host cores or T);
+the default arm reports the same oracle timing once as its cpu_baseline.
 
 --path backward times the renderer backward instead of the score replay (the gradient comparators:
 raw, detached, support- and parameter-scale-normalised gradients, all four per step).
@@ -78,8 +81,8 @@ def parse():
                          "target views at 256x448 (overrides --config)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-tiles", type=int, default=0,
-                    help="tiles per sample for the CPU oracle (0 = size for ~10-20 s)")
+    ap.add_argument("--cpu-threads", type=int, default=0,
+                    help="OpenMP threads of the CPU oracle (0 = all host cores)")
     return ap.parse_args()
 
 
@@ -163,12 +166,12 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
-def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu capture (profiles/dram_traffic.json), only
-    when the kernel's sources still hash to what was captured and the workload matches."""
+def _current_record(fname: str, kernel: str, workload: str):
+    """A kernel's entry of a committed ncu record under profiles/, only when it was captured on
+    this workload and the kernel's sources still hash to what was captured."""
     import hashlib
     try:
-        d = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))["kernels"][kernel]
+        d = json.load(open(os.path.join(ROOT, "profiles", fname)))["kernels"][kernel]
     except (OSError, KeyError, ValueError):
         return None
     if d.get("workload") != workload:
@@ -181,7 +184,22 @@ def recorded_traffic(kernel: str, workload: str):
             return None
     if m.hexdigest() != d["sha256"]:
         return None
-    return int(d["dram_read_bytes"]) + int(d["dram_write_bytes"])
+    return d
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture (profiles/dram_traffic.json)."""
+    d = _current_record("dram_traffic.json", kernel, workload)
+    return None if d is None else int(d["dram_read_bytes"]) + int(d["dram_write_bytes"])
+
+
+def recorded_pipes(kernel: str, workload: str):
+    """ncu pipe utilisation of the kernel (profiles/pipe_counters.json): FMA-pipe and ALU-pipe
+    cycles active and issue slots used, in % of peak sustained, from one captured launch."""
+    d = _current_record("pipe_counters.json", kernel, workload)
+    if d is None:
+        return None
+    return {k: d[k] for k in ("fma_pipe_pct", "alu_pipe_pct", "issue_active_pct") if k in d}
 
 
 def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dict:
@@ -223,64 +241,80 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
     }
 
 
-# algorithmic fp32 operations per traversed (pixel, list entry) pair, from the arithmetic the
-# method defines (the design notes count them): render = alpha (conic quadratic form, exp,
-# clamp/threshold tests) + transmittance + colour = 17 fp32 + 1 transcendental; replay = the same
-# alpha + suffix recovery (3 channels) + rho + masks + 7 weighted terms = 45 fp32 + 2 special;
-# backward = the same alpha + transmittance recovery + d C_hat / d alpha (two 3-channel dot
-# products) + 10 weighted terms + suffix update = 49 fp32 + 2 special; features = alpha (13 fp32 +
-# 1 special) + w + 9 channels x (mul, add) + transmittance = 35; scatter = two traversals (the
-# 9-channel map scatter, 26, and the attribution, 19) = 45
-ALU_OPS_PER_PAIR = {"render": 18, "replay": 47, "backward": 51, "features": 35, "scatter": 45}
+# Algorithmic fp32 work of the list-walking kernels, in lane operations (an fma is one; the
+# exponential is the Cody-Waite one both sides use: x log2(e) and its rounding, two reduction fmas,
+# a degree-7 Horner polynomial, the scale = 12), counted from the method's arithmetic by pair
+# class: every traversed (pixel, list entry) pair needs the exponent of G and the skip decision
+# (p - mu2D, the conic's quadratic form, the positive-exponent test and the comparison with the
+# Gaussian's precomputed exponent cut that decides alpha < 1/255 without the exponential = 13);
+# each composited pair needs alpha = min(0.99, o exp(pw)) and the 1/255 test (15) and then its
+# pass's own work:
+#   render    T (1 - alpha), the stop test, w = alpha T, C += w c (unfused)                 = 10
+#   replay    T (1 - alpha), w, w c, C_hat - P - w c (3 channels), the reciprocal of the
+#             denominator, c - C+ (3 fmas), rho, both masks, w r, w rho, w rho d, P += w c  = 31
+#   backward  1 / (1 - alpha), T, w, w r, <r, c> T - <r, S> / (1 - alpha), h = ga alpha,
+#             h d, h d d^T (3), S += w c                                                    = 28
+#   features  T (1 - alpha), w, 9 channels (mul, add)                                       = 21
+#   scatter   two traversals: the 9-channel map (T, w, 9 products) and the attribution
+#             (T, w, w, w |r|)                                                             = 12 + 5
+# so a kernel's work per step = a x traversed pairs + b x composited pairs with (a, b) below.
+ALU_OPS = {"render": (13, 25), "replay": (13, 46), "backward": (13, 43), "features": (13, 36),
+           "scatter": (26, 47)}
+
+
+def alu_ops(kernel: str, pairs: int, composited: int) -> int:
+    a, b = ALU_OPS[kernel]
+    return a * pairs + b * composited
 
 
 # ----------------------------------------------------------------------------------------------
-# CPU oracle baseline: bounded sample, extrapolated to the metric's unit
+# CPU oracle baseline: one whole view of the workload, timed as it runs
 
-def cpu_oracle_sample(sc, obs_np, seconds_hint=15.0, tiles=0, path="score"):
+def cpu_oracle_view(sc, obs_np, path="score", threads=0):
+    """The oracle (fp32 decision mode, OpenMP) over one complete view of the workload: projection
+    and binning of every Gaussian into view 0, render and the pass of `path` over every tile of
+    that view, and the per-Gaussian finalisation. Nothing is sampled or scaled: value = the
+    view's pixels / the measured wall time. threads > 0 sets the oracle's OpenMP thread count."""
     import numpy as np
     from oracle import oracle as O
+    if threads > 0:
+        O.lib().orc_set_threads(int(threads))
     one = _one_view(sc)
     t0 = time.perf_counter()
     p = O.project(one, "f")
     L = O.bin_lists(p, one.H, one.W)
     t_pb = time.perf_counter() - t0
-    TX, TY = O.n_tiles(one.H, one.W)
-    nt = TX * TY
-    rng = np.random.default_rng(0)
-    n_s = tiles or max(8, min(nt, int(nt * 0.04)))
-    sel = np.stack([np.zeros(n_s, np.int32), rng.choice(nt, n_s, replace=False).astype(np.int32)], 1)
     t1 = time.perf_counter()
-    r = O.render(p, L, one.H, one.W, one.bg, "f", sel=sel)
+    r = O.render(p, L, one.H, one.W, one.bg, "f")
     if path == "backward":
-        accb = O.backward(p, L, r, obs_np[:1], one.bg, one.H, one.W, "f", sel=sel)
+        accb = O.backward(p, L, r, obs_np[:1], one.bg, one.H, one.W, "f")
     elif path == "attributes":
         rng2 = np.random.default_rng(1)
         f = rng2.uniform(0, 1, (one.G, N_ATTR)).astype(np.float32)
         m = rng2.uniform(0, 1, (1, one.H, one.W, N_ATTR)).astype(np.float32)
-        O.render_features(p, L, r, f, one.H, one.W, "f", sel=sel)
-        O.scatter(p, L, r, m, one.H, one.W, "f", sel=sel)
-        O.attribution(p, L, r, obs_np[:1], one.H, one.W, "f", sel=sel)
+        O.render_features(p, L, r, f, one.H, one.W, "f")
+        O.scatter(p, L, r, m, one.H, one.W, "f")
+        O.attribution(p, L, r, obs_np[:1], one.H, one.W, "f")
     else:
-        O.replay(p, L, r, obs_np[:1], one.sh_degree, one.H, one.W, "f", sel=sel)
+        rp = O.replay(p, L, r, obs_np[:1], one.sh_degree, one.H, one.W, "f")
     t_rr = time.perf_counter() - t1
     t2 = time.perf_counter()
     if path == "backward":
         O.gradients(p, accb, one, "f")
     elif path == "score":
-        O.finalize(p, np.zeros((1, one.G, 8)), one)
+        O.finalize(p, rp["acc"], one)
     t_fin = time.perf_counter() - t2
     second = {"backward": "backward", "attributes": "attribute render + scatters",
               "score": "replay"}[path]
     last = {"backward": "gradient chain", "attributes": "nothing further",
             "score": "finalisation"}[path]
-    t_view = t_pb + t_rr * nt / n_s + t_fin
+    t_view = t_pb + t_rr + t_fin
     return {"value": one.H * one.W / t_view / 1e6, "unit": "Mpix/s",
             "cores": int(O.lib().orc_num_threads()), "kind": "oracle",
-            "sample": (f"1 of {sc.V} views: projection + binning of all {sc.G} Gaussians "
-                       f"({t_pb:.2f} s), render + {second} of {n_s}/{nt} random tiles "
-                       f"({t_rr:.2f} s, scaled to the view), {last} ({t_fin:.2f} s)"),
-            "seconds": t_pb + t_rr + t_fin}
+            "sample": (f"view 1 of {sc.V}, whole: projection + binning of all {sc.G} Gaussians "
+                       f"({t_pb:.2f} s), render + {second} of all {one.H}x{one.W} pixels "
+                       f"({t_rr:.2f} s), {last} ({t_fin:.2f} s)"),
+            "seconds": t_view}
 
 
 def _one_view(sc):
@@ -335,23 +369,24 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 def run_reference(args):
-    """Reference arm: the CPU oracle, as it stands, on bounded samples of the same workload."""
+    """Reference arm: the CPU oracle, as it stands, one whole view of the same workload per step
+    (every Gaussian projected and binned, every pixel rendered and replayed, every Gaussian
+    finalised); ms_per_step is the mean measured time of those steps."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import numpy as np
-    from oracle import oracle as O
     from synth import scenes
     sc = make_scene(args)
     obs = scenes.smooth_observation(99, 1, sc.H, sc.W)
     times, samples = [], []
     for it in range(args.warmup + args.steps):
-        s = cpu_oracle_sample(sc, obs, tiles=args.cpu_tiles or 0, path=args.path)
+        s = cpu_oracle_view(sc, obs, path=args.path, threads=args.cpu_threads)
         if it >= args.warmup:
             times.append(s["seconds"])
             samples.append(s)
-    val = statistics.median([s["value"] for s in samples])
-    ms = 1e3 * sc.H * sc.W / (val * 1e6)
+    # one step = one whole view, as it ran: steps x ms_per_step is the timed work
+    ms = 1e3 * sum(times) / len(times)
+    val = sc.H * sc.W * len(times) / sum(times) / 1e6
     line = {"metric": METRICS[args.path], "value": val, "unit": "Mpix/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
@@ -470,6 +505,7 @@ def main():
     pairs = ws.pair_count()
     # composited pairs: sum over this rank's pixels of the entries that contributed (n_contrib)
     composited = int(last_out["o"].n_contrib.sum(dtype=torch.int64).item())
+    pairs_rank, composited_rank = pairs, composited  # this rank's, for its kernels' rooflines
     n_total = int(sum(n_inst))
 
     # ---- timed region: device time per step (CUDA events), L2 flushed between steps ----------
@@ -599,13 +635,16 @@ def main():
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms_per_step"])
     dom_ms = per_kernel[dom]["ms_per_step"]
     lanes = torch.cuda.get_device_properties(dev).multi_processor_count * 128
-    if dom in ALU_OPS_PER_PAIR:
-        ops = ALU_OPS_PER_PAIR[dom] * pairs
+    if dom in ALU_OPS:
+        ops = alu_ops(dom, pairs_rank, composited_rank)
         achieved = ops / (dom_ms * 1e-3) / 1e12
         peak = lanes * peaks["sm_max_mhz"] * 1e6 / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "Tops/s (fp32 pipe)", "frac": achieved / peak,
                 "traffic": recorded_traffic(dom, workload_name(args, sc)),
+                "ncu_pipes": recorded_pipes(dom, workload_name(args, sc)),
+                "work": f"{ALU_OPS[dom][0]} ops x traversed pairs + {ALU_OPS[dom][1]} ops x "
+                        f"composited pairs",
                 "peak_source": f"{lanes} fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz "
                                f"({peaks['source']} max clock)"}
     else:
@@ -617,6 +656,9 @@ def main():
     for k, v in per_kernel.items():
         if k in ab:
             v["algorithmic_GBps"] = ab[k] / (v["ms_per_step"] * 1e-3) / 1e9
+        if k in ALU_OPS:
+            v["alu_frac"] = (alu_ops(k, pairs_rank, composited_rank) / (v["ms_per_step"] * 1e-3)
+                             / (lanes * peaks["sm_max_mhz"] * 1e6))
     render_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in
                     ("project", "depth_hist", "depth_scatter", "emit", "tile_hist",
                      "hist_scan", "tile_scatter", "tile_ranges", "render", "other"))
@@ -626,7 +668,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_sample(sc, obs.cpu().numpy(), tiles=args.cpu_tiles, path=args.path)
+        cpu = cpu_oracle_view(sc, obs.cpu().numpy(), path=args.path, threads=args.cpu_threads)
         cpu.pop("seconds", None)
 
     if rank == 0:

@@ -1,7 +1,8 @@
 """Host-side checks of bench.py that need no GPU: the reference arm (the CPU oracle timed on the
 host) prints exactly one JSON line with the contract's keys, a non-zero rank of it prints nothing,
-the DRAM-traffic record is reported only for the workload and sources it was captured on, the
-peaks file falls back when absent, and the algorithmic byte counts split into the parts that
+the DRAM-traffic and pipe-counter records are reported only for the workload and sources they were
+captured on, the reference arm's steps are what it ran, the fp32 work counts split by pair class,
+the peaks file falls back when absent, and the algorithmic byte counts split into the parts that
 grow with the instance count and the parts that do not."""
 import importlib.util
 import json
@@ -75,6 +76,56 @@ def test_traffic_record_follows_workload_and_sources(tmp_path, monkeypatch):
     with open(tmp_path / srcs[0], "a") as fh:  # any change to a source retires the record
         fh.write("\n")
     assert b.recorded_traffic("replay", "w1") is None
+
+
+def test_pipe_record_follows_workload_and_sources(tmp_path, monkeypatch):
+    import hashlib
+    b = _bench()
+    srcs = ["gaussian_splatting_raster_b200/csrc/raster.cu"]
+    (tmp_path / srcs[0]).parent.mkdir(parents=True, exist_ok=True)
+    shutil.copy(os.path.join(ROOT, srcs[0]), tmp_path / srcs[0])
+    rec = {"kernels": {"render": {"workload": "w1", "fma_pipe_pct": 41.5, "alu_pipe_pct": 30.0,
+                                  "issue_active_pct": 80.0, "sources": srcs,
+                                  "sha256": hashlib.sha256((tmp_path / srcs[0]).read_bytes())
+                                  .hexdigest()}}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "pipe_counters.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    assert b.recorded_pipes("render", "w1") == {"fma_pipe_pct": 41.5, "alu_pipe_pct": 30.0,
+                                                "issue_active_pct": 80.0}
+    assert b.recorded_pipes("render", "w2") is None and b.recorded_pipes("replay", "w1") is None
+    with open(tmp_path / srcs[0], "a") as fh:
+        fh.write("\n")
+    assert b.recorded_pipes("render", "w1") is None
+
+
+def test_alu_work_counts_by_pair_class():
+    """Every traversed pair costs the exponent and skip decision; only composited pairs cost
+    alpha and the pass's own arithmetic."""
+    b = _bench()
+    for k, (a, c) in b.ALU_OPS.items():
+        assert b.alu_ops(k, 1, 0) == a and b.alu_ops(k, 0, 1) == c
+        assert b.alu_ops(k, 1000, 10) == 1000 * a + 10 * c
+    # alpha (15) is part of every pass's composited cost; the replay does the most per pair
+    assert min(c for _, c in b.ALU_OPS.values()) >= 15 + 10
+    assert b.ALU_OPS["replay"][1] > b.ALU_OPS["render"][1]
+
+
+def test_reference_steps_are_what_ran():
+    """The reference arm's steps x ms_per_step is time it actually spent (no extrapolated
+    samples): it fits inside the process's own wall time."""
+    import time
+    t0 = time.perf_counter()
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "2",
+                        "--steps", "2", "--warmup", "1"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=600)
+    wall = time.perf_counter() - t0
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip())
+    assert d["steps"] == 2 and "whole" in d["cpu_baseline"]["sample"]
+    assert d["steps"] * d["ms_per_step"] * 1e-3 < wall
+    # one step is one 128 x 128 view: value and ms_per_step describe the same time
+    assert abs(d["value"] - 128 * 128 / (d["ms_per_step"] * 1e3)) < 1e-6 * d["value"]
 
 
 def test_peaks_file_and_fallback(tmp_path, monkeypatch):
