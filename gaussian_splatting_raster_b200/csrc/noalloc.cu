@@ -8,11 +8,12 @@
 // scratch is a file-scope __device__ array of fixed size, present on every GPU that loads this
 // library until the process exits. The caller passes only its input and output buffers.
 //
-// Variant of the per-tile depth sort of the tile binning (its global-memory path): one CTA runs a
-// stable least-significant-digit radix sort with 8-bit digits over the order-preserving 32-bit
-// image of the depths, keeping per-warp digit counters in shared memory.
-#include <mutex>
-
+// For the positive depths the projection produces, the result equals the binning's per-view depth
+// order (the binning sorts the raw fp32 bits of each view's visible depths, stably, and emits
+// every tile's list in that order), so it is also the order of each tile's contributors. The
+// order of negative values, -0.0 and NaNs is this entry point's own (an order-preserving map of
+// the fp32 bits). One CTA runs a stable least-significant-digit radix sort with 8-bit digits
+// over that 32-bit image of the depths, keeping per-warp digit counters in shared memory.
 #include "common.cuh"
 
 namespace splat {
@@ -24,9 +25,6 @@ constexpr int kNaThreads = kNaWarps * 32;
 
 // ping-pong keys and values: [2][kNaMax] + [2][kNaMax] 32-bit words (4 MiB at 2^18 entries)
 static __device__ __align__(256) uint32_t g_noalloc_scratch[4 * kNaMax];
-
-std::mutex g_na_mutex;
-void* g_na_ptr[64] = {nullptr};  // device address of the scratch, per device ordinal
 
 __device__ __forceinline__ uint32_t na_lanemask_lt() {
   uint32_t m;
@@ -144,25 +142,14 @@ extern "C" int splat_sort_depths_noalloc(const float* depths, int n, int* order,
   if (n < 0 || (n > 0 && (!depths || !order))) return SPLAT_ERR_INVALID_ARG;
   if (n > kNaMax) return SPLAT_ERR_CAPACITY;
   if (n == 0) return SPLAT_OK;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+  // The array's device address in the current device's context, looked up on every call: host
+  // code cannot use the symbol itself (a host-side stand-in), and a cached address would go
+  // stale when the module is loaded again (after cudaDeviceReset, or in another context). The
+  // lookup is host-side, not a stream operation; the first one on a device also loads the module.
+  void* scratch = nullptr;
+  if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch) {
     cudaGetLastError();
     return SPLAT_ERR_CUDA;
-  }
-  void* scratch = nullptr;
-  {
-    // first call on a device: resolve the array's device address (host code cannot use the
-    // symbol itself, which is only a host-side stand-in)
-    std::lock_guard<std::mutex> lock(g_na_mutex);
-    if (!g_na_ptr[dev]) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-        cudaGetLastError();
-        return SPLAT_ERR_CUDA;
-      }
-      g_na_ptr[dev] = p;
-    }
-    scratch = g_na_ptr[dev];
   }
   k_sort_depths_noalloc<<<1, kNaThreads, 0, (cudaStream_t)stream>>>(
       depths, n, static_cast<uint32_t*>(scratch), order);

@@ -290,22 +290,27 @@ const char* splat_kernel_name(int id);
  * For callers that cannot allocate device memory where they need an ordering -- code running
  * under another framework's allocator hooks or memory pool, plugins handed fixed buffers, phases
  * where cudaMalloc/cudaFree would synchronise the device or fail -- this computes, without
- * allocating anything, the order in which the tile binning lists a tile's contributors: the
- * stable ascending order of n fp32 depths (equal values keep their index order). Writes
- * order[0..n) as int32 indices into depths. Both are DEVICE pointers owned by the caller.
+ * allocating anything, the stable ascending order of n fp32 depths (equal values keep their
+ * index order). For the positive depths the projection produces this is the binning's per-view
+ * depth order, and so the order in which it lists a tile's contributors. Writes order[0..n) as
+ * int32 indices into depths. Both are DEVICE pointers owned by the caller.
  *
  * Scratch: one fixed file-scope __device__ array of 4 * SPLAT_NOALLOC_MAX_N 32-bit words
  * (4 MiB), which every GPU that loads this library holds until the process exits. No cudaMalloc,
  * cudaFree or allocating library routine is called.
  *   - n > SPLAT_NOALLOC_MAX_N returns SPLAT_ERR_CAPACITY before any work; n < 0, or NULL
  *     pointers with n > 0, return SPLAT_ERR_INVALID_ARG; n == 0 returns SPLAT_OK.
- *   - The first call on each device looks up the array's device address once
- *     (cudaGetSymbolAddress); make that first call before any stream capture on that device.
+ *   - Every call looks up the array's device address in the current context
+ *     (cudaGetSymbolAddress, host-side); the first lookup on a device also loads the module, so
+ *     make the first call on each device before any stream capture there. After
+ *     cudaDeviceReset the next call finds the array again (its contents are then undefined,
+ *     which no call depends on).
  *   - All calls share the array and it keeps the last call's contents (nothing in it needs to
  *     start at zero: every word read is written first by the same call). Calls whose kernels
  *     overlap on one GPU -- different streams, or host threads without ordering -- race and
  *     corrupt each other's results; serialise them on one stream.
- *   - Order of values: negatives before positives, -0.0 before +0.0, NaNs by bit pattern.
+ *   - Order of values (this entry point's own beyond the positive depths of the projection):
+ *     negatives before positives, -0.0 before +0.0, NaNs by bit pattern.
  *   - Enqueued on `stream` (a cudaStream_t, NULL = legacy default); returns without waiting.
  *     Kernel-launch failures return SPLAT_ERR_CUDA.
  */
