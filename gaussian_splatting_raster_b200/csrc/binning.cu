@@ -154,6 +154,11 @@ int ensure_part(Workspace& w, long long nb) {
 constexpr int kBinWarps = 8;
 constexpr int kBinThreads = kBinWarps * 32;
 constexpr int kDepthChunk = 16384;  // items per block, depth-key passes
+// widest depth digit: the varying bits are split into ceil(bits / max) passes of equal width
+#ifndef SPLAT_DEPTH_DIGIT_MAX
+#define SPLAT_DEPTH_DIGIT_MAX 11
+#endif
+constexpr int kDepthDigitMax = SPLAT_DEPTH_DIGIT_MAX;
 constexpr int kTileChunk = 16384;   // items per block, tile pass
 
 // Items of view v are [start(v), start(v + 1)); each view is cut into blocks of `chunk` items.
@@ -620,6 +625,14 @@ int launch_binning(Workspace& w, cudaStream_t st) {
       w.umask_cap = cap;
     }
   }
+  {
+    const size_t need = ((size_t)(N >> 7) + (size_t)w.V * w.nt + 1) * 1024;
+    if (need > w.lmask_cap) {
+      const size_t cap = need + need / 4;
+      if ((rc = grow(w, &w.lmask, cap, "per-pixel composited-entry masks"))) return rc;
+      w.lmask_cap = cap;
+    }
+  }
   // ---- 1. depth order of every view's Gaussians --------------------------------------------
   // highest bit that varies among any view's visible keys -> number of digit passes
   int hb = -1;
@@ -633,7 +646,7 @@ int launch_binning(Workspace& w, cudaStream_t st) {
     if (vary) hb = max(hb, 31 - __builtin_clz(vary));
   }
   const int bits = hb + 1;
-  const int passes = bits == 0 ? 0 : (bits + 10) / 11;
+  const int passes = bits == 0 ? 0 : (bits + kDepthDigitMax - 1) / kDepthDigitMax;
   const int dbits = passes ? (bits + passes - 1) / passes : 0;
   const uint32_t* order = nullptr;  // sorted Gaussian indices per view (nullptr: index order)
   if (passes > 0 && VG > 0) {

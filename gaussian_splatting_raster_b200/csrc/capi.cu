@@ -84,7 +84,7 @@ int alloc_mapped(Workspace& w, T** h, T** d, size_t n, const char* what) {
 void free_all(Workspace& w) {
   void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
-                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.accb, w.sacc,
+                 w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.lmask, w.accb, w.sacc,
                  w.acc_fix, w.accb_fix, w.tile_order};
   for (void* p : dev)
     if (p) cudaFree(p);
@@ -281,6 +281,7 @@ int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int*
   if ((rc = splat::launch_render(w, bg, img, T_final, n_contrib, (cudaStream_t)stream))) return rc;
   w.img = img;
   w.Tfin = T_final;
+  w.ncon = n_contrib;
   w.bg = bg;
   w.stage = 3;
   return SPLAT_OK;
@@ -450,9 +451,7 @@ int splat_copy_accumulators(splat_ws* ws, double* acc, void* stream) {
   if (VG == 0) return SPLAT_OK;
   int rc;
   if ((rc = check_dev_ptr(w, acc, "acc"))) return rc;
-  cudaError_t e = cudaMemcpyAsync(acc, w.acc, VG * splat::kAccN * 8, cudaMemcpyDeviceToDevice,
-                                  (cudaStream_t)stream);
-  return e == cudaSuccess ? SPLAT_OK : cuda_fail(w, "copy accumulators", e);
+  return splat::launch_acc_to_double(w, acc, (cudaStream_t)stream);
 }
 
 int splat_pair_count(splat_ws* ws, long long* pairs, void* stream) {

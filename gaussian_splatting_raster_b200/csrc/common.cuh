@@ -181,7 +181,7 @@ struct Workspace {
   int4* rect = nullptr;      // [V*G]
   int* counts = nullptr;     // [V*G] tiles touched
   long long* offs = nullptr; // [V*G + 1] exclusive scan of counts
-  double* acc = nullptr;     // [V*G*8]
+  float* acc = nullptr;      // [V*G*8] score sums: (q, w r (3)), (w rho, w rho d (2), unused)
   double* accb = nullptr;    // [max_V*max_G*10] renderer-backward sums, allocated on first use
   double* sacc = nullptr;    // [G*C] scatter sums, grown on demand
   // deterministic mode: 128-bit fixed-point (low, high) words of the replay / backward sums
@@ -194,6 +194,7 @@ struct Workspace {
   int* last = nullptr;       // [V*H*W]
   const float* img = nullptr;   // C_hat written by the last render (caller-owned)
   const float* Tfin = nullptr;  // final transmittance written by the last render (caller-owned)
+  const int* ncon = nullptr;    // contributor counts written by the last render (caller-owned)
   const float* bg = nullptr;    // background colour of the last render (caller-owned)
 
   // scan partials (int64)
@@ -220,6 +221,10 @@ struct Workspace {
   // per (tile, 32-entry chunk, warp): entries some pixel of the warp composited (render -> replay)
   uint32_t* umask = nullptr;
   size_t umask_cap = 0;
+  // per (tile, pixel, 32-entry chunk): entries that pixel composited (render -> score replay),
+  // four chunks of one pixel per 16-byte group, pixels side by side
+  uint32_t* lmask = nullptr;
+  size_t lmask_cap = 0;
 
   // tile histogram [sum_v nt * blocks_v] (int32, scanned in place)
   size_t hist_cap = 0;
@@ -313,6 +318,8 @@ int launch_features(Workspace& w, const float* feats, int C, float* out, cudaStr
 int launch_scatter(Workspace& w, const float* map, const float* obs, int C, float* out,
                    cudaStream_t st);
 int launch_pair_count(Workspace& w, cudaStream_t st);
+// the score sums widened to doubles into out [V*G*8] (the inspection copy)
+int launch_acc_to_double(Workspace& w, double* out, cudaStream_t st);
 unsigned int bounds_word_raster(cudaStream_t st);
 unsigned int bounds_word_binning(cudaStream_t st);
 unsigned int bounds_word_attributes(cudaStream_t st);

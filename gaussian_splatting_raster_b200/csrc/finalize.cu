@@ -63,7 +63,7 @@ __device__ void eig3_sym(double a00, double a01, double a02, double a11, double 
 // sum_v M_color (Swr (x) B) is added into the shared-memory column `col` (stride P) at 4 + k.
 template <int DEG, int P>
 __device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
-                                          const double* __restrict__ acc,
+                                          const float* __restrict__ acc,
                                           const float* __restrict__ views, int G, int V, int g,
                                           double& qsum, double b[3], double& sa, double A[6],
                                           float* col) {
@@ -75,13 +75,14 @@ __device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
     const int flags = __float_as_int(r3.w);
     if (!(flags & kFlagVisible)) continue;
     const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1];
-    const double2* a2 = reinterpret_cast<const double2*>(acc + i * kAccN);
-    const double2 a01 = a2[0], a23 = a2[1], a45 = a2[2], a67 = a2[3];
-    const double qgv = eps + a01.x;
+    // (q, w r (3)) and (w rho, w rho d (2), unused)
+    const float4* a4 = reinterpret_cast<const float4*>(acc + i * kAccN);
+    const float4 aq = a4[0], as = a4[1];
+    const double qgv = eps + (double)aq.x;
     qsum += qgv;
-    sa += (1.0 - (double)r1.y) * a45.x;
+    sa += (1.0 - (double)r1.y) * (double)as.x;
     // per-view products in fp32 (rounding ~1e-7 relative), sums over views in double
-    const float sd0 = (float)a45.y, sd1 = (float)a67.x;
+    const float sd0 = as.y, sd1 = as.z;
     const float sm0 = r0.z * sd0 + r0.w * sd1;
     const float sm1 = r0.w * sd0 + r1.x * sd1;
     // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
@@ -115,9 +116,9 @@ __device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
       const float il = rsqrtf(dw0 * dw0 + dw1 * dw1 + dw2 * dw2);
       sh_poly<DEG>(dw0 * il, dw1 * il, dw2 * il, B);
     }
-    const float w0 = (flags & 1) ? (float)a01.y : 0.0f;
-    const float w1 = (flags & 2) ? (float)a23.x : 0.0f;
-    const float w2 = (flags & 4) ? (float)a23.y : 0.0f;
+    const float w0 = (flags & 1) ? aq.y : 0.0f;
+    const float w1 = (flags & 2) ? aq.z : 0.0f;
+    const float w2 = (flags & 4) ? aq.w : 0.0f;
 #pragma unroll
     for (int k = 0; k < D; ++k) {
       col[(4 + 3 * k) * P] += B[k] * w0;
@@ -171,7 +172,7 @@ __device__ __forceinline__ void store_rows(const float* s_tile, int ncols, int g
 // fused single-device path: sums over all views, then the token
 template <int DEG>
 __global__ void __launch_bounds__(kFinThreads, 4)
-k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
+k_finalize(const float4* __restrict__ rec, const float* __restrict__ acc,
            const float* __restrict__ views, int G, int V, double lambda,
            float* __restrict__ tokens) {
   constexpr int D = (DEG + 1) * (DEG + 1);
@@ -197,7 +198,7 @@ k_finalize(const float4* __restrict__ rec, const double* __restrict__ acc,
 // [qsum, b(3), sa, A(6: 00 01 02 11 12 22), SH block (3d)] = 11 + 3d floats per Gaussian
 template <int DEG>
 __global__ void __launch_bounds__(kFinThreads, 4)
-k_partials(const float4* __restrict__ rec, const double* __restrict__ acc,
+k_partials(const float4* __restrict__ rec, const float* __restrict__ acc,
            const float* __restrict__ views, int G, int V, float* __restrict__ partials) {
   constexpr int D = (DEG + 1) * (DEG + 1);
   constexpr int K = 11 + 3 * D;

@@ -54,7 +54,8 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
          const long long* __restrict__ tile_off, const int* __restrict__ order,
          int G, int H, int W, int TX, int nt,
          const float* __restrict__ bgp, float* __restrict__ img, float* __restrict__ Tout,
-         int* __restrict__ ncout, int* __restrict__ last, uint32_t* __restrict__ umask) {
+         int* __restrict__ ncout, int* __restrict__ last, uint32_t* __restrict__ umask,
+         uint32_t* __restrict__ lmask) {
   int t, v;
   if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
@@ -75,13 +76,17 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   float4* wa = s_a + warp * 32;
   float4* wb = s_b + warp * 32;
   float2* wc = s_c + warp * 32;
+  // this pixel's composited-entry mask words (read by the score replay): chunk cc at
+  // lmw[1024 (cc / 4) + cc % 4]
+  uint32_t* lmw = lmask + lmask_region(s, gt) + 4 * (twarp * 32 + lane);
+  int cc = 0;  // chunks walked
   const float x0f = (float)bx, y0f = (float)by;
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int n = 0, lst = 0;
   bool done = !inside;
   const float4* recv = rec + (size_t)v * G * kRecF4;
-  for (long long base = s; base < e; base += 32) {
+  for (long long base = s; base < e; base += 32, ++cc) {
     if (__all_sync(0xffffffffu, done)) break;
     const long long k = base + lane;
     bool hit = false;
@@ -128,6 +133,7 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     }
     const uint32_t ubits = __reduce_or_sync(0xffffffffu, lbits);
     if (lane == 0) umask[chunk_index(base, gt) * 8 + twarp] = ubits;
+    lmw[(size_t)(cc >> 2) * 1024 + (cc & 3)] = lbits;
     __syncwarp();
   }
   if (inside) {
@@ -180,24 +186,27 @@ __device__ __forceinline__ void add_fixed(unsigned long long* lohi, float x) {
   if (hi) atomicAdd(lohi + 1, hi);
 }
 
-// (high, low) pairs -> doubles: dst[k] = (hi 2^64 + lo) 2^-60
-__global__ void k_fixed_to_double(const unsigned long long* __restrict__ src,
-                                  double* __restrict__ dst, long long n) {
+// (high, low) pairs -> T (double or float): dst[k] = (hi 2^64 + lo) 2^-60, rounded once to T
+template <typename T>
+__global__ void k_fixed_to(const unsigned long long* __restrict__ src, T* __restrict__ dst,
+                           long long n) {
   for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
        k += (long long)gridDim.x * blockDim.x) {
     const unsigned long long lo = src[2 * k], hi = src[2 * k + 1];
-    dst[k] = ldexp((double)(long long)hi, 64 - kFixShift) + ldexp((double)lo, -kFixShift);
+    dst[k] = (T)(ldexp((double)(long long)hi, 64 - kFixShift) + ldexp((double)lo, -kFixShift));
   }
 }
 
-template <bool kDet>
+// Score replay in deterministic mode: each warp walks the entries that some pixel of its block
+// composited, reduces the seven per-pixel terms of each entry over the warp (a fixed tree) and
+// adds the warp's sums as fixed-point integers (order-independent).
 __global__ void __launch_bounds__(kThreads, 5 * kCtaPerTile)  // 48 registers: 40 warps per SM
-k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-         const long long* __restrict__ tile_off, const int* __restrict__ order,
-         int G, int H, int W, int TX, int nt,
-         const float* __restrict__ img, const float* __restrict__ obs,
-         const int* __restrict__ last, const uint32_t* __restrict__ umask,
-         double* __restrict__ acc, unsigned long long* __restrict__ acc_fix) {
+k_replay_det(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
+             const long long* __restrict__ tile_off, const int* __restrict__ order,
+             int G, int H, int W, int TX, int nt,
+             const float* __restrict__ img, const float* __restrict__ obs,
+             const int* __restrict__ last, const uint32_t* __restrict__ umask,
+             unsigned long long* __restrict__ acc_fix) {
   int t, v;
   if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
@@ -209,7 +218,7 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   // Like the render, each warp walks the list on its own (no CTA barriers), in 32-entry chunks;
   // per chunk it stages and evaluates only the entries the render recorded as composited by some
   // pixel of the warp -- every other entry contributes nothing to any of its pixels. Its
-  // per-entry sums go straight from the seven lanes holding them to the fp64 accumulators.
+  // per-entry sums go straight from the seven lanes holding them to the fixed-point words.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
   const int twarp = tile_warp();                                 // block in the tile
   __shared__ float4 s_a[kThreads], s_b[kThreads];
@@ -234,7 +243,6 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   }
   const int wmax = __reduce_max_sync(0xffffffffu, lst);  // entries this warp must traverse
   const float4* recv = rec + (size_t)v * G * kRecF4;
-  double* accv = acc + (size_t)v * G * kAccN;
   float T = 1.0f, P2 = 0.0f;  // transmittance, prefix colour (channels 0 and 1 packed)
   float2 P01 = make_float2(0.0f, 0.0f);
   const float2 Ch01 = make_float2(Ch0, Ch1), r01 = make_float2(r0, r1);
@@ -318,15 +326,246 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
         x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
         if ((lane & 3) == 0 && slot < 7 && x[0] != 0.0f)
-        {
-          if constexpr (kDet)
-            add_fixed(acc_fix + 2 * (((size_t)v * G + wg[q]) * kAccN + slot), x[0]);
-          else
-            atomicAdd(accv + (size_t)wg[q] * kAccN + slot, (double)x[0]);
-        }
+          add_fixed(acc_fix + 2 * (((size_t)v * G + wg[q]) * kAccN + slot), x[0]);
       }
     }
     __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Score replay (the default accumulation mode): per warp, one of two traversals.
+//
+// Per-pixel walks: each lane walks only the list entries ITS pixel composited -- read from the
+// per-pixel masks the render stored -- in list order, keeping the pixel's prefix transmittance T
+// and colour P exactly as the recovery equation needs them, and adds each (pixel, entry) pair's
+// terms straight into the (view, Gaussian) sums with two 16-byte vector reductions into L2
+// (red.global.add.v4.f32: (w, w r) and, where M_alpha holds, (w rho, w rho (p - mu2D), 0)). The
+// warp runs as many iterations as its longest walk.
+//
+// Union loop: the warp visits every entry that some pixel of its block composited (the render's
+// per-warp masks), all 32 lanes evaluate it, the seven per-pixel terms are summed over the warp
+// (the transpose-reduction) and lanes 0 and 16 issue the two reductions once per (entry, warp).
+//
+// The walk does a pair's arithmetic once but costs one or two L2 reductions per pair (the L2
+// reduction rate bounds it); the union loop spends ~160 instructions per visited entry whatever
+// the number of lanes that composited it, but reduces once. So each warp counts its union entries
+// U (the render's masks) and its composited pairs P (the pixels' contributor counts) and takes
+// the union loop when P >= kUnionLanes U -- entries composited by many of its pixels at once, as
+// with large Gaussians -- and the walks otherwise (pixel-aligned scenes: ~7 lanes per entry).
+// Either way the per-pixel terms are the same fp32 values; the sums are fp32 and the order of the
+// additions is not fixed, so their last bits vary from run to run (the deterministic mode gives
+// fixed bits).
+#ifndef SPLAT_UNION_LANES
+#define SPLAT_UNION_LANES 9
+#endif
+constexpr int kUnionLanes = SPLAT_UNION_LANES;
+
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// one composited (pixel, entry) pair of the replay: the suffix numerators C_hat - P - w c per
+// channel in the recovery equation's order, unfused like the render's colour sum (at the last
+// entry C_hat - P - w c is exactly the background term), one fast reciprocal of T (1 - alpha)
+// (>= 1e-6 here), rho, the seven terms x (x[4..6] zero where M_alpha is off), then P and T
+struct PixelState {
+  float2 Ch01, r01, P01;
+  float Ch2, r2, P2, T;
+};
+__device__ __forceinline__ bool replay_pair(PixelState& ps, const Entry& E, float c0, float c1,
+                                            float c2, float x[8]) {
+  const float al = E.alpha;
+  const float den = ps.T * (1.0f - al);
+  const float w = al * ps.T;
+  const float2 ww = make_float2(w, w);
+  const float2 c01 = make_float2(c0, c1);
+  const float2 wc01 = __fmul2_rn(ww, c01);
+  const float wc2 = w * c2;
+  const float2 cp01 = __ffma2_rn(ps.P01, make_float2(-1.0f, -1.0f), ps.Ch01);
+  const float nn0 = cp01.x - wc01.x;
+  const float nn1 = cp01.y - wc01.y;
+  const float nn2 = (ps.Ch2 - ps.P2) - wc2;
+  const float inv = __fdividef(1.0f, den + 1e-12f);
+  const float2 a01 = __ffma2_rn(make_float2(nn0, nn1), make_float2(-inv, -inv), c01);
+  const float rho = fmaf(ps.r01.x, a01.x, fmaf(ps.r01.y, a01.y, ps.r2 * fmaf(-nn2, inv, c2)));
+  const float2 wr01 = __fmul2_rn(ww, ps.r01);
+  x[0] = w;
+  x[1] = wr01.x;
+  x[2] = wr01.y;
+  x[3] = w * ps.r2;
+  const bool ma = (den >= 1e-4f) && (al < 0.99f);  // M_alpha
+  if (ma) {
+    const float wr = w * rho;
+    const float2 wd = __fmul2_rn(make_float2(wr, wr), make_float2(E.dx, E.dy));
+    x[4] = wr;
+    x[5] = wd.x;
+    x[6] = wd.y;
+  }
+  ps.P01.x = ps.P01.x + wc01.x;
+  ps.P01.y = ps.P01.y + wc01.y;
+  ps.P2 = ps.P2 + wc2;
+  ps.T = den;
+  return ma;
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
+k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
+         const long long* __restrict__ tile_off, const int* __restrict__ order,
+         int G, int H, int W, int TX, int nt, const float* __restrict__ img,
+         const float* __restrict__ obs, const int* __restrict__ last,
+         const int* __restrict__ ncon, const uint32_t* __restrict__ umask,
+         const uint32_t* __restrict__ lmask, float* __restrict__ acc) {
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;  // CTA-uniform
+  const int tx = t % TX, ty = t / TX;
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
+  const bool inside = i < W && j < H;
+  const long long s = tile_off[(size_t)v * (nt + 1) + t];
+  const int gt = v * nt + t;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int twarp = tile_warp();
+  PixelState ps;
+  ps.T = 1.0f;
+  ps.P01 = make_float2(0.0f, 0.0f);
+  ps.P2 = 0.0f;
+  float Ch0 = 0.0f, Ch1 = 0.0f, r0 = 0.0f, r1 = 0.0f;
+  ps.Ch2 = 0.0f;
+  ps.r2 = 0.0f;
+  int lst = 0, nc = 0;
+  if (inside) {
+    const size_t p = ((size_t)v * H + j) * W + i;
+    Ch0 = img[3 * p];
+    Ch1 = img[3 * p + 1];
+    ps.Ch2 = img[3 * p + 2];
+    r0 = Ch0 - obs[3 * p];
+    r1 = Ch1 - obs[3 * p + 1];
+    ps.r2 = ps.Ch2 - obs[3 * p + 2];
+    lst = last[p];
+    nc = ncon[p];
+  }
+  ps.Ch01 = make_float2(Ch0, Ch1);
+  ps.r01 = make_float2(r0, r1);
+  const float px = (float)i + 0.5f, py = (float)j + 0.5f;
+  const float4* recv = rec + (size_t)v * G * kRecF4;
+  float* accv = acc + (size_t)v * G * kAccN;
+
+  // the warp's union entries U and composited pairs P
+  const int wmax = __reduce_max_sync(0xffffffffu, lst);
+  const int wch = (wmax + 31) >> 5;
+  int u = 0;
+  for (int c = lane; c < wch; c += 32) u += __popc(umask[chunk_index(s + 32LL * c, gt) * 8 + twarp]);
+  const int U = __reduce_add_sync(0xffffffffu, u);
+  const int P = __reduce_add_sync(0xffffffffu, nc);
+  if (U == 0) return;  // warp-uniform: nothing composited here
+
+  if (P >= kUnionLanes * U) {
+    // ---- union loop ----------------------------------------------------------------------
+    __shared__ float4 s_a[kThreads], s_b[kThreads];
+    __shared__ float2 s_c[kThreads];
+    __shared__ uint32_t s_g[kThreads];
+    float4* wa = s_a + warp * 32;
+    float4* wb = s_b + warp * 32;
+    float2* wc = s_c + warp * 32;
+    uint32_t* wg = s_g + warp * 32;
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    for (int base = 0; base < wmax; base += 32) {
+      uint32_t bits = umask[chunk_index(s + base, gt) * 8 + twarp];
+      if (!bits) continue;  // warp-uniform
+      bool bad = false;
+      if ((bits >> lane) & 1u) {
+        const uint32_t g = ids[s + base + lane];
+        bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
+        if (!bad) {
+          const float4* r = recv + (size_t)g * kRecF4;
+          const float4 c = r[2];
+          wa[lane] = r[0];
+          wb[lane] = r[1];
+          wc[lane] = make_float2(c.x, c.y);
+          wg[lane] = g;
+        }
+      }
+      if (kChecked) bits &= ~__ballot_sync(0xffffffffu, bad);
+      __syncwarp();
+      while (bits) {  // warp-uniform: entries some pixel of this warp composited, in list order
+        const int q = __ffs(bits) - 1;
+        bits &= bits - 1;
+        float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+        bool used = false;
+        if (base + q < lst) {
+          const float4 A = wa[q], Bq = wb[q];
+          const float2 Cq = wc[q];
+          const Entry E = eval_entry(A, Bq, Cq.y, px, py);
+          if (E.use) {
+            used = true;
+            replay_pair(ps, E, Bq.z, Bq.w, Cq.x, x);
+          }
+        }
+        if (__any_sync(0xffffffffu, used)) {
+          tr_step<4>(x, b4, 16);
+          tr_step<2>(x, b3, 8);
+          tr_step<1>(x, b2, 4);
+          x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
+          x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
+          // value k now sits in lanes 4k .. 4k + 3: lanes 0 and 16 collect four each
+          const float s1 = __shfl_down_sync(0xffffffffu, x[0], 4);
+          const float s2 = __shfl_down_sync(0xffffffffu, x[0], 8);
+          const float s3 = __shfl_down_sync(0xffffffffu, x[0], 12);
+          float* a = accv + (size_t)wg[q] * kAccN;
+          if (lane == 0) red_add4(a, x[0], s1, s2, s3);
+          if (lane == 16 && (x[0] != 0.0f || s1 != 0.0f || s2 != 0.0f))
+            red_add4(a + 4, x[0], s1, s2, 0.0f);
+        }
+      }
+      __syncwarp();
+    }
+    return;
+  }
+
+  // ---- per-pixel walks (no warp-wide operation below: lanes leave independently) ------------
+  const int cend = (lst + 31) >> 5;  // chunks holding this pixel's composited entries
+  if (cend == 0) return;
+  // this pixel's mask words: chunk c's in m, the rest of its group of four in n1..n3, the next
+  // group prefetched in pre
+  const uint4* lm = reinterpret_cast<const uint4*>(lmask + lmask_region(s, gt)) + (twarp * 32 + lane);
+  const uint4 g0 = __ldg(lm);
+  uint32_t m = g0.x, n1 = g0.y, n2 = g0.z, n3 = g0.w;
+  uint4 pre = make_uint4(0u, 0u, 0u, 0u);
+  if (4 < cend) pre = __ldg(lm + 256);
+  int c = 0;
+  for (;;) {
+    while (!m) {  // next chunk with an entry of this pixel
+      if (++c >= cend) return;
+      if ((c & 3) == 0) {
+        m = pre.x;
+        n1 = pre.y;
+        n2 = pre.z;
+        n3 = pre.w;
+        if (c + 4 < cend) pre = __ldg(lm + (size_t)((c >> 2) + 1) * 256);
+      } else {
+        m = n1;
+        n1 = n2;
+        n2 = n3;
+      }
+    }
+    const int q = __ffs(m) - 1;
+    m &= m - 1u;
+    const uint32_t g = ids[s + 32LL * c + q];
+    if (!in_bounds(g, (unsigned)G, &g_bounds_word)) continue;
+    const float4* r = recv + (size_t)g * kRecF4;
+    const float4 A = __ldg(r), Bq = __ldg(r + 1);
+    const float c2 = __ldg(reinterpret_cast<const float*>(r + 2));
+    // the render's alpha, bit for bit (a composited entry always passes the exponent cut)
+    const Entry E = eval_entry(A, Bq, -INFINITY, px, py);
+    if (!E.use) continue;
+    float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    const bool ma = replay_pair(ps, E, Bq.z, Bq.w, c2, x);
+    float* a = accv + (size_t)g * kAccN;
+    red_add4(a, x[0], x[1], x[2], x[3]);
+    if (ma) red_add4(a + 4, x[4], x[5], x[6], 0.0f);
   }
 }
 
@@ -459,6 +698,12 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   }
 }
 
+__global__ void k_widen(const float* __restrict__ src, double* __restrict__ dst, long long n) {
+  for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
+       k += (long long)gridDim.x * blockDim.x)
+    dst[k] = (double)src[k];
+}
+
 __global__ void k_pair_sum(const int* __restrict__ last, long long n, long long* out) {
   long long sacc = 0;
   for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
@@ -475,7 +720,8 @@ int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int
   dim3 grid(w.nt * kCtaPerTile, w.V);
   const int tok = prof_begin(w, st, SPLAT_K_RENDER);
   k_render<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
-                                      w.nt, bg, img, T_final, n_contrib, w.last, w.umask);
+                                      w.nt, bg, img, T_final, n_contrib, w.last, w.umask,
+                                      w.lmask);
   prof_end(w, st, tok);
   return check_launch(w, "render kernel");
 }
@@ -500,10 +746,11 @@ static int fix_buffer(Workspace& w, unsigned long long** buf, size_t& cap, int n
                     "deterministic sums clear");
 }
 
-static int fix_to_double(Workspace& w, const unsigned long long* src, double* dst, int nslot,
-                         cudaStream_t st) {
+template <typename T>
+static int fix_to(Workspace& w, const unsigned long long* src, T* dst, int nslot,
+                  cudaStream_t st) {
   const long long n = (long long)w.V * w.G * nslot;
-  k_fixed_to_double<<<(unsigned)std::min<long long>((n + 255) / 256, 8 * 148), 256, 0, st>>>(
+  k_fixed_to<T><<<(unsigned)std::min<long long>((n + 255) / 256, 8 * 148), 256, 0, st>>>(
       src, dst, n);
   return check_launch(w, "fixed-point conversion kernel");
 }
@@ -515,21 +762,21 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
   if (det) {
     rc = fix_buffer(w, &w.acc_fix, w.acc_fix_cap, kAccN, st);
   } else if (w.G > 0) {
-    rc = zero_async(w, w.acc, (size_t)w.V * w.G * kAccN * sizeof(double), st, "accumulator clear");
+    rc = zero_async(w, w.acc, (size_t)w.V * w.G * kAccN * sizeof(float), st, "accumulator clear");
   }
   if (!rc) {
     dim3 grid(w.nt * kCtaPerTile, w.V);
     if (det)
-      k_replay<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
-                                                w.nt, w.img, obs, w.last, w.umask, w.acc,
-                                                w.acc_fix);
+      k_replay_det<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H,
+                                              w.W, w.TX, w.nt, w.img, obs, w.last, w.umask,
+                                              w.acc_fix);
     else
-      k_replay<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
-                                                 w.nt, w.img, obs, w.last, w.umask, w.acc,
-                                                 nullptr);
+      k_replay<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W,
+                                          w.TX, w.nt, w.img, obs, w.last, w.ncon, w.umask,
+                                          w.lmask, w.acc);
     rc = check_launch(w, "replay kernel");
   }
-  if (!rc && det) rc = fix_to_double(w, w.acc_fix, w.acc, kAccN, st);
+  if (!rc && det) rc = fix_to<float>(w, w.acc_fix, w.acc, kAccN, st);
   prof_end(w, st, tok);
   return rc;
 }
@@ -556,9 +803,16 @@ int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {
                                                    w.umask, w.accb, nullptr);
     rc = check_launch(w, "backward kernel");
   }
-  if (!rc && det) rc = fix_to_double(w, w.accb_fix, w.accb, kAccBN, st);
+  if (!rc && det) rc = fix_to<double>(w, w.accb_fix, w.accb, kAccBN, st);
   prof_end(w, st, tok);
   return rc;
+}
+
+int launch_acc_to_double(Workspace& w, double* out, cudaStream_t st) {
+  const long long n = (long long)w.V * w.G * kAccN;
+  if (n == 0) return SPLAT_OK;
+  k_widen<<<(unsigned)std::min<long long>((n + 255) / 256, 8 * 148), 256, 0, st>>>(w.acc, out, n);
+  return check_launch(w, "accumulator copy kernel");
 }
 
 int launch_pair_count(Workspace& w, cudaStream_t st) {

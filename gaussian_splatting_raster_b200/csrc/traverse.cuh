@@ -92,6 +92,18 @@ __device__ __forceinline__ bool block_tile(const int* __restrict__ order, int nt
 // distinct for every chunk of every tile, at most N / 32 + V * nt
 __device__ __forceinline__ long long chunk_index(long long p, int gt) { return (p >> 5) + gt; }
 
+// Per-pixel composited-entry masks: the render stores, for every 32-entry chunk its warp walks,
+// one word per pixel (bit q: the pixel composited list entry 32 c + q of its tile). Four
+// consecutive chunks of one pixel form a 16-byte group, and the 256 pixels' groups of chunks
+// 4 gr .. 4 gr + 3 lie side by side (a warp stores 512 contiguous bytes per group; a pixel loads
+// one group per four chunks). The tile's region starts at word 1024 ((s >> 7) + gt) (s = the
+// tile's first list position, gt = v nt + t) and holds ceil(len / 128) groups of 1024 words; the
+// regions of consecutive tiles do not overlap because ceil(len / 128) <= (e >> 7) - (s >> 7) + 1,
+// and all of them fit in 1024 ((N >> 7) + V nt + 1) words for N list entries in total.
+__device__ __forceinline__ size_t lmask_region(long long s, int gt) {
+  return (size_t)1024 * (size_t)((s >> 7) + gt);
+}
+
 // alpha of one list entry at pixel centre (px, py), with the rasteriser's skip rules
 __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
                                             float py) {

@@ -111,9 +111,9 @@ int splat_bin_sort(splat_ws* ws, long long* n_instances_out, void* stream);
  *   img       [V,H,W,3] C_hat = sum T alpha c + T_final bg
  *   T_final   [V,H,W]   final transmittance
  *   n_contrib [V,H,W]   number of composited Gaussians (int32)
- * bg is a device pointer to 3 floats. The replay reads img back (it is C_hat), and the backward
- * img, T_final and bg, so these must stay unmodified until splat_score_replay / splat_backward
- * have run.
+ * bg is a device pointer to 3 floats. The replay reads img back (it is C_hat) and n_contrib (the
+ * per-pixel composited counts size its work per warp), and the backward img, T_final and bg, so
+ * these must stay unmodified until splat_score_replay / splat_backward have run.
  */
 int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int* n_contrib,
                  void* stream);
@@ -126,7 +126,10 @@ int splat_render(splat_ws* ws, const float* bg, float* img, float* T_final, int*
  * masks with M_alpha = (T (1 - alpha) >= 1e-4 and alpha < 0.99) and M_color (colour clamp
  * inactive), forms r = C_hat - C_obs, rho = <r, c - C+>, w = T alpha and accumulates per (g, v)
  *   q = sum w, sum w r, sum M_alpha w rho, sum M_alpha w rho (p - mu2D)
- * (reduction over each warp's pixels, then fp64 atomics). Then, per Gaussian over the views where it
+ * in fp32 (per warp either every pixel's own composited entries reduced pair by pair, or each
+ * entry summed over the warp first and reduced once; the order of the additions is not fixed, so
+ * the last bits vary between runs -- see splat_set_deterministic). Then, per Gaussian over the
+ * views where it
  * is visible: q_gv = 1e-6 + q, q_g = 1e-6 + sum_v q_gv, gamma = q_gv / q_g, and
  *   tokens[g] = [ b_mu (3) = sum_v gamma J^T Sigma2D^-1 Sd / q_gv,
  *                 s_alpha (1) = sum_v gamma (1 - o) Sa / q_gv,
@@ -222,8 +225,8 @@ int splat_attribution(splat_ws* ws, const float* obs, float* out, void* stream);
  * replay (splat_score_replay, splat_score_partials) and the renderer backward add their per-(view,
  * Gaussian) sums as 128-bit fixed-point integers (units of 2^-60; two 64-bit integer atomics with
  * an exact carry), which do not depend on the order of the adds: tokens and gradients are then
- * the same bits on every run, which exposes any race between runs. Off by default (fp64 atomics:
- * results agree to rounding order). The first deterministic call allocates 16 bytes per sum of
+ * the same bits on every run, which exposes any race between runs. Off by default (fp32
+ * reductions: results agree to rounding order). The first deterministic call allocates 16 bytes per sum of
  * the workspace maxima (SPLAT_ERR_OOM when that fails); each call then clears them and adds one
  * conversion pass. Takes effect from the next call.
  */
@@ -260,7 +263,8 @@ int splat_copy_tile_lists(splat_ws* ws, long long* tile_offsets, int* ids, void*
  * composited entry (0 when none), i.e. the number of entries both passes traverse. */
 int splat_copy_last(splat_ws* ws, int* last, void* stream);
 
-/* Per-(v, g) sums after splat_score_replay: acc [V,G,8] fp64 = q, Swr(3), Sa, Sd(2), 0. */
+/* Per-(v, g) sums after splat_score_replay: acc [V,G,8] fp64 = q, Swr(3), Sa, Sd(2), 0 (the sums
+ * are kept in fp32 and widened by this copy). */
 int splat_copy_accumulators(splat_ws* ws, double* acc, void* stream);
 
 /* Gaussian-pixel pairs traversed by the last render (sum over pixels of `last`); synchronises. */

@@ -16,12 +16,16 @@ TOKEN_FLOOR = 1e-3
 SH_COLOUR_ATOL = 4e-6
 
 
-def gpu_run(scene, obs, lam=1.0, with_acc=True):
+def gpu_run(scene, obs, lam=1.0, with_acc=True, det=False):
+    """The CUDA path over one scene; det=True uses the deterministic accumulation mode (sums
+    independent of the order of the additions)."""
     import torch
     from gaussian_splatting_raster_b200 import runner
 
     ds = runner.to_device(scene)
     ws = runner.workspace_for(ds)
+    if det:
+        ws.deterministic(True)
     out = runner.alloc_outputs(ds)
     obs_t = torch.as_tensor(np.ascontiguousarray(obs, np.float32)).cuda()
     n = runner.render_and_score(ws, ds, obs_t, out, lam)

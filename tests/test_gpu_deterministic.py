@@ -1,7 +1,7 @@
 """Deterministic accumulation (splat_set_deterministic): fixed-point integer atomics make the
 replay's and the backward's per-(view, Gaussian) sums independent of the order of the adds, so two
-runs give the same bits; the results still meet the oracle's bars and agree with the fp64-atomic
-mode to rounding."""
+runs give the same bits; the results still meet the oracle's bars and agree with the default
+(floating-point reduction) mode to rounding."""
 import numpy as np
 import pytest
 
@@ -49,7 +49,7 @@ def test_two_runs_give_the_same_bits(cfg):
     obs = O.observe(sc, "f") if cfg == 2 else scenes.smooth_observation(5, sc.V, sc.H, sc.W)
     (z1, g1), (z2, g2) = _runs(sc, obs, True)
     assert torch.equal(z1, z2) and torch.equal(g1, g2)
-    # agrees with the fp64-atomic mode to rounding
+    # agrees with the default floating-point reductions to rounding
     (z3, g3), = _runs(sc, obs, False, n=1)
     za, zb = z1.cpu().numpy().astype(np.float64), z3.cpu().numpy().astype(np.float64)
     assert PU.token_errors(za, zb).max() <= 1e-5
