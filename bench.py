@@ -203,14 +203,17 @@ def recorded_pipes(kernel: str, workload: str):
 
 
 def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dict:
-    """Bytes each kernel group must move by its definition (unique inputs + outputs), per step;
-    depth_passes = the number of depth-digit passes the binning ran."""
+    """Bytes each kernel group must move by its definition, per step; depth_passes = the number of
+    depth-digit passes the binning ran. The projection and the finalisation use the per-unit
+    figures of the path's scope table (projection: the parameters read once, 4 (11 + 3d) B per
+    Gaussian, and ~52 B written per (view, Gaussian); finalisation: 28 + 16 B read per (view,
+    Gaussian) and the (9 + 3d) x 4 B token written per Gaussian); the binning kernels, which
+    replace the table's 43-bit instance sort, count their own unique inputs and outputs."""
     G, V, H, W, d = sc.G, sc.V, sc.H, sc.W, sc.d
     px = V * H * W
     TX, TY = (W + 15) // 16, (H + 15) // 16
     return {
-        # read the parameters once, write per (v, g) record (64 B), rectangle (16 B), count (4 B)
-        "project": G * (4 * (3 + 3 + 4 + 1) + 12 * d) + V * G * (64 + 16 + 4),
+        "project": G * 4 * (11 + 3 * d) + V * G * 52,
 
         # one depth-digit pass per launch over every (v, g): histogram reads the keys, the
         # scatter reads key + index and writes both
@@ -225,8 +228,10 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
         "tile_scatter": n_inst * (4 + 4 + 4),
         # gather 36 B per list entry staged, write C_hat, T, n, last
         "render": n_inst * (4 + 36) + px * 24,
-        "replay": n_inst * (4 + 36) + px * (12 + 12 + 4) + V * G * 64,
-        "finalize": V * G * (64 + 64) + G * 4 * (9 + 3 * d),
+        # gather 36 B per list entry, read C_hat, C_obs, the list bound and the contributor
+        # count per pixel, add into 32 B of sums per (v, g)
+        "replay": n_inst * (4 + 36) + px * (12 + 12 + 4 + 4) + V * G * 32,
+        "finalize": V * G * (28 + 16) + G * 4 * (9 + 3 * d),
         # backward: list entries as the replay, per pixel C_hat, C_obs, T_final, last; ten fp64
         # sums per (v, g); the chain reads records (48 B) and sums (80 B) per (v, g), the
         # parameters, and writes four gradient rows

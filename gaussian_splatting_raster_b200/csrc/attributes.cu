@@ -72,8 +72,8 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       if (!bad) {
         const float4* r = recv + (size_t)g * kRecF4;
         wa[lane] = r[0];
-        wb[lane] = r[1];
-        wc[lane] = r[2].y;
+        wb[lane] = r[2];
+        wc[lane] = reinterpret_cast<const float*>(r + 1)[1];  // cut
         const float* fg = feats + (size_t)g * C + c0;
 #pragma unroll
         for (int k = 0; k < CB; ++k) wf[lane * CB + k] = k < nc ? fg[k] : 0.0f;
@@ -85,7 +85,9 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       const int q = __ffs(bits) - 1;
       bits &= bits - 1;
       if (base + q < lst) {
-        const Entry E = eval_entry(wa[q], wb[q], wc[q], px, py);
+        float4 A, Bq;
+        entry_operands(wa[q], wb[q], A, Bq);
+        const Entry E = eval_entry(A, Bq, wc[q], px, py);
         if (E.use) {
           const float w = E.alpha * T;
           if constexpr (CB % 2 == 0) {  // two products per packed multiply, scalar sums
@@ -176,8 +178,8 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       if (!bad) {
         const float4* r = recv + (size_t)g * kRecF4;
         wa[lane] = r[0];
-        wb[lane] = r[1];
-        wc[lane] = r[2].y;
+        wb[lane] = r[2];
+        wc[lane] = reinterpret_cast<const float*>(r + 1)[1];  // cut
         wg[lane] = g;
       }
     }
@@ -191,7 +193,9 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       for (int k = 0; k < NV; ++k) x[k] = 0.0f;
       bool used = false;
       if (base + q < lst) {
-        const Entry E = eval_entry(wa[q], wb[q], wc[q], px, py);
+        float4 A, Bq;
+        entry_operands(wa[q], wb[q], A, Bq);
+        const Entry E = eval_entry(A, Bq, wc[q], px, py);
         if (E.use) {
           used = true;
           const float w = E.alpha * T;

@@ -122,14 +122,14 @@ k_grad(const float4* __restrict__ rec, const double* __restrict__ accb,
       // all loads of the view issued together (one memory round trip per view); the record and
       // sums of a view where g is culled are read but not used
       const float4 r3 = rec[iv * kRecF4 + 3];  // (z, x_c, y_c, flags)
-      const float4 r0 = rec[iv * kRecF4], r1 = rec[iv * kRecF4 + 1];
+      const float4 r2 = rec[iv * kRecF4 + 2];  // (conic a, b, c, opacity)
       const double2* a2 = reinterpret_cast<const double2*>(accb + iv * kAccBN);
       const double2 aq = a2[0], ar = a2[1], ah = a2[2], ad = a2[3], ae = a2[4];
       const int flags = __float_as_int(r3.w);
       if (!(flags & kFlagVisible)) continue;
       // aq = (q, w r0), ar = (w r1, w r2), ah = (h, h dx), ad = (h dy, h dx dx), ae = (h dx dy, h dy dy)
       qg += eps + aq.x;
-      const double o = r1.y;
+      const double o = r2.w;
       glogit += (1.0 - o) * ah.x;
       const float* vw = views + 20 * v;
       // colour: SH block and view direction
@@ -167,7 +167,7 @@ k_grad(const float4* __restrict__ rec, const double* __restrict__ accb,
         gmu[2] += (gd[2] - u2 * dg) * il;
       }
       // projected centre (through the conic the render used) and conic
-      const double qa = r0.z, qb = r0.w, qc = r1.x;
+      const double qa = r2.x, qb = r2.y, qc = r2.z;
       const double gmx = qa * ah.y + qb * ad.x, gmy = qb * ah.y + qc * ad.x;
       const double gqa = -0.5 * ad.y, gqb2 = -0.5 * ae.x, gqc = -0.5 * ae.y;  // dL/dQ, symmetric
       // EWA Jacobian with the projection's fp32 clamp decision

@@ -412,8 +412,8 @@ int splat_copy_projection(splat_ws* ws, float* rec, int* rect, void* stream) {
   if ((rc = check_dev_ptr(w, rec, "rec"))) return rc;
   if ((rc = check_dev_ptr(w, rect, "rect"))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = cudaMemcpyAsync(rec, w.rec, VG * 64, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(rect, w.rect, VG * 16, cudaMemcpyDeviceToDevice, st);
+  if ((rc = splat::launch_copy_records(w, rec, st))) return rc;
+  cudaError_t e = cudaMemcpyAsync(rect, w.rect, VG * 16, cudaMemcpyDeviceToDevice, st);
   return e == cudaSuccess ? SPLAT_OK : cuda_fail(w, "copy projection", e);
 }
 

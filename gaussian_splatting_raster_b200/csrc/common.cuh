@@ -28,10 +28,13 @@ constexpr int kAccBN = 10;       // doubles per (v, g) renderer-backward sums
 constexpr int kFlagVisible = 256;
 constexpr int kKeyStripes = 64;  // striped copies of the per-view depth-key statistics
 
-// Record of one (view, Gaussian), 4 x float4 = 64 bytes, array-of-structures: the render and the
-// replay gather r0..r2 (48 bytes), the finaliser r0, r1, r3.
-//   r0 = (mx, my, conic a, conic b)        r1 = (conic c, opacity, colour r, colour g)
-//   r2 = (colour b, cut, ex, ey)           r3 = (depth z, x_c, y_c, flags as int bits)
+// Record of one (view, Gaussian), 4 x float4 = 64 bytes, array-of-structures: the list-walking
+// kernels gather r0..r2 (48 bytes, both 32-byte sectors); the finaliser and the gradient chain
+// need only r2, r3 -- one sector.
+//   r0 = (mx, my, colour r, colour g)      r1 = (colour b, cut, ex, ey)
+//   r2 = (conic a, conic b, conic c, opacity)   r3 = (depth z, x_c, y_c, flags as int bits)
+// (splat_copy_projection hands it out in the documented order mx, my, a, b, c, o, r, g, b, cut,
+// ex, ey, z, x_c, y_c, flags.)
 // cut = log((1/255) / o) - 1e-3: an exponent below it gives alpha < 1/255 for certain;
 // (ex, ey) = half-extents of the ellipse {exponent >= cut} widened by 1 % + 0.05 px (+inf for a
 // nearly singular conic, -1 when no pixel can pass).
@@ -320,6 +323,8 @@ int launch_scatter(Workspace& w, const float* map, const float* obs, int C, floa
 int launch_pair_count(Workspace& w, cudaStream_t st);
 // the score sums widened to doubles into out [V*G*8] (the inspection copy)
 int launch_acc_to_double(Workspace& w, double* out, cudaStream_t st);
+// the records in the documented order into out [V*G*16] (the inspection copy)
+int launch_copy_records(Workspace& w, float* out, cudaStream_t st);
 unsigned int bounds_word_raster(cudaStream_t st);
 unsigned int bounds_word_binning(cudaStream_t st);
 unsigned int bounds_word_attributes(cudaStream_t st);

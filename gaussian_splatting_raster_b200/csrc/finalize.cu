@@ -74,17 +74,17 @@ __device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
     const float4 r3 = rec[i * kRecF4 + 3];  // (z, x_c, y_c, flags)
     const int flags = __float_as_int(r3.w);
     if (!(flags & kFlagVisible)) continue;
-    const float4 r0 = rec[i * kRecF4], r1 = rec[i * kRecF4 + 1];
+    const float4 r2 = rec[i * kRecF4 + 2];  // (conic a, b, c, opacity)
     // (q, w r (3)) and (w rho, w rho d (2), unused)
     const float4* a4 = reinterpret_cast<const float4*>(acc + i * kAccN);
     const float4 aq = a4[0], as = a4[1];
     const double qgv = eps + (double)aq.x;
     qsum += qgv;
-    sa += (1.0 - (double)r1.y) * (double)as.x;
+    sa += (1.0 - (double)r2.w) * (double)as.x;
     // per-view products in fp32 (rounding ~1e-7 relative), sums over views in double
     const float sd0 = as.y, sd1 = as.z;
-    const float sm0 = r0.z * sd0 + r0.w * sd1;
-    const float sm1 = r0.w * sd0 + r1.x * sd1;
+    const float sm0 = r2.x * sd0 + r2.y * sd1;
+    const float sm1 = r2.y * sd0 + r2.z * sd1;
     // J = J_cam(x_c) R_v, unclamped pinhole Jacobian
     const float* vw = views + 20 * v;
     const float fx = vw[16], fy = vw[17];

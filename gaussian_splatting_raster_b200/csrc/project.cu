@@ -10,6 +10,8 @@
 //
 // One thread per Gaussian reads its parameters once (SH included) and writes one record per view:
 // the SH coefficients, which dominate the input bytes at degree 3, are never re-read per view.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace splat {
@@ -224,9 +226,9 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
             ex = ey = __int_as_float(0x7f800000);
           }
         }
-        r0 = make_float4(mx, my, qa, qb);
-        r1 = make_float4(qc, o, col[0], col[1]);
-        r2 = make_float4(col[2], cut, ex, ey);
+        r0 = make_float4(mx, my, col[0], col[1]);
+        r1 = make_float4(col[2], cut, ex, ey);
+        r2 = make_float4(qa, qb, qc, o);
         r3 = make_float4(z, x, y, __int_as_float(flags));
         rc = make_int4(x0, y0, x1, y1);
         cnt = (x1 - x0) * (y1 - y0);
@@ -295,6 +297,27 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
 #undef SPLAT_PROJ
   prof_end(w, st, tok);
   return check_launch(w, "project kernel");
+}
+
+// the records in the order splat_copy_projection documents: mx, my, a, b, c, o, colour r, g, b,
+// cut, ex, ey, z, x_c, y_c, flags
+__global__ void k_copy_records(const float4* __restrict__ rec, float4* __restrict__ out, long long n) {
+  for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
+       k += (long long)gridDim.x * blockDim.x) {
+    const float4 r0 = rec[4 * k], r1 = rec[4 * k + 1], r2 = rec[4 * k + 2], r3 = rec[4 * k + 3];
+    out[4 * k] = make_float4(r0.x, r0.y, r2.x, r2.y);
+    out[4 * k + 1] = make_float4(r2.z, r2.w, r0.z, r0.w);
+    out[4 * k + 2] = r1;
+    out[4 * k + 3] = r3;
+  }
+}
+
+int launch_copy_records(Workspace& w, float* out, cudaStream_t st) {
+  const long long n = (long long)w.V * w.G;
+  if (n == 0) return SPLAT_OK;
+  k_copy_records<<<(unsigned)std::min<long long>((n + 255) / 256, 8 * 148), 256, 0, st>>>(
+      w.rec, reinterpret_cast<float4*>(out), n);
+  return check_launch(w, "record copy kernel");
 }
 
 }  // namespace splat

@@ -94,11 +94,11 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       const uint32_t gi = ids[k];
       if (in_bounds(gi, (unsigned)G, &g_bounds_word)) {
         const float4* r = recv + (size_t)gi * kRecF4;
-        const float4 a = r[0], b = r[1], c = r[2];  // c = (colour b, cut, ex, ey)
-        wa[lane] = a;
-        wb[lane] = b;
-        wc[lane] = make_float2(c.x, c.y);
-        hit = reaches_block(a, c.z, c.w, x0f, y0f);
+        const float4 r0 = r[0], r1 = r[1], r2 = r[2];  // r1 = (colour b, cut, ex, ey)
+        wa[lane] = r0;
+        wb[lane] = r2;
+        wc[lane] = make_float2(r1.x, r1.y);
+        hit = reaches_block(r0, r1.z, r1.w, x0f, y0f);
       }
     }
     uint32_t bits = __ballot_sync(0xffffffffu, hit);
@@ -108,7 +108,8 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       const int q = __ffs(bits) - 1;
       bits &= bits - 1;
       if (!done) {
-        const float4 A = wa[q], Bq = wb[q];
+        float4 A, Bq;
+        entry_operands(wa[q], wb[q], A, Bq);
         const float2 Cq = wc[q];
         const Entry E = eval_entry(A, Bq, Cq.y, px, py);
         if (E.use) {
@@ -258,10 +259,10 @@ k_replay_det(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
       if (!bad) {
         const float4* r = recv + (size_t)g * kRecF4;
-        const float4 c = r[2];
+        const float2 r1 = reinterpret_cast<const float2*>(r + 1)[0];  // (colour b, cut)
         wa[lane] = r[0];
-        wb[lane] = r[1];
-        wc[lane] = make_float2(c.x, c.y);
+        wb[lane] = r[2];
+        wc[lane] = r1;
         wg[lane] = g;
       }
     }
@@ -273,7 +274,8 @@ k_replay_det(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
       bool used = false;
       if (base + q < lst) {
-        const float4 A = wa[q], Bq = wb[q];
+        float4 A, Bq;
+        entry_operands(wa[q], wb[q], A, Bq);
         const float2 Cq = wc[q];
         const Entry E = eval_entry(A, Bq, Cq.y, px, py);
         if (E.use) {
@@ -481,10 +483,10 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
         if (!bad) {
           const float4* r = recv + (size_t)g * kRecF4;
-          const float4 c = r[2];
+          const float2 r1 = reinterpret_cast<const float2*>(r + 1)[0];  // (colour b, cut)
           wa[lane] = r[0];
-          wb[lane] = r[1];
-          wc[lane] = make_float2(c.x, c.y);
+          wb[lane] = r[2];
+          wc[lane] = r1;
           wg[lane] = g;
         }
       }
@@ -496,7 +498,8 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
         bool used = false;
         if (base + q < lst) {
-          const float4 A = wa[q], Bq = wb[q];
+          float4 A, Bq;
+        entry_operands(wa[q], wb[q], A, Bq);
           const float2 Cq = wc[q];
           const Entry E = eval_entry(A, Bq, Cq.y, px, py);
           if (E.use) {
@@ -556,8 +559,9 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     const uint32_t g = ids[s + 32LL * c + q];
     if (!in_bounds(g, (unsigned)G, &g_bounds_word)) continue;
     const float4* r = recv + (size_t)g * kRecF4;
-    const float4 A = __ldg(r), Bq = __ldg(r + 1);
-    const float c2 = __ldg(reinterpret_cast<const float*>(r + 2));
+    const float4 r0 = __ldg(r), r2 = __ldg(r + 2);
+    const float c2 = __ldg(reinterpret_cast<const float*>(r + 1));  // colour b
+    const float4 A = make_float4(r0.x, r0.y, r2.x, r2.y), Bq = make_float4(r2.z, r2.w, r0.z, r0.w);
     // the render's alpha, bit for bit (a composited entry always passes the exponent cut)
     const Entry E = eval_entry(A, Bq, -INFINITY, px, py);
     if (!E.use) continue;
@@ -632,10 +636,10 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
       if (!bad) {
         const float4* r = recv + (size_t)g * kRecF4;
-        const float4 c = r[2];
+        const float2 r1 = reinterpret_cast<const float2*>(r + 1)[0];  // (colour b, cut)
         wa[lane] = r[0];
-        wb[lane] = r[1];
-        wc[lane] = make_float2(c.x, c.y);
+        wb[lane] = r[2];
+        wc[lane] = r1;
         wg[lane] = g;
       }
     }
@@ -649,7 +653,8 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       for (int k = 0; k < 16; ++k) x[k] = 0.0f;
       bool used = false;
       if (base + q < lst) {
-        const float4 A = wa[q], Bq = wb[q];
+        float4 A, Bq;
+        entry_operands(wa[q], wb[q], A, Bq);
         const float2 Cq = wc[q];
         const Entry E = eval_entry(A, Bq, Cq.y, px, py);
         if (E.use) {

@@ -104,6 +104,15 @@ __device__ __forceinline__ size_t lmask_region(long long s, int gt) {
   return (size_t)1024 * (size_t)((s >> 7) + gt);
 }
 
+// The list-walking kernels stage, per entry, the record's r0 = (mx, my, colour r, colour g) and
+// r2 = (conic a, b, c, opacity) as they are, plus (colour b, cut) from r1, and form the
+// evaluation operands from them (register moves only):
+//   A = (mx, my, conic a, conic b), B = (conic c, opacity, colour r, colour g)
+__device__ __forceinline__ void entry_operands(float4 R0, float4 R2, float4& A, float4& B) {
+  A = make_float4(R0.x, R0.y, R2.x, R2.y);
+  B = make_float4(R2.z, R2.w, R0.z, R0.w);
+}
+
 // alpha of one list entry at pixel centre (px, py), with the rasteriser's skip rules
 __device__ __forceinline__ Entry eval_entry(const float4 A, const float4 Bq, float cut, float px,
                                             float py) {
