@@ -27,93 +27,79 @@ namespace {
 
 constexpr int kMaxPass = 16;  // channels per traversal
 
-// F[c0 .. c0 + CB) of every pixel
+// F[c0 .. c0 + CB) of every pixel. Each lane walks only the entries its pixel composited (the
+// render's per-pixel masks, as in the score replay), in list order, so a warp runs its longest
+// walk instead of every entry some pixel of its block composited; every pixel's output is its own
+// (no reduction), and the sum is the same as over the render's order.
 template <int CB>
 __global__ void __launch_bounds__(kThreads)
 k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
            const long long* __restrict__ tile_off, const int* __restrict__ order,
            int G, int H, int W, int TX, int nt,
-           const int* __restrict__ last, const uint32_t* __restrict__ umask,
+           const int* __restrict__ last, const uint32_t* __restrict__ lmask,
            const float* __restrict__ feats, int C, int c0, float* __restrict__ out) {
   int t, v;
   if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
   const int tx = t % TX, ty = t / TX;
   int i, j, bx, by;
   tile_pixel(tx, ty, i, j, bx, by);
-  const bool inside = i < W && j < H;
+  if (i >= W || j >= H) return;  // no warp-wide operation below
   const long long s = tile_off[(size_t)v * (nt + 1) + t];
   const int gt = v * nt + t;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
-  const int twarp = tile_warp();                                 // block in the tile
-  __shared__ float4 s_a[kThreads], s_b[kThreads];
-  __shared__ float s_cut[kThreads];
-  __shared__ __align__(16) float s_f[kThreads * CB];
-  float4* wa = s_a + warp * 32;
-  float4* wb = s_b + warp * 32;
-  float* wc = s_cut + warp * 32;
-  float* wf = s_f + warp * 32 * CB;
+  const int lane = threadIdx.x & 31, twarp = tile_warp();
   const int nc = min(CB, C - c0);
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   const size_t p = ((size_t)v * H + j) * W + i;
-  const int lst = inside ? last[p] : 0;
-  const int wmax = __reduce_max_sync(0xffffffffu, lst);
+  const int cend = (last[p] + 31) >> 5;  // chunks holding this pixel's composited entries
   const float4* recv = rec + (size_t)v * G * kRecF4;
   float F[CB];
 #pragma unroll
   for (int k = 0; k < CB; ++k) F[k] = 0.0f;
   float T = 1.0f;
-  for (int base = 0; base < wmax; base += 32) {
-    uint32_t bits = umask[chunk_index(s + base, gt) * 8 + twarp];
-    if (!bits) continue;  // warp-uniform
-    bool bad = false;
-    if ((bits >> lane) & 1u) {
-      const uint32_t g = ids[s + base + lane];
-      bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
-      if (!bad) {
-        const float4* r = recv + (size_t)g * kRecF4;
-        wa[lane] = r[0];
-        wb[lane] = r[2];
-        wc[lane] = reinterpret_cast<const float*>(r + 1)[1];  // cut
-        const float* fg = feats + (size_t)g * C + c0;
-#pragma unroll
-        for (int k = 0; k < CB; ++k) wf[lane * CB + k] = k < nc ? fg[k] : 0.0f;
-      }
-    }
-    if (kChecked) bits &= ~__ballot_sync(0xffffffffu, bad);
-    __syncwarp();
-    while (bits) {
-      const int q = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (base + q < lst) {
-        float4 A, Bq;
-        entry_operands(wa[q], wb[q], A, Bq);
-        const Entry E = eval_entry(A, Bq, wc[q], px, py);
-        if (E.use) {
-          const float w = E.alpha * T;
-          if constexpr (CB % 2 == 0) {  // two products per packed multiply, scalar sums
-            const float2 ww = make_float2(w, w);
-            const float2* f2 = reinterpret_cast<const float2*>(wf + q * CB);
-#pragma unroll
-            for (int k = 0; k < CB; k += 2) {
-              const float2 p = __fmul2_rn(ww, f2[k / 2]);
-              F[k] = F[k] + p.x;
-              F[k + 1] = F[k + 1] + p.y;
-            }
-          } else {
-#pragma unroll
-            for (int k = 0; k < CB; ++k) F[k] = F[k] + w * wf[q * CB + k];
-          }
-          T = T * (1.0f - E.alpha);
+  if (cend > 0) {
+    const uint4* lm =
+        reinterpret_cast<const uint4*>(lmask + lmask_region(s, gt)) + (twarp * 32 + lane);
+    const uint4 g0 = __ldg(lm);
+    uint32_t m = g0.x, n1 = g0.y, n2 = g0.z, n3 = g0.w;
+    uint4 pre = make_uint4(0u, 0u, 0u, 0u);
+    if (4 < cend) pre = __ldg(lm + 256);
+    int c = 0;
+    for (;;) {
+      if (!m) {  // next chunk with an entry of this pixel
+        if (++c >= cend) break;
+        if ((c & 3) == 0) {
+          m = pre.x;
+          n1 = pre.y;
+          n2 = pre.z;
+          n3 = pre.w;
+          if (c + 4 < cend) pre = __ldg(lm + (size_t)((c >> 2) + 1) * 256);
+        } else {
+          m = n1;
+          n1 = n2;
+          n2 = n3;
         }
+        continue;
       }
-    }
-    __syncwarp();
-  }
-  if (inside) {
+      const int q = __ffs(m) - 1;
+      m &= m - 1u;
+      const uint32_t g = ids[s + 32LL * c + q];
+      if (!in_bounds(g, (unsigned)G, &g_bounds_word)) continue;
+      const float4* r = recv + (size_t)g * kRecF4;
+      float4 A, Bq;
+      entry_operands(__ldg(r), __ldg(r + 2), A, Bq);
+      const Entry E = eval_entry(A, Bq, -INFINITY, px, py);  // the render's alpha, bit for bit
+      if (!E.use) continue;
+      const float w = E.alpha * T;
+      const float* fg = feats + (size_t)g * C + c0;
 #pragma unroll
-    for (int k = 0; k < CB; ++k)
-      if (k < nc) out[p * C + c0 + k] = F[k];
+      for (int k = 0; k < CB; ++k)
+        if (k < nc) F[k] = F[k] + w * __ldg(fg + k);
+      T = T * (1.0f - E.alpha);
+    }
   }
+#pragma unroll
+  for (int k = 0; k < CB; ++k)
+    if (k < nc) out[p * C + c0 + k] = F[k];
 }
 
 // sum over pixels of w m[c0 .. c0 + NV) per (Gaussian), into acc [G, C] (fp64). RESID: the map is
@@ -253,7 +239,7 @@ int launch_features(Workspace& w, const float* feats, int C, float* out, cudaStr
     const int nc = C - c0 < kMaxPass ? C - c0 : kMaxPass;
 #define SPLAT_FEAT(CB)                                                                          \
   k_features<CB><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,    \
-                                           w.nt, w.last, w.umask, feats, C, c0, out)
+                                           w.nt, w.last, w.lmask, feats, C, c0, out)
     if (nc == 1) SPLAT_FEAT(1);
     else if (nc <= 4) SPLAT_FEAT(4);
     else if (nc <= 8) SPLAT_FEAT(8);
