@@ -249,11 +249,13 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
 # Algorithmic fp32 work of the list-walking kernels, in lane operations (an fma is one; the
 # exponential is the Cody-Waite one both sides use: x log2(e) and its rounding, two reduction fmas,
 # a degree-7 Horner polynomial, the scale = 12), counted from the method's arithmetic by pair
-# class: every traversed (pixel, list entry) pair needs the exponent of G and the skip decision
-# (p - mu2D, the conic's quadratic form, the positive-exponent test and the comparison with the
-# Gaussian's precomputed exponent cut that decides alpha < 1/255 without the exponential = 13);
-# each composited pair needs alpha = min(0.99, o exp(pw)) and the 1/255 test (15) and then its
-# pass's own work:
+# class. The render must decide every traversed (pixel, list entry) pair: the exponent of G and
+# the skip decision (p - mu2D, the conic's quadratic form, the positive-exponent test and the
+# comparison with the Gaussian's precomputed exponent cut that decides alpha < 1/255 without the
+# exponential = 13). The later passes are handed the render's decisions (its per-pixel masks of
+# composited entries) and walk only the composited pairs, except the map scatter and the
+# attribution, which still visit every entry their warp's pixels composited. Each composited pair
+# needs alpha = min(0.99, o exp(pw)) and the 1/255 test (15) and then its pass's own work:
 #   render    T (1 - alpha), the stop test, w = alpha T, C += w c (unfused)                 = 10
 #   replay    T (1 - alpha), w, w c, C_hat - P - w c (3 channels), the reciprocal of the
 #             denominator, c - C+ (3 fmas), rho, both masks, w r, w rho, w rho d, P += w c  = 31
@@ -263,8 +265,12 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
 #   scatter   two traversals: the 9-channel map (T, w, 9 products) and the attribution
 #             (T, w, w, w |r|)                                                             = 12 + 5
 # so a kernel's work per step = a x traversed pairs + b x composited pairs with (a, b) below.
-ALU_OPS = {"render": (13, 25), "replay": (13, 46), "backward": (13, 43), "features": (13, 36),
-           "scatter": (26, 47)}
+ALU_OPS = {"render": (13, 25), "replay": (0, 46), "backward": (0, 43), "features": (0, 36),
+           "scatter": (26, 47)}  # the backward visits its warps' union entries but, like the
+# replay, is handed the render's decisions: its work is counted over the composited pairs
+# kernels whose time is set by 16-byte fp32 reductions into L2 (two per composited pair in the
+# replay's per-pixel walks): reported with their reduction rate beside the fp32 figure
+L2_REDUCTIONS_PER_PAIR = {"replay": 2}
 
 
 def alu_ops(kernel: str, pairs: int, composited: int) -> int:
@@ -650,6 +656,9 @@ def main():
                 "ncu_pipes": recorded_pipes(dom, workload_name(args, sc)),
                 "work": f"{ALU_OPS[dom][0]} ops x traversed pairs + {ALU_OPS[dom][1]} ops x "
                         f"composited pairs",
+                "l2_reductions_per_s": (L2_REDUCTIONS_PER_PAIR[dom] * composited_rank
+                                        / (dom_ms * 1e-3) if dom in L2_REDUCTIONS_PER_PAIR
+                                        else None),
                 "peak_source": f"{lanes} fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz "
                                f"({peaks['source']} max clock)"}
     else:

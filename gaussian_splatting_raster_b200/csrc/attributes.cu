@@ -51,7 +51,7 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
   const size_t p = ((size_t)v * H + j) * W + i;
   const int cend = (last[p] + 31) >> 5;  // chunks holding this pixel's composited entries
-  const float4* recv = rec + (size_t)v * G * kRecF4;
+  const size_t vG = (size_t)v * G;
   float F[CB];
 #pragma unroll
   for (int k = 0; k < CB; ++k) F[k] = 0.0f;
@@ -84,9 +84,10 @@ k_features(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       m &= m - 1u;
       const uint32_t g = ids[s + 32LL * c + q];
       if (!in_bounds(g, (unsigned)G, &g_bounds_word)) continue;
-      const float4* r = recv + (size_t)g * kRecF4;
+      const float4* rl = rec + rec_lo(vG + g);  // r0, r1
+      const float4* rh = rec + rec_hi(vG + g);  // r2, r3
       float4 A, Bq;
-      entry_operands(__ldg(r), __ldg(r + 2), A, Bq);
+      entry_operands(__ldg(rl), __ldg(rh), A, Bq);
       const Entry E = eval_entry(A, Bq, -INFINITY, px, py);  // the render's alpha, bit for bit
       if (!E.use) continue;
       const float w = E.alpha * T;
@@ -150,7 +151,7 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     }
   }
   const int wmax = __reduce_max_sync(0xffffffffu, lst);
-  const float4* recv = rec + (size_t)v * G * kRecF4;
+  const size_t vG = (size_t)v * G;
   const int slot = slot_of<NV>(lane);
   const bool holder = slot_holder<NV>(lane) && slot < nc;
   float T = 1.0f;
@@ -162,10 +163,11 @@ k_scatter(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       const uint32_t g = ids[s + base + lane];
       bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
       if (!bad) {
-        const float4* r = recv + (size_t)g * kRecF4;
-        wa[lane] = r[0];
-        wb[lane] = r[2];
-        wc[lane] = reinterpret_cast<const float*>(r + 1)[1];  // cut
+        const float4* rl = rec + rec_lo(vG + g);  // r0, r1
+        const float4* rh = rec + rec_hi(vG + g);  // r2, r3
+        wa[lane] = rl[0];
+        wb[lane] = rh[0];
+        wc[lane] = reinterpret_cast<const float*>(rl + 1)[1];  // cut
         wg[lane] = g;
       }
     }

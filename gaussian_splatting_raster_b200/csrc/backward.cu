@@ -121,8 +121,9 @@ k_grad(const float4* __restrict__ rec, const double* __restrict__ accb,
       const size_t iv = (size_t)v * G + g;
       // all loads of the view issued together (one memory round trip per view); the record and
       // sums of a view where g is culled are read but not used
-      const float4 r3 = rec[iv * kRecF4 + 3];  // (z, x_c, y_c, flags)
-      const float4 r2 = rec[iv * kRecF4 + 2];  // (conic a, b, c, opacity)
+      const float4* rh = rec + rec_hi(iv);
+      const float4 r3 = rh[1];  // (z, x_c, y_c, flags)
+      const float4 r2 = rh[0];  // (conic a, b, c, opacity)
       const double2* a2 = reinterpret_cast<const double2*>(accb + iv * kAccBN);
       const double2 aq = a2[0], ar = a2[1], ah = a2[2], ad = a2[3], ae = a2[4];
       const int flags = __float_as_int(r3.w);

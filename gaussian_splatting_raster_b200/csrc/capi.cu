@@ -142,7 +142,7 @@ int splat_ws_create(splat_ws** out, int max_G, int max_V, int max_H, int max_W,
   w.max_nt = ((max_W + 15) / 16) * ((max_H + 15) / 16);
   const size_t VG = (size_t)max_V * max_G;
   int rc = 0;
-  if (!rc) rc = alloc(w, &w.rec, VG * splat::kRecF4, "records");
+  if (!rc) rc = alloc(w, &w.rec, splat::rec_f4_count(VG), "records");
   if (!rc) rc = alloc(w, &w.rect, VG, "rectangles");
   if (!rc) rc = alloc(w, &w.counts, VG, "tile counts");
   if (!rc) rc = alloc(w, &w.offs, VG + 1, "instance offsets");

@@ -22,17 +22,22 @@ namespace splat {
 
 constexpr int kTile = 16;        // 16x16 pixel tiles
 constexpr int kTilePix = 256;
-constexpr int kRecF4 = 4;        // float4 per (v, g) record
 constexpr int kAccN = 8;         // doubles per (v, g) accumulator
 constexpr int kAccBN = 10;       // doubles per (v, g) renderer-backward sums
 constexpr int kFlagVisible = 256;
 constexpr int kKeyStripes = 64;  // striped copies of the per-view depth-key statistics
 
-// Record of one (view, Gaussian), 4 x float4 = 64 bytes, array-of-structures: the list-walking
-// kernels gather r0..r2 (48 bytes, both 32-byte sectors); the finaliser and the gradient chain
-// need only r2, r3 -- one sector.
-//   r0 = (mx, my, colour r, colour g)      r1 = (colour b, cut, ex, ey)
-//   r2 = (conic a, conic b, conic c, opacity)   r3 = (depth z, x_c, y_c, flags as int bits)
+// Record of one (view, Gaussian), 4 x float4 = 64 bytes, in two halves:
+//   low  r0 = (mx, my, colour r, colour g)      r1 = (colour b, cut, ex, ey)
+//   high r2 = (conic a, conic b, conic c, opacity)   r3 = (depth z, x_c, y_c, flags as int bits)
+// stored in blocks of 32 entries (view-major (v, g) index i): the block's 32 low halves, then its
+// 32 high halves (2 KB per block). The list-walking kernels gather r0, r1 and r2; the finaliser
+// and the gradient chain need only the high halves, which lie contiguous for consecutive
+// Gaussians (DRAM is read in 64-byte pieces: with whole records side by side the finaliser read
+// all 64 bytes of each).
+__host__ __device__ __forceinline__ size_t rec_lo(size_t i) { return (i >> 5) * 128 + (i & 31) * 2; }
+__host__ __device__ __forceinline__ size_t rec_hi(size_t i) { return rec_lo(i) + 64; }
+__host__ __device__ __forceinline__ size_t rec_f4_count(size_t n) { return (n + 31) / 32 * 128; }
 // (splat_copy_projection hands it out in the documented order mx, my, a, b, c, o, r, g, b, cut,
 // ex, ey, z, x_c, y_c, flags.)
 // cut = log((1/255) / o) - 1e-3: an exponent below it gives alpha < 1/255 for certain;

@@ -71,10 +71,11 @@ __device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
   const double eps = 1e-6;
   for (int v = 0; v < V; ++v) {
     const size_t i = (size_t)v * G + g;
-    const float4 r3 = rec[i * kRecF4 + 3];  // (z, x_c, y_c, flags)
+    const float4* rh = rec + rec_hi(i);
+    const float4 r3 = rh[1];  // (z, x_c, y_c, flags)
     const int flags = __float_as_int(r3.w);
     if (!(flags & kFlagVisible)) continue;
-    const float4 r2 = rec[i * kRecF4 + 2];  // (conic a, b, c, opacity)
+    const float4 r2 = rh[0];  // (conic a, b, c, opacity)
     // (q, w r (3)) and (w rho, w rho d (2), unused)
     const float4* a4 = reinterpret_cast<const float4*>(acc + i * kAccN);
     const float4 aq = a4[0], as = a4[1];

@@ -234,11 +234,12 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
         cnt = (x1 - x0) * (y1 - y0);
       }
     }
-    float4* rp = rec + i * kRecF4;
-    rp[0] = r0;
-    rp[1] = r1;
-    rp[2] = r2;
-    rp[3] = r3;
+    float4* rl = rec + rec_lo(i);
+    float4* rh = rec + rec_hi(i);
+    rl[0] = r0;
+    rl[1] = r1;
+    rh[0] = r2;
+    rh[1] = r3;
     rect[i] = rc;
     counts[i] = cnt;
     // depth sort key (fp32 bits of z > 0 order like the values; culled entries sort last) and,
@@ -304,7 +305,8 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
 __global__ void k_copy_records(const float4* __restrict__ rec, float4* __restrict__ out, long long n) {
   for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
        k += (long long)gridDim.x * blockDim.x) {
-    const float4 r0 = rec[4 * k], r1 = rec[4 * k + 1], r2 = rec[4 * k + 2], r3 = rec[4 * k + 3];
+    const float4 r0 = rec[rec_lo(k)], r1 = rec[rec_lo(k) + 1];
+    const float4 r2 = rec[rec_hi(k)], r3 = rec[rec_hi(k) + 1];
     out[4 * k] = make_float4(r0.x, r0.y, r2.x, r2.y);
     out[4 * k + 1] = make_float4(r2.z, r2.w, r0.z, r0.w);
     out[4 * k + 2] = r1;

@@ -85,7 +85,7 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int n = 0, lst = 0;
   bool done = !inside;
-  const float4* recv = rec + (size_t)v * G * kRecF4;
+  const size_t vG = (size_t)v * G;
   for (long long base = s; base < e; base += 32, ++cc) {
     if (__all_sync(0xffffffffu, done)) break;
     const long long k = base + lane;
@@ -93,8 +93,9 @@ k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     if (k < e) {
       const uint32_t gi = ids[k];
       if (in_bounds(gi, (unsigned)G, &g_bounds_word)) {
-        const float4* r = recv + (size_t)gi * kRecF4;
-        const float4 r0 = r[0], r1 = r[1], r2 = r[2];  // r1 = (colour b, cut, ex, ey)
+        const float4* rl = rec + rec_lo(vG + gi);  // r0, r1
+        const float4* rh = rec + rec_hi(vG + gi);  // r2, r3
+        const float4 r0 = rl[0], r1 = rl[1], r2 = rh[0];  // r1 = (colour b, cut, ex, ey)
         wa[lane] = r0;
         wb[lane] = r2;
         wc[lane] = make_float2(r1.x, r1.y);
@@ -243,7 +244,7 @@ k_replay_det(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     lst = last[p];
   }
   const int wmax = __reduce_max_sync(0xffffffffu, lst);  // entries this warp must traverse
-  const float4* recv = rec + (size_t)v * G * kRecF4;
+  const size_t vG = (size_t)v * G;
   float T = 1.0f, P2 = 0.0f;  // transmittance, prefix colour (channels 0 and 1 packed)
   float2 P01 = make_float2(0.0f, 0.0f);
   const float2 Ch01 = make_float2(Ch0, Ch1), r01 = make_float2(r0, r1);
@@ -258,10 +259,11 @@ k_replay_det(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       const uint32_t g = ids[s + base + lane];
       bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
       if (!bad) {
-        const float4* r = recv + (size_t)g * kRecF4;
-        const float2 r1 = reinterpret_cast<const float2*>(r + 1)[0];  // (colour b, cut)
-        wa[lane] = r[0];
-        wb[lane] = r[2];
+        const float4* rl = rec + rec_lo(vG + g);  // r0, r1
+        const float4* rh = rec + rec_hi(vG + g);  // r2, r3
+        const float2 r1 = reinterpret_cast<const float2*>(rl + 1)[0];  // (colour b, cut)
+        wa[lane] = rl[0];
+        wb[lane] = rh[0];
         wc[lane] = r1;
         wg[lane] = g;
       }
@@ -452,7 +454,7 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   ps.Ch01 = make_float2(Ch0, Ch1);
   ps.r01 = make_float2(r0, r1);
   const float px = (float)i + 0.5f, py = (float)j + 0.5f;
-  const float4* recv = rec + (size_t)v * G * kRecF4;
+  const size_t vG = (size_t)v * G;
   float* accv = acc + (size_t)v * G * kAccN;
 
   // the warp's union entries U and composited pairs P
@@ -482,10 +484,11 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         const uint32_t g = ids[s + base + lane];
         bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
         if (!bad) {
-          const float4* r = recv + (size_t)g * kRecF4;
-          const float2 r1 = reinterpret_cast<const float2*>(r + 1)[0];  // (colour b, cut)
-          wa[lane] = r[0];
-          wb[lane] = r[2];
+          const float4* rl = rec + rec_lo(vG + g);  // r0, r1
+          const float4* rh = rec + rec_hi(vG + g);  // r2, r3
+          const float2 r1 = reinterpret_cast<const float2*>(rl + 1)[0];  // (colour b, cut)
+          wa[lane] = rl[0];
+          wb[lane] = rh[0];
           wc[lane] = r1;
           wg[lane] = g;
         }
@@ -558,9 +561,10 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     m &= m - 1u;
     const uint32_t g = ids[s + 32LL * c + q];
     if (!in_bounds(g, (unsigned)G, &g_bounds_word)) continue;
-    const float4* r = recv + (size_t)g * kRecF4;
-    const float4 r0 = __ldg(r), r2 = __ldg(r + 2);
-    const float c2 = __ldg(reinterpret_cast<const float*>(r + 1));  // colour b
+    const float4* rl = rec + rec_lo(vG + g);  // r0, r1
+    const float4* rh = rec + rec_hi(vG + g);  // r2, r3
+    const float4 r0 = __ldg(rl), r2 = __ldg(rh);
+    const float c2 = __ldg(reinterpret_cast<const float*>(rl + 1));  // colour b
     const float4 A = make_float4(r0.x, r0.y, r2.x, r2.y), Bq = make_float4(r2.z, r2.w, r0.z, r0.w);
     // the render's alpha, bit for bit (a composited entry always passes the exponent cut)
     const Entry E = eval_entry(A, Bq, -INFINITY, px, py);
@@ -624,7 +628,7 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     lst = last[p];
   }
   const int wmax = __reduce_max_sync(0xffffffffu, lst);
-  const float4* recv = rec + (size_t)v * G * kRecF4;
+  const size_t vG = (size_t)v * G;
   double* accv = accb + (size_t)v * G * kAccBN;
   const int slot = (lane >> 1) & 15;  // value index this lane holds after the reduction
   for (int base = (wmax - 1) & ~31; base >= 0; base -= 32) {
@@ -635,11 +639,11 @@ k_backward(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
       const uint32_t g = ids[s + base + lane];
       bad = !in_bounds(g, (unsigned)G, &g_bounds_word);
       if (!bad) {
-        const float4* r = recv + (size_t)g * kRecF4;
-        const float2 r1 = reinterpret_cast<const float2*>(r + 1)[0];  // (colour b, cut)
-        wa[lane] = r[0];
-        wb[lane] = r[2];
-        wc[lane] = r1;
+        const float4* rl = rec + rec_lo(vG + g);  // r0, r1
+        const float4* rh = rec + rec_hi(vG + g);  // r2, r3
+        wa[lane] = rl[0];
+        wb[lane] = rh[0];
+        wc[lane] = reinterpret_cast<const float2*>(rl + 1)[0];  // (colour b, cut)
         wg[lane] = g;
       }
     }

@@ -106,9 +106,12 @@ def test_alu_work_counts_by_pair_class():
     for k, (a, c) in b.ALU_OPS.items():
         assert b.alu_ops(k, 1, 0) == a and b.alu_ops(k, 0, 1) == c
         assert b.alu_ops(k, 1000, 10) == 1000 * a + 10 * c
-    # alpha (15) is part of every pass's composited cost; the replay does the most per pair
+    # alpha (15) is part of every pass's composited cost; the replay does the most per pair;
+    # only the render (and the passes that still visit their warps' union entries) decide
+    # traversed pairs
     assert min(c for _, c in b.ALU_OPS.values()) >= 15 + 10
     assert b.ALU_OPS["replay"][1] > b.ALU_OPS["render"][1]
+    assert b.ALU_OPS["render"][0] > 0 and b.ALU_OPS["replay"][0] == 0
 
 
 def test_reference_steps_are_what_ran():
