@@ -268,10 +268,6 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
 ALU_OPS = {"render": (13, 25), "replay": (0, 46), "backward": (0, 43), "features": (0, 36),
            "scatter": (26, 47)}  # the backward visits its warps' union entries but, like the
 # replay, is handed the render's decisions: its work is counted over the composited pairs
-# kernels whose time is set by 16-byte fp32 reductions into L2 (two per composited pair in the
-# replay's per-pixel walks): reported with their reduction rate beside the fp32 figure
-L2_REDUCTIONS_PER_PAIR = {"replay": 2}
-
 
 def alu_ops(kernel: str, pairs: int, composited: int) -> int:
     a, b = ALU_OPS[kernel]
@@ -297,6 +293,7 @@ def cpu_oracle_view(sc, obs_np, path="score", threads=0):
     t_pb = time.perf_counter() - t0
     t1 = time.perf_counter()
     r = O.render(p, L, one.H, one.W, one.bg, "f")
+    t_r = time.perf_counter() - t1
     if path == "backward":
         accb = O.backward(p, L, r, obs_np[:1], one.bg, one.H, one.W, "f")
     elif path == "attributes":
@@ -323,8 +320,9 @@ def cpu_oracle_view(sc, obs_np, path="score", threads=0):
     return {"value": one.H * one.W / t_view / 1e6, "unit": "Mpix/s",
             "cores": int(O.lib().orc_num_threads()), "kind": "oracle",
             "sample": (f"view 1 of {sc.V}, whole: projection + binning of all {sc.G} Gaussians "
-                       f"({t_pb:.2f} s), render + {second} of all {one.H}x{one.W} pixels "
-                       f"({t_rr:.2f} s), {last} ({t_fin:.2f} s)"),
+                       f"({1e3 * t_pb:.1f} ms), render of all {one.H}x{one.W} pixels "
+                       f"({1e3 * t_r:.1f} ms), {second} ({1e3 * (t_rr - t_r):.1f} ms), {last} "
+                       f"({1e3 * t_fin:.1f} ms)"),
             "seconds": t_view}
 
 
@@ -656,9 +654,6 @@ def main():
                 "ncu_pipes": recorded_pipes(dom, workload_name(args, sc)),
                 "work": f"{ALU_OPS[dom][0]} ops x traversed pairs + {ALU_OPS[dom][1]} ops x "
                         f"composited pairs",
-                "l2_reductions_per_s": (L2_REDUCTIONS_PER_PAIR[dom] * composited_rank
-                                        / (dom_ms * 1e-3) if dom in L2_REDUCTIONS_PER_PAIR
-                                        else None),
                 "peak_source": f"{lanes} fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz "
                                f"({peaks['source']} max clock)"}
     else:

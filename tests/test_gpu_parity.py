@@ -38,12 +38,47 @@ def _full_check(sc, obs, lam=1.0):
     return g, o
 
 
+def _replay_traversals(sc, o, union_lanes=9):
+    """How many warp blocks (8x4 pixels of a 16x16 tile) the score replay runs as per-pixel walks
+    and how many as the union loop: a warp takes the union loop when its pixels' composited pairs
+    P are at least union_lanes times the entries U that some pixel of the block composited.
+    Counted here from the oracle's per-pixel composited entries."""
+    p, L = o["proj"], o["lists"]
+    TX, TY = O.n_tiles(sc.H, sc.W)
+    walk = union = 0
+    for v in range(sc.V):
+        for t in range(TX * TY):
+            seg = L["ids"][L["off"][v, t]:L["off"][v, t + 1]]
+            pos = {int(gg): k for k, gg in enumerate(seg)}
+            tx, ty = t % TX, t // TX
+            for w in range(8):
+                x0, y0 = tx * 16 + (w % 2) * 8, ty * 16 + (w // 2) * 4
+                U, P = set(), 0
+                for lane in range(32):
+                    i, j = x0 + lane % 8, y0 + lane // 8
+                    if i >= sc.W or j >= sc.H:
+                        continue
+                    tr = O.trace(p, L, sc.H, sc.W, sc.bg, v, i, j, "f", cap=8192)
+                    U |= {pos[int(gg)] for gg in tr[:, 0]}
+                    P += int(o["n_contrib"][v, j, i])
+                if U:
+                    union += P >= union_lanes * len(U)
+                    walk += P < union_lanes * len(U)
+    return walk, union
+
+
 @pytest.mark.parametrize("cfg", [1, 2])
 def test_small_configs_full_parity(cfg):
+    """Full parity on the two small workloads. Both of the score replay's traversals run here:
+    on the three-layer scene about two thirds of the warp blocks walk their pixels' entries and a
+    third take the union loop (checked below), so the token comparison covers both."""
     sc = scenes.make(cfg)
     obs = O.observe(sc, "f")
     g, o = _full_check(sc, obs)
     assert g["n_contrib"].max() > 1
+    if cfg == 2:
+        walk, union = _replay_traversals(sc, o)
+        assert walk > 100 and union > 100, (walk, union)
 
 
 def test_exact_depth_ties_keep_index_order():
