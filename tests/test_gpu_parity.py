@@ -257,7 +257,7 @@ def test_full_size_sampled(cfg):
     TX, TY = O.n_tiles(sc.H, sc.W)
     # sampled Gaussians (visible somewhere, no colour near-tie) and the tiles they touch
     cand = np.nonzero(p["valid"].any(0) & ~near)[0]
-    gs = rng.choice(cand, size=24, replace=False)
+    gs = rng.choice(cand, size=64, replace=False)
     sel = set()
     for v in range(sc.V):
         for gg in gs:
