@@ -218,8 +218,9 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
         # one depth-digit pass per launch over every (v, g): histogram reads the keys, the
         # scatter reads key + index and writes both
         "depth_hist": depth_passes * V * G * 4,
-        # per pass keys and values in and out (the last writes no keys)
-        "depth_scatter": depth_passes * V * G * 16 - V * G * 4,
+        # per pass keys and values in and out; the first reads no values (the index is implicit),
+        # the last writes no keys
+        "depth_scatter": max(depth_passes * 16 - 8, 0) * V * G,
         # rectangles gathered into depth order (order 4 B + rectangle 16 B in, 16 B + count out),
         # the counts scanned (4 B in, 8 B out), instances (tile, g) emitted (rectangle, index,
         # offset in; 8 B out)

@@ -7,18 +7,21 @@
 //
 // Design (instead of one radix sort of 64-bit (tile | depth) keys over all instances):
 //   1. per view, a stable LSD radix sort of the (v, g) depth keys -- one key per Gaussian, not per
-//      instance -- over only the bits that vary among the view's visible keys (the projection
-//      records per-view ORs of the keys and of their complements), 8..11-bit digits;
+//      instance -- over the width of the view's key range: the first pass orders key - kmin(view)
+//      (the projection records each view's smallest and largest visible key), so depths in
+//      [1, 100] take 26 bits (3 passes of 9) where the varying bits of the raw keys were 31;
 //   2. the tile rectangles gathered into that depth order, their tile counts scanned, and the
 //      instances (tile, g) emitted in depth order;
 //   3. one stable counting sort of the instances by tile. Stability of 1 (index order of equal
 //      depths) and 3 (depth order inside each tile) gives exactly (depth, index) per tile, and the
 //      scanned (tile, block) histogram yields every tile's [start, end).
-// Every pass -- each depth digit and the tile pass -- is the same stable counting sort: per block
-// of 16K items, per-warp shared-memory histograms (shared-memory atomics), an int32 exclusive scan
-// of the (bucket, block) counts, and a scatter that ranks equal buckets inside each 32-item batch
-// with match.any (stable: earlier items first). Uniform, bandwidth-shaped work; no decoupled
-// look-back, so no device-side waits.
+// Every pass -- each depth digit and the tile pass -- is a stable counting sort over blocks of 16K
+// items: per-warp shared-memory histograms (shared-memory atomics), an int32 exclusive scan of the
+// (bucket, block) counts, and a scatter that ranks equal buckets inside each 32-item batch with
+// match.any (stable: earlier items first). The depth passes (512 buckets) lay each 4K-item round
+// out in bucket order in shared memory and write whole bucket runs; the tile pass (one bucket per
+// tile, ~2 items per bucket and round) writes each item straight to its place. Uniform,
+// bandwidth-shaped work; no decoupled look-back, so no device-side waits.
 #include "common.cuh"
 
 namespace splat {
@@ -161,6 +164,7 @@ constexpr int kDepthChunk = 16384;  // items per block, depth-key passes
 constexpr int kDepthDigitMax = SPLAT_DEPTH_DIGIT_MAX;
 constexpr int kTileChunk = 16384;   // items per block, tile pass
 
+
 // Items of view v are [start(v), start(v + 1)); each view is cut into blocks of `chunk` items.
 // Uniform layout (every view holds `per_view` items, blocks_per_view blocks) or tables.
 struct Segs {
@@ -207,6 +211,29 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Digit source of a depth key. The first depth pass reads the projection's keys and orders
+// key - kmin(view) (kmin = the view's smallest visible key), clamped to `top` = 2^bits - 1 where
+// bits is the width of the largest view's key range; culled entries (key 0xffffffff) clamp to the
+// top and sort last. The pass writes the mapped keys, so the later passes read them unchanged
+// (kbits == nullptr: identity).
+struct KeyMap {
+  const uint32_t* kbits;  // [V][kKeyStripes][2] statistics of the projection, or nullptr
+  uint32_t top;
+};
+
+// the view's smallest visible key: the complement of the largest complement over the stripes
+__device__ __forceinline__ uint32_t view_kmin(const uint32_t* __restrict__ kbits, int v) {
+  const int lane = threadIdx.x & 31;
+  uint32_t m = 0;
+  for (int s = lane; s < kKeyStripes; s += 32) m = max(m, kbits[2 * (v * kKeyStripes + s) + 1]);
+  return ~__reduce_max_sync(0xffffffffu, m);
+}
+
+__device__ __forceinline__ uint32_t map_key(uint32_t k, uint32_t kmin, uint32_t top) {
+  const uint32_t d = k - kmin;
+  return d < top ? d : top;
+}
+
 constexpr int kUnroll = 16;      // 32-item batches whose loads are issued together (ranking)
 constexpr int kCountUnroll = 32; // 32-item batches whose loads are issued together (counting)
 constexpr int kHistUnroll = 32;  // the same for the histogram kernel
@@ -215,9 +242,9 @@ constexpr int kHistUnroll = 32;  // the same for the histogram kernel
 // batches are issued together, then each lane adds its items with shared-memory atomics (counts
 // do not depend on the order of the adds); whole groups without tail checks, then the tail
 template <int UNR>
-__device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, int shift,
-                                            uint32_t mask, long long wb, long long we,
-                                            uint32_t* cnt) {
+__device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, uint32_t kmin,
+                                            uint32_t top, int shift, uint32_t mask, long long wb,
+                                            long long we, uint32_t* cnt) {
   const int lane = threadIdx.x & 31;
   const uint32_t* kp = keys + wb;
   const int n = we > wb ? (int)(we - wb) : 0;
@@ -225,7 +252,7 @@ __device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, i
   for (int b = 0; b < nfull; b += 32 * UNR) {
     uint32_t bk[UNR];
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) bk[u] = (kp[b + 32 * u + lane] >> shift) & mask;
+    for (int u = 0; u < UNR; ++u) bk[u] = (map_key(kp[b + 32 * u + lane], kmin, top) >> shift) & mask;
 #pragma unroll
     for (int u = 0; u < UNR; ++u) atomicAdd(cnt + bk[u], 1u);
   }
@@ -234,7 +261,7 @@ __device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, i
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
       const int o = nfull + 32 * u + lane;
-      bk[u] = o < n ? (kp[o] >> shift) & mask : 0xffffffffu;
+      bk[u] = o < n ? (map_key(kp[o], kmin, top) >> shift) & mask : 0xffffffffu;
     }
 #pragma unroll
     for (int u = 0; u < UNR; ++u)
@@ -244,16 +271,17 @@ __device__ __forceinline__ void warp_counts(const uint32_t* __restrict__ keys, i
 
 // histogram: hist[nbk * b0 + bucket * nbv + lb] = count of the block's items in the bucket
 __global__ void __launch_bounds__(kBinThreads)
-k_count_hist(const uint32_t* __restrict__ keys, int shift, uint32_t mask, int nbk, Segs sg,
-             int* __restrict__ hist) {
+k_count_hist(const uint32_t* __restrict__ keys, KeyMap km, int shift, uint32_t mask, int nbk,
+             Segs sg, int* __restrict__ hist) {
   extern __shared__ uint32_t s_cnt[];  // [kBinWarps][nbk]
   const BlockRange r = block_range(sg, blockIdx.x);
   for (int t = threadIdx.x; t < kBinWarps * nbk; t += blockDim.x) s_cnt[t] = 0;
+  const uint32_t kmin = km.kbits ? view_kmin(km.kbits, r.v) : 0u;
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   const long long wb = r.beg + (long long)warp * (sg.chunk / kBinWarps);
   const long long we = min(wb + (long long)(sg.chunk / kBinWarps), r.end);
-  warp_counts<kHistUnroll>(keys, shift, mask, wb, we, s_cnt + warp * nbk);
+  warp_counts<kHistUnroll>(keys, kmin, km.top, shift, mask, wb, we, s_cnt + warp * nbk);
   __syncthreads();
   int* h = hist + (size_t)nbk * r.b0;
   for (int t = threadIdx.x; t < nbk; t += blockDim.x) {
@@ -267,8 +295,8 @@ k_count_hist(const uint32_t* __restrict__ keys, int shift, uint32_t mask, int nb
 // stable scatter of (key, value) by bucket; vals == nullptr means value = index within the view;
 // kout == nullptr drops the keys
 __global__ void __launch_bounds__(kBinThreads)
-k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ vals, int shift,
-                uint32_t mask, int nbk, Segs sg, const int* __restrict__ hist_scan,
+k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ vals, KeyMap km,
+                int shift, uint32_t mask, int nbk, Segs sg, const int* __restrict__ hist_scan,
                 uint32_t* __restrict__ kout, uint32_t* __restrict__ vout) {
   extern __shared__ uint32_t s_cnt[];  // [kBinWarps][nbk]
   const BlockRange r = block_range(sg, blockIdx.x);
@@ -278,7 +306,8 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
   uint32_t* cnt = s_cnt + warp * nbk;
   const long long wb = r.beg + (long long)warp * (sg.chunk / kBinWarps);
   const long long we = min(wb + (long long)(sg.chunk / kBinWarps), r.end);
-  warp_counts<kCountUnroll>(keys, shift, mask, wb, we, cnt);
+  const uint32_t kmin = km.kbits ? view_kmin(km.kbits, r.v) : 0u;
+  warp_counts<kCountUnroll>(keys, kmin, km.top, shift, mask, wb, we, cnt);
   __syncthreads();
   // per bucket: global start of this block's run, then one sub-run per warp in warp order
   const int* h = hist_scan + (size_t)nbk * r.b0;
@@ -306,7 +335,7 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int o = b + 32 * u + lane;
-      key[u] = kp[o];
+      key[u] = map_key(kp[o], kmin, km.top);
       val[u] = vp ? vp[o] : vbase + (uint32_t)o;
     }
 #pragma unroll
@@ -326,7 +355,7 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
   for (int b = nfull; b < n; b += 32) {
     const int o = b + lane;
     const bool ok = o < n;
-    const uint32_t key = ok ? kp[o] : 0u;
+    const uint32_t key = ok ? map_key(kp[o], kmin, km.top) : 0u;
     const uint32_t val = ok ? (vp ? vp[o] : vbase + (uint32_t)o) : 0u;
     const uint32_t bk = ok ? (key >> shift) & mask : (0x80000000u | lane);
     const uint32_t peers = __match_any_sync(0xffffffffu, bk);
@@ -340,6 +369,140 @@ k_count_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ 
     __syncwarp();
     if (ok && lane == __ffs(peers) - 1) cnt[bk] += __popc(peers);
     __syncwarp();
+  }
+}
+
+// Stable scatter of (key, value) by bucket, one round of kRound consecutive items at a time
+// (vals == nullptr: value = index within the view; kout == nullptr drops the keys). In a round
+// each warp ranks its kWarpRound items in order -- match.any inside each 32-item batch and a
+// per-warp count per bucket -- and a block scan over (bucket, warp), bucket-major, turns the
+// counts into every item's place in the round's bucket order (stable: a warp's items in order,
+// the warps in order). The round is laid out in shared memory in that order and then written
+// out: thread j stores place j at base(bucket) + j - start(bucket), so a warp's stores fall on a
+// few bucket runs instead of 32 scattered words. base(bucket) starts at the block's entry of the
+// scanned (bucket, block) histogram and advances by the bucket's count after every round.
+constexpr int kRoundIpt = 16;                        // items per thread per round
+constexpr int kRound = kBinThreads * kRoundIpt;      // items per round
+constexpr int kWarpRound = kRound / kBinWarps;       // items per warp per round
+
+// buckets per thread in the (bucket, warp) scan: odd, so that the threads' strided reads of the
+// counts fall on distinct banks
+__host__ __device__ __forceinline__ int scan_bpt(int nbk) {
+  return ((nbk + 1 + kBinThreads - 1) / kBinThreads) | 1;
+}
+
+// dynamic shared memory of k_rank_scatter: counts [kBinWarps][nbk + 1], bases [nbk], the round's
+// keys and values [kRound] each
+__host__ __device__ __forceinline__ size_t rank_scatter_smem(int nbk) {
+  return ((size_t)kBinWarps * (nbk + 1) + nbk + 2 * (size_t)kRound) * sizeof(uint32_t);
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t* dst, const uint32_t* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src));
+}
+
+__global__ void __launch_bounds__(kBinThreads, 4)
+k_rank_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ vals, KeyMap km,
+               int shift, uint32_t mask, int nbk, Segs sg, const int* __restrict__ hist_scan,
+               uint32_t* __restrict__ kout, uint32_t* __restrict__ vout) {
+  extern __shared__ uint32_t s_mem[];
+  __shared__ uint32_t s_warp[32];
+  const int ncol = nbk + 1;                       // column nbk: the items past the end
+  uint32_t* s_cnt = s_mem;                        // [kBinWarps][ncol]
+  uint32_t* s_base = s_cnt + kBinWarps * ncol;    // [nbk]
+  uint32_t* s_key = s_base + nbk;                 // [kRound] values as read, then keys in bucket order
+  uint32_t* s_val = s_key + kRound;               // [kRound] values in bucket order
+  const BlockRange r = block_range(sg, blockIdx.x);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t kmin = km.kbits ? view_kmin(km.kbits, r.v) : 0u;
+  const int* h = hist_scan + (size_t)nbk * r.b0;
+  for (int t = threadIdx.x; t < nbk; t += kBinThreads) s_base[t] = (uint32_t)h[(size_t)t * r.nbv + r.lb];
+  const uint32_t lt = lanemask_lt();
+  const unsigned long long lim =
+      sg.per_view >= 0 ? (unsigned long long)sg.per_view * sg.V : (unsigned long long)sg.vstart[sg.V];
+  const int bpt = scan_bpt(nbk);
+  const int sb0 = threadIdx.x * bpt, sb1 = min(sb0 + bpt, ncol);
+  const int wo = warp * kWarpRound + lane;
+  uint32_t* cnt = s_cnt + warp * ncol;
+  for (long long rb = r.beg; rb < r.end; rb += kRound) {
+    const int n = (int)min((long long)kRound, r.end - rb);
+    for (int t = threadIdx.x; t < kBinWarps * ncol; t += kBinThreads) s_cnt[t] = 0;
+    // the values go to shared memory asynchronously (read at the layout step), the keys to
+    // registers
+    if (vals)
+      for (int j = threadIdx.x; j < n; j += kBinThreads) cp_async4(s_key + j, vals + rb + j);
+    asm volatile("cp.async.commit_group;\n" ::);
+    const uint32_t* kq = keys + rb + wo;
+    uint32_t key[kRoundIpt], rank[kRoundIpt / 2];  // ranks: two 16-bit halves per word
+    if (n == kRound) {
+#pragma unroll
+      for (int u = 0; u < kRoundIpt; ++u) key[u] = map_key(kq[32 * u], kmin, km.top);
+    } else {
+#pragma unroll
+      for (int u = 0; u < kRoundIpt; ++u)
+        key[u] = wo + 32 * u < n ? map_key(kq[32 * u], kmin, km.top) : 0u;
+    }
+    __syncthreads();
+    // rank inside the warp: earlier items of the same bucket, in (batch, lane) order
+#pragma unroll
+    for (int u = 0; u < kRoundIpt; ++u) {
+      const uint32_t bk = wo + 32 * u < n ? (key[u] >> shift) & mask : (uint32_t)nbk;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bk);
+      const uint32_t c = cnt[bk];
+      const uint32_t rk = c + __popc(peers & lt);  // < kWarpRound
+      rank[u / 2] = (u & 1) ? rank[u / 2] | (rk << 16) : rk;
+      __syncwarp();
+      if (lane == __ffs(peers) - 1) cnt[bk] = c + __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    // exclusive scan of the counts in (bucket, warp) order; row 0 then holds the bucket starts
+    uint32_t sum = 0;
+    for (int b = sb0; b < sb1; ++b)
+#pragma unroll
+      for (int ww = 0; ww < kBinWarps; ++ww) sum += s_cnt[ww * ncol + b];
+    uint32_t off = block_exclusive_scan<uint32_t>(sum, s_warp, nullptr);
+    for (int b = sb0; b < sb1; ++b)
+#pragma unroll
+      for (int ww = 0; ww < kBinWarps; ++ww) {
+        const uint32_t c = s_cnt[ww * ncol + b];
+        s_cnt[ww * ncol + b] = off;
+        off += c;
+      }
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    __syncthreads();
+    // the round in bucket order: first the values (read from where they landed in s_key), then,
+    // once every value is read, the keys
+    const uint32_t vbase = (uint32_t)(rb - r.vbeg) + (uint32_t)wo;
+#pragma unroll
+    for (int u = 0; u < kRoundIpt; ++u) {
+      if (wo + 32 * u < n) {
+        const uint32_t lp = cnt[(key[u] >> shift) & mask] + ((rank[u / 2] >> (16 * (u & 1))) & 0xffffu);
+        s_val[lp] = vals ? s_key[wo + 32 * u] : vbase + 32 * u;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kRoundIpt; ++u) {
+      if (wo + 32 * u < n) {
+        const uint32_t lp = cnt[(key[u] >> shift) & mask] + ((rank[u / 2] >> (16 * (u & 1))) & 0xffffu);
+        s_key[lp] = key[u];
+      }
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < n; j += kBinThreads) {
+      const uint32_t k = s_key[j];
+      const uint32_t bk = (k >> shift) & mask;
+      const uint32_t pos = s_base[bk] + (uint32_t)j - s_cnt[bk];
+      if (in_bounds(pos, lim, &g_bounds_word)) {
+        if (kout) kout[pos] = k;
+        vout[pos] = s_val[j];
+      }
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < nbk; b += kBinThreads) s_base[b] += s_cnt[b + 1] - s_cnt[b];
+    __syncthreads();
   }
 }
 
@@ -582,16 +745,16 @@ int scan_i32_inplace(Workspace& w, int* data, long long n, cudaStream_t st) {
 }
 
 
-// one stable counting-sort pass (histogram, scan, scatter)
+// one stable counting-sort pass (histogram, scan, scatter; runs: the scatter through bucket runs)
 static int count_pass(Workspace& w, cudaStream_t st, const uint32_t* keys, const uint32_t* vals,
-                      int shift, uint32_t mask, int nbk, const Segs& sg, int nblocks,
-                      uint32_t* kout, uint32_t* vout, int id_hist, int id_scatter) {
+                      KeyMap km, int shift, uint32_t mask, int nbk, const Segs& sg, int nblocks,
+                      uint32_t* kout, uint32_t* vout, int id_hist, int id_scatter, bool runs) {
   int rc;
   const size_t hist_n = (size_t)nbk * nblocks;
   if ((rc = ensure_hist(w, hist_n))) return rc;
   const size_t smem = (size_t)kBinWarps * nbk * sizeof(uint32_t);
   int tok = prof_begin(w, st, id_hist);
-  k_count_hist<<<nblocks, kBinThreads, smem, st>>>(keys, shift, mask, nbk, sg, w.hist);
+  k_count_hist<<<nblocks, kBinThreads, smem, st>>>(keys, km, shift, mask, nbk, sg, w.hist);
   prof_end(w, st, tok);
   if ((rc = check_launch(w, "histogram kernel"))) return rc;
   tok = prof_begin(w, st, SPLAT_K_HIST_SCAN);
@@ -599,8 +762,12 @@ static int count_pass(Workspace& w, cudaStream_t st, const uint32_t* keys, const
   prof_end(w, st, tok);
   if (rc) return rc;
   tok = prof_begin(w, st, id_scatter);
-  k_count_scatter<<<nblocks, kBinThreads, smem, st>>>(keys, vals, shift, mask, nbk, sg, w.hist,
-                                                       kout, vout);
+  if (runs)
+    k_rank_scatter<<<nblocks, kBinThreads, rank_scatter_smem(nbk), st>>>(keys, vals, km, shift, mask,
+                                                                        nbk, sg, w.hist, kout, vout);
+  else
+    k_count_scatter<<<nblocks, kBinThreads, smem, st>>>(keys, vals, km, shift, mask, nbk, sg, w.hist,
+                                                         kout, vout);
   prof_end(w, st, tok);
   return check_launch(w, "scatter kernel");
 }
@@ -634,18 +801,18 @@ int launch_binning(Workspace& w, cudaStream_t st) {
     }
   }
   // ---- 1. depth order of every view's Gaussians --------------------------------------------
-  // highest bit that varies among any view's visible keys -> number of digit passes
-  int hb = -1;
+  // width of the widest view's visible key range -> number of digit passes
+  uint32_t range = 0;
   for (int v = 0; v < w.V; ++v) {
-    uint32_t k1 = 0, k0 = 0;
+    uint32_t khi = 0, klo = 0;
     for (int sidx = 0; sidx < kKeyStripes; ++sidx) {
-      k1 |= w.h_kbits[2 * (v * kKeyStripes + sidx)];
-      k0 |= w.h_kbits[2 * (v * kKeyStripes + sidx) + 1];
+      khi = max(khi, w.h_kbits[2 * (v * kKeyStripes + sidx)]);
+      klo = max(klo, w.h_kbits[2 * (v * kKeyStripes + sidx) + 1]);
     }
-    const uint32_t vary = k1 & k0;
-    if (vary) hb = max(hb, 31 - __builtin_clz(vary));
+    if (khi) range = max(range, khi - ~klo);  // no visible key: both stay 0
   }
-  const int bits = hb + 1;
+  const int bits = range ? 32 - __builtin_clz(range) : 0;
+  const KeyMap map0{w.kbits, bits >= 32 ? 0xffffffffu : (1u << bits) - 1u};
   const int passes = bits == 0 ? 0 : (bits + kDepthDigitMax - 1) / kDepthDigitMax;
   const int dbits = passes ? (bits + passes - 1) / passes : 0;
   const uint32_t* order = nullptr;  // sorted Gaussian indices per view (nullptr: index order)
@@ -662,8 +829,9 @@ int launch_binning(Workspace& w, cudaStream_t st) {
       const uint32_t mask = (width >= 32) ? 0xffffffffu : ((1u << width) - 1u);
       uint32_t* kout = (p + 1 < passes) ? kb[p & 1] : nullptr;
       uint32_t* vout = vb[p & 1];
-      if ((rc = count_pass(w, st, kin, vin, shift, mask, (int)mask + 1, sg, nblocks, kout, vout,
-                           SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER)))
+      const KeyMap km = p == 0 ? map0 : KeyMap{nullptr, 0xffffffffu};
+      if ((rc = count_pass(w, st, kin, vin, km, shift, mask, (int)mask + 1, sg, nblocks, kout,
+                           vout, SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER, true)))
         return rc;
       kin = kout;
       vin = vout;
@@ -695,8 +863,9 @@ int launch_binning(Workspace& w, cudaStream_t st) {
     return rc;
   if (N > 0) {
     Segs sg{-1, 0, w.d_vstart, w.d_bstart, w.V, kTileChunk};
-    if ((rc = count_pass(w, st, w.inst_tile, w.inst_g, 0, 0xffffffffu, w.nt, sg, w.n_blocks,
-                         nullptr, w.sval, SPLAT_K_TILE_HIST, SPLAT_K_TILE_SCATTER)))
+    if ((rc = count_pass(w, st, w.inst_tile, w.inst_g, KeyMap{nullptr, 0xffffffffu}, 0,
+                         0xffffffffu, w.nt, sg, w.n_blocks, nullptr, w.sval, SPLAT_K_TILE_HIST,
+                         SPLAT_K_TILE_SCATTER, false)))
       return rc;
   } else if ((rc = ensure_hist(w, 1))) {
     return rc;
@@ -719,12 +888,15 @@ int launch_binning(Workspace& w, cudaStream_t st) {
 
 // shared-memory opt-in for the counting-sort kernels (called once per workspace)
 int binning_configure(Workspace& w) {
-  const int need = kBinWarps * max(w.max_nt, 2048) * (int)sizeof(uint32_t);
+  const int nbk = max(w.max_nt, 2048);
+  const size_t need_hist = (size_t)kBinWarps * nbk * sizeof(uint32_t);
   cudaError_t e2 = cudaFuncSetAttribute(k_count_hist, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        need);
-  cudaError_t e3 = cudaFuncSetAttribute(k_count_scatter,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, need);
-  if (e2 != cudaSuccess || e3 != cudaSuccess) {
+                                        (int)need_hist);
+  cudaError_t e3 = cudaFuncSetAttribute(k_rank_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)rank_scatter_smem(nbk));
+  cudaError_t e4 = cudaFuncSetAttribute(k_count_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)need_hist);
+  if (e2 != cudaSuccess || e3 != cudaSuccess || e4 != cudaSuccess) {
     cudaGetLastError();
     return set_err(w, SPLAT_ERR_CAPACITY,
                    "image has too many tiles for the binning kernels' shared memory");

@@ -211,7 +211,7 @@ struct Workspace {
 
   // per-(v, g) depth order
   uint32_t* dkey = nullptr;    // [V*G] depth sort keys (written by the projection)
-  uint32_t* kbits = nullptr;   // [V][kKeyStripes][2]: OR of visible keys, OR of complements
+  uint32_t* kbits = nullptr;   // [V][kKeyStripes][2]: max visible key, max complement of one
   unsigned long long* ntot = nullptr;  // [V][kKeyStripes] instance counts (striped)
   unsigned long long* h_ntot = nullptr;  // pinned, mapped (hd_ntot: its device address)
   unsigned long long* hd_ntot = nullptr;

@@ -23,6 +23,10 @@ namespace splat {
 namespace {
 
 constexpr int kFinThreads = 128;
+// 7 blocks of 128 threads per SM: 72 registers a thread (the shared-memory token tile, 29 KB a
+// block at degree 3, also allows 7)
+constexpr int kFinMinBlocks = 7;
+
 
 // eigenvalues of a symmetric 3x3 matrix, descending, by the trigonometric solution of the
 // characteristic cubic (O. K. Smith, "Eigenvalues of a symmetric 3x3 matrix", CACM 4(4), 1961)
@@ -125,6 +129,10 @@ __device__ __forceinline__ void view_sums(const float4* __restrict__ rec,
       col[(4 + 3 * k) * P] += B[k] * w0;
       col[(5 + 3 * k) * P] += B[k] * w1;
       col[(6 + 3 * k) * P] += B[k] * w2;
+      // (a compiler-only fence every four coefficients: without it the 3 x D shared-memory
+      // loads of the block are all hoisted ahead of their adds, which holds ~48 more registers
+      // and caps the kernel at 16 warps per SM)
+      if ((k & 3) == 3) asm volatile("" ::: "memory");
     }
   }
 }
@@ -172,7 +180,7 @@ __device__ __forceinline__ void store_rows(const float* s_tile, int ncols, int g
 
 // fused single-device path: sums over all views, then the token
 template <int DEG>
-__global__ void __launch_bounds__(kFinThreads, 4)
+__global__ void __launch_bounds__(kFinThreads, kFinMinBlocks)
 k_finalize(const float4* __restrict__ rec, const float* __restrict__ acc,
            const float* __restrict__ views, int G, int V, double lambda,
            float* __restrict__ tokens) {
@@ -198,7 +206,7 @@ k_finalize(const float4* __restrict__ rec, const float* __restrict__ acc,
 // sharded path, part 1: this device's per-Gaussian partial sums over its views,
 // [qsum, b(3), sa, A(6: 00 01 02 11 12 22), SH block (3d)] = 11 + 3d floats per Gaussian
 template <int DEG>
-__global__ void __launch_bounds__(kFinThreads, 4)
+__global__ void __launch_bounds__(kFinThreads, kFinMinBlocks)
 k_partials(const float4* __restrict__ rec, const float* __restrict__ acc,
            const float* __restrict__ views, int G, int V, float* __restrict__ partials) {
   constexpr int D = (DEG + 1) * (DEG + 1);

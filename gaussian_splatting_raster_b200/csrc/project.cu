@@ -243,21 +243,21 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
     rect[i] = rc;
     counts[i] = cnt;
     // depth sort key (fp32 bits of z > 0 order like the values; culled entries sort last) and,
-    // per view, the OR of the visible keys and of their complements: a bit varies among the
-    // visible keys exactly where both ORs have it set
+    // per view, the largest visible key and the largest complement of one (the complement of the
+    // smallest visible key): the sort orders key - smallest, over the bits of the key range
     const uint32_t key = cnt > 0 ? __float_as_uint(z) : 0xffffffffu;
     dkey[i] = key;
     const unsigned lanes = __activemask();
-    const uint32_t k1 = __reduce_or_sync(lanes, cnt > 0 ? key : 0u);
-    const uint32_t k0 = __reduce_or_sync(lanes, cnt > 0 ? ~key : 0u);
+    const uint32_t khi = __reduce_max_sync(lanes, cnt > 0 ? key : 0u);
+    const uint32_t klo = __reduce_max_sync(lanes, cnt > 0 ? ~key : 0u);
     const unsigned int ntile = __reduce_add_sync(lanes, (unsigned int)cnt);
-    if ((threadIdx.x & 31) == __ffs(lanes) - 1 && (k1 | k0)) {
+    if ((threadIdx.x & 31) == __ffs(lanes) - 1 && khi) {
       // one of kKeyStripes copies per view, chosen by block, keeps same-address atomics rare;
-      // the host folds the stripes (OR of the key statistics, sum of the instance counts)
+      // the stripes are folded later (maxima of the key statistics, sum of the instance counts)
       const int stripe = v * kKeyStripes + (blockIdx.x & (kKeyStripes - 1));
       uint32_t* kb = kbits + 2 * stripe;
-      atomicOr(kb, k1);
-      atomicOr(kb + 1, k0);
+      atomicMax(kb, khi);
+      atomicMax(kb + 1, klo);
       atomicAdd(ntot + stripe, (unsigned long long)ntile);
     }
   }
