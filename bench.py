@@ -221,10 +221,10 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
         # per pass keys and values in and out; the first reads no values (the index is implicit),
         # the last writes no keys
         "depth_scatter": max(depth_passes * 16 - 8, 0) * V * G,
-        # rectangles gathered into depth order (order 4 B + rectangle 16 B in, 16 B + count out),
-        # the counts scanned (4 B in, 8 B out), instances (tile, g) emitted (rectangle, index,
-        # offset in; 8 B out)
-        "emit": V * G * (20 + 20 + 12 + 28) + n_inst * 8,
+        # rectangles (4 x 16 bit) gathered into depth order (order 4 B + rectangle 8 B in, 8 B +
+        # count 4 B out), the counts scanned in place (4 B in, 4 B out), instances (tile, g)
+        # emitted (rectangle, index, offset in; 8 B out)
+        "emit": V * G * (12 + 12 + 8 + 16) + n_inst * 8,
         "tile_hist": n_inst * 4,
         "tile_scatter": n_inst * (4 + 4 + 4),
         # gather 36 B per list entry staged, write C_hat, T, n, last

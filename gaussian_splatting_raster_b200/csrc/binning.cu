@@ -136,8 +136,6 @@ k_scan_down(const TI* in, TO* out, long long n, const long long* __restrict__ pa
   }
 }
 
-__global__ void k_store_total(const long long* part, int nb, long long* dst) { *dst = part[nb]; }
-
 int ensure_part(Workspace& w, long long nb) {
   if ((size_t)(nb + 1) <= w.part_cap) return SPLAT_OK;
   if (w.part) cudaFree(w.part);
@@ -506,17 +504,17 @@ k_rank_scatter(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ v
   }
 }
 
-// tile rectangles and counts in depth order (order == nullptr: index order)
-__global__ void k_gather_rects(const int4* __restrict__ rect, const uint32_t* __restrict__ order,
-                               long long VG, int G, int4* __restrict__ rect_s,
+// tile rectangles and their tile counts in depth order (order == nullptr: index order)
+__global__ void k_gather_rects(const ushort4* __restrict__ rect, const uint32_t* __restrict__ order,
+                               long long VG, int G, ushort4* __restrict__ rect_s,
                                int* __restrict__ cnt_s) {
   const long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= VG) return;
   const long long v = k / G;
   const uint32_t g = order ? order[k] : (uint32_t)(k - v * G);
-  const int4 rc = rect[v * G + g];
+  const ushort4 rc = rect[v * G + g];
   rect_s[k] = rc;
-  cnt_s[k] = (rc.z - rc.x) * (rc.w - rc.y);
+  cnt_s[k] = ((int)rc.z - (int)rc.x) * ((int)rc.w - (int)rc.y);
 }
 
 // instances (tile, g) in depth order. One warp per 32 consecutive entries: the lanes write the
@@ -524,27 +522,30 @@ __global__ void k_gather_rects(const int4* __restrict__ rect, const uint32_t* __
 // however many tiles each entry covers); each position finds its entry by a binary search over
 // the 32 entry offsets, then its tile from its index inside the entry's rectangle (row-major).
 __global__ void __launch_bounds__(256)
-k_emit(const int4* __restrict__ rect_s, const uint32_t* __restrict__ order,
-       const long long* __restrict__ offs, long long VG, int G, int TX,
+k_emit(const ushort4* __restrict__ rect_s, const uint32_t* __restrict__ order,
+       const int* __restrict__ offs, long long VG, long long n_inst, int G, int TX,
        uint32_t* __restrict__ inst_tile, uint32_t* __restrict__ inst_g) {
   const int lane = threadIdx.x & 31;
   const long long k0 = (long long)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
   if (k0 >= VG) return;  // warp-uniform
   const long long k = k0 + lane;
   const bool ok = k < VG;
-  int4 rc = make_int4(0, 0, 0, 0);
+  int x0e = 0, y0e = 0, wdt = 0;
   uint32_t g = 0;
   if (ok) {
-    rc = rect_s[k];
+    const ushort4 rc = rect_s[k];
+    x0e = rc.x;
+    y0e = rc.y;
+    wdt = (int)rc.z - (int)rc.x;
     const long long v = k / G;
     g = order ? order[k] : (uint32_t)(k - v * G);
   }
-  const long long start = offs[k0];
-  const int total = (int)(offs[min(k0 + 32, VG)] - start);
+  // offs: exclusive scan of the entries' tile counts (int32: the instance total is below 2^31)
+  const int start = offs[k0];
+  const int total = (k0 + 32 < VG ? offs[k0 + 32] : (int)n_inst) - start;
   // entry start relative to the warp's range; lanes past the end sit at the end (never chosen)
-  const int rel = ok ? (int)(offs[k] - start) : total;
-  const int wdt = rc.z - rc.x;
-  const unsigned long long lim = kChecked ? (unsigned long long)offs[VG] : 0ull;
+  const int rel = ok ? offs[k] - start : total;
+  const unsigned long long lim = kChecked ? (unsigned long long)n_inst : 0ull;
   for (int b = 0; b < total; b += 32) {
     const int p = b + lane;
     // the last entry whose start is <= p (starts are non-decreasing; entry 0 starts at 0)
@@ -552,8 +553,8 @@ k_emit(const int4* __restrict__ rect_s, const uint32_t* __restrict__ order,
 #pragma unroll
     for (int s = 16; s >= 1; s >>= 1)
       if (__shfl_sync(0xffffffffu, rel, j + s) <= p) j += s;
-    const int x0 = __shfl_sync(0xffffffffu, rc.x, j);
-    const int y0 = __shfl_sync(0xffffffffu, rc.y, j);
+    const int x0 = __shfl_sync(0xffffffffu, x0e, j);
+    const int y0 = __shfl_sync(0xffffffffu, y0e, j);
     const int wj = __shfl_sync(0xffffffffu, wdt, j);
     const int rj = __shfl_sync(0xffffffffu, rel, j);
     const uint32_t gj = __shfl_sync(0xffffffffu, g, j);
@@ -673,25 +674,6 @@ int ensure_hist(Workspace& w, size_t n) {
 }
 
 }  // namespace
-
-// ---------------------------------------------------------------------------------------------
-int scan_i32_to_i64(Workspace& w, const int* in, long long* out, long long n, cudaStream_t st) {
-  const long long nb = (n + kScanTile - 1) / kScanTile;
-  int rc = ensure_part(w, nb > 0 ? nb : 1);
-  if (rc) return rc;
-  if (nb > 0) {
-    k_scan_reduce<int><<<(unsigned)nb, kScanThreads, 0, st>>>(in, n, w.part);
-    if ((rc = check_launch(w, "scan reduce"))) return rc;
-  }
-  k_scan_partials<<<1, 1024, 0, st>>>(w.part, (int)nb);
-  if ((rc = check_launch(w, "scan partials"))) return rc;
-  if (nb > 0) {
-    k_scan_down<int, long long><<<(unsigned)nb, kScanThreads, 0, st>>>(in, out, n, w.part);
-    if ((rc = check_launch(w, "scan downsweep"))) return rc;
-  }
-  k_store_total<<<1, 1, 0, st>>>(w.part, (int)nb, out + n);
-  return check_launch(w, "scan total");
-}
 
 namespace {
 __global__ void k_zero(uint4* __restrict__ p16, size_t n16, uint32_t* __restrict__ p4, size_t n4) {
@@ -844,8 +826,9 @@ int launch_binning(Workspace& w, cudaStream_t st) {
     const unsigned grid = (unsigned)((VG + 255) / 256);
     k_gather_rects<<<grid, 256, 0, st>>>(w.rect, order, VG, w.G, w.rect_s, w.counts);
     if ((rc = check_launch(w, "rectangle gather kernel"))) return rc;
-    if ((rc = scan_i32_to_i64(w, w.counts, w.offs, VG, st))) return rc;
-    k_emit<<<grid, 256, 0, st>>>(w.rect_s, order, w.offs, VG, w.G, w.TX, w.inst_tile, w.inst_g);
+    if ((rc = scan_i32_inplace(w, w.counts, VG, st))) return rc;
+    k_emit<<<grid, 256, 0, st>>>(w.rect_s, order, w.counts, VG, N, w.G, w.TX, w.inst_tile,
+                                 w.inst_g);
     prof_end(w, st, tok);
     if ((rc = check_launch(w, "emit kernel"))) return rc;
   }
@@ -892,8 +875,9 @@ int binning_configure(Workspace& w) {
   const size_t need_hist = (size_t)kBinWarps * nbk * sizeof(uint32_t);
   cudaError_t e2 = cudaFuncSetAttribute(k_count_hist, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)need_hist);
+  // (the runs scatter serves only the depth passes: at most 2^kDepthDigitMax buckets)
   cudaError_t e3 = cudaFuncSetAttribute(k_rank_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)rank_scatter_smem(nbk));
+                                        (int)rank_scatter_smem(1 << kDepthDigitMax));
   cudaError_t e4 = cudaFuncSetAttribute(k_count_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)need_hist);
   if (e2 != cudaSuccess || e3 != cudaSuccess || e4 != cudaSuccess) {

@@ -82,7 +82,7 @@ int alloc_mapped(Workspace& w, T** h, T** d, size_t n, const char* what) {
 }
 
 void free_all(Workspace& w) {
-  void* dev[] = {w.rec, w.rect, w.counts, w.offs, w.acc, w.views, w.last, w.part,
+  void* dev[] = {w.rec, w.rect, w.counts, w.acc, w.views, w.last, w.part,
                  w.inst_tile, w.inst_g, w.sval, w.hist, w.tile_off, w.d_vstart, w.d_bstart,
                  w.d_scratch, w.dkey, w.kbits, w.dk1, w.dk2, w.dv0, w.dv1, w.rect_s, w.ntot, w.umask, w.lmask, w.accb, w.sacc,
                  w.acc_fix, w.accb_fix, w.tile_order};
@@ -144,8 +144,7 @@ int splat_ws_create(splat_ws** out, int max_G, int max_V, int max_H, int max_W,
   int rc = 0;
   if (!rc) rc = alloc(w, &w.rec, splat::rec_f4_count(VG), "records");
   if (!rc) rc = alloc(w, &w.rect, VG, "rectangles");
-  if (!rc) rc = alloc(w, &w.counts, VG, "tile counts");
-  if (!rc) rc = alloc(w, &w.offs, VG + 1, "instance offsets");
+  if (!rc) rc = alloc(w, &w.counts, VG, "tile counts in depth order, then their scan");
   if (!rc) rc = alloc(w, &w.acc, VG * splat::kAccN, "accumulators");
   if (!rc) rc = alloc(w, &w.views, (size_t)max_V * 20, "views");
   if (!rc) rc = alloc(w, &w.last, (size_t)max_V * max_H * max_W, "list bounds");
@@ -413,8 +412,7 @@ int splat_copy_projection(splat_ws* ws, float* rec, int* rect, void* stream) {
   if ((rc = check_dev_ptr(w, rect, "rect"))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   if ((rc = splat::launch_copy_records(w, rec, st))) return rc;
-  cudaError_t e = cudaMemcpyAsync(rect, w.rect, VG * 16, cudaMemcpyDeviceToDevice, st);
-  return e == cudaSuccess ? SPLAT_OK : cuda_fail(w, "copy projection", e);
+  return splat::launch_copy_rects(w, rect, st);
 }
 
 int splat_copy_tile_lists(splat_ws* ws, long long* tile_offsets, int* ids, void* stream) {

@@ -186,9 +186,8 @@ struct Workspace {
 
   // per (v, g)
   float4* rec = nullptr;     // [V*G*4]
-  int4* rect = nullptr;      // [V*G]
-  int* counts = nullptr;     // [V*G] tiles touched
-  long long* offs = nullptr; // [V*G + 1] exclusive scan of counts
+  ushort4* rect = nullptr;   // [V*G] tile rectangle x0, y0, x1, y1 (16-bit tile coordinates)
+  int* counts = nullptr;     // [V*G] tile counts in depth order, then their exclusive scan
   float* acc = nullptr;      // [V*G*8] score sums: (q, w r (3)), (w rho, w rho d (2), unused)
   double* accb = nullptr;    // [max_V*max_G*10] renderer-backward sums, allocated on first use
   double* sacc = nullptr;    // [G*C] scatter sums, grown on demand
@@ -219,7 +218,7 @@ struct Workspace {
   uint32_t* dk2 = nullptr;     // [V*G]
   uint32_t* dv0 = nullptr;     // [V*G] radix values (Gaussian index), ping
   uint32_t* dv1 = nullptr;     // [V*G] pong
-  int4* rect_s = nullptr;      // [V*G] tile rectangles in depth order
+  ushort4* rect_s = nullptr;   // [V*G] tile rectangles in depth order
 
   // instances
   size_t inst_cap = 0;
@@ -330,6 +329,7 @@ int launch_pair_count(Workspace& w, cudaStream_t st);
 int launch_acc_to_double(Workspace& w, double* out, cudaStream_t st);
 // the records in the documented order into out [V*G*16] (the inspection copy)
 int launch_copy_records(Workspace& w, float* out, cudaStream_t st);
+int launch_copy_rects(Workspace& w, int* out, cudaStream_t st);
 unsigned int bounds_word_raster(cudaStream_t st);
 unsigned int bounds_word_binning(cudaStream_t st);
 unsigned int bounds_word_attributes(cudaStream_t st);
@@ -337,7 +337,6 @@ int binning_configure(Workspace& w);
 
 // reduce-then-scan over n int32 values into int64 exclusive prefixes (out has n + 1 entries; the
 // last is the total). Uses w.part as scratch.
-int scan_i32_to_i64(Workspace& w, const int* in, long long* out, long long n, cudaStream_t st);
 // same, int32 in place (values and total < 2^31)
 int scan_i32_inplace(Workspace& w, int* data, long long n, cudaStream_t st);
 // Stream-ordered clear and word copy done by kernels on the SMs, never by a copy engine: inside a

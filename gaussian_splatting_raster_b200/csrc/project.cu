@@ -30,8 +30,8 @@ __global__ void __launch_bounds__(kProjThreads)
 k_project(const float* __restrict__ means, const float* __restrict__ lsc,
           const float* __restrict__ quats, const float* __restrict__ opac,
           const float* __restrict__ sh, const float* __restrict__ views_in, int G, int V, int H,
-          int W, int TX, int TY, float4* __restrict__ rec, int4* __restrict__ rect,
-          int* __restrict__ counts, uint32_t* __restrict__ dkey, uint32_t* __restrict__ kbits,
+          int W, int TX, int TY, float4* __restrict__ rec, ushort4* __restrict__ rect,
+          uint32_t* __restrict__ dkey, uint32_t* __restrict__ kbits,
           unsigned long long* __restrict__ ntot) {
   constexpr int D = (DEG + 1) * (DEG + 1);
   constexpr int NSH = D * 3;
@@ -132,7 +132,7 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
     const size_t i = (size_t)v * G + g;
     const float* vw = s_views + 20 * v;
     float4 r0 = make_float4(0, 0, 0, 0), r1 = r0, r2 = r0, r3 = r0;
-    int4 rc = make_int4(0, 0, 0, 0);
+    ushort4 rc = make_ushort4(0, 0, 0, 0);
     int cnt = 0;
     bool vis = ok;
     float Rv[3][3], t[3];
@@ -230,7 +230,8 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
         r1 = make_float4(col[2], cut, ex, ey);
         r2 = make_float4(qa, qb, qc, o);
         r3 = make_float4(z, x, y, __int_as_float(flags));
-        rc = make_int4(x0, y0, x1, y1);
+        rc = make_ushort4((unsigned short)x0, (unsigned short)y0, (unsigned short)x1,
+                          (unsigned short)y1);
         cnt = (x1 - x0) * (y1 - y0);
       }
     }
@@ -241,7 +242,6 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
     rh[0] = r2;
     rh[1] = r3;
     rect[i] = rc;
-    counts[i] = cnt;
     // depth sort key (fp32 bits of z > 0 order like the values; culled entries sort last) and,
     // per view, the largest visible key and the largest complement of one (the complement of the
     // smallest visible key): the sort orders key - smallest, over the bits of the key range
@@ -286,7 +286,7 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
       return set_err(w, SPLAT_ERR_CAPACITY, "too many views for the projection kernel");        \
     k_project<DEG><<<blocks, kProjThreads, smem, st>>>(means, lsc, quats, opac, sh, w.views,     \
                                                        w.G, w.V, w.H, w.W, w.TX, w.TY, w.rec,    \
-                                                       w.rect, w.counts, w.dkey, w.kbits,        \
+                                                       w.rect, w.dkey, w.kbits,                  \
                                                        w.ntot);                                  \
   }
   switch (w.deg) {
@@ -314,12 +314,29 @@ __global__ void k_copy_records(const float4* __restrict__ rec, float4* __restric
   }
 }
 
+// the tile rectangles widened to the documented int32 [V, G, 4]
+__global__ void k_copy_rects(const ushort4* __restrict__ rect, int4* __restrict__ out, long long n) {
+  for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < n;
+       k += (long long)gridDim.x * blockDim.x) {
+    const ushort4 r = rect[k];
+    out[k] = make_int4(r.x, r.y, r.z, r.w);
+  }
+}
+
 int launch_copy_records(Workspace& w, float* out, cudaStream_t st) {
   const long long n = (long long)w.V * w.G;
   if (n == 0) return SPLAT_OK;
   k_copy_records<<<(unsigned)std::min<long long>((n + 255) / 256, 8 * 148), 256, 0, st>>>(
       w.rec, reinterpret_cast<float4*>(out), n);
   return check_launch(w, "record copy kernel");
+}
+
+int launch_copy_rects(Workspace& w, int* out, cudaStream_t st) {
+  const long long n = (long long)w.V * w.G;
+  if (n == 0) return SPLAT_OK;
+  k_copy_rects<<<(unsigned)std::min<long long>((n + 255) / 256, 8 * 148), 256, 0, st>>>(
+      w.rect, reinterpret_cast<int4*>(out), n);
+  return check_launch(w, "rectangle copy kernel");
 }
 
 }  // namespace splat

@@ -61,7 +61,9 @@ typedef enum splat_status {
  * Create a workspace on the current device for problems with at most max_G Gaussians, max_V
  * views of at most max_H x max_W pixels and SH degree <= max_sh_degree (0..3). Allocates the
  * per-(Gaussian, view) records and accumulators up front; the instance (tile, Gaussian) lists
- * grow on demand inside splat_bin_sort. *ws is set to NULL on failure.
+ * grow on demand inside splat_bin_sort. *ws is set to NULL on failure. SPLAT_ERR_CAPACITY when
+ * an image has more 16x16 tiles, ceil(max_W/16) ceil(max_H/16), than the binning kernels' shared
+ * memory holds per-warp counts for (7,264 tiles).
  */
 int splat_ws_create(splat_ws** ws, int max_G, int max_V, int max_H, int max_W,
                     int max_sh_degree);

@@ -242,6 +242,18 @@ def test_calls_out_of_order_and_bad_arguments():
     ws.close()
 
 
+def test_most_tiles_a_workspace_holds():
+    """An image of 7,264 16x16 tiles (the largest the binning's per-warp shared-memory counts
+    hold) renders and scores like the oracle; one tile more is refused at workspace creation."""
+    from gaussian_splatting_raster_b200 import SplatError, Workspace
+    with pytest.raises(SplatError) as e:
+        Workspace(16, 1, 16, 16 * 7265, 1)
+    assert e.value.code == -2
+    sc = scenes.tiny_scene(61, 300, 16, 16 * 7264, V=1, deg=1)
+    obs = np.random.default_rng(61).uniform(0, 1, (1, 16, 16 * 7264, 3)).astype(np.float32)
+    _full_check(sc, obs)
+
+
 @pytest.mark.parametrize("cfg", [3, 4, 5])
 def test_full_size_sampled(cfg):
     """Full-size workloads: projection and every tile list compared in full; render on sampled
