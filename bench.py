@@ -79,6 +79,9 @@ def parse():
     ap.add_argument("--views", type=int, default=0,
                     help="view-count scaling: the ReSplat-scale layout with this many context and "
                          "target views at 256x448 (overrides --config)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="score path: splat_render then splat_score_replay (two kernels) instead "
+                         "of splat_render_score (one kernel)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-threads", type=int, default=0,
@@ -229,6 +232,9 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
         "tile_scatter": n_inst * (4 + 4 + 4),
         # gather 36 B per list entry staged, write C_hat, T, n, last
         "render": n_inst * (4 + 36) + px * 24,
+        # render and replay in one kernel: the list entries gathered by both phases, C_hat, T,
+        # n, last written, C_obs read, 32 B of sums per (v, g)
+        "render_replay": n_inst * 2 * (4 + 36) + px * (24 + 12) + V * G * 32,
         # gather 36 B per list entry, read C_hat, C_obs, the list bound and the contributor
         # count per pixel, add into 32 B of sums per (v, g)
         "replay": n_inst * (4 + 36) + px * (12 + 12 + 4 + 4) + V * G * 32,
@@ -267,8 +273,10 @@ def algorithmic_bytes(sc, n_inst: int, pairs: int, depth_passes: int = 3) -> dic
 #             (T, w, w, w |r|)                                                             = 12 + 5
 # so a kernel's work per step = a x traversed pairs + b x composited pairs with (a, b) below.
 ALU_OPS = {"render": (13, 25), "replay": (0, 46), "backward": (0, 43), "features": (0, 36),
-           "scatter": (26, 47)}  # the backward visits its warps' union entries but, like the
-# replay, is handed the render's decisions: its work is counted over the composited pairs
+           "scatter": (26, 47), "render_replay": (13, 25 + 46)}
+# the backward visits its warps' union entries but, like the replay, is handed the render's
+# decisions: its work is counted over the composited pairs; render_replay is the render and the
+# replay in one kernel (splat_render_score)
 
 def alu_ops(kernel: str, pairs: int, composited: int) -> int:
     a, b = ALU_OPS[kernel]
@@ -495,7 +503,7 @@ def main():
             ws.scatter(pmap, attr_["S"])
             ws.attribution(obs_, attr_["A"])
             return n
-        return runner.render_and_score(ws, ds_, obs_, out_)
+        return runner.render_and_score(ws, ds_, obs_, out_, fused=not args.unfused)
 
     last_out = {}
 
@@ -546,6 +554,19 @@ def main():
             "torch_reserved_gb": torch.cuda.memory_reserved(dev) / 1e9,
             "device_total_gb": total_b / 1e9}
     kern = ws.profile_read(reset=True)
+    # The fused score path runs the render and the replay as one kernel, so the render's own
+    # time -- the denominator of the replay's cost -- is taken from separate render-only steps
+    # (projection, binning, render; same L2 flush), outside the timed region.
+    fused = args.path == "score" and not args.unfused and not shard and "render_replay" in kern
+    render_alone_ms = None
+    if fused:
+        for _ in range(args.steps):
+            l2_flush.zero_()
+            runner.render(ws, ds, out)
+        torch.cuda.synchronize()
+        render_alone_ms = ws.profile_read(reset=True)["render"][0] / args.steps
+        runner.render_and_score(ws, ds, obs, out)  # leave the workspace as the timed steps did
+        torch.cuda.synchronize()
     ws.profile(False)
 
     total_ms = max_over_ranks(sum(step_ms), world)
@@ -675,6 +696,12 @@ def main():
     second = {"backward": ("backward", "grad"), "attributes": ("features", "scatter"),
               "score": ("replay", "finalize")}[args.path]
     replay_ms = sum(per_kernel.get(k, {}).get("ms_per_step", 0.0) for k in second)
+    if fused:
+        # render side: the render kernel timed alone; replay side: what the fused kernel takes
+        # beyond it, plus the finalisation
+        per_kernel["render_replay"]["render_alone_ms"] = render_alone_ms
+        render_ms += render_alone_ms
+        replay_ms += per_kernel["render_replay"]["ms_per_step"] - render_alone_ms
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -691,7 +718,9 @@ def main():
                        "height": sc.H, "width": sc.W, "sh_degree": sc.sh_degree,
                        "path": PATHS[args.path],
                        "accumulation": "fixed-point (deterministic)" if args.deterministic
-                       else "fp64 atomics",
+                       else "fp32 vector reductions",
+                       "calls": ("splat_render_score (render and replay in one kernel)" if fused
+                                 else "separate calls"),
                        "instances_per_step": n_total, "pairs_per_step": pairs,
                        "composited_pairs_per_step": composited,
                        "l2": "256 MiB buffer written between timed steps",

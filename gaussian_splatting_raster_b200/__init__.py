@@ -23,7 +23,8 @@ _ERRORS = {
 # every symbol include/splat.h declares (checked against the header by the tests)
 EXPORTS = [
     "splat_ws_create", "splat_ws_destroy", "splat_last_error", "splat_project",
-    "splat_bin_sort", "splat_render", "splat_score_replay", "splat_copy_projection",
+    "splat_bin_sort", "splat_render", "splat_score_replay", "splat_render_score",
+    "splat_copy_projection",
     "splat_copy_tile_lists", "splat_copy_last", "splat_copy_accumulators", "splat_pair_count",
     "splat_launch_count", "splat_profile_enable", "splat_profile_read", "splat_kernel_name",
     "splat_sort_depths_noalloc", "splat_score_partials", "splat_finalize_partials",
@@ -32,7 +33,7 @@ EXPORTS = [
 ]
 
 
-KERNEL_GROUPS = 16  # SPLAT_NUM_KERNELS
+KERNEL_GROUPS = 17  # SPLAT_NUM_KERNELS
 
 
 class SplatError(RuntimeError):
@@ -68,6 +69,8 @@ def load_library(path: str | None = None):
     L.splat_render.restype = I
     L.splat_score_replay.argtypes = [V, V, F, V, V]
     L.splat_score_replay.restype = I
+    L.splat_render_score.argtypes = [V, V, V, F, V, V, V, V, V]
+    L.splat_render_score.restype = I
     L.splat_copy_projection.argtypes = [V, V, V, V]
     L.splat_copy_projection.restype = I
     L.splat_copy_tile_lists.argtypes = [V, V, V, V]
@@ -225,6 +228,20 @@ class Workspace:
         V, H, W = self.V, self.H, self.W
         self._check(self._L.splat_score_replay(
             self._h, _ptr(obs, "obs", torch.float32, (V, H, W, 3)), ctypes.c_float(lam),
+            _ptr(tokens, "tokens", torch.float32, (self.G, token_dim(self.deg))),
+            _stream(stream)))
+
+    def render_score(self, bg, obs, img, T_final, n_contrib, tokens, lam: float = 1.0,
+                     stream=None):
+        """render followed by score_replay in one call (one fused kernel in the default mode)."""
+        import torch
+        V, H, W = self.V, self.H, self.W
+        self._check(self._L.splat_render_score(
+            self._h, _ptr(bg, "bg", torch.float32, (3,)),
+            _ptr(obs, "obs", torch.float32, (V, H, W, 3)), ctypes.c_float(lam),
+            _ptr(img, "img", torch.float32, (V, H, W, 3)),
+            _ptr(T_final, "T_final", torch.float32, (V, H, W)),
+            _ptr(n_contrib, "n_contrib", torch.int32, (V, H, W)),
             _ptr(tokens, "tokens", torch.float32, (self.G, token_dim(self.deg))),
             _stream(stream)))
 

@@ -100,7 +100,7 @@ void free_all(Workspace& w) {
 const char* const kKernelNames[SPLAT_NUM_KERNELS] = {
     "project", "depth_hist", "depth_scatter", "emit", "tile_hist", "hist_scan",
     "tile_scatter", "tile_ranges", "render", "replay", "finalize", "backward", "grad", "features", "scatter",
-    "other"};
+    "render_replay", "other"};
 
 // fold every recorded (start, end) pair into the per-kernel sums
 int fold_events(Workspace& w) {
@@ -299,6 +299,37 @@ int splat_score_replay(splat_ws* ws, const float* obs, float lambda, float* toke
   if ((rc = check_dev_ptr(w, tokens, "tokens", w.G == 0))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   if ((rc = splat::launch_replay(w, obs, st))) return rc;
+  if ((rc = splat::launch_finalize(w, lambda, tokens, st))) return rc;
+  w.stage = 4;
+  return SPLAT_OK;
+}
+
+int splat_render_score(splat_ws* ws, const float* bg, const float* obs, float lambda, float* img,
+                       float* T_final, int* n_contrib, float* tokens, void* stream) {
+  if (!ws) return SPLAT_ERR_INVALID_ARG;
+  Workspace& w = ws->w;
+  w.err.clear();
+  if (w.stage < 2) return fail(w, SPLAT_ERR_STATE, "splat_render_score before splat_bin_sort");
+  if (!(lambda >= 0.0f) || !std::isfinite(lambda))
+    return fail(w, SPLAT_ERR_INVALID_ARG, "lambda must be finite and >= 0");
+  int rc;
+  if ((rc = check_dev_ptr(w, bg, "bg"))) return rc;
+  if ((rc = check_dev_ptr(w, obs, "obs"))) return rc;
+  if ((rc = check_dev_ptr(w, img, "img"))) return rc;
+  if ((rc = check_dev_ptr(w, T_final, "T_final"))) return rc;
+  if ((rc = check_dev_ptr(w, n_contrib, "n_contrib"))) return rc;
+  if ((rc = check_dev_ptr(w, tokens, "tokens", w.G == 0))) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  w.img = img;
+  w.Tfin = T_final;
+  w.ncon = n_contrib;
+  w.bg = bg;
+  if (w.det) {
+    if ((rc = splat::launch_render(w, bg, img, T_final, n_contrib, st))) return rc;
+    if ((rc = splat::launch_replay(w, obs, st))) return rc;
+  } else if ((rc = splat::launch_render_replay(w, bg, obs, img, T_final, n_contrib, st))) {
+    return rc;
+  }
   if ((rc = splat::launch_finalize(w, lambda, tokens, st))) return rc;
   w.stage = 4;
   return SPLAT_OK;

@@ -314,6 +314,8 @@ int launch_binning(Workspace& w, cudaStream_t st);
 int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int* n_contrib,
                   cudaStream_t st);
 int launch_replay(Workspace& w, const float* obs, cudaStream_t st);
+int launch_render_replay(Workspace& w, const float* bg, const float* obs, float* img,
+                         float* T_final, int* n_contrib, cudaStream_t st);
 int launch_finalize(Workspace& w, float lambda, float* tokens, cudaStream_t st);
 int launch_partials(Workspace& w, float* partials, cudaStream_t st);
 cudaError_t launch_finalize_partials(const float* partials, int G, int deg, double lambda,

@@ -49,106 +49,6 @@ SPLAT_BOUNDS_WORD(bounds_word_raster)
 
 namespace {
 
-__global__ void __launch_bounds__(kThreads)
-k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-         const long long* __restrict__ tile_off, const int* __restrict__ order,
-         int G, int H, int W, int TX, int nt,
-         const float* __restrict__ bgp, float* __restrict__ img, float* __restrict__ Tout,
-         int* __restrict__ ncout, int* __restrict__ last, uint32_t* __restrict__ umask,
-         uint32_t* __restrict__ lmask) {
-  int t, v;
-  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
-  const int tx = t % TX, ty = t / TX;
-  int i, j, bx, by;
-  tile_pixel(tx, ty, i, j, bx, by);
-  const bool inside = i < W && j < H;
-  const long long s = tile_off[(size_t)v * (nt + 1) + t];
-  const long long e = tile_off[(size_t)v * (nt + 1) + t + 1];
-  const int gt = v * nt + t;
-  // Each warp walks the whole list on its own (no CTA barriers): it stages 32 entries into its
-  // slice of shared memory, ballots which of them can reach its pixel block, evaluates only
-  // those, and leaves as soon as its 32 pixels are done. Per 32-entry chunk it records which
-  // entries some pixel of the warp composited: the replay visits exactly those.
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
-  const int twarp = tile_warp();                                 // block in the tile
-  __shared__ float4 s_a[kThreads], s_b[kThreads];
-  __shared__ float2 s_c[kThreads];  // (colour b, exponent cut)
-  float4* wa = s_a + warp * 32;
-  float4* wb = s_b + warp * 32;
-  float2* wc = s_c + warp * 32;
-  // this pixel's composited-entry mask words (read by the score replay): chunk cc at
-  // lmw[1024 (cc / 4) + cc % 4]
-  uint32_t* lmw = lmask + lmask_region(s, gt) + 4 * (twarp * 32 + lane);
-  int cc = 0;  // chunks walked
-  const float x0f = (float)bx, y0f = (float)by;
-  const float px = (float)i + 0.5f, py = (float)j + 0.5f;
-  float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
-  int n = 0, lst = 0;
-  bool done = !inside;
-  const size_t vG = (size_t)v * G;
-  for (long long base = s; base < e; base += 32, ++cc) {
-    if (__all_sync(0xffffffffu, done)) break;
-    const long long k = base + lane;
-    bool hit = false;
-    if (k < e) {
-      const uint32_t gi = ids[k];
-      if (in_bounds(gi, (unsigned)G, &g_bounds_word)) {
-        const float4* rl = rec + rec_lo(vG + gi);  // r0, r1
-        const float4* rh = rec + rec_hi(vG + gi);  // r2, r3
-        const float4 r0 = rl[0], r1 = rl[1], r2 = rh[0];  // r1 = (colour b, cut, ex, ey)
-        wa[lane] = r0;
-        wb[lane] = r2;
-        wc[lane] = make_float2(r1.x, r1.y);
-        hit = reaches_block(r0, r1.z, r1.w, x0f, y0f);
-      }
-    }
-    uint32_t bits = __ballot_sync(0xffffffffu, hit);
-    uint32_t lbits = 0u;  // entries of this chunk this lane composited
-    __syncwarp();
-    while (bits) {  // warp-uniform: entries that can reach this warp's rows, in list order
-      const int q = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (!done) {
-        float4 A, Bq;
-        entry_operands(wa[q], wb[q], A, Bq);
-        const float2 Cq = wc[q];
-        const Entry E = eval_entry(A, Bq, Cq.y, px, py);
-        if (E.use) {
-          const float Tn = T * (1.0f - E.alpha);
-          if (Tn < 1e-4f) {
-            done = true;
-          } else {
-            const float wgt = E.alpha * T;
-            // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is
-            // then exactly the background term, and the suffix recovery sees no rounding mismatch
-            const float2 wc01 = __fmul2_rn(make_float2(wgt, wgt), make_float2(Bq.z, Bq.w));
-            C0 = C0 + wc01.x;
-            C1 = C1 + wc01.y;
-            C2 = C2 + wgt * Cq.x;
-            T = Tn;
-            ++n;
-            lst = (int)(base - s) + q + 1;
-            lbits |= 1u << q;
-          }
-        }
-      }
-    }
-    const uint32_t ubits = __reduce_or_sync(0xffffffffu, lbits);
-    if (lane == 0) umask[chunk_index(base, gt) * 8 + twarp] = ubits;
-    lmw[(size_t)(cc >> 2) * 1024 + (cc & 3)] = lbits;
-    __syncwarp();
-  }
-  if (inside) {
-    const size_t p = ((size_t)v * H + j) * W + i;
-    img[3 * p + 0] = C0 + T * bgp[0];
-    img[3 * p + 1] = C1 + T * bgp[1];
-    img[3 * p + 2] = C2 + T * bgp[2];
-    Tout[p] = T;
-    ncout[p] = n;
-    last[p] = lst;
-  }
-}
-
 // Deterministic accumulation: each warp's partial sum x (fp32) is turned into the signed 128-bit
 // fixed-point integer X = x 2^60 (exact for |x| >= 2^-37; smaller values are truncated toward
 // zero, the same way every run) and added with two 64-bit integer atomics -- the low word, then
@@ -415,66 +315,24 @@ __device__ __forceinline__ bool replay_pair(PixelState& ps, const Entry& E, floa
   return ma;
 }
 
-__global__ void __launch_bounds__(kThreads, 4)
-k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
-         const long long* __restrict__ tile_off, const int* __restrict__ order,
-         int G, int H, int W, int TX, int nt, const float* __restrict__ img,
-         const float* __restrict__ obs, const int* __restrict__ last,
-         const int* __restrict__ ncon, const uint32_t* __restrict__ umask,
-         const uint32_t* __restrict__ lmask, float* __restrict__ acc) {
-  int t, v;
-  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;  // CTA-uniform
-  const int tx = t % TX, ty = t / TX;
-  int i, j, bx, by;
-  tile_pixel(tx, ty, i, j, bx, by);
-  const bool inside = i < W && j < H;
-  const long long s = tile_off[(size_t)v * (nt + 1) + t];
-  const int gt = v * nt + t;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// The replay of one warp block, given its pixel's state (C_hat, r = C_hat - C_obs, T = 1, P = 0),
+// list bound lst and the warp's union entries U and composited pairs P. kFresh: the composited-
+// entry masks were stored by this same launch (read through the coherent path, not the
+// read-only one).
+template <bool kFresh>
+__device__ __forceinline__ void replay_walk(const float4* __restrict__ rec,
+                                            const uint32_t* __restrict__ ids, long long s, int gt,
+                                            int G, size_t vG, float px, float py, PixelState ps,
+                                            int lst, int U, int P, const uint32_t* umask,
+                                            const uint32_t* lmask, float* __restrict__ accv,
+                                            float4* wa, float4* wb, float2* wc, uint32_t* wg) {
+  const int lane = threadIdx.x & 31;
   const int twarp = tile_warp();
-  PixelState ps;
-  ps.T = 1.0f;
-  ps.P01 = make_float2(0.0f, 0.0f);
-  ps.P2 = 0.0f;
-  float Ch0 = 0.0f, Ch1 = 0.0f, r0 = 0.0f, r1 = 0.0f;
-  ps.Ch2 = 0.0f;
-  ps.r2 = 0.0f;
-  int lst = 0, nc = 0;
-  if (inside) {
-    const size_t p = ((size_t)v * H + j) * W + i;
-    Ch0 = img[3 * p];
-    Ch1 = img[3 * p + 1];
-    ps.Ch2 = img[3 * p + 2];
-    r0 = Ch0 - obs[3 * p];
-    r1 = Ch1 - obs[3 * p + 1];
-    ps.r2 = ps.Ch2 - obs[3 * p + 2];
-    lst = last[p];
-    nc = ncon[p];
-  }
-  ps.Ch01 = make_float2(Ch0, Ch1);
-  ps.r01 = make_float2(r0, r1);
-  const float px = (float)i + 0.5f, py = (float)j + 0.5f;
-  const size_t vG = (size_t)v * G;
-  float* accv = acc + (size_t)v * G * kAccN;
-
-  // the warp's union entries U and composited pairs P
-  const int wmax = __reduce_max_sync(0xffffffffu, lst);
-  const int wch = (wmax + 31) >> 5;
-  int u = 0;
-  for (int c = lane; c < wch; c += 32) u += __popc(umask[chunk_index(s + 32LL * c, gt) * 8 + twarp]);
-  const int U = __reduce_add_sync(0xffffffffu, u);
-  const int P = __reduce_add_sync(0xffffffffu, nc);
   if (U == 0) return;  // warp-uniform: nothing composited here
+  const int wmax = __reduce_max_sync(0xffffffffu, lst);
 
   if (P >= kUnionLanes * U) {
     // ---- union loop ----------------------------------------------------------------------
-    __shared__ float4 s_a[kThreads], s_b[kThreads];
-    __shared__ float2 s_c[kThreads];
-    __shared__ uint32_t s_g[kThreads];
-    float4* wa = s_a + warp * 32;
-    float4* wb = s_b + warp * 32;
-    float2* wc = s_c + warp * 32;
-    uint32_t* wg = s_g + warp * 32;
     const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
     for (int base = 0; base < wmax; base += 32) {
       uint32_t bits = umask[chunk_index(s + base, gt) * 8 + twarp];
@@ -502,7 +360,7 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         bool used = false;
         if (base + q < lst) {
           float4 A, Bq;
-        entry_operands(wa[q], wb[q], A, Bq);
+          entry_operands(wa[q], wb[q], A, Bq);
           const float2 Cq = wc[q];
           const Entry E = eval_entry(A, Bq, Cq.y, px, py);
           if (E.use) {
@@ -537,10 +395,10 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
   // this pixel's mask words: chunk c's in m, the rest of its group of four in n1..n3, the next
   // group prefetched in pre
   const uint4* lm = reinterpret_cast<const uint4*>(lmask + lmask_region(s, gt)) + (twarp * 32 + lane);
-  const uint4 g0 = __ldg(lm);
+  const uint4 g0 = kFresh ? lm[0] : __ldg(lm);
   uint32_t m = g0.x, n1 = g0.y, n2 = g0.z, n3 = g0.w;
   uint4 pre = make_uint4(0u, 0u, 0u, 0u);
-  if (4 < cend) pre = __ldg(lm + 256);
+  if (4 < cend) pre = kFresh ? lm[256] : __ldg(lm + 256);
   int c = 0;
   for (;;) {
     while (!m) {  // next chunk with an entry of this pixel
@@ -550,7 +408,10 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
         n1 = pre.y;
         n2 = pre.z;
         n3 = pre.w;
-        if (c + 4 < cend) pre = __ldg(lm + (size_t)((c >> 2) + 1) * 256);
+        if (c + 4 < cend) {
+          const uint4* nx = lm + (size_t)((c >> 2) + 1) * 256;
+          pre = kFresh ? nx[0] : __ldg(nx);
+        }
       } else {
         m = n1;
         n1 = n2;
@@ -576,6 +437,198 @@ k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
     if (ma) red_add4(a + 4, x[4], x[5], x[6], 0.0f);
   }
 }
+
+// pixel state of the replay from the rendered colour and the observation
+__device__ __forceinline__ PixelState replay_state(float Ch0, float Ch1, float Ch2, float o0,
+                                                   float o1, float o2) {
+  PixelState ps;
+  ps.T = 1.0f;
+  ps.P01 = make_float2(0.0f, 0.0f);
+  ps.P2 = 0.0f;
+  ps.Ch01 = make_float2(Ch0, Ch1);
+  ps.Ch2 = Ch2;
+  ps.r01 = make_float2(Ch0 - o0, Ch1 - o1);
+  ps.r2 = Ch2 - o2;
+  return ps;
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
+k_replay(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
+         const long long* __restrict__ tile_off, const int* __restrict__ order,
+         int G, int H, int W, int TX, int nt, const float* __restrict__ img,
+         const float* __restrict__ obs, const int* __restrict__ last,
+         const int* __restrict__ ncon, const uint32_t* __restrict__ umask,
+         const uint32_t* __restrict__ lmask, float* __restrict__ acc) {
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;  // CTA-uniform
+  const int tx = t % TX, ty = t / TX;
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
+  const bool inside = i < W && j < H;
+  const long long s = tile_off[(size_t)v * (nt + 1) + t];
+  const int gt = v * nt + t;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int twarp = tile_warp();
+  float Ch0 = 0.0f, Ch1 = 0.0f, Ch2 = 0.0f, o0 = 0.0f, o1 = 0.0f, o2 = 0.0f;
+  int lst = 0, nc = 0;
+  if (inside) {
+    const size_t p = ((size_t)v * H + j) * W + i;
+    Ch0 = img[3 * p];
+    Ch1 = img[3 * p + 1];
+    Ch2 = img[3 * p + 2];
+    o0 = obs[3 * p];
+    o1 = obs[3 * p + 1];
+    o2 = obs[3 * p + 2];
+    lst = last[p];
+    nc = ncon[p];
+  }
+  // the warp's union entries U (the render's per-warp masks) and composited pairs P
+  const int wmax = __reduce_max_sync(0xffffffffu, lst);
+  const int wch = (wmax + 31) >> 5;
+  int u = 0;
+  for (int c = lane; c < wch; c += 32) u += __popc(umask[chunk_index(s + 32LL * c, gt) * 8 + twarp]);
+  const int U = __reduce_add_sync(0xffffffffu, u);
+  const int P = __reduce_add_sync(0xffffffffu, nc);
+  __shared__ float4 s_a[kThreads], s_b[kThreads];
+  __shared__ float2 s_c[kThreads];
+  __shared__ uint32_t s_g[kThreads];
+  replay_walk<false>(rec, ids, s, gt, G, (size_t)v * G, (float)i + 0.5f, (float)j + 0.5f,
+                     replay_state(Ch0, Ch1, Ch2, o0, o1, o2), lst, U, P, umask, lmask,
+                     acc + (size_t)v * G * kAccN, s_a + warp * 32, s_b + warp * 32,
+                     s_c + warp * 32, s_g + warp * 32);
+}
+
+// The render (kReplay = false), or render and score replay in one launch (kReplay): each warp
+// renders its block, stores the render's outputs and masks, and replays its composited entries
+// at once with the pixel state still in registers. Across an SM the warps are in different
+// phases, so the render's issue-bound work and the replay's L2 reductions overlap instead of
+// following one another. The arithmetic and the decisions are those of the separate passes.
+template <bool kReplay>
+__global__ void __launch_bounds__(kThreads)
+k_render(const float4* __restrict__ rec, const uint32_t* __restrict__ ids,
+         const long long* __restrict__ tile_off, const int* __restrict__ order,
+         int G, int H, int W, int TX, int nt,
+         const float* __restrict__ bgp, float* __restrict__ img, float* __restrict__ Tout,
+         int* __restrict__ ncout, int* __restrict__ last, uint32_t* __restrict__ umask,
+         uint32_t* __restrict__ lmask, const float* __restrict__ obs, float* __restrict__ acc) {
+  int t, v;
+  if (!block_tile(order, nt, &g_bounds_word, t, v)) return;
+  const int tx = t % TX, ty = t / TX;
+  int i, j, bx, by;
+  tile_pixel(tx, ty, i, j, bx, by);
+  const bool inside = i < W && j < H;
+  const long long s = tile_off[(size_t)v * (nt + 1) + t];
+  const long long e = tile_off[(size_t)v * (nt + 1) + t + 1];
+  const int gt = v * nt + t;
+  // Each warp walks the whole list on its own (no CTA barriers): it stages 32 entries into its
+  // slice of shared memory, ballots which of them can reach its pixel block, evaluates only
+  // those, and leaves as soon as its 32 pixels are done. Per 32-entry chunk it records which
+  // entries some pixel of the warp composited: the replay visits exactly those.
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp in the CTA
+  const int twarp = tile_warp();                                 // block in the tile
+  __shared__ float4 s_a[kThreads], s_b[kThreads];
+  __shared__ float2 s_c[kThreads];  // (colour b, exponent cut)
+  float4* wa = s_a + warp * 32;
+  float4* wb = s_b + warp * 32;
+  float2* wc = s_c + warp * 32;
+  // this pixel's composited-entry mask words (read by the score replay): chunk cc at
+  // lmw[1024 (cc / 4) + cc % 4]
+  uint32_t* lmw = lmask + lmask_region(s, gt) + 4 * (twarp * 32 + lane);
+  int cc = 0;  // chunks walked
+  const float x0f = (float)bx, y0f = (float)by;
+  const float px = (float)i + 0.5f, py = (float)j + 0.5f;
+  float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
+  int n = 0, lst = 0;
+  int U = 0;  // (kReplay) entries some pixel of the warp composited
+  bool done = !inside;
+  const size_t vG = (size_t)v * G;
+  for (long long base = s; base < e; base += 32, ++cc) {
+    if (__all_sync(0xffffffffu, done)) break;
+    const long long k = base + lane;
+    bool hit = false;
+    if (k < e) {
+      const uint32_t gi = ids[k];
+      if (in_bounds(gi, (unsigned)G, &g_bounds_word)) {
+        const float4* rl = rec + rec_lo(vG + gi);  // r0, r1
+        const float4* rh = rec + rec_hi(vG + gi);  // r2, r3
+        const float4 r0 = rl[0], r1 = rl[1], r2 = rh[0];  // r1 = (colour b, cut, ex, ey)
+        wa[lane] = r0;
+        wb[lane] = r2;
+        wc[lane] = make_float2(r1.x, r1.y);
+        hit = reaches_block(r0, r1.z, r1.w, x0f, y0f);
+      }
+    }
+    uint32_t bits = __ballot_sync(0xffffffffu, hit);
+    uint32_t lbits = 0u;  // entries of this chunk this lane composited
+    __syncwarp();
+    while (bits) {  // warp-uniform: entries that can reach this warp's rows, in list order
+      const int q = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (!done) {
+        float4 A, Bq;
+        entry_operands(wa[q], wb[q], A, Bq);
+        const float2 Cq = wc[q];
+        const Entry E = eval_entry(A, Bq, Cq.y, px, py);
+        if (E.use) {
+          const float Tn = T * (1.0f - E.alpha);
+          if (Tn < 1e-4f) {
+            done = true;
+          } else {
+            const float wgt = E.alpha * T;
+            // unfused, as the replay accumulates its prefix P: at the last entry C_hat - P is
+            // then exactly the background term, and the suffix recovery sees no rounding mismatch
+            const float2 wc01 = __fmul2_rn(make_float2(wgt, wgt), make_float2(Bq.z, Bq.w));
+            C0 = C0 + wc01.x;
+            C1 = C1 + wc01.y;
+            C2 = C2 + wgt * Cq.x;
+            T = Tn;
+            ++n;
+            lst = (int)(base - s) + q + 1;
+            lbits |= 1u << q;
+          }
+        }
+      }
+    }
+    const uint32_t ubits = __reduce_or_sync(0xffffffffu, lbits);
+    if (kReplay) U += __popc(ubits);
+    if (lane == 0) umask[chunk_index(base, gt) * 8 + twarp] = ubits;
+    lmw[(size_t)(cc >> 2) * 1024 + (cc & 3)] = lbits;
+    __syncwarp();
+  }
+  if constexpr (!kReplay) {
+    if (inside) {
+      const size_t p = ((size_t)v * H + j) * W + i;
+      img[3 * p + 0] = C0 + T * bgp[0];
+      img[3 * p + 1] = C1 + T * bgp[1];
+      img[3 * p + 2] = C2 + T * bgp[2];
+      Tout[p] = T;
+      ncout[p] = n;
+      last[p] = lst;
+    }
+  } else {
+    float Ch0 = 0.0f, Ch1 = 0.0f, Ch2 = 0.0f, o0 = 0.0f, o1 = 0.0f, o2 = 0.0f;
+    if (inside) {
+      const size_t p = ((size_t)v * H + j) * W + i;
+      Ch0 = C0 + T * bgp[0];
+      Ch1 = C1 + T * bgp[1];
+      Ch2 = C2 + T * bgp[2];
+      img[3 * p + 0] = Ch0;
+      img[3 * p + 1] = Ch1;
+      img[3 * p + 2] = Ch2;
+      Tout[p] = T;
+      ncout[p] = n;
+      last[p] = lst;
+      o0 = obs[3 * p];
+      o1 = obs[3 * p + 1];
+      o2 = obs[3 * p + 2];
+    }
+    const int P = __reduce_add_sync(0xffffffffu, n);
+    __shared__ uint32_t s_g[kThreads];
+    replay_walk<true>(rec, ids, s, gt, G, vG, px, py, replay_state(Ch0, Ch1, Ch2, o0, o1, o2),
+                      lst, U, P, umask, lmask, acc + vG * kAccN, wa, wb, wc, s_g + warp * 32);
+  }
+}
+
 
 // Renderer backward of L = 1/2 sum |C_hat - C_obs|^2 with the render's decisions held fixed.
 // Each warp walks its composited entries BACK TO FRONT (chunks from the last one down, entries in
@@ -728,9 +781,9 @@ int launch_render(Workspace& w, const float* bg, float* img, float* T_final, int
                   cudaStream_t st) {
   dim3 grid(w.nt * kCtaPerTile, w.V);
   const int tok = prof_begin(w, st, SPLAT_K_RENDER);
-  k_render<<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H, w.W, w.TX,
-                                      w.nt, bg, img, T_final, n_contrib, w.last, w.umask,
-                                      w.lmask);
+  k_render<false><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H,
+                                             w.W, w.TX, w.nt, bg, img, T_final, n_contrib, w.last,
+                                             w.umask, w.lmask, nullptr, nullptr);
   prof_end(w, st, tok);
   return check_launch(w, "render kernel");
 }
@@ -788,6 +841,26 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
   if (!rc && det) rc = fix_to<float>(w, w.acc_fix, w.acc, kAccN, st);
   prof_end(w, st, tok);
   return rc;
+}
+
+// render and replay in one launch (default accumulation mode only; the deterministic mode runs
+// launch_render and launch_replay)
+int launch_render_replay(Workspace& w, const float* bg, const float* obs, float* img,
+                         float* T_final, int* n_contrib, cudaStream_t st) {
+  const int tok = prof_begin(w, st, SPLAT_K_RENDER_REPLAY);
+  int rc = SPLAT_OK;
+  if (w.G > 0)
+    rc = zero_async(w, w.acc, (size_t)w.V * w.G * kAccN * sizeof(float), st, "accumulator clear");
+  if (rc) {
+    prof_end(w, st, tok);
+    return rc;
+  }
+  dim3 grid(w.nt * kCtaPerTile, w.V);
+  k_render<true><<<grid, kThreads, 0, st>>>(w.rec, w.sval, w.tile_off, w.tile_order, w.G, w.H,
+                                            w.W, w.TX, w.nt, bg, img, T_final, n_contrib, w.last,
+                                            w.umask, w.lmask, obs, w.acc);
+  prof_end(w, st, tok);
+  return check_launch(w, "render and replay kernel");
 }
 
 int launch_backward(Workspace& w, const float* obs, cudaStream_t st) {

@@ -69,9 +69,17 @@ def render(ws: Workspace, ds: DeviceScene, out: Outputs, stream=None) -> list[in
 
 
 def render_and_score(ws: Workspace, ds: DeviceScene, obs, out: Outputs, lam: float = 1.0,
-                     stream=None) -> list[int]:
-    n = render(ws, ds, out, stream)
-    ws.score_replay(obs, out.tokens, lam, stream)
+                     stream=None, fused: bool = True) -> list[int]:
+    """Project, bin, render and score. fused: render and replay through splat_render_score (one
+    kernel); otherwise splat_render, then splat_score_replay."""
+    if not fused:
+        n = render(ws, ds, out, stream)
+        ws.score_replay(obs, out.tokens, lam, stream)
+        return n
+    ws.project(ds.means, ds.log_scales, ds.quats, ds.opac, ds.sh, ds.viewmats, ds.intrin, ds.H,
+               ds.W, stream)
+    n = ws.bin_sort(stream)
+    ws.render_score(ds.bg, obs, out.img, out.T, out.n_contrib, out.tokens, lam, stream)
     return n
 
 

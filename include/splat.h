@@ -147,6 +147,20 @@ int splat_score_replay(splat_ws* ws, const float* obs, float lambda, float* toke
                        void* stream);
 
 /*
+ * splat_render followed by splat_score_replay in one call, with the same outputs (img, T_final,
+ * n_contrib, tokens) and the same arithmetic and decisions: in the default accumulation mode the
+ * render and the replay run as one kernel -- each warp renders its 8x4 pixel block and replays
+ * the entries it composited at once, with the pixel state still in registers, so that across the
+ * GPU the render's issue-bound work and the replay's L2 reductions overlap. (Deterministic mode:
+ * the two kernels of splat_render and splat_score_replay, one after the other.) The tokens agree
+ * with the two-call sequence up to the order of the fp32 reductions. Afterwards the workspace is
+ * in the state splat_score_replay leaves (splat_backward, splat_render_features, splat_scatter
+ * and splat_attribution may follow, with img, T_final and bg unchanged).
+ */
+int splat_render_score(splat_ws* ws, const float* bg, const float* obs, float lambda, float* img,
+                       float* T_final, int* n_contrib, float* tokens, void* stream);
+
+/*
  * View-sharded replay ([P1] "Exact Score Operators": every cross-view quantity of the token --
  * q_g, the covector pullback, s^alpha, s^SH and A -- is a per-Gaussian sum over views, so the sums
  * of disjoint view sets add). splat_score_partials runs the replay of splat_score_replay for this
@@ -283,7 +297,7 @@ enum {
   SPLAT_K_PROJECT = 0, SPLAT_K_DEPTH_HIST, SPLAT_K_DEPTH_SCATTER,
   SPLAT_K_EMIT, SPLAT_K_TILE_HIST, SPLAT_K_HIST_SCAN, SPLAT_K_TILE_SCATTER, SPLAT_K_TILE_RANGES,
   SPLAT_K_RENDER, SPLAT_K_REPLAY, SPLAT_K_FINALIZE, SPLAT_K_BACKWARD, SPLAT_K_GRAD,
-  SPLAT_K_FEATURES, SPLAT_K_SCATTER, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
+  SPLAT_K_FEATURES, SPLAT_K_SCATTER, SPLAT_K_RENDER_REPLAY, SPLAT_K_OTHER, SPLAT_NUM_KERNELS
 };
 int splat_profile_enable(splat_ws* ws, int enable);
 int splat_profile_read(splat_ws* ws, double* ms, long long* launches, int reset);

@@ -16,9 +16,10 @@ TOKEN_FLOOR = 1e-3
 SH_COLOUR_ATOL = 4e-6
 
 
-def gpu_run(scene, obs, lam=1.0, with_acc=True, det=False):
+def gpu_run(scene, obs, lam=1.0, with_acc=True, det=False, fused=True):
     """The CUDA path over one scene; det=True uses the deterministic accumulation mode (sums
-    independent of the order of the additions)."""
+    independent of the order of the additions); fused=False renders and scores with two calls
+    (splat_render, splat_score_replay) instead of splat_render_score."""
     import torch
     from gaussian_splatting_raster_b200 import runner
 
@@ -28,7 +29,7 @@ def gpu_run(scene, obs, lam=1.0, with_acc=True, det=False):
         ws.deterministic(True)
     out = runner.alloc_outputs(ds)
     obs_t = torch.as_tensor(np.ascontiguousarray(obs, np.float32)).cuda()
-    n = runner.render_and_score(ws, ds, obs_t, out, lam)
+    n = runner.render_and_score(ws, ds, obs_t, out, lam, fused=fused)
     V, G, H, W = ds.V, ds.G, ds.H, ds.W
     TX, TY = O.n_tiles(H, W)
     res = dict(n_per_view=n, img=out.img, T=out.T, n_contrib=out.n_contrib, tokens=out.tokens)

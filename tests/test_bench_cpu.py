@@ -147,7 +147,7 @@ def test_algorithmic_bytes_split_by_what_they_scale_with():
     a = b.algorithmic_bytes(sc, 1000, 0)
     a2 = b.algorithmic_bytes(sc, 2000, 0)
     per_instance = {"emit": 8, "tile_hist": 4, "tile_scatter": 12, "render": 40, "replay": 40,
-                    "backward": 40, "features": 40, "scatter": 80}
+                    "backward": 40, "features": 40, "scatter": 80, "render_replay": 80}
     for k, v in a.items():
         assert v >= 0, k
         assert a2[k] - v == 1000 * per_instance.get(k, 0), k

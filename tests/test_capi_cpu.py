@@ -62,7 +62,7 @@ def test_missing_library_fails_loudly(tmp_path):
 # to store it): a NULL there is an argument error reported before any device work
 _HANDLE_CALLS = [
     "splat_ws_create", "splat_project", "splat_bin_sort", "splat_render", "splat_score_replay",
-    "splat_score_partials", "splat_backward", "splat_render_features", "splat_scatter",
+    "splat_render_score", "splat_score_partials", "splat_backward", "splat_render_features", "splat_scatter",
     "splat_attribution", "splat_copy_projection", "splat_copy_tile_lists", "splat_copy_last",
     "splat_copy_accumulators", "splat_pair_count", "splat_check_status", "splat_set_deterministic",
     "splat_profile_enable", "splat_profile_read",

@@ -26,8 +26,8 @@ def _lib():
     load_library()
 
 
-def _full_check(sc, obs, lam=1.0):
-    g = PU.gpu_run(sc, obs, lam)
+def _full_check(sc, obs, lam=1.0, fused=True):
+    g = PU.gpu_run(sc, obs, lam, fused=fused)
     o = O.run(sc, obs, "f", lam=lam)
     near = PU.compare_projection(sc, g, o["proj"]) if sc.G > 0 else np.zeros(0, bool)
     PU.compare_lists(g, o["lists"])
@@ -67,14 +67,17 @@ def _replay_traversals(sc, o, union_lanes=9):
     return walk, union
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["render_score", "two_calls"])
 @pytest.mark.parametrize("cfg", [1, 2])
-def test_small_configs_full_parity(cfg):
-    """Full parity on the two small workloads. Both of the score replay's traversals run here:
-    on the three-layer scene about two thirds of the warp blocks walk their pixels' entries and a
-    third take the union loop (checked below), so the token comparison covers both."""
+def test_small_configs_full_parity(cfg, fused):
+    """Full parity on the two small workloads, through splat_render_score (render and replay in
+    one kernel) and through splat_render + splat_score_replay. Both of the score replay's
+    traversals run here: on the three-layer scene about two thirds of the warp blocks walk their
+    pixels' entries and a third take the union loop (checked below), so the token comparison
+    covers both."""
     sc = scenes.make(cfg)
     obs = O.observe(sc, "f")
-    g, o = _full_check(sc, obs)
+    g, o = _full_check(sc, obs, fused=fused)
     assert g["n_contrib"].max() > 1
     if cfg == 2:
         walk, union = _replay_traversals(sc, o)
@@ -240,6 +243,21 @@ def test_calls_out_of_order_and_bad_arguments():
         ws.project(z.cpu(), z, z, z[:, 0], torch.zeros((16, 4, 3), device="cuda"),
                    torch.eye(4, device="cuda")[None], torch.ones((1, 4), device="cuda"), 16, 16)
     ws.close()
+
+
+def test_render_score_equals_two_calls():
+    """ReSplat-scale workload: splat_render_score gives the image, final T, contributor counts,
+    list bounds and tile lists of splat_render bit for bit, and the tokens of splat_score_replay
+    up to the order of the fp32 reductions."""
+    sc = scenes.make(3)
+    obs = scenes.smooth_observation(91, sc.V, sc.H, sc.W)
+    a = PU.gpu_run(sc, obs, fused=True)
+    b = PU.gpu_run(sc, obs, fused=False)
+    for k in ("img", "T", "n_contrib", "last", "off", "ids", "rec", "rect"):
+        assert np.array_equal(a[k], b[k]), k
+    err = PU.token_errors(a["tokens"].astype(np.float64), b["tokens"].astype(np.float64))
+    assert err.max() <= 1e-5, err.max()
+    assert np.abs(a["acc"] - b["acc"]).max() <= 1e-5 * np.abs(b["acc"]).max()
 
 
 def test_most_tiles_a_workspace_holds():
