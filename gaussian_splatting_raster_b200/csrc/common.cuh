@@ -189,6 +189,7 @@ struct Workspace {
   ushort4* rect = nullptr;   // [V*G] tile rectangle x0, y0, x1, y1 (16-bit tile coordinates)
   int* counts = nullptr;     // [V*G] tile counts in depth order, then their exclusive scan
   float* acc = nullptr;      // [V*G*8] score sums: (q, w r (3)), (w rho, w rho d (2), unused)
+  bool acc_clean = false;    // acc is all zero (the projection clears it; a replay uses it up)
   double* accb = nullptr;    // [max_V*max_G*10] renderer-backward sums, allocated on first use
   double* sacc = nullptr;    // [G*C] scatter sums, grown on demand
   // deterministic mode: 128-bit fixed-point (low, high) words of the replay / backward sums

@@ -31,7 +31,7 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
           const float* __restrict__ quats, const float* __restrict__ opac,
           const float* __restrict__ sh, const float* __restrict__ views_in, int G, int V, int H,
           int W, int TX, int TY, float4* __restrict__ rec, ushort4* __restrict__ rect,
-          uint32_t* __restrict__ dkey, uint32_t* __restrict__ kbits,
+          uint32_t* __restrict__ dkey, uint32_t* __restrict__ kbits, float4* __restrict__ acc,
           unsigned long long* __restrict__ ntot) {
   constexpr int D = (DEG + 1) * (DEG + 1);
   constexpr int NSH = D * 3;
@@ -242,6 +242,10 @@ k_project(const float* __restrict__ means, const float* __restrict__ lsc,
     rh[0] = r2;
     rh[1] = r3;
     rect[i] = rc;
+    // the score replay's (view, Gaussian) sums start from zero: cleared here, where every row is
+    // written anyway, instead of by a separate pass over 32 B per (view, Gaussian)
+    acc[2 * i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    acc[2 * i + 1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     // depth sort key (fp32 bits of z > 0 order like the values; culled entries sort last) and,
     // per view, the largest visible key and the largest complement of one (the complement of the
     // smallest visible key): the sort orders key - smallest, over the bits of the key range
@@ -287,6 +291,7 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
     k_project<DEG><<<blocks, kProjThreads, smem, st>>>(means, lsc, quats, opac, sh, w.views,     \
                                                        w.G, w.V, w.H, w.W, w.TX, w.TY, w.rec,    \
                                                        w.rect, w.dkey, w.kbits,                  \
+                                                       reinterpret_cast<float4*>(w.acc),         \
                                                        w.ntot);                                  \
   }
   switch (w.deg) {
@@ -297,7 +302,9 @@ int launch_project(Workspace& w, const float* means, const float* lsc, const flo
   }
 #undef SPLAT_PROJ
   prof_end(w, st, tok);
-  return check_launch(w, "project kernel");
+  const int rc2 = check_launch(w, "project kernel");
+  w.acc_clean = rc2 == SPLAT_OK;
+  return rc2;
 }
 
 // the records in the order splat_copy_projection documents: mx, my, a, b, c, o, colour r, g, b,

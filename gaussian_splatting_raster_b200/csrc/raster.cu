@@ -823,9 +823,10 @@ int launch_replay(Workspace& w, const float* obs, cudaStream_t st) {
   const bool det = w.det && w.G > 0;
   if (det) {
     rc = fix_buffer(w, &w.acc_fix, w.acc_fix_cap, kAccN, st);
-  } else if (w.G > 0) {
+  } else if (w.G > 0 && !w.acc_clean) {
     rc = zero_async(w, w.acc, (size_t)w.V * w.G * kAccN * sizeof(float), st, "accumulator clear");
   }
+  w.acc_clean = false;
   if (!rc) {
     dim3 grid(w.nt * kCtaPerTile, w.V);
     if (det)
@@ -849,8 +850,9 @@ int launch_render_replay(Workspace& w, const float* bg, const float* obs, float*
                          float* T_final, int* n_contrib, cudaStream_t st) {
   const int tok = prof_begin(w, st, SPLAT_K_RENDER_REPLAY);
   int rc = SPLAT_OK;
-  if (w.G > 0)
+  if (w.G > 0 && !w.acc_clean)
     rc = zero_async(w, w.acc, (size_t)w.V * w.G * kAccN * sizeof(float), st, "accumulator clear");
+  w.acc_clean = false;
   if (rc) {
     prof_end(w, st, tok);
     return rc;
