@@ -32,13 +32,14 @@
 // multiplied by one fast reciprocal of T (1 - alpha) + eps (T (1 - alpha) >= 1e-6 wherever the
 // result is used; relative error a few 1e-8). (Rewriting rho through
 // running dot products <r, P> is algebraically the same but moves that cancellation and costs
-// ~4e-4 relative token error.) Per entry and warp the seven per-pixel terms
-// (w, w r (3), w rho, w rho (p - mu2D) (2)) are summed by a transpose-reduction (each exchange
-// step halves the values a lane carries: 9 shuffles instead of 35), and the seven lanes holding a
-// result add it to the (view, Gaussian) accumulator with one fp64 atomic each -- seven global
-// atomics per (Gaussian, warp block). The SH block never enters the pixel loop: M_color w (B (x) r)
-// factors into M_color B (x) (sum w r); the mean block Sigma^-1 (sum w rho d) is formed once per
-// (Gaussian, view) in finalisation.
+// ~4e-4 relative token error.) The seven per-pixel terms (w, w r (3), w rho, w rho (p - mu2D) (2))
+// reach the (view, Gaussian) sums either pair by pair (two 16-byte fp32 vector reductions) or,
+// where many pixels of a warp composite the same entry, summed over the warp first by a
+// transpose-reduction (each exchange step halves the values a lane carries: 9 shuffles instead of
+// 35) and reduced once per (entry, warp block) -- see k_replay. The SH block never enters the
+// pixel loop: M_color w (B (x) r) factors into M_color B (x) (sum w r); the mean block
+// Sigma^-1 (sum w rho d) is formed once per (Gaussian, view) in finalisation. The render and the
+// replay also run as one kernel (k_render<true>, splat_render_score).
 #include <algorithm>
 
 #include "traverse.cuh"
