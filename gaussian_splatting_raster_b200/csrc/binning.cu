@@ -155,7 +155,7 @@ int ensure_part(Workspace& w, long long nb) {
 constexpr int kBinWarps = 8;
 constexpr int kBinThreads = kBinWarps * 32;
 constexpr int kDepthChunk = 16384;  // items per block, depth-key passes
-// widest depth digit: the varying bits are split into ceil(bits / max) passes of equal width
+// widest depth digit: the key range's bits are split into ceil(bits / max) passes of equal width
 #ifndef SPLAT_DEPTH_DIGIT_MAX
 #define SPLAT_DEPTH_DIGIT_MAX 11
 #endif

@@ -98,8 +98,9 @@ int splat_project(splat_ws* ws, const float* means, const float* log_scales, con
 /*
  * Stage 1 tile binning and contributor sort ([P1] Stage 1 step 1): every visible (g, v) emits one
  * instance per tile of its rectangle; each tile's list is ordered by (camera depth z, Gaussian
- * index) -- a stable radix sort of one fp32 depth key per (view, Gaussian) over the key bits
- * that vary, emission of the instances in that order, and one stable counting sort by tile.
+ * index) -- a stable radix sort of one fp32 depth key per (view, Gaussian), less the view's
+ * smallest visible key, over the width of the key range; emission of the instances in that
+ * order; and one stable counting sort by tile.
  * The lists stay in the workspace ([P1] Stage 1: not exposed as a per-pixel tensor).
  * n_instances_out (HOST pointer, may be NULL) receives V counts. Synchronises with the stream
  * once (the counts size the sort).
