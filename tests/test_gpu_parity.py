@@ -260,6 +260,31 @@ def test_render_score_equals_two_calls():
     assert np.abs(a["acc"] - b["acc"]).max() <= 1e-5 * np.abs(b["acc"]).max()
 
 
+def test_repeated_replays_start_from_cleared_sums():
+    """The projection clears the replay's per-(view, Gaussian) sums; a replay that finds them
+    already used (a second replay after one projection, here after splat_render_score) clears them
+    itself, so every call gives the same tokens (up to the order of the fp32 reductions); twice
+    the sums would double q_g and change every token."""
+    import torch
+    from gaussian_splatting_raster_b200 import runner
+    sc = scenes.make(2)
+    obs = O.observe(sc, "f")
+    ds = runner.to_device(sc)
+    ws = runner.workspace_for(ds)
+    out = runner.alloc_outputs(ds)
+    obs_t = torch.as_tensor(obs).cuda()
+    runner.render_and_score(ws, ds, obs_t, out)
+    z1 = out.tokens.cpu().numpy().astype(np.float64)
+    for _ in range(2):
+        ws.score_replay(obs_t, out.tokens)
+        z = out.tokens.cpu().numpy().astype(np.float64)
+        assert PU.token_errors(z, z1).max() <= 1e-5
+    ws.render_score(ds.bg, obs_t, out.img, out.T, out.n_contrib, out.tokens)
+    z = out.tokens.cpu().numpy().astype(np.float64)
+    assert PU.token_errors(z, z1).max() <= 1e-5
+    ws.close()
+
+
 def test_most_tiles_a_workspace_holds():
     """An image of 7,264 16x16 tiles (the largest the binning's per-warp shared-memory counts
     hold) renders and scores like the oracle; one tile more is refused at workspace creation."""
