@@ -11,7 +11,7 @@
 //   attribution        [sum w, sum w |r|, sum w |r| / (sum w + 1e-6)] per Gaussian, r = C_hat - C_obs
 // with w = T alpha of the composited entries (the render's decisions; no background term).
 //
-// Same traversal as the score replay: one CTA per (tile, view); each warp walks the list for its
+// Same traversal as the score replay (kCtaPerTile CTAs per (tile, view)); each warp walks the list for its
 // 8x4 pixel block on its own in 32-entry chunks, staging only the entries the render marked as
 // composited by some pixel of the warp. The attribute render keeps up to 16 channels per pixel in
 // registers (more channels take further passes); the scatter reduces each entry's per-pixel

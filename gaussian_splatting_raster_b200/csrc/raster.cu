@@ -8,10 +8,10 @@
 // (o = sigmoid(a), alpha = o G, w = T alpha, rho = <r, c - C+>, q = sum w; the opacity-logit,
 // SH and projected-centre scores).
 //
-// One CTA per (tile, view), one thread per pixel of the 16x16 tile, the CTAs taking the tiles in
-// the binning's launch order (longest list first, so that no long list starts in the last wave);
-// the eight warps (an 8x4 pixel block each) walk the tile's list independently, with no CTA
-// barrier: each warp stages 32-entry
+// One thread per pixel of the 16x16 tile in kCtaPerTile CTAs per (tile, view), the CTAs taking
+// the tiles in the binning's launch order (longest list first, so that no long list starts in the
+// last wave); the eight warps (an 8x4 pixel block each) walk the tile's list independently, with
+// no CTA barrier: each warp stages 32-entry
 // chunks of records in its own shared-memory slice, keeps by ballot the entries whose precomputed
 // box reaches its block, and stops when all its pixels are saturated. Both passes evaluate alpha
 // through the same device function, so the replay takes exactly the render's decisions; the

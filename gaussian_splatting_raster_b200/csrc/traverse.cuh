@@ -22,11 +22,11 @@
 namespace splat {
 namespace {
 
-// A tile's eight warp blocks run in kCtaPerTile CTAs of kCtaWarps warps each. The warps walk the
-// lists independently (no CTA barriers), so a CTA is only a residency unit: smaller CTAs let the
-// warps of a finished block make room sooner.
+// A tile's eight warp blocks run in kCtaPerTile CTAs of kCtaWarps warps each (two of four by
+// default). The warps walk the lists independently (no CTA barriers), so a CTA is only a residency
+// unit: smaller CTAs let the warps of a finished block make room sooner.
 #ifndef SPLAT_CTA_WARPS
-#define SPLAT_CTA_WARPS 8
+#define SPLAT_CTA_WARPS 4
 #endif
 constexpr int kCtaWarps = SPLAT_CTA_WARPS;
 static_assert(kCtaWarps == 1 || kCtaWarps == 2 || kCtaWarps == 4 || kCtaWarps == 8,
