@@ -169,23 +169,60 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
+def code_text(src: str) -> str:
+    """C/C++/CUDA source with its comments removed (each replaced by one space, as the compiler
+    does), trailing blanks cut and empty lines dropped: what remains is the code the compiler
+    sees, so rewording a comment leaves it unchanged while any change to the code changes it.
+    String and character literals are copied as they are."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == "/" and src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif c == "/" and src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c and src[j] != "\n":
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).split("\n"))
+    return "\n".join(ln for ln in lines if ln)
+
+
+def code_digest(paths) -> str:
+    """sha256 over the code (code_text) of the given repository files, in order."""
+    import hashlib
+    m = hashlib.sha256()
+    for f in paths:
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            m.update(code_text(fh.read()).encode())
+        m.update(b"\0")
+    return m.hexdigest()
+
+
 def _current_record(fname: str, kernel: str, workload: str):
     """A kernel's entry of a committed ncu record under profiles/, only when it was captured on
-    this workload and the kernel's sources still hash to what was captured."""
-    import hashlib
+    this workload and the code of the kernel's sources (comments aside) is still what was
+    captured."""
     try:
         d = json.load(open(os.path.join(ROOT, "profiles", fname)))["kernels"][kernel]
     except (OSError, KeyError, ValueError):
         return None
     if d.get("workload") != workload:
         return None
-    m = hashlib.sha256()
-    for f in d["sources"]:
-        try:
-            m.update(open(os.path.join(ROOT, f), "rb").read())
-        except OSError:
+    try:
+        if code_digest(d["sources"]) != d["code_sha256"]:
             return None
-    if m.hexdigest() != d["sha256"]:
+    except (OSError, KeyError, UnicodeDecodeError):
         return None
     return d
 

@@ -40,8 +40,8 @@ struct Entry {
   float alpha, dx, dy;
 };
 
-// Pixel blocks of the warps. A tile's CTA has eight warps; warp w covers a kWarpW x kWarpH block
-// of the 16x16 tile (blocks in row-major order), lane l the pixel (l % kWarpW, l / kWarpW) of its
+// Pixel blocks of the warps. A tile has eight warps (over its CTAs); warp w covers a kWarpW x
+// kWarpH block of the 16x16 tile (row-major), lane l the pixel (l % kWarpW, l / kWarpW) of its
 // block. Every kernel that walks the lists uses this one mapping: the render records per warp
 // which entries some pixel of the block composited, and the later passes read those masks.
 #ifndef SPLAT_WARP_W

@@ -1,7 +1,7 @@
 """Host-side checks of bench.py that need no GPU: the reference arm (the CPU oracle timed on the
 host) prints exactly one JSON line with the contract's keys, a non-zero rank of it prints nothing,
-the DRAM-traffic and pipe-counter records are reported only for the workload and sources they were
-captured on, the reference arm's steps are what it ran, the fp32 work counts split by pair class,
+the DRAM-traffic and pipe-counter records are reported only for the workload and code they were
+captured on (comments aside), the reference arm's steps are what it ran, the fp32 work counts split by pair class,
 the peaks file falls back when absent, and the algorithmic byte counts split into the parts that
 grow with the instance count and the parts that do not."""
 import importlib.util
@@ -53,50 +53,59 @@ def test_reference_arm_other_ranks_do_no_work():
     assert r.stdout.strip() == ""
 
 
-def test_traffic_record_follows_workload_and_sources(tmp_path, monkeypatch):
-    """A record answers only for its workload and only while its sources hash the same."""
-    import hashlib
-    b = _bench()
-    srcs = ["gaussian_splatting_raster_b200/csrc/traverse.cuh",
-            "gaussian_splatting_raster_b200/csrc/raster.cu"]
+def _copy_sources(tmp_path, srcs):
     for f in srcs:
         (tmp_path / f).parent.mkdir(parents=True, exist_ok=True)
         shutil.copy(os.path.join(ROOT, f), tmp_path / f)
-    m = hashlib.sha256()
-    for f in srcs:
-        m.update((tmp_path / f).read_bytes())
+
+
+def test_traffic_record_follows_workload_and_code(tmp_path, monkeypatch):
+    """A record answers only for its workload and only while its sources' code is unchanged:
+    rewording a comment keeps it, changing one token of code retires it."""
+    b = _bench()
+    srcs = ["gaussian_splatting_raster_b200/csrc/traverse.cuh",
+            "gaussian_splatting_raster_b200/csrc/raster.cu"]
+    _copy_sources(tmp_path, srcs)
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
     rec = {"kernels": {"replay": {"workload": "w1", "dram_read_bytes": 300, "dram_write_bytes": 45,
-                                  "sources": srcs, "sha256": m.hexdigest()}}}
+                                  "sources": srcs, "code_sha256": b.code_digest(srcs)}}}
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
-    monkeypatch.setattr(b, "ROOT", str(tmp_path))
     assert b.recorded_traffic("replay", "w1") == 345
     assert b.recorded_traffic("replay", "w2") is None
     assert b.recorded_traffic("render", "w1") is None
-    with open(tmp_path / srcs[0], "a") as fh:  # any change to a source retires the record
-        fh.write("\n")
+    f0 = tmp_path / srcs[0]
+    text = f0.read_text()
+    f0.write_text("// a reworded note\n/* and a block\n   comment */\n" + text + "\n\n")
+    assert b.recorded_traffic("replay", "w1") == 345
+    f0.write_text(text.replace("kAlphaMin = 1.0f / 255.0f", "kAlphaMin = 1.0f / 256.0f", 1))
     assert b.recorded_traffic("replay", "w1") is None
 
 
-def test_pipe_record_follows_workload_and_sources(tmp_path, monkeypatch):
-    import hashlib
+def test_pipe_record_follows_workload_and_code(tmp_path, monkeypatch):
     b = _bench()
     srcs = ["gaussian_splatting_raster_b200/csrc/raster.cu"]
-    (tmp_path / srcs[0]).parent.mkdir(parents=True, exist_ok=True)
-    shutil.copy(os.path.join(ROOT, srcs[0]), tmp_path / srcs[0])
+    _copy_sources(tmp_path, srcs)
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
     rec = {"kernels": {"render": {"workload": "w1", "fma_pipe_pct": 41.5, "alu_pipe_pct": 30.0,
                                   "issue_active_pct": 80.0, "sources": srcs,
-                                  "sha256": hashlib.sha256((tmp_path / srcs[0]).read_bytes())
-                                  .hexdigest()}}}
+                                  "code_sha256": b.code_digest(srcs)}}}
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "pipe_counters.json").write_text(json.dumps(rec))
-    monkeypatch.setattr(b, "ROOT", str(tmp_path))
     assert b.recorded_pipes("render", "w1") == {"fma_pipe_pct": 41.5, "alu_pipe_pct": 30.0,
                                                 "issue_active_pct": 80.0}
     assert b.recorded_pipes("render", "w2") is None and b.recorded_pipes("replay", "w1") is None
     with open(tmp_path / srcs[0], "a") as fh:
-        fh.write("\n")
+        fh.write("static int extra;\n")
     assert b.recorded_pipes("render", "w1") is None
+
+
+def test_code_text_drops_comments_only():
+    b = _bench()
+    src = ('int a = 1; // note\n/* block\n   x */ const char* s = "// kept"; char q = \'/\';\n'
+           '\n#define X 1 /* y */\nfloat f = 2.0f;   \n')
+    assert b.code_text(src) == ('int a = 1;\n  const char* s = "// kept"; char q = \'/\';\n'
+                                '#define X 1\nfloat f = 2.0f;')
 
 
 def test_alu_work_counts_by_pair_class():
