@@ -323,11 +323,13 @@ def alu_ops(kernel: str, pairs: int, composited: int) -> int:
 # ----------------------------------------------------------------------------------------------
 # CPU oracle baseline: one whole view of the workload, timed as it runs
 
-def cpu_oracle_view(sc, obs_np, path="score", threads=0):
+def cpu_oracle_view(sc, obs_np, path="score", threads=0, keep_outputs=False):
     """The oracle (fp32 decision mode, OpenMP) over one complete view of the workload: projection
     and binning of every Gaussian into view 0, render and the pass of `path` over every tile of
     that view, and the per-Gaussian finalisation. Nothing is sampled or scaled: value = the
-    view's pixels / the measured wall time. threads > 0 sets the oracle's OpenMP thread count."""
+    view's pixels / the measured wall time. threads > 0 sets the oracle's OpenMP thread count.
+    keep_outputs (score path): also return the view's image, final transmittance, contributor
+    counts and tokens under "outputs", for the whole-view comparison with the CUDA path."""
     import numpy as np
     from oracle import oracle as O
     if threads > 0:
@@ -353,28 +355,120 @@ def cpu_oracle_view(sc, obs_np, path="score", threads=0):
         rp = O.replay(p, L, r, obs_np[:1], one.sh_degree, one.H, one.W, "f")
     t_rr = time.perf_counter() - t1
     t2 = time.perf_counter()
+    tokens = None
     if path == "backward":
         O.gradients(p, accb, one, "f")
     elif path == "score":
-        O.finalize(p, rp["acc"], one)
+        tokens = O.finalize(p, rp["acc"], one)
     t_fin = time.perf_counter() - t2
     second = {"backward": "backward", "attributes": "attribute render + scatters",
               "score": "replay"}[path]
     last = {"backward": "gradient chain", "attributes": "nothing further",
             "score": "finalisation"}[path]
     t_view = t_pb + t_rr + t_fin
+    outputs = None
+    if keep_outputs and path == "score":
+        outputs = {"img": r["img"], "T": r["T"], "n_contrib": r["n_contrib"], "tokens": tokens}
     return {"value": one.H * one.W / t_view / 1e6, "unit": "Mpix/s",
             "cores": int(O.lib().orc_num_threads()), "kind": "oracle",
             "sample": (f"view 1 of {sc.V}, whole: projection + binning of all {sc.G} Gaussians "
                        f"({1e3 * t_pb:.1f} ms), render of all {one.H}x{one.W} pixels "
                        f"({1e3 * t_r:.1f} ms), {second} ({1e3 * (t_rr - t_r):.1f} ms), {last} "
                        f"({1e3 * t_fin:.1f} ms)"),
-            "seconds": t_view}
+            "seconds": t_view, "outputs": outputs}
 
 
 def _one_view(sc):
     import dataclasses
     return dataclasses.replace(sc, viewmats=sc.viewmats[:1], intrin=sc.intrin[:1])
+
+
+def token_blocks(d: int) -> dict:
+    """Column ranges of the token's blocks: [b (3), s^alpha, s^SH (3d), log q, eig (3), log tr]."""
+    return {"b_mu": (0, 3), "s_alpha": (3, 4), "s_sh": (4, 4 + 3 * d),
+            "log_q": (4 + 3 * d, 5 + 3 * d), "eig": (5 + 3 * d, 8 + 3 * d),
+            "log_tr": (8 + 3 * d, 9 + 3 * d)}
+
+
+COLOUR_ATOL, TOKEN_RTOL, NORM_FLOOR = 1e-5, 1e-4, 1e-3
+
+
+def parity_report(g: dict, o: dict, d: int, chunk: int = 1 << 16) -> dict:
+    """d = SH coefficients per channel ((degree + 1)^2). Element-by-element comparison of one whole view of the workload, CUDA path (g) against the
+    oracle in fp32 decision mode (o): image, final transmittance, contributor counts and every
+    Gaussian's token. The bars are the parity tests': colour within 1e-5 absolute, transmittance
+    and counts exact, tokens within 1e-4 relative L2 per Gaussian (floor 1e-3 x the median token
+    norm); per token block the same ratio with the block's own floor (1e-3 x its median non-zero
+    norm). Reported, not asserted: the tests assert."""
+    import numpy as np
+    img_err = float(np.abs(g["img"].astype(np.float64) - o["img"]).max(initial=0.0))
+    t_mis = int((g["T"] != np.asarray(o["T"]).astype(np.float32)).sum())
+    nc_mis = int((g["n_contrib"] != o["n_contrib"]).sum())
+    zg, zo = g["tokens"], o["tokens"]
+    G = zo.shape[0]
+    if zg.shape != zo.shape or zo.shape[1] != 9 + 3 * d:
+        raise ValueError(f"token arrays {zg.shape} / {zo.shape} for {d} SH coefficients")
+    blocks = token_blocks(d)
+    names = list(blocks)
+
+    def block_norms(x):  # [n, K] -> [n, blocks] L2 norms of each block, and [n] of the row
+        sq = np.stack([np.einsum("ij,ij->i", x[:, a:b], x[:, a:b]) for a, b in blocks.values()],
+                      axis=1)
+        return np.sqrt(sq), np.sqrt(sq.sum(axis=1))
+
+    bn = np.empty((G, len(names)))
+    norms = np.empty(G)
+    for s in range(0, G, chunk):
+        bn[s:s + chunk], norms[s:s + chunk] = block_norms(np.asarray(zo[s:s + chunk], np.float64))
+
+    def floor_of(n):
+        nz = n[n > 0]
+        return NORM_FLOOR * (float(np.median(nz)) if nz.size else 0.0) or 1e-30
+
+    floor = floor_of(norms)
+    bfloor = np.array([floor_of(bn[:, i]) for i in range(len(names))])
+    err = np.empty(G)
+    be = np.empty((G, len(names)))
+    for s in range(0, G, chunk):
+        dz = np.asarray(zg[s:s + chunk], np.float64) - np.asarray(zo[s:s + chunk], np.float64)
+        dbn, dn = block_norms(dz)
+        err[s:s + chunk] = dn / np.maximum(norms[s:s + chunk], floor)
+        be[s:s + chunk] = dbn / np.maximum(bn[s:s + chunk], bfloor)
+    berr = {k: be[:, i] for i, k in enumerate(names)}
+    covered = np.exp(np.asarray(zo[:, 4 + 3 * d], np.float64)) >= 1e-3  # q_g >= 1e-3
+    ok = err <= TOKEN_RTOL
+
+    def q(a, p):
+        return float(np.percentile(a, p)) if a.size else 0.0
+
+    return {"pixels": int(np.asarray(o["n_contrib"]).size), "gaussians": int(G),
+            "colour_max_abs_err": img_err, "colour_bar": COLOUR_ATOL,
+            "T_final_mismatches": t_mis, "n_contrib_mismatches": nc_mis,
+            "token_rel_err_max": float(err.max(initial=0.0)), "token_rel_err_p99": q(err, 99),
+            "token_bar": TOKEN_RTOL,
+            "token_block_rel_err_max": {k: float(v.max(initial=0.0)) for k, v in berr.items()},
+            "token_block_rel_err_p99": {k: q(v, 99) for k, v in berr.items()},
+            "gaussians_qg_ge_1e-3": int(covered.sum()),
+            "frac_pass_qg_ge_1e-3": float(ok[covered].mean()) if covered.any() else None,
+            "frac_pass_all": float(ok.mean()) if G else None}
+
+
+def gpu_view_outputs(sc, obs, fused: bool, deterministic: bool) -> dict:
+    """The CUDA path over view 0 of the workload alone (its own workspace), as host arrays."""
+    import torch
+    from gaussian_splatting_raster_b200 import runner
+    ds1 = runner.to_device(_one_view(sc))
+    ws1 = runner.workspace_for(ds1)
+    try:
+        if deterministic:
+            ws1.deterministic(True)
+        out1 = runner.alloc_outputs(ds1)
+        runner.render_and_score(ws1, ds1, obs[:1].contiguous(), out1, fused=fused)
+        torch.cuda.synchronize()
+        return {"img": out1.img.cpu().numpy(), "T": out1.T.cpu().numpy(),
+                "n_contrib": out1.n_contrib.cpu().numpy(), "tokens": out1.tokens.cpu().numpy()}
+    finally:
+        ws1.close()
 
 
 # ----------------------------------------------------------------------------------------------
@@ -757,10 +851,24 @@ def main():
         render_ms += render_alone_ms
         replay_ms += per_kernel["render_replay"]["ms_per_step"] - render_alone_ms
 
+    # The oracle's view is also compared with the CUDA path over the same view, element by
+    # element (score path, whole view: every pixel and every Gaussian's token).
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_view(sc, obs.cpu().numpy(), path=args.path, threads=args.cpu_threads)
+        want = args.path == "score" and not shard
+        cpu = cpu_oracle_view(sc, obs.cpu().numpy(), path=args.path, threads=args.cpu_threads,
+                              keep_outputs=want)
         cpu.pop("seconds", None)
+        ora = cpu.pop("outputs", None)
+        if ora is not None:
+            try:
+                parity = {"view": f"1 of {sc.V}, whole",
+                          **parity_report(gpu_view_outputs(sc, obs, not args.unfused,
+                                                           args.deterministic), ora, sc.d)}
+            except Exception as e:  # a report: its failure must not cost the line
+                parity = {"error": f"{type(e).__name__}: {e}"[:300]}
+        del ora
 
     if rank == 0:
         line = {
@@ -788,6 +896,7 @@ def main():
             "gpu_launches": int(launches), "per_kernel": per_kernel,
             "ms_per_step_with_kernel_events": max_over_ranks(sum(prof_step_ms), world) / args.steps,
             "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "vram": vram,
+            "parity_vs_oracle": parity,
         }
         os.write(json_fd, (json.dumps(line) + "\n").encode())
     ws.close()

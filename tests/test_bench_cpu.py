@@ -165,3 +165,62 @@ def test_algorithmic_bytes_split_by_what_they_scale_with():
     VG = sc.V * sc.G
     assert a4["depth_hist"] - a["depth_hist"] == 4 * VG
     assert a4["depth_scatter"] - a["depth_scatter"] == 16 * VG
+
+
+def test_parity_report_locates_differences():
+    """The whole-view comparison the bench prints: identical outputs give zero errors; a token
+    block or a pixel changed on one side shows up in that block's and that output's figures."""
+    import numpy as np
+    b = _bench()
+    rng = np.random.default_rng(3)
+    d, G, H, W = 4, 500, 8, 16
+    K = 9 + 3 * d
+    zo = rng.normal(size=(G, K))
+    zo[:, 4 + 3 * d] = np.log(rng.uniform(1e-5, 2.0, G))  # log q_g: some below 1e-3
+    o = {"img": rng.uniform(size=(1, H, W, 3)), "T": rng.uniform(size=(1, H, W)),
+         "n_contrib": rng.integers(0, 9, (1, H, W)).astype(np.int32), "tokens": zo}
+    g = {"img": o["img"].astype(np.float32), "T": o["T"].astype(np.float32),
+         "n_contrib": o["n_contrib"].copy(), "tokens": zo.astype(np.float32)}
+    r = b.parity_report(g, o, d, chunk=64)
+    assert r["T_final_mismatches"] == 0 and r["n_contrib_mismatches"] == 0
+    assert r["colour_max_abs_err"] < 1e-7 and r["token_rel_err_max"] < 1e-6
+    assert r["frac_pass_all"] == 1.0 and r["frac_pass_qg_ge_1e-3"] == 1.0
+    assert r["gaussians_qg_ge_1e-3"] == int((np.exp(zo[:, 4 + 3 * d]) >= 1e-3).sum())
+    assert set(r["token_block_rel_err_max"]) == {"b_mu", "s_alpha", "s_sh", "log_q", "eig",
+                                                 "log_tr"}
+    # one Gaussian's SH block off by 1 %, one pixel's colour by 1e-4, one count and one T changed
+    g["tokens"][7, 4:4 + 3 * d] *= 1.01
+    g["img"][0, 2, 3, 1] += 1e-4
+    g["n_contrib"][0, 1, 1] += 1
+    g["T"][0, 5, 5] = np.nextafter(g["T"][0, 5, 5], np.float32(2))
+    r = b.parity_report(g, o, d, chunk=64)
+    assert r["T_final_mismatches"] == 1 and r["n_contrib_mismatches"] == 1
+    assert 0.9e-4 < r["colour_max_abs_err"] < 1.1e-4
+    blk = r["token_block_rel_err_max"]
+    assert 0.9e-2 < blk["s_sh"] < 1.1e-2
+    assert all(v < 1e-6 for k, v in blk.items() if k != "s_sh")
+    assert r["frac_pass_all"] == (G - 1) / G
+    assert r["token_rel_err_max"] > 1e-4
+
+
+def test_oracle_view_outputs_feed_the_report():
+    """cpu_oracle_view(keep_outputs=True) hands back the arrays parity_report reads, shaped as the
+    CUDA path's outputs of one view (compared here with themselves, rounded to fp32)."""
+    import numpy as np
+    b = _bench()
+    sys.path.insert(0, ROOT)
+    from synth import scenes
+    sc = scenes.make(2)
+    obs = np.random.default_rng(0).uniform(0, 1, (sc.V, sc.H, sc.W, 3)).astype(np.float32)
+    s = b.cpu_oracle_view(sc, obs, keep_outputs=True)
+    o = s["outputs"]
+    assert o["img"].shape == (1, sc.H, sc.W, 3) and o["T"].shape == (1, sc.H, sc.W)
+    assert o["n_contrib"].shape == (1, sc.H, sc.W)
+    assert o["tokens"].shape == (sc.G, 9 + 3 * sc.d)
+    g = {"img": o["img"].astype(np.float32), "T": np.asarray(o["T"]).astype(np.float32),
+         "n_contrib": o["n_contrib"].astype(np.int32), "tokens": o["tokens"].astype(np.float32)}
+    r = b.parity_report(g, o, sc.d)
+    assert r["pixels"] == sc.H * sc.W and r["gaussians"] == sc.G
+    assert r["T_final_mismatches"] == 0 and r["n_contrib_mismatches"] == 0
+    assert r["token_rel_err_max"] < 1e-6 and r["frac_pass_all"] == 1.0
+    assert b.cpu_oracle_view(sc, obs)["outputs"] is None
