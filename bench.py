@@ -715,6 +715,10 @@ def main():
 
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
+    # every rank takes part in these reductions, in the same order
+    median_ms = max_over_ranks(statistics.median(step_ms), world)
+    min_ms = max_over_ranks(min(step_ms), world)
+    prof_ms_per_step = max_over_ranks(sum(prof_step_ms), world) / args.steps
     px_step = sc.V * sc.H * sc.W
     # replicas: every rank does the whole workload; views: the ranks split one workload
     units = 1 if shard else world
@@ -894,7 +898,8 @@ def main():
             "render_ms_per_view": render_ms / sc.V, f"{second[0]}_ms_per_view": replay_ms / sc.V,
             f"{second[0]}_over_render": replay_ms / render_ms if render_ms else None,
             "gpu_launches": int(launches), "per_kernel": per_kernel,
-            "ms_per_step_with_kernel_events": max_over_ranks(sum(prof_step_ms), world) / args.steps,
+            "ms_per_step_with_kernel_events": prof_ms_per_step,
+            "ms_per_step_median": median_ms, "ms_per_step_min": min_ms,
             "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "vram": vram,
             "parity_vs_oracle": parity,
         }

@@ -224,3 +224,27 @@ def test_oracle_view_outputs_feed_the_report():
     assert r["T_final_mismatches"] == 0 and r["n_contrib_mismatches"] == 0
     assert r["token_rel_err_max"] < 1e-6 and r["frac_pass_all"] == 1.0
     assert b.cpu_oracle_view(sc, obs)["outputs"] is None
+
+
+def test_no_collective_under_a_rank_branch():
+    """Every rank must take the same collective steps: no reduction or barrier of bench.py sits
+    inside a branch taken by some ranks only (a test of `rank`), where the other ranks would wait
+    for it forever."""
+    import ast
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
+    collectives = {"max_over_ranks", "pairs_sum_over_ranks", "barrier", "all_reduce",
+                   "all_gather", "reduce_scatter_tensor", "broadcast"}
+
+    def names(node):
+        return {n.id for n in ast.walk(node) if isinstance(n, ast.Name)}
+
+    bad = []
+    for node in ast.walk(tree):
+        if isinstance(node, (ast.If, ast.IfExp)) and "rank" in names(node.test):
+            for sub in ast.walk(node):
+                if isinstance(sub, ast.Call):
+                    f = sub.func
+                    name = f.id if isinstance(f, ast.Name) else getattr(f, "attr", None)
+                    if name in collectives:
+                        bad.append((sub.lineno, name))
+    assert not bad, bad
