@@ -106,6 +106,9 @@ def test_code_text_drops_comments_only():
            '\n#define X 1 /* y */\nfloat f = 2.0f;   \n')
     assert b.code_text(src) == ('int a = 1;\n  const char* s = "// kept"; char q = \'/\';\n'
                                 '#define X 1\nfloat f = 2.0f;')
+    # an escaped quote does not end a literal; a comment marker after it is still literal text
+    src = 'printf("a\\"// b"); // c\nchar e = \'\\\'\'; /* d */ int z;\n'
+    assert b.code_text(src) == 'printf("a\\"// b");\nchar e = \'\\\'\';   int z;'
 
 
 def test_alu_work_counts_by_pair_class():
