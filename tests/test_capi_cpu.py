@@ -99,3 +99,33 @@ def test_kernel_group_names_and_build_flavour(lib_path):
     assert {"project", "render", "replay", "finalize", "backward"} <= set(names)
     assert L.splat_kernel_name(-1) == b"?" and L.splat_kernel_name(P.KERNEL_GROUPS) == b"?"
     assert L.splat_checked_build() == 0  # the release library
+
+
+def test_argument_errors_come_before_any_device_work(lib_path):
+    """The refusals include/splat.h documents as taken before any work: they return their codes
+    here, where there is no device (a call that reached CUDA would fail with SPLAT_ERR_CUDA or
+    SPLAT_ERR_OOM instead)."""
+    import gaussian_splatting_raster_b200 as P
+    L = P.load_library()
+    INVALID, CAPACITY, OK = -1, -2, 0
+    h = ctypes.c_void_p()
+    for args in ((-1, 1, 8, 8, 0), (1, 0, 8, 8, 0), (1, 1025, 8, 8, 0), (1, 1, 0, 8, 0),
+                 (1, 1, 8, 0, 0), (1, 1, 8, 8, -1), (1, 1, 8, 8, 4)):
+        assert L.splat_ws_create(ctypes.byref(h), *args) == INVALID, args
+        assert h.value is None  # *ws is set to NULL on failure
+    assert L.splat_ws_create(None, 1, 1, 8, 8, 0) == INVALID
+    fin = L.splat_finalize_partials
+    some = ctypes.c_void_p(4096)  # never dereferenced: every call below returns first
+    for G, deg, lam in ((-1, 0, 1.0), (4, -1, 1.0), (4, 4, 1.0), (4, 0, -1.0),
+                        (4, 0, float("nan")), (4, 0, float("inf"))):
+        assert fin(some, G, deg, ctypes.c_float(lam), some, None) == INVALID, (G, deg, lam)
+    assert fin(None, 4, 0, ctypes.c_float(1.0), some, None) == INVALID
+    assert fin(ctypes.c_void_p(4098), 4, 0, ctypes.c_float(1.0), some, None) == INVALID  # align
+    assert fin(None, 0, 3, ctypes.c_float(1.0), None, None) == OK  # nothing to do
+    srt = L.splat_sort_depths_noalloc
+    srt.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    srt.restype = ctypes.c_int
+    assert srt(some, -1, some, None) == INVALID
+    assert srt(None, 5, some, None) == INVALID and srt(some, 5, None, None) == INVALID
+    assert srt(some, 262144 + 1, some, None) == CAPACITY  # SPLAT_NOALLOC_MAX_N + 1
+    assert srt(None, 0, None, None) == OK
