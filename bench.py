@@ -93,58 +93,87 @@ def parse():
 # clocks during the timed region
 
 class ClockSampler:
+    """nvidia-smi samples of the SM clock and the throttle reasons, kept only when they arrived
+    inside the timed region (mark() .. stop())."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 100
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_id: str | None):
         self.gpu_id = gpu_id
         self.proc = None
-        self.lines: list[str] = []
+        self.lines: list[tuple[float, str]] = []  # (arrival time, line)
+        self.t0 = None
+        self._first = threading.Event()
 
-    def start(self):
+    def start(self, wait_s: float = 5.0):
+        """Start sampling and wait (up to wait_s) for the first sample, so that sampling is live
+        before the timed region begins."""
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-               "-lms", "200"]
+               "-lms", str(self.INTERVAL_MS)]
         if self.gpu_id:
             cmd += ["-i", self.gpu_id]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
         except OSError:
             self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        self._first.wait(wait_s)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+            self._first.set()
+
+    def mark(self):
+        """The timed region starts now."""
+        self.t0 = time.monotonic()
 
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        t1 = time.monotonic()
+        time.sleep(2 * self.INTERVAL_MS / 1e3)  # let a sample taken at the end arrive
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0 = self.t0 if self.t0 is not None else 0.0
+        return self.summarize(list(self.lines), t0, t1 + self.INTERVAL_MS / 1e3)
+
+    @classmethod
+    def summarize(cls, lines, t0: float, t1: float) -> dict:
+        """Median SM clock, largest max clock and the throttle reasons seen in the samples that
+        arrived in [t0, t1]. A region shorter than the sampling interval may hold none: then the
+        first sample after t0 stands for it, and `window` says so."""
+        parsed = []
+        for t, ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 7:
                 continue
             try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
+                sm, smax = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            for n, p in zip(names, parts[3:7]):
-                if p.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            act = {n for n, p in zip(cls.REASONS, parts[3:7]) if p.lower().startswith("active")}
+            parsed.append((t, sm, smax, act))
+        inside = [x for x in parsed if t0 <= x[0] <= t1]
+        window = "timed region"
+        if not inside:
+            after = [x for x in parsed if x[0] >= t0]
+            inside = after[:1]
+            window = "first sample after the timed region began" if inside else "no sample"
+        return {"sm_mhz": statistics.median(x[1] for x in inside) if inside else None,
+                "sm_max_mhz": max(x[2] for x in inside) if inside else None,
+                "reasons": sorted(set().union(*(x[3] for x in inside))) if inside else [],
+                "samples": len(inside), "window": window,
+                "interval_ms": cls.INTERVAL_MS}
 
 
 def gpu_id_for(dev) -> str | None:
@@ -678,9 +707,11 @@ def main():
         return ms
 
     ws.profile(False)
+    if sampler:
+        sampler.start()  # returns once sampling is live
     barrier(world)
     if sampler:
-        sampler.start()
+        sampler.mark()
     launches_before = ws.launch_count
     step_ms = timed_steps()
     launches = ws.launch_count - launches_before

@@ -251,3 +251,46 @@ def test_no_collective_under_a_rank_branch():
                     if name in collectives:
                         bad.append((sub.lineno, name))
     assert not bad, bad
+
+
+def test_clock_samples_are_those_of_the_timed_region():
+    b = _bench()
+    S = b.ClockSampler
+    idle, busy = "1200, 1965, 90.5, Not Active, Not Active, Not Active, Not Active", \
+        "1965, 1965, 700.0, Not Active, Not Active, Not Active, Active"
+    lines = [(0.0, idle), (1.0, idle), (2.0, busy), (2.1, busy), (2.2, "garbage"),
+             (2.3, busy.replace("1965, 1965", "1905, 1965")), (5.0, idle)]
+    r = S.summarize(lines, 1.5, 2.5)
+    assert r["samples"] == 3 and r["window"] == "timed region"
+    assert r["sm_mhz"] == 1965.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"]
+    # a region shorter than the interval: the first sample after its start stands for it
+    r = S.summarize(lines, 2.35, 2.4)
+    assert r["samples"] == 1 and r["sm_mhz"] == 1200.0 and r["window"].startswith("first")
+    assert S.summarize(lines, 9.0, 9.5)["window"] == "no sample"
+
+
+def test_clock_sampler_reads_a_live_sampler(tmp_path, monkeypatch):
+    """The sampler against a stand-in nvidia-smi that prints one CSV sample every 20 ms: start()
+    returns once a sample has arrived, and stop() keeps only the samples of the marked region."""
+    import time
+    b = _bench()
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!" + sys.executable + "\n"
+                    "import sys, time\n"
+                    "while True:\n"
+                    "    print('1965, 1965, 500, Not Active, Not Active, Not Active, Active',"
+                    " flush=True)\n"
+                    "    time.sleep(0.02)\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ["PATH"])
+    s = b.ClockSampler(None)
+    t = time.monotonic()
+    s.start()
+    assert s.lines and time.monotonic() - t < 5
+    s.mark()
+    time.sleep(0.3)
+    r = s.stop()
+    assert r["window"] == "timed region" and r["samples"] >= 5
+    assert r["sm_mhz"] == 1965.0 and r["reasons"] == ["sw_power_cap"]
+    assert s.proc.poll() is not None  # the sampler process has ended
