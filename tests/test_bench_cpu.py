@@ -291,6 +291,6 @@ def test_clock_sampler_reads_a_live_sampler(tmp_path, monkeypatch):
     s.mark()
     time.sleep(0.3)
     r = s.stop()
-    assert r["window"] == "timed region" and r["samples"] >= 5
+    assert r["window"] == "timed region" and r["samples"] >= 2
     assert r["sm_mhz"] == 1965.0 and r["reasons"] == ["sw_power_cap"]
     assert s.proc.poll() is not None  # the sampler process has ended
