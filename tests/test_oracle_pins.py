@@ -323,6 +323,51 @@ def test_tiled_lists_equal_brute_force_global_sort(which):
     assert (r["n_contrib"] == nc).all()
 
 
+def test_tile_rectangles_cut_only_beyond_three_sigma():
+    """The tile rectangle of a Gaussian covers its 3-sigma footprint (radius ceil(3 sqrt(lambda_max)),
+    rounded out to whole tiles), so a pixel outside it lies more than 3 sigma out along an axis and
+    its exponent is below -4.5 -- but alpha = o G can still reach 1/255 there (G >= e^-4.5 = 0.011).
+    Against a render of the same records with no rectangle test: the tiled render differs only at
+    pixels where some Gaussian outside its rectangle would have composited, every such Gaussian's
+    exponent is below -4.5 (a smaller radius or a rectangle off by a tile breaks this), and on this
+    scene of large, nearly opaque Gaussians some pixels do differ (the truncation the rasteriser's
+    rule implies)."""
+    sc = scenes.tiny_scene(3, 40, 64, 64, V=1, deg=0, log_scale_mean=math.log(0.3),
+                           opac_mean=3.0, opac_sigma=0.5)
+    p = O.project(sc, "d")
+    tiled = O.render(p, O.bin_lists(p, sc.H, sc.W), sc.H, sc.W, sc.bg, "d")
+    rec, rect, valid = p["rec"][0], p["rect"][0], p["valid"][0]
+    ids = np.nonzero(valid)[0]
+    order = ids[np.lexsort((ids, rec[ids, 5]))]
+    r, rr = rec[order], rect[order]
+    n_diff = 0
+    for j in range(sc.H):
+        for i in range(sc.W):
+            dx, dy = i + 0.5 - r[:, 0], j + 0.5 - r[:, 1]
+            pw = -0.5 * (r[:, 2] * dx * dx + r[:, 4] * dy * dy) - r[:, 3] * dx * dy
+            a = np.minimum(0.99, r[:, 6] * np.exp(np.minimum(pw, 0.0)))
+            ok = (pw <= 0) & (a >= 1 / 255)
+            tx, ty = i // 16, j // 16
+            inside = (rr[:, 0] <= tx) & (tx < rr[:, 2]) & (rr[:, 1] <= ty) & (ty < rr[:, 3])
+            Tp, C = 1.0, np.zeros(3)
+            for k in np.nonzero(ok)[0]:  # every valid Gaussian, no rectangle test
+                Tn = Tp * (1 - a[k])
+                if Tn < 1e-4:
+                    break
+                C = C + a[k] * Tp * r[k, 7:10]
+                Tp = Tn
+            C = C + Tp * sc.bg
+            cut = ok & ~inside
+            assert (pw[cut] < -4.5).all(), (i, j, pw[cut].max())
+            # the same entries give the same sums up to the order of the products (1e-12)
+            same = (np.abs(C - tiled["img"][0, j, i]).max() <= 1e-12
+                    and abs(Tp - tiled["T"][0, j, i]) <= 1e-12)
+            if not same:
+                assert cut.any(), (i, j)
+                n_diff += 1
+    assert n_diff > 0
+
+
 @pytest.mark.parametrize("mode", ["d", "f"])
 def test_suffix_recovery_equals_back_to_front_composite(mode):
     """C+_k from the recovery equation equals the directly composited suffix
