@@ -10,7 +10,13 @@ target views. Default workload: the DepthSplat-scale dense scene (5,898,240 Gaus
                   [--path score|backward|attributes] [--cpu-threads T]
 
 --impl reference times the CPU oracle instead (one whole view per step, all host cores or T);
-the default arm reports the same oracle timing once as its cpu_baseline.
+the default arm reports the same oracle timing once as its cpu_baseline, and (score path)
+compares that view, element by element, with the CUDA path run on the same view alone
+(parity_vs_oracle).
+
+Timing: K timed steps with the library's per-kernel event pairs off give value, ms_per_step and
+its median and minimum; K more with them on give the per-kernel times, the rooflines and
+ms_per_step_with_kernel_events. Clocks are sampled during both.
 
 --path backward times the renderer backward instead of the score replay (the gradient comparators:
 raw, detached, support- and parameter-scale-normalised gradients, all four per step).
