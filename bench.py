@@ -429,12 +429,16 @@ COLOUR_ATOL, TOKEN_RTOL, NORM_FLOOR = 1e-5, 1e-4, 1e-3
 
 
 def parity_report(g: dict, o: dict, d: int, chunk: int = 1 << 16) -> dict:
-    """d = SH coefficients per channel ((degree + 1)^2). Element-by-element comparison of one whole view of the workload, CUDA path (g) against the
-    oracle in fp32 decision mode (o): image, final transmittance, contributor counts and every
-    Gaussian's token. The bars are the parity tests': colour within 1e-5 absolute, transmittance
-    and counts exact, tokens within 1e-4 relative L2 per Gaussian (floor 1e-3 x the median token
-    norm); per token block the same ratio with the block's own floor (1e-3 x its median non-zero
-    norm). Reported, not asserted: the tests assert."""
+    """Element-by-element comparison of one whole view of the workload, CUDA path (g) against the
+    oracle in fp32 decision mode (o); d = SH coefficients per channel ((degree + 1)^2): image,
+    final transmittance, contributor counts and every Gaussian's token. The bars are the parity
+    tests': colour within 1e-5 absolute, transmittance and counts exact, tokens within 1e-4
+    relative L2 per Gaussian (floor 1e-3 x the median token norm); per token block the same ratio
+    with the block's own floor (1e-3 x its median non-zero norm). Also the correctness metrics the
+    experiment plan names for its score check ("Block 0": sign accuracy, blockwise cosine), over
+    the Gaussians with q_g >= 1e-3: the fraction of token entries whose sign agrees (entries
+    larger than 1e-4 of their token's norm) and each block's cosine between the two sides.
+    Reported, not asserted: the tests assert."""
     import numpy as np
     img_err = float(np.abs(g["img"].astype(np.float64) - o["img"]).max(initial=0.0))
     t_mis = int((g["T"] != np.asarray(o["T"]).astype(np.float32)).sum())
@@ -462,16 +466,36 @@ def parity_report(g: dict, o: dict, d: int, chunk: int = 1 << 16) -> dict:
 
     floor = floor_of(norms)
     bfloor = np.array([floor_of(bn[:, i]) for i in range(len(names))])
+    covered = np.exp(np.asarray(zo[:, 4 + 3 * d], np.float64)) >= 1e-3  # q_g >= 1e-3
     err = np.empty(G)
     be = np.empty((G, len(names)))
+    cos = np.full((G, len(names)), np.nan, np.float32)
+    n_sign = n_agree = 0
     for s in range(0, G, chunk):
-        dz = np.asarray(zg[s:s + chunk], np.float64) - np.asarray(zo[s:s + chunk], np.float64)
-        dbn, dn = block_norms(dz)
+        a64 = np.asarray(zg[s:s + chunk], np.float64)
+        b64 = np.asarray(zo[s:s + chunk], np.float64)
+        dbn, dn = block_norms(a64 - b64)
         err[s:s + chunk] = dn / np.maximum(norms[s:s + chunk], floor)
         be[s:s + chunk] = dbn / np.maximum(bn[s:s + chunk], bfloor)
+        cov = covered[s:s + chunk]
+        big = (np.abs(b64) > 1e-4 * norms[s:s + chunk, None]) & cov[:, None]
+        n_sign += int(np.count_nonzero(big))
+        n_agree += int(np.count_nonzero(big & (a64 * b64 > 0)))  # b != 0 where big
+        gbn, _ = block_norms(a64)
+        dots = np.stack([np.einsum("ij,ij->i", a64[:, a:b], b64[:, a:b])
+                         for a, b in blocks.values()], axis=1)
+        den = gbn * bn[s:s + chunk]
+        with np.errstate(invalid="ignore", divide="ignore"):
+            c = np.where(den > 0, dots / den, np.nan)
+        c[~cov] = np.nan
+        cos[s:s + chunk] = c
     berr = {k: be[:, i] for i, k in enumerate(names)}
-    covered = np.exp(np.asarray(zo[:, 4 + 3 * d], np.float64)) >= 1e-3  # q_g >= 1e-3
     ok = err <= TOKEN_RTOL
+
+    def cos_stat(i, f):
+        v = cos[:, i]
+        v = v[~np.isnan(v)]
+        return float(f(v)) if v.size else None
 
     def q(a, p):
         return float(np.percentile(a, p)) if a.size else 0.0
@@ -485,7 +509,11 @@ def parity_report(g: dict, o: dict, d: int, chunk: int = 1 << 16) -> dict:
             "token_block_rel_err_p99": {k: q(v, 99) for k, v in berr.items()},
             "gaussians_qg_ge_1e-3": int(covered.sum()),
             "frac_pass_qg_ge_1e-3": float(ok[covered].mean()) if covered.any() else None,
-            "frac_pass_all": float(ok.mean()) if G else None}
+            "frac_pass_all": float(ok.mean()) if G else None,
+            "sign_agreement_qg_ge_1e-3": n_agree / n_sign if n_sign else None,
+            "block_cosine_min_qg_ge_1e-3": {k: cos_stat(i, np.min) for i, k in enumerate(names)},
+            "block_cosine_median_qg_ge_1e-3": {k: cos_stat(i, np.median)
+                                               for i, k in enumerate(names)}}
 
 
 def gpu_view_outputs(sc, obs, fused: bool, deterministic: bool) -> dict:

@@ -294,3 +294,31 @@ def test_clock_sampler_reads_a_live_sampler(tmp_path, monkeypatch):
     assert r["window"] == "timed region" and r["samples"] >= 2
     assert r["sm_mhz"] == 1965.0 and r["reasons"] == ["sw_power_cap"]
     assert s.proc.poll() is not None  # the sampler process has ended
+
+
+def test_parity_report_sign_and_cosine():
+    """The experiment plan's score-check metrics in the report: identical tokens agree in sign
+    everywhere and every block's cosine is 1; one flipped entry of one Gaussian's SH block lowers
+    the sign agreement by one entry and that block's cosine only."""
+    import numpy as np
+    b = _bench()
+    rng = np.random.default_rng(4)
+    d, G = 9, 300
+    K = 9 + 3 * d
+    zo = rng.normal(size=(G, K))
+    zo[:, 4 + 3 * d] = np.log(2.0)  # q_g = 2: every Gaussian counts
+    o = {"img": np.zeros((1, 4, 4, 3)), "T": np.ones((1, 4, 4)),
+         "n_contrib": np.zeros((1, 4, 4), np.int32), "tokens": zo}
+    g = {"img": np.zeros((1, 4, 4, 3), np.float32), "T": np.ones((1, 4, 4), np.float32),
+         "n_contrib": np.zeros((1, 4, 4), np.int32), "tokens": zo.copy()}
+    r = b.parity_report(g, o, d, chunk=50)
+    assert r["sign_agreement_qg_ge_1e-3"] == 1.0
+    assert all(abs(c - 1) < 1e-12 for c in r["block_cosine_min_qg_ge_1e-3"].values())
+    n_big = int((np.abs(zo) > 1e-4 * np.linalg.norm(zo, axis=1)[:, None]).sum())
+    g["tokens"][11, 4 + 5] *= -1.0
+    r = b.parity_report(g, o, d, chunk=50)
+    assert r["sign_agreement_qg_ge_1e-3"] == (n_big - 1) / n_big
+    cmin = r["block_cosine_min_qg_ge_1e-3"]
+    assert cmin["s_sh"] < 1 - 1e-6
+    assert all(abs(c - 1) < 1e-12 for k, c in cmin.items() if k != "s_sh")
+    assert abs(r["block_cosine_median_qg_ge_1e-3"]["s_sh"] - 1) < 1e-12
